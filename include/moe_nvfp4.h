@@ -1,0 +1,206 @@
+/*
+ * moe_nvfp4.h - C ABI of the B200 (sm_100a) NVFP4 mixture-of-experts layer library.
+ *
+ * The layer follows the Basalt pages:
+ *   - "What Basalt changes in a Blackwell local inference stack", section "Experts can move
+ *     without becoming free": the model selects a subset of its experts for each token.
+ *   - "Basalt" project page, section "Expert tiers" (and FAQ "Can it use a second GPU or
+ *     system RAM?"): each token uses only a few experts; the most routed experts form the
+ *     hot tier.
+ *   - "Basalt" project page, "All the numbers", list "Engines: commit, and what is not
+ *     NVIDIA's weights": routed experts are NVIDIA's NVFP4, kept bit-exact, including an
+ *     activation input_scale.
+ * The pages define neither NVFP4 nor the routing rule. This library uses:
+ *   NVFP4  - E2M1 codes (two per byte, element 2i in the low nibble), one E4M3 scale per 16
+ *            consecutive elements of a row ([rows][cols/16] bytes), one float32 tensor scale;
+ *            value = e2m1 * e4m3 * ts. Dynamic tensor scale ts = amax / (6 * 448).
+ *            Conversions round to nearest even and saturate; a negative value that rounds
+ *            to zero keeps its sign (code 0x8); a block whose scale rounds to 0 stores +0s.
+ *   router - logits = x Wr^T + br (float32); top-k by logit, ties to the lower expert id;
+ *            weights = softmax over all experts restricted to the top-k and renormalised.
+ *   FFN    - SwiGLU: h = silu(x Wg^T) * (x Wu^T); h is re-quantised to NVFP4 with tensor
+ *            scale 1.0; o = h Wd^T. A shared expert, if given, is added with weight 1.
+ *   order  - the token permutation is a stable counting sort of assignments a = t*k + j.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller; the library never
+ *     allocates device memory. Scratch comes from a caller-provided workspace `ws` of
+ *     `ws_bytes` bytes (see moe_workspace_size); it must be 256-byte aligned.
+ *   - Tensor pointers must be 16-byte aligned. bf16 values are passed as uint16_t bits.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Argument errors are detected on the host before anything is launched and
+ *     returned synchronously; nothing is enqueued in that case.
+ *   - Device-side problems (a bounded wait that ran out) are recorded in a device status
+ *     word, read with moe_get_device_status (which synchronises the stream).
+ *   - Functions never abort and never throw across the ABI.
+ */
+#ifndef MOE_NVFP4_H
+#define MOE_NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, negative size, misaligned pointer ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* sizes outside what the kernels handle */
+  MOE_ERR_CUDA = 3,               /* a CUDA runtime call failed (see moe_last_error) */
+  MOE_ERR_TIMEOUT = 4,            /* a bounded device-side wait ran out */
+  MOE_ERR_WORKSPACE = 5           /* ws too small or misaligned */
+} moe_status;
+
+/* FFN output modes */
+#define MOE_FFN_ACCUMULATE 0  /* out = float32 y_acc [T][d] = sum_j w[t,j] o[t,j] + shared */
+#define MOE_FFN_PER_ASSIGN 1  /* out = float32 [T*k][d], row p = o of sorted_assign[p];
+                                 shared_out = float32 [T][d] (unweighted) */
+/* FFN kernel paths */
+#define MOE_PATH_AUTO 0       /* PREFILL when available and T is large, else DECODE */
+#define MOE_PATH_DECODE 1     /* CUDA-core GEMV path (any T; meant for 1-64 tokens) */
+#define MOE_PATH_PREFILL 2    /* tcgen05 block-scaled grouped GEMM path */
+
+/* workspace query operations */
+#define MOE_OP_LAYER 0        /* enough for every call of one layer forward */
+#define MOE_OP_ROUTE 1
+#define MOE_OP_QUANT 2
+#define MOE_OP_FFN 3
+
+/*
+ * Expert weights of one expert group (E routed experts, or E = 1 for the shared expert),
+ * natural NVFP4 layout as a checkpoint stores it. All pointers are device pointers.
+ *   gu_codes  [E][2I][d/2]   gate rows 0..I-1, then up rows I..2I-1
+ *   gu_scales [E][2I][d/16]  E4M3 bytes
+ *   gu_ts     [E][2]         float32 tensor scales (gate, up)
+ *   dn_codes  [E][d][I/2]
+ *   dn_scales [E][d][I/16]
+ *   dn_ts     [E]            float32
+ *   gu_sf_tiled, dn_sf_tiled: the same scale bytes re-tiled for the tensor-core path by
+ *            moe_pack_experts (NULL if not packed; the PREFILL path then refuses).
+ */
+typedef struct moe_expert_weights {
+  int32_t E, d, I;
+  const uint8_t* gu_codes;
+  const uint8_t* gu_scales;
+  const float* gu_ts;
+  const uint8_t* dn_codes;
+  const uint8_t* dn_scales;
+  const float* dn_ts;
+  const uint8_t* gu_sf_tiled;
+  const uint8_t* dn_sf_tiled;
+} moe_expert_weights_t;
+
+typedef struct moe_experts {
+  moe_expert_weights_t routed;
+  moe_expert_weights_t shared;  /* used when has_shared != 0; shared.E must be 1 */
+  int32_t has_shared;
+} moe_experts_t;
+
+/*
+ * nvfp4_quantize_act - NVFP4 quantisation of a bf16 matrix (activations, or weights at
+ * load time). Steps: amax over the whole matrix (unless ts_in is given), then per 16-block
+ *   sb = (amax_b / 6) / ts; s = E4M3(sb); q_i = E2M1(x_i / (E4M3value(s) * ts)).
+ *   x_bf16  [rows][cols] device; cols % 16 == 0
+ *   ts_in   device float32[1] static tensor scale, or NULL for the dynamic amax/2688
+ *   codes   [rows][cols/2] out; scales [rows][cols/16] out; ts_out float32[1] out (may be
+ *           NULL); ws needs moe_workspace_size(MOE_OP_QUANT, rows*cols/... ) bytes.
+ * rows == 0 is allowed (writes only ts_out = 1 or *ts_in).
+ */
+moe_status nvfp4_quantize_act(const uint16_t* x_bf16, int64_t rows, int32_t cols,
+                              const float* ts_in, uint8_t* codes, uint8_t* scales,
+                              float* ts_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_route - router (A1), softmax/top-k/renormalisation (A2) and permutation (A3).
+ *   x_bf16 [T][d]; Wr float32 [E][d]; br float32 [E] or NULL.
+ *   topk_idx int32 [T][k] (descending logit), topk_w float32 [T][k],
+ *   counts int32 [E], offsets int32 [E+1], sorted_assign int32 [T*k] (assignment ids
+ *   a = t*k + j grouped by expert, increasing a within an expert), assign_pos int32 [T*k]
+ *   (inverse of sorted_assign). 1 <= k <= 32, k <= E <= 1024, d % 16 == 0.
+ */
+moe_status moe_route(const uint16_t* x_bf16, int32_t T, int32_t d, const float* Wr,
+                     const float* br, int32_t E, int32_t k, int32_t* topk_idx,
+                     float* topk_w, int32_t* counts, int32_t* offsets,
+                     int32_t* sorted_assign, int32_t* assign_pos, void* ws,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * moe_permute - the permutation step (A3) alone, from given top-k indices: a stable
+ * counting sort of the T*k assignments by expert, with the per-expert histogram.
+ * Same outputs and limits as moe_route.
+ */
+moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
+                       int32_t* counts, int32_t* offsets, int32_t* sorted_assign,
+                       int32_t* assign_pos, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_pack_experts - re-tile the E4M3 scale bytes of an expert group for the tensor-core
+ * (PREFILL) path. gu_sf_tiled needs E*2I*d/16 bytes, dn_sf_tiled E*d*I/16 bytes. Run once
+ * per weight load; the natural-layout weights stay in use by the DECODE path.
+ * Requires d % 128 == 0 and I % 64 == 0.
+ */
+moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
+                            uint8_t* dn_sf_tiled, void* stream);
+
+/*
+ * moe_expert_ffn - expert SwiGLU FFN for all routed assignments (A5-A7) and the shared
+ * expert (A8).
+ *   xq_codes [T][d/2], xq_scales [T][d/16], xq_ts float32[1]: the NVFP4 activation.
+ *   offsets [E+1], sorted_assign [T*k], topk_w [T][k]: from moe_route / moe_permute.
+ *   mode MOE_FFN_ACCUMULATE: out = float32 [T][d] (overwritten), shared_out unused.
+ *   mode MOE_FFN_PER_ASSIGN: out = float32 [T*k][d] in sorted order (unweighted);
+ *        shared_out = float32 [T][d] when the layer has a shared expert, else NULL.
+ *   path: MOE_PATH_AUTO / DECODE / PREFILL.
+ * Limits: d % 16 == 0, I % 16 == 0, d <= 8192, I <= 8192 (PREFILL: d % 256 == 0,
+ * I % 64 == 0, scales packed). Accumulation order in ACCUMULATE mode is not fixed.
+ */
+moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales,
+                          const float* xq_ts, int32_t T, const moe_experts_t* W, int32_t k,
+                          const int32_t* offsets, const int32_t* sorted_assign,
+                          const float* topk_w, int32_t mode, int32_t path, float* out,
+                          float* shared_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine - weighted combine (A9) and cast to bf16.
+ *   mode MOE_FFN_ACCUMULATE: expert_out = y_acc float32 [T][d]; y = bf16(y_acc).
+ *   mode MOE_FFN_PER_ASSIGN: y[t] = sum_j topk_w[t,j] * expert_out[assign_pos[t*k+j]]
+ *        + shared_out[t] (shared_out may be NULL).
+ *   rms_renorm != 0: each output row is scaled to unit root-mean-square before the cast
+ *        (an all-zero row stays zero); used to chain layers of a decode stack.
+ *   y_bf16 [T][d] out.
+ */
+moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const float* expert_out,
+                       const float* shared_out, const float* topk_w,
+                       const int32_t* assign_pos, int32_t rms_renorm, uint16_t* y_bf16,
+                       void* stream);
+
+/*
+ * moe_expert_hist - cumulative routing counts and hot-to-cold ranking (A10).
+ *   counts int32 [E] (this call's histogram), cum int64 [E] in/out (cum += counts, or
+ *   cum = counts when reset != 0), rank_out int32 [E] or NULL: expert ids from most to
+ *   least routed, equal counts by lower id. E <= 4096.
+ */
+moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32_t* rank_out,
+                           int32_t reset, void* stream);
+
+/* Bytes of workspace needed by one op (MOE_OP_*) for these sizes (MOE_OP_LAYER: max). */
+size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k, int32_t I);
+
+/* Synchronise `stream` and return the device status word (MOE_OK or MOE_ERR_TIMEOUT);
+ * `clear` != 0 resets it afterwards. */
+moe_status moe_get_device_status(void* stream, int32_t clear, int32_t* status_out);
+
+/* Static description of a status code, and a per-thread detail of the last failure. */
+const char* moe_status_string(moe_status s);
+const char* moe_last_error(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_NVFP4_H */

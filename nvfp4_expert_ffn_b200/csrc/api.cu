@@ -1,0 +1,313 @@
+// C ABI entry points (declared in include/moe_nvfp4.h): argument validation on the host,
+// workspace carving, and kernel launches on the caller's stream.
+#include <mutex>
+#include <string>
+
+#include "../../include/moe_nvfp4.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+__device__ int32_t g_device_status = 0;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+moe_status fail(moe_status s, const std::string& msg) {
+  t_last_error = msg;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  t_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return MOE_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Per-device one-time setup: SM count and dynamic shared memory limits.
+moe_status device_info(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_CUDA, "device index out of range");
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (major != 10 || minor != 0)
+      return fail(MOE_ERR_CUDA, "this library is built for sm_100a (B200); device is sm_" +
+                                    std::to_string(major * 10 + minor));
+    e = cudaDeviceGetAttribute(&di.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = init_kernel_attributes();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel attribute setup");
+    di.ready = true;
+  }
+  *num_sms = di.num_sms;
+  return MOE_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+size_t quant_ws_bytes() { return align256(kMaxPartials * sizeof(float)); }
+
+size_t ffn_ws_bytes(int64_t T, int d, int E, int k, int I) {
+  return ffn_decode_ws_bytes(T, d, E, k, I);
+}
+
+moe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return MOE_OK;
+  if (!ws || ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "workspace too small: need " + std::to_string(need) + " bytes, got " +
+                                       std::to_string(ws_bytes));
+  if (((uintptr_t)ws & 255u) != 0) return fail(MOE_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  return MOE_OK;
+}
+
+moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E, int d, int I) {
+  const std::string n(name);
+  if (w.E != E || w.d != d || w.I != I) return fail(MOE_ERR_INVALID_ARG, n + ": inconsistent E/d/I");
+  const void* ps[6] = {w.gu_codes, w.gu_scales, w.gu_ts, w.dn_codes, w.dn_scales, w.dn_ts};
+  for (const void* p : ps) {
+    if (!p) return fail(MOE_ERR_INVALID_ARG, n + ": null weight pointer");
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, n + ": weight pointer not 16-byte aligned");
+  }
+  return MOE_OK;
+}
+
+ExpertGroup to_group(const moe_expert_weights_t& w) {
+  return ExpertGroup{w.gu_codes, w.gu_scales, w.gu_ts, w.dn_codes, w.dn_scales, w.dn_ts,
+                     w.gu_sf_tiled, w.dn_sf_tiled};
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_version(void) { return 100; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_WORKSPACE: return "workspace too small or misaligned";
+  }
+  return "unknown status";
+}
+
+const char* moe_last_error(void) { return t_last_error.c_str(); }
+
+size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k, int32_t I) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || I <= 0) return 0;
+  const size_t q = quant_ws_bytes();
+  const size_t r = align256(route_ws_bytes(T, d, E, k));
+  const size_t f = align256(ffn_ws_bytes(T, d, E, k, I));
+  switch (op) {
+    case MOE_OP_QUANT: return q;
+    case MOE_OP_ROUTE: return r;
+    case MOE_OP_FFN: return f;
+    case MOE_OP_LAYER: {
+      size_t m = q > r ? q : r;
+      return m > f ? m : f;
+    }
+  }
+  return 0;
+}
+
+moe_status nvfp4_quantize_act(const uint16_t* x, int64_t rows, int32_t cols, const float* ts_in,
+                              uint8_t* codes, uint8_t* scales, float* ts_out, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (rows < 0 || cols <= 0) return fail(MOE_ERR_INVALID_ARG, "rows must be >= 0 and cols > 0");
+  if (cols % kBlock) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "cols must be a multiple of 16");
+  if (rows > 0) {
+    if (!x || !codes || !scales) return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(x) || !aligned16(codes))
+      return fail(MOE_ERR_INVALID_ARG, "x and codes must be 16-byte aligned");
+  }
+  if (ts_in && !aligned16(ts_in)) return fail(MOE_ERR_INVALID_ARG, "ts_in must be 16-byte aligned");
+  const int64_t nblk = rows * (int64_t)(cols / kBlock);
+  if (nblk > 4096 && !ts_in) {
+    moe_status s = check_ws(ws, ws_bytes, quant_ws_bytes());
+    if (s != MOE_OK) return s;
+  }
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_quantize(x, rows, cols, ts_in, codes, scales, ts_out, ws, sms,
+                                  (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "nvfp4_quantize_act launch");
+}
+
+static moe_status check_route_common(int32_t T, int32_t E, int32_t k, int32_t* counts,
+                                     int32_t* offsets, int32_t* sorted_assign,
+                                     int32_t* assign_pos) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (k < 1 || k > 32) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "k must be in [1, 32]");
+  if (E < k || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E must be in [k, 1024]");
+  if ((int64_t)T * k > (int64_t)1 << 30) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "T*k too large");
+  if (!counts || !offsets) return fail(MOE_ERR_INVALID_ARG, "null counts/offsets");
+  if (T > 0 && (!sorted_assign || !assign_pos)) return fail(MOE_ERR_INVALID_ARG, "null permutation output");
+  return MOE_OK;
+}
+
+moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E, int32_t* counts,
+                       int32_t* offsets, int32_t* sorted_assign, int32_t* assign_pos, void* ws,
+                       size_t ws_bytes, void* stream) {
+  moe_status s = check_route_common(T, E, k, counts, offsets, sorted_assign, assign_pos);
+  if (s != MOE_OK) return s;
+  if (T > 0 && !topk_idx) return fail(MOE_ERR_INVALID_ARG, "null topk_idx");
+  if ((int64_t)T * k > 4096) {
+    s = check_ws(ws, ws_bytes, permute_ws_bytes(T, k, E));
+    if (s != MOE_OK) return s;
+  }
+  int sms = 0;
+  s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_permute(topk_idx, T, k, E, counts, offsets, sorted_assign, assign_pos, ws,
+                                 (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_permute launch");
+}
+
+moe_status moe_route(const uint16_t* x, int32_t T, int32_t d, const float* Wr, const float* br,
+                     int32_t E, int32_t k, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                     int32_t* offsets, int32_t* sorted_assign, int32_t* assign_pos, void* ws,
+                     size_t ws_bytes, void* stream) {
+  moe_status s = check_route_common(T, E, k, counts, offsets, sorted_assign, assign_pos);
+  if (s != MOE_OK) return s;
+  if (d <= 0 || d % kBlock || d > 8192) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "d must be a multiple of 16 in [16, 8192]");
+  if (T > 0) {
+    if (!x || !Wr || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+    if (!aligned16(x) || !aligned16(Wr)) return fail(MOE_ERR_INVALID_ARG, "x and Wr must be 16-byte aligned");
+    s = check_ws(ws, ws_bytes, route_ws_bytes(T, d, E, k));
+    if (s != MOE_OK) return s;
+  }
+  int sms = 0;
+  s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_route(x, T, d, Wr, br, E, k, topk_idx, topk_w, counts, offsets,
+                               sorted_assign, assign_pos, ws, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
+}
+
+moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
+                            uint8_t* dn_sf_tiled, void* stream) {
+  (void)W; (void)gu_sf_tiled; (void)dn_sf_tiled; (void)stream;
+  return fail(MOE_ERR_UNSUPPORTED_SHAPE, "tensor-core path not built yet");
+}
+
+moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, const float* xq_ts,
+                          int32_t T, const moe_experts_t* W, int32_t k, const int32_t* offsets,
+                          const int32_t* sorted_assign, const float* topk_w, int32_t mode,
+                          int32_t path, float* out, float* shared_out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (!W) return fail(MOE_ERR_INVALID_ARG, "null weights");
+  const int E = W->routed.E, d = W->routed.d, I = W->routed.I;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (k < 1 || k > 32 || E < k || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "need 1 <= k <= 32, k <= E <= 1024");
+  if (d <= 0 || I <= 0 || d % kBlock || I % kBlock || d > 8192 || I > 8192)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "d and I must be multiples of 16 in [16, 8192]");
+  if (mode != MOE_FFN_ACCUMULATE && mode != MOE_FFN_PER_ASSIGN) return fail(MOE_ERR_INVALID_ARG, "bad mode");
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL)
+    return fail(MOE_ERR_INVALID_ARG, "bad path");
+  moe_status s = check_weights(W->routed, "routed", E, d, I);
+  if (s != MOE_OK) return s;
+  if (W->has_shared) {
+    s = check_weights(W->shared, "shared", 1, d, I);
+    if (s != MOE_OK) return s;
+  }
+  if (T == 0) return MOE_OK;
+  if (!xq_codes || !xq_scales || !xq_ts || !offsets || !sorted_assign || !topk_w || !out)
+    return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(xq_codes) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "xq_codes/out must be 16-byte aligned");
+  if (mode == MOE_FFN_PER_ASSIGN && W->has_shared && !shared_out)
+    return fail(MOE_ERR_INVALID_ARG, "shared_out needed in PER_ASSIGN mode with a shared expert");
+  if (path == MOE_PATH_PREFILL) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "tensor-core path not built yet");
+  const size_t need = ffn_ws_bytes(T, d, E, k, I);
+  s = check_ws(ws, ws_bytes, need);
+  if (s != MOE_OK) return s;
+  int sms = 0;
+  s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  FfnArgs a;
+  a.xq_codes = xq_codes;
+  a.xq_scales = xq_scales;
+  a.xq_ts = xq_ts;
+  a.T = T; a.d = d; a.I = I; a.E = E; a.k = k;
+  a.routed = to_group(W->routed);
+  a.shared = W->has_shared ? to_group(W->shared) : ExpertGroup{};
+  a.has_shared = W->has_shared ? 1 : 0;
+  a.offsets = offsets;
+  a.sorted_assign = sorted_assign;
+  a.topk_w = topk_w;
+  a.mode = mode;
+  a.out = out;
+  a.shared_out = shared_out;
+  const size_t slots = (size_t)T * k + T;
+  a.h_codes = reinterpret_cast<uint8_t*>(ws);
+  a.h_scales = reinterpret_cast<uint8_t*>(ws) + align256(slots * (I / 2));
+  cudaError_t e = launch_ffn_decode(a, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
+}
+
+moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const float* expert_out,
+                       const float* shared_out, const float* topk_w, const int32_t* assign_pos,
+                       int32_t rms_renorm, uint16_t* y, void* stream) {
+  if (T < 0 || d <= 0 || d % kBlock) return fail(MOE_ERR_INVALID_ARG, "T >= 0 and d a positive multiple of 16");
+  if (mode != MOE_FFN_ACCUMULATE && mode != MOE_FFN_PER_ASSIGN) return fail(MOE_ERR_INVALID_ARG, "bad mode");
+  if (T == 0) return MOE_OK;
+  if (!expert_out || !y) return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+  if (mode == MOE_FFN_PER_ASSIGN && (k < 1 || !topk_w || !assign_pos))
+    return fail(MOE_ERR_INVALID_ARG, "PER_ASSIGN combine needs k >= 1, topk_w and assign_pos");
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_combine(T, d, k, mode, expert_out, shared_out, topk_w, assign_pos,
+                                 rms_renorm ? 1 : 0, y, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_combine launch");
+}
+
+moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32_t* rank_out,
+                           int32_t reset, void* stream) {
+  if (E < 1 || E > 4096) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "E must be in [1, 4096]");
+  if (!counts || !cum) return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_hist(counts, E, cum, rank_out, reset ? 1 : 0, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_hist launch");
+}
+
+moe_status moe_get_device_status(void* stream, int32_t clear, int32_t* status_out) {
+  if (!status_out) return fail(MOE_ERR_INVALID_ARG, "null status_out");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemcpyFromSymbol(status_out, g_device_status, sizeof(int32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "read device status");
+  if (clear) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "clear device status");
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

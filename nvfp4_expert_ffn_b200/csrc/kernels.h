@@ -1,0 +1,77 @@
+// Internal launchers (host side) of the sm_100a kernels. Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Device-side view of one expert group (natural NVFP4 layout, see moe_nvfp4.h).
+struct ExpertGroup {
+  const uint8_t* gu_codes;
+  const uint8_t* gu_scales;
+  const float* gu_ts;
+  const uint8_t* dn_codes;
+  const uint8_t* dn_scales;
+  const float* dn_ts;
+  const uint8_t* gu_sf_tiled;
+  const uint8_t* dn_sf_tiled;
+};
+
+struct FfnArgs {
+  const uint8_t* xq_codes;
+  const uint8_t* xq_scales;
+  const float* xq_ts;
+  int T, d, I, E, k;
+  ExpertGroup routed, shared;
+  int has_shared;
+  const int32_t* offsets;
+  const int32_t* sorted_assign;
+  const float* topk_w;
+  int mode;  // 0 accumulate, 1 per-assignment
+  float* out;
+  float* shared_out;
+  // workspace: NVFP4 h of every (assignment slot, h-block); slots 0..T*k-1 are sorted
+  // positions of routed assignments, T*k + t is token t of the shared expert
+  uint8_t* h_codes;   // [(T*k + T)][I/2]
+  uint8_t* h_scales;  // [(T*k + T)][I/16]
+};
+
+cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int cols, const float* ts_in,
+                            uint8_t* codes, uint8_t* scales, float* ts_out, void* ws, int num_sms,
+                            cudaStream_t st);
+
+cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const float* br, int E,
+                         int k, int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                         int32_t* sorted_assign, int32_t* assign_pos, void* ws, int num_sms,
+                         cudaStream_t st);
+size_t route_ws_bytes(int64_t T, int d, int E, int k);
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
+                           int32_t* offsets, int32_t* sorted_assign, int32_t* assign_pos, void* ws,
+                           cudaStream_t st);
+size_t permute_ws_bytes(int64_t T, int k, int E);
+
+cudaError_t launch_hist(const int32_t* counts, int E, int64_t* cum, int32_t* rank_out, int reset,
+                        cudaStream_t st);
+
+cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, cudaStream_t st);
+size_t ffn_decode_ws_bytes(int64_t T, int d, int E, int k, int I);
+size_t ffn_decode_smem_gateup(int d, int E);
+size_t ffn_decode_smem_down(int I, int E);
+
+cudaError_t launch_combine(int T, int d, int k, int mode, const float* expert_out,
+                           const float* shared_out, const float* topk_w, const int32_t* assign_pos,
+                           int rms, uint16_t* y, cudaStream_t st);
+
+// one-time per-device kernel attribute setup (dynamic shared memory limits)
+cudaError_t init_route_attributes();
+cudaError_t init_ffn_decode_attributes();
+inline cudaError_t init_kernel_attributes() {
+  cudaError_t e = init_route_attributes();
+  if (e != cudaSuccess) return e;
+  return init_ffn_decode_attributes();
+}
+
+}  // namespace moe

@@ -1,0 +1,416 @@
+// Router (logits), softmax/top-k/renormalisation, token permutation and expert histogram.
+//
+// Basalt pages: "What Basalt changes in a Blackwell local inference stack", section
+// "Experts can move without becoming free" (each token selects a subset of experts) and
+// the "Basalt" project page, section "Expert tiers" (the most routed experts are the hot
+// ones). Reading used here: logits = x Wr^T + br in float32, top-k by logit with ties to
+// the lower expert id, weights = softmax restricted to the top-k and renormalised; the
+// permutation is a stable counting sort of assignments a = t*k + j by expert.
+//
+// Precision: a float32 sum over d = 2048 products accumulates ~1e-6 of rounding error,
+// the size of the top-k tie margin. Dot products therefore use float64 accumulation
+// (decode GEMV: exact float64 FMAs; prefill GEMM: float32 partial sums over 32 products
+// folded into float64 totals), and each logit is rounded to float32 once.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- router GEMV (T <= 8)
+// One warp per expert row of Wr; x (T x d bf16) staged in shared memory.
+constexpr int kGemvMaxT = 8;
+
+__global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                          const float* __restrict__ Wr,
+                                                          const float* __restrict__ br, int E,
+                                                          float* __restrict__ logits) {
+  extern __shared__ __align__(16) uint16_t xs[];  // [T][d]
+  const int nvec = T * d / 8;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x)
+    reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  for (int e = blockIdx.x * warps + (threadIdx.x >> 5); e < E; e += gridDim.x * warps) {
+    double acc[kGemvMaxT];
+#pragma unroll
+    for (int t = 0; t < kGemvMaxT; ++t) acc[t] = 0.0;
+    const float4* w4 = reinterpret_cast<const float4*>(Wr + (size_t)e * d);
+    for (int c = lane; c < d / 4; c += 32) {
+      const float4 w = __ldg(w4 + c);
+#pragma unroll
+      for (int t = 0; t < kGemvMaxT; ++t) {
+        if (t < T) {
+          const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * d + 4 * c);
+          acc[t] = fma((double)bf16_to_f32(xv.x & 0xFFFFu), (double)w.x, acc[t]);
+          acc[t] = fma((double)bf16_to_f32(xv.x >> 16), (double)w.y, acc[t]);
+          acc[t] = fma((double)bf16_to_f32(xv.y & 0xFFFFu), (double)w.z, acc[t]);
+          acc[t] = fma((double)bf16_to_f32(xv.y >> 16), (double)w.w, acc[t]);
+        }
+      }
+    }
+    const double b = br ? (double)__ldg(br + e) : 0.0;
+#pragma unroll
+    for (int t = 0; t < kGemvMaxT; ++t) {
+      if (t < T) {
+        double s = warp_sum_f64(acc[t]);
+        if (lane == 0) logits[(size_t)t * E + e] = (float)(s + b);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- router GEMM (large T)
+// 64 tokens x 64 experts per CTA, 256 threads with 4x4 outputs each, K tiles of 32.
+constexpr int kRgBM = 64, kRgBN = 64, kRgBK = 32;
+
+__global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __restrict__ x, int T, int d,
+                                                          const float* __restrict__ Wr,
+                                                          const float* __restrict__ br, int E,
+                                                          float* __restrict__ logits) {
+  __shared__ float xs[kRgBK][kRgBM + 4];
+  __shared__ float ws[kRgBK][kRgBN + 4];
+  const int m0 = blockIdx.y * kRgBM, n0 = blockIdx.x * kRgBN;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double tot[4][4];
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tot[i][j] = 0.0, acc[i][j] = 0.0f;
+  for (int k0 = 0; k0 < d; k0 += kRgBK) {
+    // x tile: 64 rows x 32 cols bf16 = 256 x 8 elements
+    {
+      const int r = threadIdx.x >> 2, c8 = (threadIdx.x & 3) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (m0 + r < T && k0 + c8 < d) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(m0 + r) * d + k0 + c8));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        xs[c8 + 2 * i][r] = bf16_to_f32(w[i] & 0xFFFFu);
+        xs[c8 + 2 * i + 1][r] = bf16_to_f32(w[i] >> 16);
+      }
+    }
+    // W tile: 64 rows x 32 cols fp32 = 256 x 8 elements
+    {
+      const int r = threadIdx.x >> 2, c8 = (threadIdx.x & 3) * 8;
+      float4 a = make_float4(0, 0, 0, 0), b = a;
+      if (n0 + r < E && k0 + c8 < d) {
+        const float4* p = reinterpret_cast<const float4*>(Wr + (size_t)(n0 + r) * d + k0 + c8);
+        a = __ldg(p);
+        b = __ldg(p + 1);
+      }
+      ws[c8 + 0][r] = a.x; ws[c8 + 1][r] = a.y; ws[c8 + 2][r] = a.z; ws[c8 + 3][r] = a.w;
+      ws[c8 + 4][r] = b.x; ws[c8 + 5][r] = b.y; ws[c8 + 6][r] = b.z; ws[c8 + 7][r] = b.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kRgBK; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tot[i][j] += (double)acc[i][j], acc[i][j] = 0.0f;
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < E) logits[(size_t)m * E + n] = (float)(tot[i][j] + (br ? (double)br[n] : 0.0));
+    }
+  }
+}
+
+// ---------------------------------------------------------------- top-k + weights
+// One warp per token. Lane L holds logits L, L+32, ...; k rounds of a warp arg-max with
+// ties to the lower index. Weights: exp(l_j - l_max) / sum over the chosen k.
+constexpr int kTopkMaxPerLane = 32;  // E <= 1024
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                   int32_t* __restrict__ topk_idx,
+                                                   float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + (size_t)t * E;
+  float v[kTopkMaxPerLane];
+  const int nper = (E + 31) >> 5;
+#pragma unroll
+  for (int j = 0; j < kTopkMaxPerLane; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (j < nper && e < E) ? row[e] : -INFINITY;
+  }
+  uint32_t taken = 0;
+  float top0 = 0.0f, mysel_l = 0.0f;
+  int mysel_e = 0;
+  for (int r = 0; r < k; ++r) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < kTopkMaxPerLane; ++j) {
+      const int e = lane + 32 * j;
+      if (j < nper && e < E && !((taken >> j) & 1u)) {
+        if (v[j] > bv || (v[j] == bv && e < be)) bv = v[j], be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (r == 0) top0 = bv;
+    if (lane == r) mysel_l = bv, mysel_e = be;
+  }
+  // lane j < k holds the j-th selection
+  const float ex = (lane < k) ? expf(mysel_l - top0) : 0.0f;
+  const float sum = warp_sum(ex);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = mysel_e;
+    topk_w[(size_t)t * k + lane] = ex / sum;
+  }
+}
+
+// ---------------------------------------------------------------- permutation
+// Stable counting sort of n = T*k assignments by expert. Chunk c covers assignments
+// [c*kPermChunk, (c+1)*kPermChunk). Pass 1: per-chunk histograms (warp-aggregated shared
+// atomics). Pass 2: counts, offsets and each chunk's base per expert. Pass 3: each chunk
+// assigns positions in assignment order (warps in turn, lanes ranked with match_any).
+constexpr int kPermChunk = 4096;
+constexpr int kPermThreads = 512;
+
+MOE_DEV void warp_aggregated_add(int* hist, int e) {
+  const uint32_t peers = __match_any_sync(__activemask(), e);
+  const int leader = __ffs(peers) - 1;
+  if ((threadIdx.x & 31) == leader) atomicAdd(hist + e, __popc(peers));
+}
+
+MOE_DEV void chunk_histogram(const int32_t* idx, int n, int c, int E, int* sh) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sh[e] = 0;
+  __syncthreads();
+  const int beg = c * kPermChunk, end = min(n, beg + kPermChunk);
+  for (int a = beg + threadIdx.x; a < end; a += blockDim.x) warp_aggregated_add(sh, idx[a]);
+  __syncthreads();
+}
+
+// Positions for chunk c given run[e] = first free position of expert e for this chunk.
+MOE_DEV void chunk_scatter(const int32_t* idx, int n, int c, int* run, int32_t* sorted_assign,
+                           int32_t* assign_pos) {
+  const int beg = c * kPermChunk, end = min(n, beg + kPermChunk);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int base = beg; base < end; base += blockDim.x) {
+    const int a = base + threadIdx.x;
+    const bool valid = a < end;
+    const int e = valid ? idx[a] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const bool last = (peers >> lane) == 1u;  // highest lane of its group
+    for (int w = 0; w < nw; ++w) {
+      if (warp == w && valid) {
+        const int p = run[e] + rank;
+        sorted_assign[p] = a;
+        assign_pos[a] = p;
+      }
+      __syncthreads();
+      if (warp == w && valid && last) run[e] += __popc(peers);
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* __restrict__ idx, int n,
+                                                                 int E, int32_t* __restrict__ chunk_hist) {
+  extern __shared__ int sh[];
+  chunk_histogram(idx, n, blockIdx.x, E, sh);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = sh[e];
+}
+
+// One CTA: counts, offsets, and chunk_hist[c][e] := base position of chunk c for expert e.
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_hist, int nchunk,
+                                                         int E, int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets) {
+  __shared__ int tmp[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    int run = 0;
+    if (e < E) {
+      for (int c = 0; c < nchunk; ++c) {
+        const int h = chunk_hist[(size_t)c * E + e];
+        chunk_hist[(size_t)c * E + e] = run;
+        run += h;
+      }
+    }
+    int total;
+    const int excl = block_exclusive_scan(run, tmp, &total) + carry;
+    if (e < E) {
+      counts[e] = run;
+      offsets[e] = excl;
+      for (int c = 0; c < nchunk; ++c) chunk_hist[(size_t)c * E + e] += excl;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offsets[E] = carry;
+}
+
+__global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_t* __restrict__ idx, int n,
+                                                                    int E,
+                                                                    const int32_t* __restrict__ chunk_base,
+                                                                    int32_t* __restrict__ sorted_assign,
+                                                                    int32_t* __restrict__ assign_pos) {
+  extern __shared__ int run[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = chunk_base[(size_t)blockIdx.x * E + e];
+  __syncthreads();
+  chunk_scatter(idx, n, blockIdx.x, run, sorted_assign, assign_pos);
+}
+
+// Single CTA for n <= kPermChunk: histogram, scan and scatter in one launch.
+__global__ void __launch_bounds__(kPermThreads) perm_small_kernel(const int32_t* __restrict__ idx, int n,
+                                                                  int E, int32_t* __restrict__ counts,
+                                                                  int32_t* __restrict__ offsets,
+                                                                  int32_t* __restrict__ sorted_assign,
+                                                                  int32_t* __restrict__ assign_pos) {
+  extern __shared__ int sh[];  // [E]
+  __shared__ int tmp[32];
+  __shared__ int carry;
+  chunk_histogram(idx, n, 0, E, sh);
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    const int h = e < E ? sh[e] : 0;
+    int total;
+    const int excl = block_exclusive_scan(h, tmp, &total) + carry;
+    if (e < E) {
+      counts[e] = h;
+      offsets[e] = excl;
+      sh[e] = excl;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offsets[E] = carry;
+  __syncthreads();
+  chunk_scatter(idx, n, 0, sh, sorted_assign, assign_pos);
+}
+
+__global__ void zero_counts_kernel(int E, int32_t* counts, int32_t* offsets) {
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+    if (e < E) counts[e] = 0;
+    offsets[e] = 0;
+  }
+}
+
+cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
+                           int32_t* offsets, int32_t* sorted_assign, int32_t* assign_pos,
+                           void* ws, cudaStream_t st) {
+  const int n = T * k;
+  if (n == 0) {
+    zero_counts_kernel<<<1, 1024, 0, st>>>(E, counts, offsets);
+    return cudaGetLastError();
+  }
+  const size_t smem = (size_t)E * sizeof(int);
+  if (n <= kPermChunk) {
+    perm_small_kernel<<<1, kPermThreads, smem, st>>>(idx, n, E, counts, offsets, sorted_assign,
+                                                     assign_pos);
+    return cudaGetLastError();
+  }
+  const int nchunk = (n + kPermChunk - 1) / kPermChunk;
+  int32_t* chunk_hist = reinterpret_cast<int32_t*>(ws);
+  perm_hist_kernel<<<nchunk, kPermThreads, smem, st>>>(idx, n, E, chunk_hist);
+  perm_scan_kernel<<<1, 1024, 0, st>>>(chunk_hist, nchunk, E, counts, offsets);
+  perm_scatter_kernel<<<nchunk, kPermThreads, smem, st>>>(idx, n, E, chunk_hist, sorted_assign,
+                                                          assign_pos);
+  return cudaGetLastError();
+}
+
+size_t permute_ws_bytes(int64_t T, int k, int E) {
+  const int64_t n = T * k;
+  const int64_t nchunk = (n + kPermChunk - 1) / kPermChunk;
+  return (size_t)(nchunk * E * sizeof(int32_t));
+}
+
+size_t route_ws_bytes(int64_t T, int d, int E, int k) {
+  const size_t logits = ((size_t)T * E * sizeof(float) + 255) & ~(size_t)255;
+  return logits + permute_ws_bytes(T, k, E);
+}
+
+cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const float* br,
+                         int E, int k, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                         int32_t* offsets, int32_t* sorted_assign, int32_t* assign_pos, void* ws,
+                         int num_sms, cudaStream_t st) {
+  if (T == 0) return launch_permute(nullptr, 0, k, E, counts, offsets, sorted_assign, assign_pos,
+                                    nullptr, st);
+  float* logits = reinterpret_cast<float*>(ws);
+  const size_t logits_bytes = ((size_t)T * E * sizeof(float) + 255) & ~(size_t)255;
+  void* perm_ws = reinterpret_cast<char*>(ws) + logits_bytes;
+  if (T <= kGemvMaxT) {
+    const size_t smem = (size_t)T * d * sizeof(uint16_t);
+    const int grid = (E + 7) / 8;
+    router_gemv_kernel<<<grid, 256, smem, st>>>(x, T, d, Wr, br, E, logits);
+  } else {
+    dim3 grid((E + kRgBN - 1) / kRgBN, (T + kRgBM - 1) / kRgBM);
+    router_gemm_kernel<<<grid, 256, 0, st>>>(x, T, d, Wr, br, E, logits);
+  }
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  return launch_permute(topk_idx, T, k, E, counts, offsets, sorted_assign, assign_pos, perm_ws, st);
+}
+
+// ---------------------------------------------------------------- cumulative histogram
+// One CTA: cum[e] += counts[e] (or = on reset); rank position of e is the number of experts
+// that are hotter, or equally hot with a lower id.
+__global__ void __launch_bounds__(1024) hist_kernel(const int32_t* __restrict__ counts, int E,
+                                                    int64_t* __restrict__ cum,
+                                                    int32_t* __restrict__ rank_out, int reset) {
+  extern __shared__ long long sc[];  // [E]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const long long v = (reset ? 0 : cum[e]) + counts[e];
+    sc[e] = v;
+    cum[e] = v;
+  }
+  __syncthreads();
+  if (!rank_out) return;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const long long v = sc[e];
+    int r = 0;
+    for (int f = 0; f < E; ++f) {
+      const long long w = sc[f];
+      r += (w > v) || (w == v && f < e);
+    }
+    rank_out[r] = e;
+  }
+}
+
+cudaError_t init_route_attributes() {
+  return cudaFuncSetAttribute(router_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kGemvMaxT * 8192 * (int)sizeof(uint16_t));
+}
+
+cudaError_t launch_hist(const int32_t* counts, int E, int64_t* cum, int32_t* rank_out, int reset,
+                        cudaStream_t st) {
+  hist_kernel<<<1, 1024, (size_t)E * sizeof(long long), st>>>(counts, E, cum, rank_out, reset);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,89 @@
+"""One MoE layer forward through the C ABI: buffers on the GPU and the five calls in order.
+
+    quantise x -> route (router, top-k, permutation) -> expert FFN -> combine -> histogram
+
+Each step is one call of libmoe_nvfp4.so; this module only allocates device buffers
+(torch) and passes pointers.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+from . import synth
+
+
+def quantize_weights_gpu(seed: int, cfg: synth.LayerShape, layer: int = 0, device="cuda",
+                         experts: Optional[range] = None, shared: bool = False,
+                         ws: Optional[torch.Tensor] = None) -> B.ExpertWeights:
+    """Generate an expert group's bf16 weights on the GPU and quantise each matrix
+    (gate, up, down of every expert, one tensor scale each) with nvfp4_quantize_act."""
+    E = 1 if shared else cfg.E
+    d, I = cfg.d, cfg.I
+    w = B.ExpertWeights(
+        gu_codes=torch.empty(E, 2 * I, d // 2, dtype=torch.uint8, device=device),
+        gu_scales=torch.empty(E, 2 * I, d // 16, dtype=torch.uint8, device=device),
+        gu_ts=torch.empty(E, 2, dtype=torch.float32, device=device),
+        dn_codes=torch.empty(E, d, I // 2, dtype=torch.uint8, device=device),
+        dn_scales=torch.empty(E, d, I // 16, dtype=torch.uint8, device=device),
+        dn_ts=torch.empty(E, dtype=torch.float32, device=device))
+    if ws is None:
+        ws = torch.empty(B.moe_workspace_size(B.MOE_OP_QUANT, 1, d, 1, 1, I),
+                         dtype=torch.uint8, device=device)
+    for e in range(E):
+        g, u, dn = synth.make_expert_weights_bf16(seed, cfg, e, layer, shared, device)
+        B.nvfp4_quantize_act(g, w.gu_codes[e, :I], w.gu_scales[e, :I], w.gu_ts[e, 0:1], ws=ws)
+        B.nvfp4_quantize_act(u, w.gu_codes[e, I:], w.gu_scales[e, I:], w.gu_ts[e, 1:2], ws=ws)
+        B.nvfp4_quantize_act(dn, w.dn_codes[e], w.dn_scales[e], w.dn_ts[e:e + 1], ws=ws)
+    return w
+
+
+class MoeLayer:
+    """Device buffers for one layer and up to T_max tokens per call."""
+
+    def __init__(self, experts: B.Experts, Wr: torch.Tensor, br: Optional[torch.Tensor], k: int,
+                 T_max: int, static_ts: Optional[torch.Tensor] = None, device="cuda"):
+        self.experts, self.Wr, self.br, self.k = experts, Wr, br, k
+        r = experts.routed
+        self.E, self.d, self.I = r.E, r.d, r.I
+        self.T_max = T_max
+        self.static_ts = static_ts
+        d, E, k, I = self.d, self.E, k, self.I
+        dev = device
+        self.xq_codes = torch.empty(T_max, d // 2, dtype=torch.uint8, device=dev)
+        self.xq_scales = torch.empty(T_max, d // 16, dtype=torch.uint8, device=dev)
+        self.xq_ts = torch.empty(4, dtype=torch.float32, device=dev)
+        self.topk_idx = torch.empty(T_max, k, dtype=torch.int32, device=dev)
+        self.topk_w = torch.empty(T_max, k, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.sorted_assign = torch.empty(max(1, T_max * k), dtype=torch.int32, device=dev)
+        self.assign_pos = torch.empty(max(1, T_max * k), dtype=torch.int32, device=dev)
+        self.y_acc = torch.empty(T_max, d, dtype=torch.float32, device=dev)
+        self.y = torch.empty(T_max, d, dtype=torch.int16, device=dev)
+        self.cum = torch.zeros(E, dtype=torch.int64, device=dev)
+        self.rank = torch.empty(E, dtype=torch.int32, device=dev)
+        ws = B.moe_workspace_size(B.MOE_OP_LAYER, T_max, d, E, k, I)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        self.path = B.MOE_PATH_AUTO
+
+    def forward(self, x: torch.Tensor, rms_renorm: bool = False, stream=None) -> torch.Tensor:
+        """x: bf16 bits (int16 or bfloat16) [T][d] on the GPU. Returns y bf16 bits [T][d]
+        (a view into this layer's output buffer)."""
+        T, k = x.shape[0], self.k
+        assert T <= self.T_max
+        B.nvfp4_quantize_act(x, self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
+                             ts_in=self.static_ts, ws=self.ws, stream=stream)
+        B.moe_route(x, self.Wr, self.br, k, self.topk_idx[:T], self.topk_w[:T], self.counts,
+                    self.offsets, self.sorted_assign[:T * k], self.assign_pos[:T * k], self.ws,
+                    stream=stream)
+        B.moe_expert_ffn(self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1], self.experts, k,
+                         self.offsets, self.sorted_assign[:T * k], self.topk_w[:T],
+                         B.MOE_FFN_ACCUMULATE, self.path, self.y_acc[:T], None, self.ws,
+                         stream=stream)
+        B.moe_combine(T, self.d, k, B.MOE_FFN_ACCUMULATE, self.y_acc[:T], None, self.topk_w[:T],
+                      self.assign_pos[:T * k], rms_renorm, self.y[:T], stream=stream)
+        B.moe_expert_hist(self.counts, self.cum, self.rank, stream=stream)
+        return self.y[:T]

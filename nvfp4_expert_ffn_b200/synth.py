@@ -160,13 +160,21 @@ def make_router(seed: int, cfg: LayerShape, layer: int = 0, epoch: int = 0, devi
     return Wr, br
 
 
-def make_expert_weights_f32(seed: int, cfg: LayerShape, expert: int, layer: int = 0,
-                            shared: bool = False, device="cpu"):
-    """Unquantised float32 weights of one expert: gate [I][d], up [I][d], down [d][I]."""
+def make_expert_weights_bf16(seed: int, cfg: LayerShape, expert: int, layer: int = 0,
+                             shared: bool = False, device="cpu"):
+    """Unquantised weights of one expert as bf16 bit patterns (int16), the precision a
+    checkpoint holds before NVFP4 quantisation: gate [I][d], up [I][d], down [d][I],
+    each ~N(0, weight_std^2)."""
     tg, tu, td = (TID_SGATE, TID_SUP, TID_SDOWN) if shared else (TID_GATE, TID_UP, TID_DOWN)
     base = (seed, cfg.cid, layer)
     n = cfg.I * cfg.d
-    gate = normal_f32(stream_key(*base, tg, expert), n, cfg.weight_std, device).view(cfg.I, cfg.d)
-    up = normal_f32(stream_key(*base, tu, expert), n, cfg.weight_std, device).view(cfg.I, cfg.d)
-    down = normal_f32(stream_key(*base, td, expert), n, cfg.weight_std, device).view(cfg.d, cfg.I)
-    return gate, up, down
+    mk = lambda tid: f32_to_bf16_bits(  # noqa: E731
+        normal_f32(stream_key(*base, tid, expert), n, cfg.weight_std, device))
+    return mk(tg).view(cfg.I, cfg.d), mk(tu).view(cfg.I, cfg.d), mk(td).view(cfg.d, cfg.I)
+
+
+def make_expert_weights_f32(seed: int, cfg: LayerShape, expert: int, layer: int = 0,
+                            shared: bool = False, device="cpu"):
+    """The same weights widened (exactly) to float32."""
+    return tuple(bf16_bits_to_f32(w) for w in
+                 make_expert_weights_bf16(seed, cfg, expert, layer, shared, device))

@@ -1,0 +1,99 @@
+"""The C ABI library: it loads, exports every function include/*.h declares, and rejects bad
+arguments on the host before touching the GPU (CPU only)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from nvfp4_expert_ffn_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", src, flags=re.M):
+            name = m.group(1)
+            if name not in ("defined",):
+                names.add(name)
+    return names
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = B.lib()
+    declared = _declared()
+    assert {"moe_route", "nvfp4_quantize_act", "moe_expert_ffn", "moe_combine",
+            "moe_expert_hist"} <= declared
+    for name in declared:
+        assert hasattr(L, name), f"{name} declared but not exported"
+    assert declared == set(B.EXPORTS), declared ^ set(B.EXPORTS)
+    assert L.moe_version() >= 100
+
+
+def _status(call):
+    return int(call)
+
+
+def test_host_validation_without_gpu():
+    L = B.lib()
+    INV, SHAPE, WS = 1, 2, 5
+    # quantiser: cols not a multiple of 16 / negative rows
+    assert L.nvfp4_quantize_act(None, 4, 24, None, None, None, None, None, 0, None) == SHAPE
+    assert L.nvfp4_quantize_act(None, -1, 32, None, None, None, None, None, 0, None) == INV
+    # misaligned pointer
+    assert L.nvfp4_quantize_act(ctypes.c_void_p(0x1008), 4, 32, None, ctypes.c_void_p(0x2000),
+                                ctypes.c_void_p(0x3000), None, None, 0, None) == INV
+    # large input needs workspace
+    assert L.nvfp4_quantize_act(ctypes.c_void_p(0x1000), 100000, 64, None, ctypes.c_void_p(0x2000),
+                                ctypes.c_void_p(0x3000), None, None, 0, None) == WS
+    p = ctypes.c_void_p(0x10000)
+    # route: k out of range, E < k, d not /16
+    assert L.moe_route(p, 4, 64, p, None, 8, 0, p, p, p, p, p, p, p, 1 << 20, None) == SHAPE
+    assert L.moe_route(p, 4, 64, p, None, 4, 8, p, p, p, p, p, p, p, 1 << 20, None) == SHAPE
+    assert L.moe_route(p, 4, 72, p, None, 8, 2, p, p, p, p, p, p, p, 1 << 20, None) == SHAPE
+    assert L.moe_route(p, 4, 64, p, None, 2000, 2, p, p, p, p, p, p, p, 1 << 20, None) == SHAPE
+    # route: workspace too small
+    assert L.moe_route(p, 4, 64, p, None, 8, 2, p, p, p, p, p, p, p, 16, None) == WS
+    # permute: null outputs
+    assert L.moe_permute(p, 4, 2, 8, None, p, p, p, p, 1 << 20, None) == INV
+    # ffn: null weights, bad mode
+    assert L.moe_expert_ffn(p, p, p, 4, None, 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == INV
+    # combine: bad d, bad mode
+    assert L.moe_combine(4, 24, 2, 0, p, None, None, None, 0, p, None) == INV
+    assert L.moe_combine(4, 32, 2, 7, p, None, None, None, 0, p, None) == INV
+    # hist: E out of range
+    assert L.moe_expert_hist(p, 0, p, None, 0, None) == SHAPE
+    assert b"E must be" in L.moe_last_error()
+    assert L.moe_status_string(5) == b"workspace too small or misaligned"
+
+
+def test_ffn_weight_validation():
+    L = B.lib()
+    p = ctypes.c_void_p(0x10000)
+    w = B._WeightsC(8, 64, 32, p.value, p.value, p.value, p.value, p.value, p.value, None, None)
+    bad = B._WeightsC(8, 64, 32, p.value, None, p.value, p.value, p.value, p.value, None, None)
+    ex = B._ExpertsC(w, B._WeightsC(), 0)
+    assert L.moe_expert_ffn(p, p, p, 0, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 0, None) in (0, 3)
+    ex = B._ExpertsC(bad, B._WeightsC(), 0)
+    assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == 1
+    # shared expert with E != 1
+    ex = B._ExpertsC(w, w, 1)
+    assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == 1
+    # I not a multiple of 16
+    w2 = B._WeightsC(8, 64, 40, p.value, p.value, p.value, p.value, p.value, p.value, None, None)
+    ex = B._ExpertsC(w2, B._WeightsC(), 0)
+    assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == 2
+
+
+def test_workspace_sizes_monotone():
+    small = B.moe_workspace_size(B.MOE_OP_LAYER, 8, 2048, 512, 10, 512)
+    big = B.moe_workspace_size(B.MOE_OP_LAYER, 16384, 2048, 512, 10, 512)
+    assert 0 < small < big
+    assert B.moe_workspace_size(B.MOE_OP_LAYER, 8, 2048, 512, 10, 512) >= \
+        B.moe_workspace_size(B.MOE_OP_FFN, 8, 2048, 512, 10, 512)
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, -1, 2048, 512, 10, 512) == 0

@@ -1,0 +1,141 @@
+"""moe_expert_ffn and moe_combine on the GPU vs the oracle (routing given by the oracle)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe as omoe
+from oracle import nvfp4 as onv
+from nvfp4_expert_ffn_b200 import binding as B
+from nvfp4_expert_ffn_b200 import layer as L
+from nvfp4_expert_ffn_b200 import synth
+
+from helpers import (OracleWeights, assert_close_layer, bits_to_f32, oracle_expert_from_bf16,
+                     weights_to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_route(xf, Wr, br, k, E):
+    logits = omoe.router_logits(xf, Wr, br)
+    idx = omoe.topk_fast(logits, k)
+    w = omoe.routing_weights(logits, idx)
+    counts, offsets, sa, pos = omoe.permute(idx, E)
+    return idx, w, offsets, sa, pos
+
+
+def _run_ffn(xq, routing, experts_gpu, k, mode, path, T, d):
+    idx, w, offsets, sa, pos = routing
+    xc, xs, xts = xq
+    cu = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()  # noqa: E731
+    E, I = experts_gpu.routed.E, experts_gpu.routed.I
+    out = torch.empty((T if mode == 0 else T * k), d, dtype=torch.float32, device="cuda")
+    sh = torch.empty(T, d, dtype=torch.float32, device="cuda") \
+        if (mode == 1 and experts_gpu.shared is not None) else None
+    ws = torch.empty(B.moe_workspace_size(B.MOE_OP_FFN, T, d, E, k, I), dtype=torch.uint8,
+                     device="cuda")
+    B.moe_expert_ffn(cu(xc), cu(xs), cu(np.array([xts], np.float32)), experts_gpu, k,
+                     cu(offsets), cu(sa), cu(w), mode, path, out, sh, ws)
+    y = torch.empty(T, d, dtype=torch.int16, device="cuda")
+    B.moe_combine(T, d, k, mode, out, sh, cu(w), cu(pos), False, y)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), None if sh is None else sh.cpu().numpy(), y.cpu().numpy()
+
+
+def _oracle_outputs(xq, routing, experts, shared, T, d, k, tokens=None):
+    idx, w, offsets, sa, pos = routing
+    xh = onv.dequantize(*xq)
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    want = np.zeros(T, bool)
+    want[tokens] = True
+    o = np.full((T * k, d), np.nan)
+    for e in np.unique(idx[tokens]):
+        seg = sa[offsets[e]:offsets[e + 1]]
+        seg = seg[want[seg // k]]
+        o[seg] = omoe.expert_ffn(xh[seg // k], experts[int(e)])
+    os_ = None
+    if shared is not None:
+        os_ = np.full((T, d), np.nan)
+        os_[tokens] = omoe.expert_ffn(xh[tokens], shared)
+    y = omoe.combine(len(tokens), d, idx[tokens], w[tokens],
+                     np.concatenate([o[t * k:(t + 1) * k] for t in tokens]),
+                     None if os_ is None else os_[tokens])
+    return o, os_, y
+
+
+def _tiny_case(seed, d, E, k, I, T, shared, zipf=0.0):
+    cfg = synth.LayerShape("t", cid=100 + seed, d=d, E=E, k=k, I=I, shared=shared, zipf_s=zipf,
+                           router_std=0.02)
+    experts = [oracle_expert_from_bf16(*synth.make_expert_weights_bf16(seed, cfg, e))
+               for e in range(E)]
+    sh = oracle_expert_from_bf16(*synth.make_expert_weights_bf16(seed, cfg, 0, shared=True)) \
+        if shared else None
+    x = synth.make_x(seed, cfg, T).numpy()
+    Wr, br = synth.make_router(seed, cfg)
+    xf = bits_to_f32(x)
+    xq = onv.quantize(xf)
+    routing = _oracle_route(xf, Wr.numpy(), br.numpy(), k, E)
+    gpu = B.Experts(weights_to_gpu(experts), weights_to_gpu([sh]) if shared else None)
+    return experts, sh, xq, routing, gpu
+
+
+@pytest.mark.parametrize("mode", [B.MOE_FFN_ACCUMULATE, B.MOE_FFN_PER_ASSIGN])
+@pytest.mark.parametrize("d,E,k,I,T,shared", [
+    (256, 8, 2, 128, 16, False),      # tiny layer
+    (256, 8, 2, 128, 16, True),
+    (128, 16, 3, 64, 1, True),        # single token
+    (512, 32, 4, 96, 37, True),       # ragged: experts with 0..many tokens, I not /32
+    (64, 64, 8, 32, 200, False),      # many tokens per expert (> token chunk)
+    (2048, 16, 2, 512, 5, True),      # decode-like widths
+    (48, 8, 2, 32, 9, True),          # d not a multiple of 32
+])
+def test_ffn_decode_path_matches_oracle(mode, d, E, k, I, T, shared):
+    experts, sh, xq, routing, gpu = _tiny_case(11, d, E, k, I, T, shared)
+    o_g, os_g, y_g = _run_ffn(xq, routing, gpu, k, mode, B.MOE_PATH_DECODE, T, d)
+    o_r, os_r, y_r = _oracle_outputs(xq, routing, experts, sh, T, d, k)
+    idx, w, offsets, sa, pos = routing
+    if mode == B.MOE_FFN_PER_ASSIGN:
+        assert_close_layer(o_g, o_r[sa], "per-assignment o")
+        if sh is not None:
+            assert_close_layer(os_g, os_r, "shared o")
+    else:
+        assert_close_layer(o_g, y_r, "y_acc")
+    assert_close_layer(bits_to_f32(y_g), y_r, "y bf16")
+
+
+@pytest.fixture(scope="module")
+def decode_layer():
+    cfg = synth.CONFIGS["decode"]
+    routed = L.quantize_weights_gpu(0, cfg)
+    shared = L.quantize_weights_gpu(0, cfg, shared=True)
+    return cfg, B.Experts(routed, shared), OracleWeights(0, cfg)
+
+
+@pytest.mark.parametrize("T", [1, 4, 8])
+def test_ffn_decode_config_full_size(decode_layer, T):
+    cfg, gpu, ow = decode_layer
+    x = synth.make_x(0, cfg, T).numpy()
+    Wr, br = synth.make_router(0, cfg)
+    xf = bits_to_f32(x)
+    xq = onv.quantize(xf)
+    routing = _oracle_route(xf, Wr.numpy(), br.numpy(), cfg.k, cfg.E)
+    _, _, y_g = _run_ffn(xq, routing, gpu, cfg.k, B.MOE_FFN_ACCUMULATE, B.MOE_PATH_DECODE, T, cfg.d)
+    _, _, y_r = _oracle_outputs(xq, routing, ow, ow.shared, T, cfg.d, cfg.k)
+    assert_close_layer(bits_to_f32(y_g), y_r, f"decode T={T}")
+    # the GPU-quantised weights of the touched experts equal the oracle's
+    for e in np.unique(routing[0])[:4]:
+        assert np.array_equal(gpu.routed.gu_codes[int(e)].cpu().numpy(), ow[int(e)].gu_codes)
+        assert np.array_equal(gpu.routed.dn_scales[int(e)].cpu().numpy(), ow[int(e)].dn_scales)
+
+
+def test_combine_rms_renorm():
+    T, d, k = 7, 64, 3
+    rng = np.random.default_rng(5)
+    y_acc = rng.standard_normal((T, d)).astype(np.float32)
+    y_acc[3] = 0
+    y = torch.empty(T, d, dtype=torch.int16, device="cuda")
+    B.moe_combine(T, d, k, B.MOE_FFN_ACCUMULATE, torch.from_numpy(y_acc).cuda(), None, None, None,
+                  True, y)
+    torch.cuda.synchronize()
+    ref = omoe.rms_renorm(y_acc)
+    assert_close_layer(bits_to_f32(y.cpu().numpy()), ref, "rms renorm")
+    assert not bits_to_f32(y.cpu().numpy())[3].any()

@@ -1,0 +1,85 @@
+"""Whole layer through the C ABI (MoeLayer.forward) vs the oracle's layer_forward, plus the
+cumulative expert histogram."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe as omoe
+from nvfp4_expert_ffn_b200 import binding as B
+from nvfp4_expert_ffn_b200 import layer as L
+from nvfp4_expert_ffn_b200 import synth
+
+from helpers import (OracleWeights, assert_close_layer, bits_to_f32, compare_topk,
+                     oracle_expert_from_bf16, weights_to_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+def _layer(cfg_name, seed=0, T_max=64):
+    cfg = synth.CONFIGS[cfg_name]
+    routed = L.quantize_weights_gpu(seed, cfg)
+    shared = L.quantize_weights_gpu(seed, cfg, shared=True) if cfg.shared else None
+    Wr, br = synth.make_router(seed, cfg)
+    lay = L.MoeLayer(B.Experts(routed, shared), Wr.cuda(), br.cuda(), cfg.k, T_max)
+    return cfg, lay, Wr.numpy(), br.numpy()
+
+
+@pytest.mark.parametrize("cfg_name,T", [("tiny", 16), ("decode", 1), ("decode", 8)])
+def test_layer_matches_oracle(cfg_name, T):
+    cfg, lay, Wr, br = _layer(cfg_name)
+    ow = OracleWeights(0, cfg)
+    x = synth.make_x(0, cfg, T, step=3)
+    y = lay.forward(x.cuda())
+    torch.cuda.synchronize()
+    ref = omoe.layer_forward(x.numpy(), Wr, br, cfg.k, ow, ow.shared if cfg.shared else None)
+    excused = compare_topk(lay.topk_idx[:T].cpu().numpy(), ref["idx"], ref["logits"], cfg.k)
+    keep = [t for t in range(T) if t not in set(excused)]
+    assert_close_layer(bits_to_f32(y.cpu().numpy())[keep], ref["y"][keep], cfg_name)
+    assert np.array_equal(lay.xq_codes[:T].cpu().numpy(), ref["x_codes"])
+    if not excused:
+        assert np.array_equal(lay.counts.cpu().numpy(), ref["counts"])
+        cum, rank = omoe.hist_update(ref["counts"])
+        assert np.array_equal(lay.cum.cpu().numpy(), cum)
+        assert np.array_equal(lay.rank.cpu().numpy(), rank)
+
+
+def test_hist_over_calls():
+    rng = np.random.default_rng(3)
+    E = 512
+    counts = [rng.integers(0, 50, E).astype(np.int32) for _ in range(5)]
+    counts[2][:] = 7  # all tied
+    cum_g = torch.zeros(E, dtype=torch.int64, device="cuda")
+    rank_g = torch.empty(E, dtype=torch.int32, device="cuda")
+    cum = None
+    for i, c in enumerate(counts):
+        reset = i == 3
+        B.moe_expert_hist(torch.from_numpy(c).cuda(), cum_g, rank_g, reset=reset)
+        cum, rank = omoe.hist_update(c, cum, reset=reset)
+        torch.cuda.synchronize()
+        assert np.array_equal(cum_g.cpu().numpy(), cum)
+        assert np.array_equal(rank_g.cpu().numpy(), rank)
+
+
+def test_stack_chaining_with_rms_renorm():
+    """Two decode layers chained with per-token RMS renormalisation (decode-stack input)."""
+    cfg = synth.CONFIGS["stack48"]
+    T = 8
+    layers, owl = [], []
+    for li in range(2):
+        routed = L.quantize_weights_gpu(0, cfg, layer=li)
+        shared = L.quantize_weights_gpu(0, cfg, layer=li, shared=True)
+        Wr, br = synth.make_router(0, cfg, layer=li)
+        layers.append(L.MoeLayer(B.Experts(routed, shared), Wr.cuda(), br.cuda(), cfg.k, T))
+        owl.append((OracleWeights(0, cfg, li), Wr.numpy(), br.numpy()))
+    x = synth.make_x(0, cfg, T)
+    h = x.cuda()
+    for lay in layers:
+        h = lay.forward(h, rms_renorm=True).clone()
+    torch.cuda.synchronize()
+    xr = x.numpy()
+    for ow, Wr, br in owl:
+        ref = omoe.layer_forward(xr, Wr, br, cfg.k, ow, ow.shared)
+        yr = omoe.rms_renorm(ref["y"])
+        xr = synth.f32_to_bf16_bits(torch.from_numpy(yr.astype(np.float32))).numpy()
+    # bf16 re-rounding between layers can flip an h code; compare loosely on the final layer
+    assert_close_layer(bits_to_f32(h.cpu().numpy()), yr, "2-layer stack")
