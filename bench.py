@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s (decode T=1–8, prefill T=16K); % of HBM BW / FP4 MMA peak"
 SEED = 0
-N_LAYER_COPIES = 4
+N_LAYER_COPIES = 4  # overridden by --layers
 
 
 def _peaks():
@@ -100,13 +100,13 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- GPU arm
-def build_layers(T: int, device):
+def build_layers(T: int, device, n_layers: int):
     from nvfp4_expert_ffn_b200 import binding as B
     from nvfp4_expert_ffn_b200 import layer as L
     from nvfp4_expert_ffn_b200 import synth
     cfg = synth.CONFIGS["decode"]
     layers = []
-    for li in range(N_LAYER_COPIES):
+    for li in range(n_layers):
         routed = L.quantize_weights_gpu(SEED, cfg, layer=li, device=device)
         shared = L.quantize_weights_gpu(SEED, cfg, layer=li, shared=True, device=device)
         Wr, br = synth.make_router(SEED, cfg, layer=li)
@@ -139,8 +139,10 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    global N_LAYER_COPIES
+    N_LAYER_COPIES = args.layers
     T, K, W = args.T, args.steps, args.warmup
-    cfg, layers = build_layers(T, device)
+    cfg, layers = build_layers(T, device, N_LAYER_COPIES)
     stream = torch.cuda.Stream(device)
     sampler = ClockSampler(local)
     sampler.start()
@@ -193,14 +195,24 @@ def run_gpu(args):
             g_step.replay()
             g_ffn.replay()
     torch.cuda.synchronize()
+    if args.eager:
+        # profiling aid: the same steps launched directly (no graph), inside an NVTX range
+        with torch.cuda.stream(stream):
+            torch.cuda.nvtx.range_push("timed")
+            for i in range(K):
+                layers[i % N_LAYER_COPIES].forward(layers[i % N_LAYER_COPIES].x_static)
+            torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed_graph")
     ms_total, win1 = timed(g_step, reps)
     ms_ffn, win2 = timed(g_ffn, reps)
+    torch.cuda.nvtx.range_pop()
 
     # end to end through the public API: pinned host x -> device, forward, y -> pinned host
     xs_host = [lay.x_static.cpu().pin_memory() for lay in layers]
     y_host = torch.empty(T, cfg.d, dtype=torch.int16).pin_memory()
     x_dev = [torch.empty_like(lay.x_static) for lay in layers]
-    e2e_steps = min(K, 2000)
+    e2e_steps = 0 if args.no_e2e else min(K, 2000)
     with torch.cuda.stream(stream):
         for i in range(min(W, 8)):
             li = i % N_LAYER_COPIES
@@ -230,7 +242,7 @@ def run_gpu(args):
 
     ms_step = ms_total / K
     tokens_per_s = world * T * K / (ms_total / 1e3)
-    e2e_tps = world * T * e2e_steps / (ms_e2e / 1e3)
+    e2e_tps = world * T * e2e_steps / (ms_e2e / 1e3) if e2e_steps else None
     hbm_peak, _, peak_kind = _peaks()
     U_avg = float(np.mean([b[0] for b in bytes_info]))
     ffn_bytes = float(np.mean([b[1] for b in bytes_info]))
@@ -254,7 +266,7 @@ def run_gpu(args):
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
                      "bytes_per_launch": int(ffn_bytes), "avg_launch_us": round(ffn_ms * 1e3, 3),
                      "traffic": None},
-        "e2e": {"value": round(e2e_tps, 1), "unit": "tokens/s",
+        "e2e": {"value": None if e2e_tps is None else round(e2e_tps, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2,
                 "steps": e2e_steps},
         "gpu_launches": launches_per_step * K,
@@ -331,6 +343,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=4, help="distinct layer copies rotated")
+    ap.add_argument("--eager", action="store_true",
+                    help="also run K eager steps in an NVTX range 'timed' (for ncu)")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

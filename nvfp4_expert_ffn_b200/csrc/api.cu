@@ -31,12 +31,13 @@ constexpr int kMaxDevices = 64;
 struct DeviceInfo {
   bool ready = false;
   int num_sms = 0;
+  int32_t* status = nullptr;  // device address of g_device_status on this device
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
 // Per-device one-time setup: SM count and dynamic shared memory limits.
-moe_status device_info(int* num_sms) {
+moe_status device_info(int* num_sms, int32_t** status = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -54,9 +55,12 @@ moe_status device_info(int* num_sms) {
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
     e = init_kernel_attributes();
     if (e != cudaSuccess) return cuda_fail(e, "kernel attribute setup");
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(&di.status), g_device_status);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_device_status)");
     di.ready = true;
   }
   *num_sms = di.num_sms;
+  if (status) *status = di.status;
   return MOE_OK;
 }
 
@@ -245,7 +249,8 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   s = check_ws(ws, ws_bytes, need);
   if (s != MOE_OK) return s;
   int sms = 0;
-  s = device_info(&sms);
+  int32_t* dstatus = nullptr;
+  s = device_info(&sms, &dstatus);
   if (s != MOE_OK) return s;
   FfnArgs a;
   a.xq_codes = xq_codes;
@@ -264,7 +269,7 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const size_t slots = (size_t)T * k + T;
   a.h_codes = reinterpret_cast<uint8_t*>(ws);
   a.h_scales = reinterpret_cast<uint8_t*>(ws) + align256(slots * (I / 2));
-  cudaError_t e = launch_ffn_decode(a, sms, (cudaStream_t)stream);
+  cudaError_t e = launch_ffn_decode(a, sms, dstatus, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
 }
 

@@ -16,12 +16,12 @@
 // the offsets array.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace moe {
 
 constexpr int kTokChunk = 8;      // tokens processed together per unit pass
 constexpr int kFfnThreads = 256;  // 8 warps
-constexpr int kDownRows = 32;     // output rows per down unit (4 per warp)
 
 __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 
@@ -119,219 +119,388 @@ MOE_DEV void row_dots(const uint8_t* wc, const uint8_t* wsc, int K, const uint32
   }
 }
 
-// ---------------------------------------------------------------- gate/up + SwiGLU + h quant
-__global__ void __launch_bounds__(kFfnThreads) ffn_gateup_decode_kernel(FfnArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int d = a.d, I = a.I;
-  int* s_act = reinterpret_cast<int*>(smem);
-  size_t off = align16((size_t)(a.E + 1) * sizeof(int));
-  uint32_t* s_x = reinterpret_cast<uint32_t*>(smem + off);
-  off += align16((size_t)kTokChunk * (d / 2) * sizeof(uint32_t));
-  float* s_xs = reinterpret_cast<float*>(smem + off);
-  off += align16((size_t)kTokChunk * (d / kBlock) * sizeof(float));
-  __shared__ float s_g[kTokChunk][16], s_u[kTokChunk][16];
-  __shared__ int s_rows[kTokChunk], s_slot[kTokChunk];
-  __shared__ int tmp[32];
+// ---------------------------------------------------------------- fused persistent kernel
+// One CTA per SM. Warp 8 is the producer: it streams the weights of this CTA's work units
+// into a ring of shared-memory stages with cp.async.bulk. Warps 0-7 consume:
+//   phase 1 unit (active expert a, 16 h-rows): gate and up rows -> SwiGLU -> NVFP4 h, written
+//     to the workspace; then the unit is counted in done[a];
+//   phase 2 unit (active expert a, r2 output rows): waits until done[a] == I/16 (all of the
+//     expert's h is written), then the down projection and the weighted scatter into y.
+// Every CTA takes a contiguous range of phase-1 units, then a contiguous range of phase-2
+// units, so a CTA reaches phase 2 only after finishing its phase-1 work; all CTAs are
+// resident (grid <= SM count, one CTA per SM), so the waits always end.
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kFusedThreads = kConsumers + 32;
+constexpr int kMaxStages = 6;
 
-  // ACCUMULATE mode: zero y_acc here; the down kernel runs after this grid completes.
-  if (a.mode == 0) {
-    const size_t n4 = (size_t)a.T * d / 4;
-    float4* o4 = reinterpret_cast<float4*>(a.out);
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
-         i += (size_t)gridDim.x * blockDim.x)
-      o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+struct DecodeCfg {
+  int stage_bytes;  // bytes of one stage (phase-1 unit: 32 rows x (d/2 + d/16))
+  int nstages;
+  int r2;           // output rows per phase-2 unit
+  int kmax;         // max(d, I): staged activation row length
+  int32_t* done;    // [E+1] phase-1 units finished per active slot (zeroed before launch)
+  int32_t* status;  // device status word
+};
+
+struct UnitRange {
+  int beg, end;
+};
+
+MOE_DEV UnitRange block_range(int n, int cta, int ncta) {
+  return UnitRange{(int)((long long)n * cta / ncta), (int)((long long)n * (cta + 1) / ncta)};
+}
+
+MOE_DEV int32_t ld_acquire(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Stage nt rows of NVFP4 written earlier in this kernel by other CTAs (read through L2).
+MOE_DEV void stage_rows_cg(const uint8_t* codes, const uint8_t* scales, int K, const int* rows, int nt,
+                           uint32_t* s_f16, float* s_sc, int tid, int nthr) {
+  const int q_per_row = K / 8;
+  for (int i = tid; i < nt * q_per_row; i += nthr) {
+    const int j = i / q_per_row, q = i - j * q_per_row;
+    const uint32_t w = __ldcg(reinterpret_cast<const uint32_t*>(codes + (size_t)rows[j] * (K / 2)) + q);
+    uint32_t o[4];
+    e2m1x8_to_f16x2x4(w, o);
+    *reinterpret_cast<uint4*>(s_f16 + (size_t)j * (K / 2) + 4 * q) = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  const int nb = K / kBlock;
+  for (int i = tid; i < nt * nb; i += nthr) {
+    const int j = i / nb, b = i - j * nb;
+    s_sc[i] = e4m3_to_f32(__ldcg(scales + (size_t)rows[j] * nb + b));
+  }
+}
 
-  const int n_act = build_active_list(a, s_act, tmp);
-  const int nhb = I / kBlock;
-  const int units = n_act * nhb;
-  const float ts_x = *a.xq_ts;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+MOE_DEV void stage_rows_nc(const uint8_t* codes, const uint8_t* scales, int K, const int* rows, int nt,
+                           uint32_t* s_f16, float* s_sc, int tid, int nthr) {
+  const int q_per_row = K / 8;
+  for (int i = tid; i < nt * q_per_row; i += nthr) {
+    const int j = i / q_per_row, q = i - j * q_per_row;
+    const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(codes + (size_t)rows[j] * (K / 2)) + q);
+    uint32_t o[4];
+    e2m1x8_to_f16x2x4(w, o);
+    *reinterpret_cast<uint4*>(s_f16 + (size_t)j * (K / 2) + 4 * q) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  const int nb = K / kBlock;
+  for (int i = tid; i < nt * nb; i += nthr) {
+    const int j = i / nb, b = i - j * nb;
+    s_sc[i] = e4m3_to_f32(__ldg(scales + (size_t)rows[j] * nb + b));
+  }
+}
 
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int hb = u % nhb;
-    const UnitExpert ue = unit_expert(a, s_act[u / nhb]);
-    const ExpertGroup& G = *ue.G;
-    const float ts_g = G.gu_ts[2 * ue.eloc] * ts_x;
-    const float ts_u = G.gu_ts[2 * ue.eloc + 1] * ts_x;
-    // this warp's rows: h-rows i0, i0+1 (gate rows i, up rows I+i); 8 warps x 2 = 16
-    const int i0 = hb * kBlock + 2 * warp;
-    const size_t rowstride_c = (size_t)(d / 2), rowstride_s = (size_t)(d / kBlock);
-    const size_t ebase = (size_t)ue.eloc * 2 * I;
-    for (int c0 = 0; c0 < ue.cnt; c0 += kTokChunk) {
-      const int nt = min(kTokChunk, ue.cnt - c0);
-      __syncthreads();
-      if (threadIdx.x < nt) {
-        const int j = threadIdx.x;
-        if (ue.shared) {
-          s_rows[j] = c0 + j;
-          s_slot[j] = a.T * a.k + c0 + j;
-        } else {
-          s_rows[j] = a.sorted_assign[ue.off + c0 + j] / a.k;
-          s_slot[j] = ue.off + c0 + j;
-        }
-      }
-      __syncthreads();
-      stage_rows(a.xq_codes, a.xq_scales, d, s_rows, nt, s_x, s_xs);
-      __syncthreads();
+// Partial dots of one smem weight row (codes, scales) with nt staged rows.
+MOE_DEV void row_dots_smem(const uint8_t* wc, const uint8_t* wsc, int K, const uint32_t* s_f16,
+                           const float* s_sc, int nt, float part[kTokChunk]) {
+  const int lane = threadIdx.x & 31;
+  const int nb = K / kBlock;
+  for (int b = lane; b < nb; b += 32) {
+    const uint2 cw = *reinterpret_cast<const uint2*>(wc + 8 * b);
+    const float sw = e4m3_to_f32(wsc[b]);
+    uint32_t wf[8];
+    e2m1x8_to_f16x2x4(cw.x, wf);
+    e2m1x8_to_f16x2x4(cw.y, wf + 4);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = i0 + (r & 1);
-        const int row = (r < 2) ? i : I + i;
-        float part[kTokChunk];
-#pragma unroll
-        for (int j = 0; j < kTokChunk; ++j) part[j] = 0.0f;
-        row_dots(G.gu_codes + (ebase + row) * rowstride_c, G.gu_scales + (ebase + row) * rowstride_s,
-                 d, s_x, s_xs, nt, part);
-#pragma unroll
-        for (int j = 0; j < kTokChunk; ++j) {
-          const float v = warp_sum(part[j]);
-          if (lane == 0 && j < nt) {
-            if (r < 2) s_g[j][2 * warp + (r & 1)] = v * ts_g;
-            else s_u[j][2 * warp + (r & 1)] = v * ts_u;
-          }
-        }
-      }
-      __syncthreads();
-      // SwiGLU + NVFP4 quantisation of h (tensor scale 1.0): 16 lanes per token
-      if (threadIdx.x < kTokChunk * 16) {
-        const int j = threadIdx.x >> 4, ii = threadIdx.x & 15;
-        const float g = s_g[j][ii], uu = s_u[j][ii];
-        const float h = __fdiv_rn(g, 1.0f + expf(-g)) * uu;
-        float amax = fabsf(h);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o, 16));
-        const uint32_t s = f32_to_e4m3_sat(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), 1.0f));
-        const float sval = e4m3_to_f32(s);
-        const float q = (sval != 0.0f) ? __fdiv_rn(h, __fmul_rn(sval, 1.0f)) : 0.0f;
-        uint32_t code = f32x2_to_e2m1x2(q, 0.0f) & 0xFu;
-        if (sval == 0.0f) code = 0;
-        uint32_t b = code | (__shfl_down_sync(0xffffffffu, code, 1, 16) << 4);
-        b |= __shfl_down_sync(0xffffffffu, b, 2, 16) << 8;
-        b |= __shfl_down_sync(0xffffffffu, b, 4, 16) << 16;
-        const uint32_t hi = __shfl_down_sync(0xffffffffu, b, 8, 16);
-        if (ii == 0 && j < nt) {
-          const size_t slot = (size_t)s_slot[j];
-          *reinterpret_cast<uint2*>(a.h_codes + slot * (I / 2) + hb * 8) = make_uint2(b, hi);
-          a.h_scales[slot * (I / kBlock) + hb] = (uint8_t)s;
-        }
+    for (int j = 0; j < kTokChunk; ++j) {
+      if (j < nt) {
+        const float sdot = block_dot(wf, s_f16 + (size_t)j * (K / 2) + 8 * b);
+        part[j] = fmaf(sdot, sw * s_sc[j * nb + b], part[j]);
       }
     }
   }
 }
 
-// ---------------------------------------------------------------- down projection
-__global__ void __launch_bounds__(kFfnThreads) ffn_down_decode_kernel(FfnArgs a) {
-  extern __shared__ __align__(16) uint8_t smem[];
+__global__ void __launch_bounds__(kFusedThreads, 1) ffn_decode_fused_kernel(FfnArgs a, DecodeCfg c) {
+  extern __shared__ __align__(128) uint8_t smem[];
   const int d = a.d, I = a.I;
-  int* s_act = reinterpret_cast<int*>(smem);
-  size_t off = align16((size_t)(a.E + 1) * sizeof(int));
-  uint32_t* s_h = reinterpret_cast<uint32_t*>(smem + off);
-  off += align16((size_t)kTokChunk * (I / 2) * sizeof(uint32_t));
-  float* s_hs = reinterpret_cast<float*>(smem + off);
-  __shared__ int s_rows[kTokChunk], s_tok[kTokChunk];
+  const int nst = c.nstages;
+  uint8_t* stages = smem;
+  size_t off = (size_t)nst * c.stage_bytes;
+  uint32_t* s_x = reinterpret_cast<uint32_t*>(smem + off);
+  off += align16((size_t)kTokChunk * (c.kmax / 2) * sizeof(uint32_t));
+  float* s_xs = reinterpret_cast<float*>(smem + off);
+  off += align16((size_t)kTokChunk * (c.kmax / kBlock) * sizeof(float));
+  int* s_act = reinterpret_cast<int*>(smem + off);
+  off += align16((size_t)(a.E + 1) * sizeof(int));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + off);
+  uint64_t* empty = full + kMaxStages;
+  __shared__ float s_g[kTokChunk][16], s_u[kTokChunk][16];
+  __shared__ int s_rows[kTokChunk], s_slot[kTokChunk], s_tok[kTokChunk];
   __shared__ float s_w[kTokChunk];
   __shared__ int tmp[32];
+  __shared__ volatile int s_abort;
 
-  const int n_act = build_active_list(a, s_act, tmp);
-  const int ntile = (d + kDownRows - 1) / kDownRows;
-  const int units = n_act * ntile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nst; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kConsumerWarps);
+    }
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  const int n_act = build_active_list(a, s_act, tmp);  // contains __syncthreads
+  const int nhb = I / kBlock;
+  const int nrt = (d + c.r2 - 1) / c.r2;
+  const UnitRange r1 = block_range(n_act * nhb, blockIdx.x, gridDim.x);
+  const UnitRange r2 = block_range(n_act * nrt, blockIdx.x, gridDim.x);
+  const int n_units = (r1.end - r1.beg) + (r2.end - r2.beg);
 
-  for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int tile = u % ntile;
-    const UnitExpert ue = unit_expert(a, s_act[u / ntile]);
-    const ExpertGroup& G = *ue.G;
-    const float ts_o = G.dn_ts[ue.eloc];  // h tensor scale is 1.0
-    for (int c0 = 0; c0 < ue.cnt; c0 += kTokChunk) {
-      const int nt = min(kTokChunk, ue.cnt - c0);
-      __syncthreads();
-      if (threadIdx.x < nt) {
-        const int j = threadIdx.x;
-        if (ue.shared) {
-          s_rows[j] = a.T * a.k + c0 + j;
-          s_tok[j] = c0 + j;
-          s_w[j] = 1.0f;
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      for (; it < n_units && !s_abort; ++it) {
+        const int s = it % nst;
+        if (!mbar_wait(&empty[s], ((it / nst) & 1) ^ 1, &s_abort, c.status)) break;
+        uint8_t* dst = stages + (size_t)s * c.stage_bytes;
+        const bool ph1 = it < (r1.end - r1.beg);
+        const int v = ph1 ? r1.beg + it : r2.beg + (it - (r1.end - r1.beg));
+        const int e = s_act[ph1 ? v / nhb : v / nrt];
+        const bool sh = (e == a.E);
+        const ExpertGroup& G = sh ? a.shared : a.routed;
+        const size_t eloc = sh ? 0 : (size_t)e;
+        if (ph1) {
+          const int i0 = (v % nhb) * kBlock;
+          const uint32_t cb = 16u * (uint32_t)(d / 2), sb = 16u * (uint32_t)(d / kBlock);
+          mbar_arrive_expect_tx(&full[s], 2 * cb + 2 * sb);
+          bulk_g2s(dst, G.gu_codes + (eloc * 2 * I + i0) * (d / 2), cb, &full[s]);
+          bulk_g2s(dst + cb, G.gu_codes + (eloc * 2 * I + I + i0) * (d / 2), cb, &full[s]);
+          bulk_g2s(dst + 2 * cb, G.gu_scales + (eloc * 2 * I + i0) * (d / kBlock), sb, &full[s]);
+          bulk_g2s(dst + 2 * cb + sb, G.gu_scales + (eloc * 2 * I + I + i0) * (d / kBlock), sb, &full[s]);
         } else {
-          const int p = ue.off + c0 + j;
-          const int asg = a.sorted_assign[p];
-          s_rows[j] = p;
-          s_tok[j] = asg / a.k;
-          s_w[j] = a.topk_w[asg];
+          const int n0 = (v % nrt) * c.r2;
+          const int R = min(c.r2, d - n0);
+          const uint32_t cb = (uint32_t)R * (I / 2), sb = (uint32_t)R * (I / kBlock);
+          mbar_arrive_expect_tx(&full[s], cb + sb);
+          bulk_g2s(dst, G.dn_codes + (eloc * d + n0) * (I / 2), cb, &full[s]);
+          bulk_g2s(dst + (size_t)c.r2 * (I / 2), G.dn_scales + (eloc * d + n0) * (I / kBlock), sb,
+                   &full[s]);
         }
       }
-      __syncthreads();
-      stage_rows(a.h_codes, a.h_scales, I, s_rows, nt, s_h, s_hs);
-      __syncthreads();
+      // never leave copies in flight: wait for the last issued stage of each slot
+      for (int j = (it > nst ? it - nst : 0); j < it; ++j) {
+        volatile int no_abort = 0;
+        mbar_wait(&full[j % nst], (j / nst) & 1, &no_abort, c.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int tid = threadIdx.x;
+    int staged_e = -1, staged_c0 = -1;
+    const float ts_x = *a.xq_ts;
+    for (int it = 0; it < n_units; ++it) {
+      const int s = it % nst;
+      // one thread waits, the barrier publishes both the data and the abort decision
+      if (tid == 0) mbar_wait(&full[s], (it / nst) & 1, &s_abort, c.status);
+      named_bar_sync(1, kConsumers);
+      if (s_abort) break;
+      const uint8_t* st = stages + (size_t)s * c.stage_bytes;
+      const bool ph1 = it < (r1.end - r1.beg);
+      const int v = ph1 ? r1.beg + it : r2.beg + (it - (r1.end - r1.beg));
+      const int ai = ph1 ? v / nhb : v / nrt;
+      const UnitExpert ue = unit_expert(a, s_act[ai]);
+      const ExpertGroup& G = *ue.G;
+      if (ph1) {
+        const int hb = v % nhb;
+        const float ts_g = G.gu_ts[2 * ue.eloc] * ts_x;
+        const float ts_u = G.gu_ts[2 * ue.eloc + 1] * ts_x;
+        const uint8_t* gc = st;
+        const uint8_t* uc = st + 16 * (d / 2);
+        const uint8_t* gs = st + 32 * (d / 2);
+        const uint8_t* us = gs + 16 * (d / kBlock);
+        for (int c0 = 0; c0 < ue.cnt; c0 += kTokChunk) {
+          const int nt = min(kTokChunk, ue.cnt - c0);
+          if (staged_e != s_act[ai] || staged_c0 != c0) {
+            named_bar_sync(1, kConsumers);
+            if (tid < nt) {
+              const int j = tid;
+              s_rows[j] = ue.shared ? c0 + j : a.sorted_assign[ue.off + c0 + j] / a.k;
+            }
+            named_bar_sync(1, kConsumers);
+            stage_rows_nc(a.xq_codes, a.xq_scales, d, s_rows, nt, s_x, s_xs, tid, kConsumers);
+            if (tid < nt) s_slot[tid] = ue.shared ? a.T * a.k + c0 + tid : ue.off + c0 + tid;
+            named_bar_sync(1, kConsumers);
+            staged_e = s_act[ai];
+            staged_c0 = c0;
+          }
 #pragma unroll
-      for (int r = 0; r < kDownRows / 8; ++r) {
-        const int n = tile * kDownRows + warp * (kDownRows / 8) + r;
-        if (n >= d) continue;  // warp-uniform: d % 16 == 0 but not always % 32
-        const size_t row = (size_t)ue.eloc * d + n;
-        float part[kTokChunk];
+          for (int r = 0; r < 4; ++r) {
+            const int rr = 2 * warp + (r & 1);  // row within the unit's 16 h-rows
+            float part[kTokChunk];
 #pragma unroll
-        for (int j = 0; j < kTokChunk; ++j) part[j] = 0.0f;
-        row_dots(G.dn_codes + row * (I / 2), G.dn_scales + row * (I / kBlock), I, s_h, s_hs, nt, part);
+            for (int j = 0; j < kTokChunk; ++j) part[j] = 0.0f;
+            if (r < 2)
+              row_dots_smem(gc + rr * (d / 2), gs + rr * (d / kBlock), d, s_x, s_xs, nt, part);
+            else
+              row_dots_smem(uc + rr * (d / 2), us + rr * (d / kBlock), d, s_x, s_xs, nt, part);
 #pragma unroll
-        for (int j = 0; j < kTokChunk; ++j) {
-          const float v = warp_sum(part[j]);
-          if (lane == j && j < nt) {
-            const float o = v * ts_o;
-            if (a.mode == 0) {
-              atomicAdd(a.out + (size_t)s_tok[j] * d + n, s_w[j] * o);
-            } else if (ue.shared) {
-              a.shared_out[(size_t)s_tok[j] * d + n] = o;
-            } else {
-              a.out[(size_t)s_rows[j] * d + n] = o;
+            for (int j = 0; j < kTokChunk; ++j) {
+              const float vsum = warp_sum(part[j]);
+              if (lane == 0 && j < nt) {
+                if (r < 2) s_g[j][rr] = vsum * ts_g;
+                else s_u[j][rr] = vsum * ts_u;
+              }
+            }
+          }
+          named_bar_sync(1, kConsumers);
+          if (tid < kTokChunk * 16) {
+            const int j = tid >> 4, ii = tid & 15;
+            const float g = s_g[j][ii], uu = s_u[j][ii];
+            const float h = __fdiv_rn(g, 1.0f + expf(-g)) * uu;
+            float amax = fabsf(h);
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o, 16));
+            const uint32_t sbyte = f32_to_e4m3_sat(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), 1.0f));
+            const float sval = e4m3_to_f32(sbyte);
+            uint32_t code = 0;
+            if (sval != 0.0f) code = f32x2_to_e2m1x2(__fdiv_rn(h, __fmul_rn(sval, 1.0f)), 0.0f) & 0xFu;
+            uint32_t b = code | (__shfl_down_sync(0xffffffffu, code, 1, 16) << 4);
+            b |= __shfl_down_sync(0xffffffffu, b, 2, 16) << 8;
+            b |= __shfl_down_sync(0xffffffffu, b, 4, 16) << 16;
+            const uint32_t hi = __shfl_down_sync(0xffffffffu, b, 8, 16);
+            if (ii == 0 && j < nt) {
+              const size_t slot = (size_t)s_slot[j];
+              *reinterpret_cast<uint2*>(a.h_codes + slot * (I / 2) + hb * 8) = make_uint2(b, hi);
+              a.h_scales[slot * (I / kBlock) + hb] = (uint8_t)sbyte;
+            }
+            __threadfence();
+          }
+          named_bar_sync(1, kConsumers);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        if (tid == 0) atomicAdd(c.done + ai, 1);
+      } else {
+        // phase 2: wait for all h-blocks of this expert
+        const int rt = v % nrt;
+        const int n0 = rt * c.r2;
+        const int R = min(c.r2, d - n0);
+        if (tid == 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire(c.done + ai) < nhb) {
+            if (s_abort) break;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              s_abort = 1;
+              atomicExch(c.status, kStatusTimeout);
+              break;
             }
           }
         }
+        named_bar_sync(1, kConsumers);
+        if (s_abort) break;
+        __threadfence();
+        const float ts_o = G.dn_ts[ue.eloc];
+        const uint8_t* dc = st;
+        const uint8_t* ds = st + (size_t)c.r2 * (I / 2);
+        for (int c0 = 0; c0 < ue.cnt; c0 += kTokChunk) {
+          const int nt = min(kTokChunk, ue.cnt - c0);
+          named_bar_sync(1, kConsumers);
+          if (tid < nt) {
+            const int j = tid;
+            if (ue.shared) {
+              s_rows[j] = a.T * a.k + c0 + j;
+              s_tok[j] = c0 + j;
+              s_w[j] = 1.0f;
+            } else {
+              const int p = ue.off + c0 + j;
+              const int asg = a.sorted_assign[p];
+              s_rows[j] = p;
+              s_tok[j] = asg / a.k;
+              s_w[j] = a.topk_w[asg];
+            }
+          }
+          named_bar_sync(1, kConsumers);
+          stage_rows_cg(a.h_codes, a.h_scales, I, s_rows, nt, s_x, s_xs, tid, kConsumers);
+          named_bar_sync(1, kConsumers);
+          staged_e = -1;  // s_x now holds h, not x
+          for (int rr = warp; rr < R; rr += kConsumerWarps) {
+            const int n = n0 + rr;
+            float part[kTokChunk];
+#pragma unroll
+            for (int j = 0; j < kTokChunk; ++j) part[j] = 0.0f;
+            row_dots_smem(dc + (size_t)rr * (I / 2), ds + (size_t)rr * (I / kBlock), I, s_x, s_xs, nt, part);
+#pragma unroll
+            for (int j = 0; j < kTokChunk; ++j) {
+              const float vsum = warp_sum(part[j]);
+              if (lane == j && j < nt) {
+                const float o = vsum * ts_o;
+                if (a.mode == 0) {
+                  atomicAdd(a.out + (size_t)s_tok[j] * d + n, s_w[j] * o);
+                } else if (ue.shared) {
+                  a.shared_out[(size_t)s_tok[j] * d + n] = o;
+                } else {
+                  a.out[(size_t)s_rows[j] * d + n] = o;
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
   }
+  __syncthreads();
 }
 
-size_t ffn_decode_smem_gateup(int d, int E) {
-  return align16((size_t)(E + 1) * sizeof(int)) + align16((size_t)kTokChunk * (d / 2) * 4) +
-         align16((size_t)kTokChunk * (d / kBlock) * 4);
+size_t ffn_decode_smem_fused(int d, int I, int E, int stage_bytes, int nstages) {
+  const int kmax = d > I ? d : I;
+  return (size_t)nstages * stage_bytes + align16((size_t)kTokChunk * (kmax / 2) * 4) +
+         align16((size_t)kTokChunk * (kmax / kBlock) * 4) + align16((size_t)(E + 1) * sizeof(int)) +
+         2 * kMaxStages * sizeof(uint64_t);
 }
 
-size_t ffn_decode_smem_down(int I, int E) {
-  return align16((size_t)(E + 1) * sizeof(int)) + align16((size_t)kTokChunk * (I / 2) * 4) +
-         align16((size_t)kTokChunk * (I / kBlock) * 4);
-}
+constexpr size_t kFusedSmemLimit = 227 * 1024 - 2048;  // leave room for static shared memory
 
 size_t ffn_decode_ws_bytes(int64_t T, int d, int E, int k, int I) {
   const size_t slots = (size_t)(T * k + T);
-  return ((slots * (I / 2) + 255) & ~(size_t)255) + ((slots * (I / kBlock) + 255) & ~(size_t)255);
+  return ((slots * (I / 2) + 255) & ~(size_t)255) + ((slots * (I / kBlock) + 255) & ~(size_t)255) +
+         (((size_t)(E + 1) * sizeof(int32_t) + 255) & ~(size_t)255);
 }
 
-cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, cudaStream_t st) {
-  const int max_act = (a.T * a.k < a.E ? a.T * a.k : a.E) + (a.has_shared ? 1 : 0);
-  const int gu_units = max_act * (a.I / kBlock);
-  const int dn_units = max_act * ((a.d + kDownRows - 1) / kDownRows);
-  int g1 = gu_units < num_sms * 4 ? gu_units : num_sms * 4;
-  int g2 = dn_units < num_sms * 4 ? dn_units : num_sms * 4;
-  if (a.mode == 0) {
-    // the gate/up grid also zeroes y_acc: make sure it covers it reasonably
-    if (g1 < num_sms) g1 = num_sms;
+cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, int32_t* status, cudaStream_t st) {
+  DecodeCfg c;
+  c.stage_bytes = 32 * (a.d / 2 + a.d / kBlock);  // 16 gate + 16 up rows
+  c.kmax = a.d > a.I ? a.d : a.I;
+  int r2 = c.stage_bytes / (a.I / 2 + a.I / kBlock);
+  r2 = r2 > 256 ? 256 : r2;
+  r2 = (r2 / 16) * 16;
+  if (r2 < 16) {
+    // very wide I: grow the stage to hold 16 down rows
+    r2 = 16;
+    c.stage_bytes = 16 * (a.I / 2 + a.I / kBlock);
   }
-  if (g1 < 1) g1 = 1;
-  if (g2 < 1) g2 = 1;
-  ffn_gateup_decode_kernel<<<g1, kFfnThreads, ffn_decode_smem_gateup(a.d, a.E), st>>>(a);
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
-  ffn_down_decode_kernel<<<g2, kFfnThreads, ffn_decode_smem_down(a.I, a.E), st>>>(a);
+  c.r2 = r2;
+  int nst = kMaxStages;
+  while (nst > 2 && ffn_decode_smem_fused(a.d, a.I, a.E, c.stage_bytes, nst) > kFusedSmemLimit) --nst;
+  if (ffn_decode_smem_fused(a.d, a.I, a.E, c.stage_bytes, nst) > kFusedSmemLimit)
+    return cudaErrorInvalidConfiguration;
+  c.nstages = nst;
+  const size_t slots = (size_t)a.T * a.k + a.T;
+  c.done = reinterpret_cast<int32_t*>(a.h_codes + (((slots * (a.I / 2) + 255) & ~(size_t)255) +
+                                                   ((slots * (a.I / kBlock) + 255) & ~(size_t)255)));
+  c.status = status;
+  cudaError_t e = cudaMemsetAsync(c.done, 0, (size_t)(a.E + 1) * sizeof(int32_t), st);
+  if (e != cudaSuccess) return e;
+  if (a.mode == 0) {
+    e = cudaMemsetAsync(a.out, 0, (size_t)a.T * a.d * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+  }
+  const int max_act = (a.T * a.k < a.E ? a.T * a.k : a.E) + (a.has_shared ? 1 : 0);
+  const int units = max_act * (a.I / kBlock);
+  const int grid = units < num_sms ? (units > 0 ? units : 1) : num_sms;
+  const size_t smem = ffn_decode_smem_fused(a.d, a.I, a.E, c.stage_bytes, nst);
+  ffn_decode_fused_kernel<<<grid, kFusedThreads, smem, st>>>(a, c);
   return cudaGetLastError();
 }
 
 cudaError_t init_ffn_decode_attributes() {
-  cudaError_t e = cudaFuncSetAttribute(ffn_gateup_decode_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)ffn_decode_smem_gateup(8192, 1024));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(ffn_down_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)ffn_decode_smem_down(8192, 1024));
+  return cudaFuncSetAttribute(ffn_decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kFusedSmemLimit);
 }
 
 }  // namespace moe

@@ -56,10 +56,8 @@ size_t permute_ws_bytes(int64_t T, int k, int E);
 cudaError_t launch_hist(const int32_t* counts, int E, int64_t* cum, int32_t* rank_out, int reset,
                         cudaStream_t st);
 
-cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, int32_t* status, cudaStream_t st);
 size_t ffn_decode_ws_bytes(int64_t T, int d, int E, int k, int I);
-size_t ffn_decode_smem_gateup(int d, int E);
-size_t ffn_decode_smem_down(int I, int E);
 
 cudaError_t launch_combine(int T, int d, int k, int mode, const float* expert_out,
                            const float* shared_out, const float* topk_w, const int32_t* assign_pos,
