@@ -69,7 +69,9 @@ size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 size_t quant_ws_bytes() { return align256(kMaxPartials * sizeof(float)); }
 
 size_t ffn_ws_bytes(int64_t T, int d, int E, int k, int I) {
-  return ffn_decode_ws_bytes(T, d, E, k, I);
+  const size_t a = ffn_decode_ws_bytes(T, d, E, k, I);
+  const size_t b = ffn_tc_ws_bytes(T, d, E, k, I);
+  return a > b ? a : b;
 }
 
 moe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -214,8 +216,18 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t d, const float* Wr, c
 
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
                             uint8_t* dn_sf_tiled, void* stream) {
-  (void)W; (void)gu_sf_tiled; (void)dn_sf_tiled; (void)stream;
-  return fail(MOE_ERR_UNSUPPORTED_SHAPE, "tensor-core path not built yet");
+  if (!W || !gu_sf_tiled || !dn_sf_tiled) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if (W->E < 1 || W->d <= 0 || W->I <= 0) return fail(MOE_ERR_INVALID_ARG, "bad E/d/I");
+  if (W->d % 128 || W->I % 64) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "packing needs d % 128 == 0 and I % 64 == 0");
+  if (!W->gu_scales || !W->dn_scales) return fail(MOE_ERR_INVALID_ARG, "null scales");
+  if (!aligned16(W->gu_scales) || !aligned16(W->dn_scales) || !aligned16(gu_sf_tiled) || !aligned16(dn_sf_tiled))
+    return fail(MOE_ERR_INVALID_ARG, "scale pointers must be 16-byte aligned");
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_pack_sf(to_group(*W), W->E, W->d, W->I, gu_sf_tiled, dn_sf_tiled, sms,
+                                 (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_pack_experts launch");
 }
 
 moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, const float* xq_ts,
@@ -244,8 +256,14 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   if (!aligned16(xq_codes) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "xq_codes/out must be 16-byte aligned");
   if (mode == MOE_FFN_PER_ASSIGN && W->has_shared && !shared_out)
     return fail(MOE_ERR_INVALID_ARG, "shared_out needed in PER_ASSIGN mode with a shared expert");
-  if (path == MOE_PATH_PREFILL) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "tensor-core path not built yet");
-  const size_t need = ffn_ws_bytes(T, d, E, k, I);
+  const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
+                      (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
+  const bool tc_ok = ffn_tc_supported(d, I) && packed;
+  if (path == MOE_PATH_PREFILL && !tc_ok)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                "tensor-core path needs d % 256 == 0, I % 256 == 0 and scales packed by moe_pack_experts");
+  const bool use_tc = (path == MOE_PATH_PREFILL) || (path == MOE_PATH_AUTO && tc_ok);
+  const size_t need = use_tc ? ffn_tc_ws_bytes(T, d, E, k, I) : ffn_decode_ws_bytes(T, d, E, k, I);
   s = check_ws(ws, ws_bytes, need);
   if (s != MOE_OK) return s;
   int sms = 0;
@@ -269,7 +287,8 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const size_t slots = (size_t)T * k + T;
   a.h_codes = reinterpret_cast<uint8_t*>(ws);
   a.h_scales = reinterpret_cast<uint8_t*>(ws) + align256(slots * (I / 2));
-  cudaError_t e = launch_ffn_decode(a, sms, dstatus, (cudaStream_t)stream);
+  cudaError_t e = use_tc ? launch_ffn_tc(a, ws, sms, dstatus, (cudaStream_t)stream)
+                         : launch_ffn_decode(a, sms, dstatus, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
 }
 

@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) ffn_decode_fused_kernel(FfnA
   __shared__ float s_w[kTokChunk];
   __shared__ int tmp[32];
   __shared__ volatile int s_abort;
+  __shared__ int s_go[2];  // decision of the waiting thread, by unit parity
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -294,10 +295,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) ffn_decode_fused_kernel(FfnA
     const float ts_x = *a.xq_ts;
     for (int it = 0; it < n_units; ++it) {
       const int s = it % nst;
-      // one thread waits, the barrier publishes both the data and the abort decision
-      if (tid == 0) mbar_wait(&full[s], (it / nst) & 1, &s_abort, c.status);
+      // one thread waits, the barrier publishes both the data and the decision
+      if (tid == 0) s_go[it & 1] = mbar_wait(&full[s], (it / nst) & 1, &s_abort, c.status) ? 1 : 0;
       named_bar_sync(1, kConsumers);
-      if (s_abort) break;
+      if (!s_go[it & 1]) break;
       const uint8_t* st = stages + (size_t)s * c.stage_bytes;
       const bool ph1 = it < (r1.end - r1.beg);
       const int v = ph1 ? r1.beg + it : r2.beg + (it - (r1.end - r1.beg));
@@ -380,18 +381,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1) ffn_decode_fused_kernel(FfnA
         const int n0 = rt * c.r2;
         const int R = min(c.r2, d - n0);
         if (tid == 0) {
+          int ok = 1;
           const uint64_t t0 = globaltimer_ns();
           while (ld_acquire(c.done + ai) < nhb) {
-            if (s_abort) break;
+            if (s_abort) {
+              ok = 0;
+              break;
+            }
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
               s_abort = 1;
               atomicExch(c.status, kStatusTimeout);
+              ok = 0;
               break;
             }
           }
+          s_go[it & 1] = ok;
         }
         named_bar_sync(1, kConsumers);
-        if (s_abort) break;
+        if (!s_go[it & 1]) break;
         __threadfence();
         const float ts_o = G.dn_ts[ue.eloc];
         const uint8_t* dc = st;

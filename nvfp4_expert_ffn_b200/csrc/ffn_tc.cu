@@ -1,0 +1,627 @@
+// Expert SwiGLU FFN on the tcgen05 tensor cores: block-scaled NVFP4 x NVFP4 grouped GEMMs.
+//
+// The MoE layer of the Basalt pages ("What Basalt changes in a Blackwell local inference
+// stack", section "Experts can move without becoming free": each token runs a subset of
+// experts; "Basalt" project page, "Engines": routed experts are NVFP4) computes, per
+// expert, h = silu(x Wg^T) * (x Wu^T), h re-quantised to NVFP4 (tensor scale 1), then
+// o = h Wd^T, and y += w * o. Here both products are tcgen05.mma kind::mxf4nvf4 with the
+// E4M3 block scales staged into tensor memory: the tensor core consumes E2M1 codes and
+// scales directly, nothing is decoded on the CUDA cores.
+//
+// Three launches per call:
+//   1. tc_schedule_kernel (1 CTA): 128-row m-tiles over each expert's tokens (the shared
+//      expert is slot E); zeroes the per-m-tile completion counters.
+//   2. tc_gather_kernel: copies the activation rows of every m-tile into a padded,
+//      expert-major buffer (codes row-major, scales re-tiled into 512-byte scale atoms)
+//      and records (token, weight, output slot) per row; zeroes y in accumulate mode.
+//   3. tc_ffn_kernel (persistent, one CTA per SM, warp-specialised):
+//        warp 0   TMA producer (A rows, B weight tiles, scale atoms) into a 5-stage ring
+//        warp 1   TMEM allocation and the MMA issuer (single thread)
+//        warps 2-5 epilogue: TMEM -> registers
+//      phase-1 tiles (m-tile, 64 gate + 64 up rows): SwiGLU and NVFP4 h quantisation in
+//      the epilogue, h written to the workspace; phase-2 tiles (m-tile, 128 output rows)
+//      wait until all phase-1 tiles of their m-tile are done (bounded wait), then the down
+//      GEMM, whose epilogue adds w * o into y (red.global.add.v4.f32) or stores o.
+//      Accumulators are double-buffered in TMEM so an epilogue overlaps the next tile.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+constexpr int kTcStages = 5;
+constexpr int kTileM = 128;                // tokens per m-tile (MMA M)
+constexpr int kTileN = 128;                // weight rows per tile (MMA N)
+constexpr int kStageK = 256;               // elements of K per pipeline stage (4 MMAs)
+constexpr int kAtom = 512;                 // bytes of one 128-row x 4-block scale atom
+constexpr int kABytes = kTileM * kStageK / 2;   // 16 KB
+constexpr int kBBytes = kTileN * kStageK / 2;   // 16 KB
+constexpr int kSfBytes = 4 * kAtom;             // 2 KB per operand per stage
+constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
+constexpr int kTcThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kIdesc = idesc_mxf4nvf4(kTileM, kTileN);
+
+MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+MOE_DEV int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+struct TcParams {
+  // schedule and gathered rows (workspace)
+  int32_t* n_mtiles;
+  int32_t* mt_expert;
+  int32_t* mt_valid;
+  int32_t* mt_first;  // local row index (within its expert) of the m-tile's first row
+  int32_t* done1;
+  int32_t* row_token;
+  float* row_weight;
+  int32_t* row_slot;
+  uint8_t* a1_codes;  // [rows_cap][d/2]
+  uint8_t* sfa1;      // [m][d/64][512]
+  uint8_t* h_codes;   // [rows_cap][I/2]
+  uint8_t* sfa2;      // [m][I/64][512]
+  int max_m;
+  // inputs
+  const uint8_t* xq_codes;
+  const uint8_t* xq_scales;
+  const float* xq_ts;
+  const int32_t* offsets;
+  const int32_t* sorted_assign;
+  const float* topk_w;
+  ExpertGroup routed, shared;
+  int has_shared;
+  int E, d, I, T, k, mode;
+  float* out;
+  float* shared_out;
+  int32_t* status;
+};
+
+// ---------------------------------------------------------------- 1. schedule
+__global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
+  __shared__ int tmp[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int nslots = p.E + (p.has_shared ? 1 : 0);
+  for (int e0 = 0; e0 < nslots; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    int cnt = 0;
+    if (e < p.E) cnt = p.offsets[e + 1] - p.offsets[e];
+    else if (e < nslots) cnt = p.T;
+    const int nm = (cnt + kTileM - 1) / kTileM;
+    int total;
+    const int base = block_exclusive_scan(nm, tmp, &total) + carry;
+    for (int i = 0; i < nm; ++i) {
+      const int m = base + i;
+      if (m < p.max_m) {
+        p.mt_expert[m] = e;
+        p.mt_valid[m] = min(kTileM, cnt - i * kTileM);
+        p.mt_first[m] = i * kTileM;
+        p.done1[m] = 0;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *p.n_mtiles = min(carry, p.max_m);
+}
+
+// ---------------------------------------------------------------- 2. gather
+// One warp per padded row; row r of m-tile m is local token index mt_first[m] + r of its
+// expert.
+__global__ void __launch_bounds__(256) tc_gather_kernel(TcParams p) {
+  const int n_m = *p.n_mtiles;
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  const int d = p.d;
+  if (p.mode == 0) {
+    const size_t n4 = (size_t)p.T * d / 4;
+    float4* o4 = reinterpret_cast<float4*>(p.out);
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x)
+      o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (int w = gw; w < n_m * kTileM; w += nw) {
+    const int m = w / kTileM, r = w % kTileM;
+    if (r >= p.mt_valid[m]) continue;
+    const int e = p.mt_expert[m];
+    const int i = p.mt_first[m] + r;
+    int t, slot;
+    float wgt;
+    if (e < p.E) {
+      const int q = p.offsets[e] + i;
+      const int a = p.sorted_assign[q];
+      t = a / p.k;
+      wgt = p.topk_w[a];
+      slot = q;
+    } else {
+      t = i;
+      wgt = 1.0f;
+      slot = -1;
+    }
+    const size_t prow = (size_t)m * kTileM + r;
+    const uint4* src = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
+    uint4* dst = reinterpret_cast<uint4*>(p.a1_codes + prow * (d / 2));
+    for (int c = lane; c < d / 32; c += 32) dst[c] = __ldg(src + c);
+    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
+    for (int kc = lane; kc < d / 64; kc += 32) {
+      uint8_t* atom = p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom;
+      *reinterpret_cast<uint32_t*>(atom + (r % 32) * 16 + (r / 32) * 4) = __ldg(ssrc + kc);
+    }
+    if (lane == 0) {
+      p.row_token[prow] = t;
+      p.row_weight[prow] = wgt;
+      p.row_slot[prow] = slot;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- pack weight scales
+// gate/up: [E][I/64][d/64][512], atom row r < 64 -> gate row 64j + r, else up row 64j + r - 64
+// down:    [E][d/128][I/64][512], atom row r -> down row 128j + r
+// Within an atom, row r = 32*r1 + r0 and block kb of the 4-block chunk sit at r0*16+r1*4+kb.
+__global__ void pack_sf_kernel(const uint8_t* __restrict__ gu_scales, const uint8_t* __restrict__ dn_scales,
+                               int E, int d, int I, uint8_t* __restrict__ gu_t, uint8_t* __restrict__ dn_t) {
+  const size_t n_gu = (size_t)E * (I / 64) * (d / 64) * 128;  // 32-bit words
+  const size_t n_dn = (size_t)E * (d / 128) * (I / 64) * 128;
+  for (size_t w = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w < n_gu + n_dn;
+       w += (size_t)gridDim.x * blockDim.x) {
+    if (w < n_gu) {
+      const size_t atom = w / 128;
+      const int slot = (int)(w % 128);  // r0 * 4 + r1
+      const int r = (slot % 4) * 32 + slot / 4;
+      const int kc = (int)(atom % (d / 64));
+      const int j = (int)((atom / (d / 64)) % (I / 64));
+      const size_t e = atom / ((size_t)(d / 64) * (I / 64));
+      const int row = r < 64 ? 64 * j + r : I + 64 * j + (r - 64);
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(gu_scales + (e * 2 * I + row) * (d / kBlock) + 4 * kc);
+      *reinterpret_cast<uint32_t*>(gu_t + atom * kAtom + (slot / 4) * 16 + (slot % 4) * 4) = v;
+    } else {
+      const size_t ww = w - n_gu;
+      const size_t atom = ww / 128;
+      const int slot = (int)(ww % 128);
+      const int r = (slot % 4) * 32 + slot / 4;
+      const int kc = (int)(atom % (I / 64));
+      const int j = (int)((atom / (I / 64)) % (d / 128));
+      const size_t e = atom / ((size_t)(I / 64) * (d / 128));
+      const int row = 128 * j + r;
+      const uint32_t v = *reinterpret_cast<const uint32_t*>(dn_scales + (e * d + row) * (I / kBlock) + 4 * kc);
+      *reinterpret_cast<uint32_t*>(dn_t + atom * kAtom + (slot / 4) * 16 + (slot % 4) * 4) = v;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- 3. persistent FFN kernel
+struct TcMaps {
+  CUtensorMap a1;    // gathered x codes  [rows_cap][d/2]
+  CUtensorMap a2;    // h codes           [rows_cap][I/2]
+  CUtensorMap b1;    // routed gate/up    {d/2, I, 2, E}
+  CUtensorMap b1s;   // shared gate/up    {d/2, I, 2, 1}
+  CUtensorMap b2;    // routed down       {I/2, d, E}
+  CUtensorMap b2s;   // shared down       {I/2, d, 1}
+};
+
+struct TileInfo {
+  int phase, m, j;
+};
+
+MOE_DEV TileInfo decode_tile(int t, int n_m, int nt1, int nt2) {
+  TileInfo ti;
+  if (t < n_m * nt1) {
+    ti.phase = 1;
+    ti.m = t / nt1;
+    ti.j = t % nt1;
+  } else {
+    const int u = t - n_m * nt1;
+    ti.phase = 2;
+    ti.m = u / nt2;
+    ti.j = u % nt2;
+  }
+  return ti;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t full[kTcStages], empty[kTcStages], acc_full[2], acc_empty[2], final_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = p.d, I = p.I;
+  const int nt1 = I / 64, nt2 = d / kTileN;
+  const int nks1 = d / kStageK, nks2 = I / kStageK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(&final_bar, 1);
+    fence_barrier_init();
+    s_abort = 0;
+    prefetch_tensormap(&maps.a1);
+    prefetch_tensormap(&maps.a2);
+    prefetch_tensormap(&maps.b1);
+    prefetch_tensormap(&maps.b2);
+  }
+  if (warp == 1) tmem_alloc(&s_tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int n_m = *p.n_mtiles;
+  const int total = n_m * (nt1 + nt2);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
+        const TileInfo ti = decode_tile(t, n_m, nt1, nt2);
+        const int e = p.mt_expert[ti.m];
+        const bool sh = (e == p.E);
+        const int eloc = sh ? 0 : e;
+        const int nq = (p.mt_valid[ti.m] + 31) / 32;
+        if (ti.phase == 2) {
+          // h of this m-tile is produced by phase-1 tiles of any CTA
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(p.done1 + ti.m) < nt1) {
+            if (s_abort) break;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              s_abort = 1;
+              atomicExch(p.status, kStatusTimeout);
+              break;
+            }
+          }
+          if (s_abort) break;
+          fence_proxy_async_global();
+        }
+        const int nks = ti.phase == 1 ? nks1 : nks2;
+        for (int ks = 0; ks < nks; ++ks, ++it) {
+          const int s = it % kTcStages;
+          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1, &s_abort, p.status)) break;
+          uint8_t* st = smem + (size_t)s * kStageBytes;
+          uint8_t* sA = st;
+          uint8_t* sB = st + kABytes;
+          uint8_t* sSFA = sB + kBBytes;
+          uint8_t* sSFB = sSFA + kSfBytes;
+          mbar_arrive_expect_tx(&full[s], (uint32_t)(nq * 4096 + kBBytes + 2 * kSfBytes));
+          const CUtensorMap* ma = ti.phase == 1 ? &maps.a1 : &maps.a2;
+          for (int q = 0; q < nq; ++q)
+            tma_load_2d(sA + q * 4096, ma, &full[s], ks * 128, ti.m * kTileM + 32 * q);
+          const uint8_t* sfa;
+          const uint8_t* sfb;
+          if (ti.phase == 1) {
+            tma_load_4d(sB, sh ? &maps.b1s : &maps.b1, &full[s], ks * 128, 64 * ti.j, 0, eloc);
+            sfa = p.sfa1 + ((size_t)ti.m * (d / 64) + 4 * ks) * kAtom;
+            const ExpertGroup& G = sh ? p.shared : p.routed;
+            sfb = G.gu_sf_tiled + (((size_t)eloc * nt1 + ti.j) * (d / 64) + 4 * ks) * kAtom;
+          } else {
+            tma_load_3d(sB, sh ? &maps.b2s : &maps.b2, &full[s], ks * 128, kTileN * ti.j, eloc);
+            sfa = p.sfa2 + ((size_t)ti.m * (I / 64) + 4 * ks) * kAtom;
+            const ExpertGroup& G = sh ? p.shared : p.routed;
+            sfb = G.dn_sf_tiled + (((size_t)eloc * nt2 + ti.j) * (I / 64) + 4 * ks) * kAtom;
+          }
+          bulk_g2s(sSFA, sfa, kSfBytes, &full[s]);
+          bulk_g2s(sSFB, sfb, kSfBytes, &full[s]);
+        }
+      }
+      // no copies left in flight: the last issued stage of each slot has landed
+      for (uint32_t j = (it > (uint32_t)kTcStages ? it - kTcStages : 0); j < it; ++j) {
+        volatile int no_abort = 0;
+        mbar_wait(&full[j % kTcStages], (j / kTcStages) & 1, &no_abort, p.status);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tc = 0;
+      for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x, ++tc) {
+        const TileInfo ti = decode_tile(t, n_m, nt1, nt2);
+        const int buf = tc & 1;
+        if (!mbar_wait(&acc_empty[buf], ((tc >> 1) & 1) ^ 1, &s_abort, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + buf * kTileN;
+        const int nks = ti.phase == 1 ? nks1 : nks2;
+        bool ok = true;
+        for (int ks = 0; ks < nks; ++ks, ++it) {
+          const int s = it % kTcStages;
+          if (!mbar_wait(&full[s], (it / kTcStages) & 1, &s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint8_t* st = smem + (size_t)s * kStageBytes;
+          const uint32_t aA = smem_u32(st), aB = smem_u32(st + kABytes);
+          const uint32_t aSFA = smem_u32(st + kABytes + kBBytes), aSFB = aSFA + kSfBytes;
+          const uint32_t sfa_col = tmem + 256 + 32 * s, sfb_col = sfa_col + 16;
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            tmem_cp_sf(sfa_col + 4 * kc, sdesc_sf(aSFA + kAtom * kc));
+            tmem_cp_sf(sfb_col + 4 * kc, sdesc_sf(aSFB + kAtom * kc));
+          }
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            mma_mxf4nvf4(d_tmem, sdesc_sw128(aA + 32 * kc), sdesc_sw128(aB + 32 * kc), kIdesc,
+                         sfa_col + 4 * kc, sfb_col + 4 * kc, (ks | kc) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+      }
+      // all issued tensor-core work has completed before TMEM is released
+      mma_commit(&final_bar);
+      volatile int no_abort = 0;
+      mbar_wait(&final_bar, 0, &no_abort, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    // one thread waits for the accumulator; a named barrier publishes data and decision
+    __shared__ int s_epi_go[2];  // by tile parity: a slow warp never reads the next tile's value
+    const int q = warp & 3;            // TMEM lane quarter of this warp
+    const int row = 32 * q + lane;     // accumulator row = token row of the m-tile
+    const float ts_x = *p.xq_ts;
+    uint32_t tc = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
+      const TileInfo ti = decode_tile(t, n_m, nt1, nt2);
+      const int buf = tc & 1;
+      if (warp == 2 && lane == 0)
+        s_epi_go[buf] = mbar_wait(&acc_full[buf], (tc >> 1) & 1, &s_abort, p.status) ? 1 : 0;
+      named_bar_sync(2, 128);
+      if (!s_epi_go[buf]) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kTileN;
+      const int e = p.mt_expert[ti.m];
+      const bool sh = (e == p.E);
+      const int eloc = sh ? 0 : e;
+      const ExpertGroup& G = sh ? p.shared : p.routed;
+      const bool valid = row < p.mt_valid[ti.m];
+      const size_t prow = (size_t)ti.m * kTileM + row;
+      if (ti.phase == 1) {
+        const float sg = G.gu_ts[2 * eloc] * ts_x, su = G.gu_ts[2 * eloc + 1] * ts_x;
+        uint32_t sfbytes = 0;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + 32 * c, g);
+          tmem_ld32(taddr + 64 + 32 * c, u);
+          tmem_ld_wait();
+          float h[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gv = __uint_as_float(g[i]) * sg, uv = __uint_as_float(u[i]) * su;
+            h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
+          }
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            uint2 codes;
+            const uint32_t sb = quantize_block16(h + 16 * b, 1.0f, &codes);
+            sfbytes |= sb << (8 * (2 * c + b));
+            if (valid)
+              *reinterpret_cast<uint2*>(p.h_codes + prow * (I / 2) + 32 * ti.j + 16 * c + 8 * b) = codes;
+          }
+        }
+        if (valid)
+          *reinterpret_cast<uint32_t*>(p.sfa2 + ((size_t)ti.m * (I / 64) + ti.j) * kAtom + (row % 32) * 16 +
+                                       (row / 32) * 4) = sfbytes;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        // publish h of this tile: generic writes -> visible to other CTAs' TMA reads
+        fence_proxy_async_global();
+        __threadfence();
+        named_bar_sync(2, 128);
+        if (warp == 2 && lane == 0) atomicAdd(p.done1 + ti.m, 1);
+      } else {
+        const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
+        int tok = 0, slot = 0;
+        float wgt = 0.0f;
+        if (valid) {
+          tok = p.row_token[prow];
+          wgt = p.row_weight[prow];
+          slot = p.row_slot[prow];
+        }
+#pragma unroll 1
+        for (int c = 0; c < kTileN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + 32 * c, v);
+          tmem_ld_wait();
+          if (valid) {
+            const int n0 = kTileN * ti.j + 32 * c;
+            if (p.mode == 0) {
+              float* dst = p.out + (size_t)tok * d + n0;
+              const float f = wgt * ts_o;
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                red_add_v4(dst + 4 * i, __uint_as_float(v[4 * i]) * f, __uint_as_float(v[4 * i + 1]) * f,
+                           __uint_as_float(v[4 * i + 2]) * f, __uint_as_float(v[4 * i + 3]) * f);
+            } else {
+              float* dst = sh ? p.shared_out + (size_t)tok * d + n0 : p.out + (size_t)slot * d + n0;
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                reinterpret_cast<float4*>(dst)[i] =
+                    make_float4(__uint_as_float(v[4 * i]) * ts_o, __uint_as_float(v[4 * i + 1]) * ts_o,
+                                __uint_as_float(v[4 * i + 2]) * ts_o, __uint_as_float(v[4 * i + 3]) * ts_o);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+cudaError_t get_encode() {
+  if (g_encode) return cudaSuccess;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess) return e;
+  if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return cudaSuccess;
+}
+
+cudaError_t encode_u8(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                      const cuuint64_t* strides, const cuuint32_t* box) {
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), dims,
+                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct TcLayout {
+  int max_m;
+  size_t rows_cap;
+  size_t off_hdr, off_expert, off_valid, off_first, off_done, off_tok, off_w, off_slot, off_a1, off_sfa1, off_h, off_sfa2,
+      total;
+};
+
+TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
+  TcLayout L;
+  const int64_t n = T * k;
+  L.max_m = (int)((n + kTileM - 1) / kTileM + (n < E ? n : E) + (T + kTileM - 1) / kTileM + 2);
+  L.rows_cap = (size_t)L.max_m * kTileM;
+  size_t o = 0;
+  L.off_hdr = o; o += 256;
+  L.off_expert = o; o += a256((size_t)L.max_m * 4);
+  L.off_valid = o; o += a256((size_t)L.max_m * 4);
+  L.off_first = o; o += a256((size_t)L.max_m * 4);
+  L.off_done = o; o += a256((size_t)L.max_m * 4);
+  L.off_tok = o; o += a256(L.rows_cap * 4);
+  L.off_w = o; o += a256(L.rows_cap * 4);
+  L.off_slot = o; o += a256(L.rows_cap * 4);
+  L.off_a1 = o; o += a256(L.rows_cap * (d / 2));
+  L.off_sfa1 = o; o += a256(L.rows_cap * (d / kBlock));
+  L.off_h = o; o += a256(L.rows_cap * (I / 2));
+  L.off_sfa2 = o; o += a256(L.rows_cap * (I / kBlock));
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+
+size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I) {
+  if (d % kStageK || I % kStageK) return 0;
+  return tc_layout(T, d, E, k, I).total;
+}
+
+bool ffn_tc_supported(int d, int I) { return d % kStageK == 0 && I % kStageK == 0 && d <= 16384 && I <= 16384; }
+
+size_t ffn_tc_smem_bytes() { return (size_t)kTcStages * kStageBytes + 1024; }
+
+cudaError_t init_ffn_tc_attributes() {
+  return cudaFuncSetAttribute(tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ffn_tc_smem_bytes());
+}
+
+cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t, int num_sms,
+                           cudaStream_t st) {
+  pack_sf_kernel<<<num_sms * 4, 256, 0, st>>>(g.gu_scales, g.dn_scales, E, d, I, gu_t, dn_t);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st) {
+  cudaError_t e = get_encode();
+  if (e != cudaSuccess) return e;
+  const TcLayout L = tc_layout(a.T, a.d, a.E, a.k, a.I);
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  TcParams p;
+  p.n_mtiles = reinterpret_cast<int32_t*>(w + L.off_hdr);
+  p.mt_expert = reinterpret_cast<int32_t*>(w + L.off_expert);
+  p.mt_valid = reinterpret_cast<int32_t*>(w + L.off_valid);
+  p.mt_first = reinterpret_cast<int32_t*>(w + L.off_first);
+  p.done1 = reinterpret_cast<int32_t*>(w + L.off_done);
+  p.row_token = reinterpret_cast<int32_t*>(w + L.off_tok);
+  p.row_weight = reinterpret_cast<float*>(w + L.off_w);
+  p.row_slot = reinterpret_cast<int32_t*>(w + L.off_slot);
+  p.a1_codes = w + L.off_a1;
+  p.sfa1 = w + L.off_sfa1;
+  p.h_codes = w + L.off_h;
+  p.sfa2 = w + L.off_sfa2;
+  p.max_m = L.max_m;
+  p.xq_codes = a.xq_codes;
+  p.xq_scales = a.xq_scales;
+  p.xq_ts = a.xq_ts;
+  p.offsets = a.offsets;
+  p.sorted_assign = a.sorted_assign;
+  p.topk_w = a.topk_w;
+  p.routed = a.routed;
+  p.shared = a.shared;
+  p.has_shared = a.has_shared;
+  p.E = a.E; p.d = a.d; p.I = a.I; p.T = a.T; p.k = a.k; p.mode = a.mode;
+  p.out = a.out;
+  p.shared_out = a.shared_out;
+  p.status = status;
+
+  TcMaps maps;
+  const int d = a.d, I = a.I;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)L.rows_cap};
+    cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
+    cuuint32_t box[2] = {128, 32};
+    if ((e = encode_u8(&maps.a1, p.a1_codes, 2, dims, strides, box)) != cudaSuccess) return e;
+  }
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)(I / 2), (cuuint64_t)L.rows_cap};
+    cuuint64_t strides[1] = {(cuuint64_t)(I / 2)};
+    cuuint32_t box[2] = {128, 32};
+    if ((e = encode_u8(&maps.a2, p.h_codes, 2, dims, strides, box)) != cudaSuccess) return e;
+  }
+  for (int which = 0; which < 2; ++which) {
+    const ExpertGroup& g = which ? a.shared : a.routed;
+    const int E = which ? 1 : a.E;
+    CUtensorMap* m1 = which ? &maps.b1s : &maps.b1;
+    CUtensorMap* m2 = which ? &maps.b2s : &maps.b2;
+    if (which && !a.has_shared) {
+      *m1 = maps.b1;
+      *m2 = maps.b2;
+      continue;
+    }
+    cuuint64_t dims1[4] = {(cuuint64_t)(d / 2), (cuuint64_t)I, 2, (cuuint64_t)E};
+    cuuint64_t str1[3] = {(cuuint64_t)(d / 2), (cuuint64_t)I * (d / 2), (cuuint64_t)2 * I * (d / 2)};
+    cuuint32_t box1[4] = {128, 64, 2, 1};
+    if ((e = encode_u8(m1, g.gu_codes, 4, dims1, str1, box1)) != cudaSuccess) return e;
+    cuuint64_t dims2[3] = {(cuuint64_t)(I / 2), (cuuint64_t)d, (cuuint64_t)E};
+    cuuint64_t str2[2] = {(cuuint64_t)(I / 2), (cuuint64_t)d * (I / 2)};
+    cuuint32_t box2[3] = {128, 128, 1};
+    if ((e = encode_u8(m2, g.dn_codes, 3, dims2, str2, box2)) != cudaSuccess) return e;
+  }
+  tc_schedule_kernel<<<1, 1024, 0, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc_gather_kernel<<<num_sms * 4, 256, 0, st>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc_ffn_kernel<<<num_sms, kTcThreads, ffn_tc_smem_bytes(), st>>>(maps, p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

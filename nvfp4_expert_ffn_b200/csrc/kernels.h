@@ -63,13 +63,23 @@ cudaError_t launch_combine(int T, int d, int k, int mode, const float* expert_ou
                            const float* shared_out, const float* topk_w, const int32_t* assign_pos,
                            int rms, uint16_t* y, cudaStream_t st);
 
+// tensor-core (tcgen05) FFN path
+bool ffn_tc_supported(int d, int I);
+size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I);
+cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
+cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
+                           int num_sms, cudaStream_t st);
+
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t init_route_attributes();
 cudaError_t init_ffn_decode_attributes();
+cudaError_t init_ffn_tc_attributes();
 inline cudaError_t init_kernel_attributes() {
   cudaError_t e = init_route_attributes();
   if (e != cudaSuccess) return e;
-  return init_ffn_decode_attributes();
+  e = init_ffn_decode_attributes();
+  if (e != cudaSuccess) return e;
+  return init_ffn_tc_attributes();
 }
 
 }  // namespace moe

@@ -17,9 +17,10 @@ from . import synth
 
 def quantize_weights_gpu(seed: int, cfg: synth.LayerShape, layer: int = 0, device="cuda",
                          experts: Optional[range] = None, shared: bool = False,
-                         ws: Optional[torch.Tensor] = None) -> B.ExpertWeights:
+                         ws: Optional[torch.Tensor] = None, pack: bool = True) -> B.ExpertWeights:
     """Generate an expert group's bf16 weights on the GPU and quantise each matrix
-    (gate, up, down of every expert, one tensor scale each) with nvfp4_quantize_act."""
+    (gate, up, down of every expert, one tensor scale each) with nvfp4_quantize_act; then
+    re-tile the scales for the tensor-core path (moe_pack_experts) when the shape allows."""
     E = 1 if shared else cfg.E
     d, I = cfg.d, cfg.I
     w = B.ExpertWeights(
@@ -37,6 +38,8 @@ def quantize_weights_gpu(seed: int, cfg: synth.LayerShape, layer: int = 0, devic
         B.nvfp4_quantize_act(g, w.gu_codes[e, :I], w.gu_scales[e, :I], w.gu_ts[e, 0:1], ws=ws)
         B.nvfp4_quantize_act(u, w.gu_codes[e, I:], w.gu_scales[e, I:], w.gu_ts[e, 1:2], ws=ws)
         B.nvfp4_quantize_act(dn, w.dn_codes[e], w.dn_scales[e], w.dn_ts[e:e + 1], ws=ws)
+    if pack and d % 128 == 0 and I % 64 == 0:
+        B.moe_pack_experts(w)
     return w
 
 

@@ -50,8 +50,9 @@ def oracle_expert_from_bf16(g, u, dn) -> omoe.Expert:
                                 bits_to_f32(dn.cpu().numpy()))
 
 
-def weights_to_gpu(experts, device="cuda") -> B.ExpertWeights:
-    """Upload a list of oracle Expert objects (their codes) as one GPU expert group."""
+def weights_to_gpu(experts, device="cuda", pack=False) -> B.ExpertWeights:
+    """Upload a list of oracle Expert objects (their codes) as one GPU expert group;
+    optionally re-tile its scales for the tensor-core path."""
     gu_c = np.stack([e.gu_codes for e in experts])
     gu_s = np.stack([e.gu_scales for e in experts])
     gu_t = np.array([[e.gate_ts, e.up_ts] for e in experts], dtype=F32)
@@ -59,7 +60,10 @@ def weights_to_gpu(experts, device="cuda") -> B.ExpertWeights:
     dn_s = np.stack([e.dn_scales for e in experts])
     dn_t = np.array([e.dn_ts for e in experts], dtype=F32)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)  # noqa: E731
-    return B.ExpertWeights(t(gu_c), t(gu_s), t(gu_t), t(dn_c), t(dn_s), t(dn_t))
+    w = B.ExpertWeights(t(gu_c), t(gu_s), t(gu_t), t(dn_c), t(dn_s), t(dn_t))
+    if pack:
+        B.moe_pack_experts(w)
+    return w
 
 
 class OracleWeights:

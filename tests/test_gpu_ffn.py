@@ -62,7 +62,7 @@ def _oracle_outputs(xq, routing, experts, shared, T, d, k, tokens=None):
     return o, os_, y
 
 
-def _tiny_case(seed, d, E, k, I, T, shared, zipf=0.0):
+def _tiny_case(seed, d, E, k, I, T, shared, zipf=0.0, pack=False):
     cfg = synth.LayerShape("t", cid=100 + seed, d=d, E=E, k=k, I=I, shared=shared, zipf_s=zipf,
                            router_std=0.02)
     experts = [oracle_expert_from_bf16(*synth.make_expert_weights_bf16(seed, cfg, e))
@@ -74,7 +74,7 @@ def _tiny_case(seed, d, E, k, I, T, shared, zipf=0.0):
     xf = bits_to_f32(x)
     xq = onv.quantize(xf)
     routing = _oracle_route(xf, Wr.numpy(), br.numpy(), k, E)
-    gpu = B.Experts(weights_to_gpu(experts), weights_to_gpu([sh]) if shared else None)
+    gpu = B.Experts(weights_to_gpu(experts, pack=pack), weights_to_gpu([sh], pack=pack) if shared else None)
     return experts, sh, xq, routing, gpu
 
 
@@ -102,6 +102,29 @@ def test_ffn_decode_path_matches_oracle(mode, d, E, k, I, T, shared):
     assert_close_layer(bits_to_f32(y_g), y_r, "y bf16")
 
 
+@pytest.mark.parametrize("mode", [B.MOE_FFN_ACCUMULATE, B.MOE_FFN_PER_ASSIGN])
+@pytest.mark.parametrize("d,E,k,I,T,shared,zipf", [
+    (256, 8, 2, 256, 16, False, 0.0),     # one k-stage per GEMM
+    (512, 16, 4, 256, 1, True, 0.0),      # single token
+    (512, 16, 4, 512, 37, True, 1.0),     # ragged, Zipf: experts with 0..many tokens
+    (256, 4, 2, 256, 700, True, 0.0),     # several 128-row m-tiles per expert
+    (2048, 32, 4, 512, 300, True, 0.8),   # decode/prefill widths
+    (1024, 8, 1, 768, 129, False, 0.0),   # k=1, m-tile boundary +1, 3 k-stages of h
+])
+def test_ffn_tensor_core_path_matches_oracle(mode, d, E, k, I, T, shared, zipf):
+    experts, sh, xq, routing, gpu = _tiny_case(12, d, E, k, I, T, shared, zipf=zipf, pack=True)
+    o_g, os_g, y_g = _run_ffn(xq, routing, gpu, k, mode, B.MOE_PATH_PREFILL, T, d)
+    o_r, os_r, y_r = _oracle_outputs(xq, routing, experts, sh, T, d, k)
+    idx, w, offsets, sa, pos = routing
+    if mode == B.MOE_FFN_PER_ASSIGN:
+        assert_close_layer(o_g, o_r[sa], "per-assignment o")
+        if sh is not None:
+            assert_close_layer(os_g, os_r, "shared o")
+    else:
+        assert_close_layer(o_g, y_r, "y_acc")
+    assert_close_layer(bits_to_f32(y_g), y_r, "y bf16")
+
+
 @pytest.fixture(scope="module")
 def decode_layer():
     cfg = synth.CONFIGS["decode"]
@@ -110,15 +133,16 @@ def decode_layer():
     return cfg, B.Experts(routed, shared), OracleWeights(0, cfg)
 
 
+@pytest.mark.parametrize("path", [B.MOE_PATH_DECODE, B.MOE_PATH_PREFILL])
 @pytest.mark.parametrize("T", [1, 4, 8])
-def test_ffn_decode_config_full_size(decode_layer, T):
+def test_ffn_decode_config_full_size(decode_layer, T, path):
     cfg, gpu, ow = decode_layer
     x = synth.make_x(0, cfg, T).numpy()
     Wr, br = synth.make_router(0, cfg)
     xf = bits_to_f32(x)
     xq = onv.quantize(xf)
     routing = _oracle_route(xf, Wr.numpy(), br.numpy(), cfg.k, cfg.E)
-    _, _, y_g = _run_ffn(xq, routing, gpu, cfg.k, B.MOE_FFN_ACCUMULATE, B.MOE_PATH_DECODE, T, cfg.d)
+    _, _, y_g = _run_ffn(xq, routing, gpu, cfg.k, B.MOE_FFN_ACCUMULATE, path, T, cfg.d)
     _, _, y_r = _oracle_outputs(xq, routing, ow, ow.shared, T, cfg.d, cfg.k)
     assert_close_layer(bits_to_f32(y_g), y_r, f"decode T={T}")
     # the GPU-quantised weights of the touched experts equal the oracle's
@@ -139,3 +163,27 @@ def test_combine_rms_renorm():
     ref = omoe.rms_renorm(y_acc)
     assert_close_layer(bits_to_f32(y.cpu().numpy()), ref, "rms renorm")
     assert not bits_to_f32(y.cpu().numpy())[3].any()
+
+
+@pytest.mark.parametrize("cfg_name,n_sample", [("prefill", 8), ("wide", 3)])
+def test_ffn_prefill_configs_sampled(cfg_name, n_sample):
+    """Full-size prefill FFN on the tensor-core path; the oracle checks sampled tokens."""
+    cfg = synth.CONFIGS[cfg_name]
+    T = cfg.T_list[0]
+    routed = L.quantize_weights_gpu(0, cfg)
+    shared = L.quantize_weights_gpu(0, cfg, shared=True)
+    gpu = B.Experts(routed, shared)
+    ow = OracleWeights(0, cfg)
+    x = synth.make_x(0, cfg, T).numpy()
+    Wr, br = synth.make_router(0, cfg)
+    xf = bits_to_f32(x)
+    xq = onv.quantize(xf)
+    routing = _oracle_route(xf, Wr.numpy(), br.numpy(), cfg.k, cfg.E)
+    _, _, y_g = _run_ffn(xq, routing, gpu, cfg.k, B.MOE_FFN_ACCUMULATE, B.MOE_PATH_PREFILL, T, cfg.d)
+    rng = np.random.default_rng(1)
+    tokens = np.sort(rng.choice(T, n_sample, replace=False))
+    _, _, y_r = _oracle_outputs(xq, routing, ow, ow.shared, T, cfg.d, cfg.k, tokens=tokens)
+    assert_close_layer(bits_to_f32(y_g)[tokens], y_r, f"{cfg_name} sampled")
+    # every output row is finite and not all zero
+    yf = bits_to_f32(y_g)
+    assert np.isfinite(yf).all() and (np.abs(yf).sum(1) > 0).all()
