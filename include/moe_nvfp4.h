@@ -185,6 +185,28 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
 moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32_t* rank_out,
                            int32_t reset, void* stream);
 
+/*
+ * moe_route_noalloc - moe_route for callers that cannot give the library any scratch
+ * memory: for instance a serving process that reserves all device memory up front and
+ * allows no later allocation, a C host with no device allocator of its own, or code that is
+ * capturing a CUDA graph, where cudaMalloc may not be called. The Basalt pages have no
+ * counterpart of this call; it exists for such callers only.
+ *   Same arguments, outputs and results as moe_route, minus ws/ws_bytes. The scratch is one
+ *   256 KiB array compiled into the library and held by every GPU that loads it until the
+ *   process exits; calls whose scratch need (moe_workspace_size(MOE_OP_ROUTE, ...)) exceeds
+ *   256 KiB return MOE_ERR_UNSUPPORTED_SHAPE. With T*k <= 4096 that allows T*E <= 65536
+ *   (e.g. 64 tokens with 1024 experts, or 128 tokens with 512 experts).
+ *   It allocates nothing. The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before capturing any stream.
+ *   All calls share the one array, which keeps the last call's contents (nothing in it needs
+ *   to start at zero). Calls that overlap on the GPU - on different streams or from
+ *   different host threads - race on it and give undefined results.
+ */
+moe_status moe_route_noalloc(const uint16_t* x_bf16, int32_t T, int32_t d, const float* Wr,
+                             const float* br, int32_t E, int32_t k, int32_t* topk_idx,
+                             float* topk_w, int32_t* counts, int32_t* offsets,
+                             int32_t* sorted_assign, int32_t* assign_pos, void* stream);
+
 /* Bytes of workspace needed by one op (MOE_OP_*) for these sizes (MOE_OP_LAYER: max). */
 size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k, int32_t I);
 

@@ -28,6 +28,7 @@ EXPORTS = {
     "nvfp4_quantize_act": (_I32, [_P, _I64, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_route": (_I32, [_P, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_route_noalloc": (_I32, [_P, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "moe_pack_experts": (_I32, [_P, _P, _P, _P]),
     "moe_expert_ffn": (_I32, [_P, _P, _P, _I32, _P, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P,
                               _SZ, _P]),
@@ -165,6 +166,17 @@ def moe_route(x, Wr, br, k, topk_idx, topk_w, counts, offsets, sorted_assign, as
         _ptr(x), T, d, _ptr(Wr), _ptr(br), E, k, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
         _ptr(offsets), _ptr(sorted_assign), _ptr(assign_pos), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_route_noalloc(x, Wr, br, k, topk_idx, topk_w, counts, offsets, sorted_assign, assign_pos,
+                      stream=None):
+    """moe_route without a workspace: the library uses its own fixed 256 KiB scratch array
+    (for callers that cannot allocate device memory; see include/moe_nvfp4.h)."""
+    T, d = x.shape
+    E = Wr.shape[0]
+    _check("moe_route_noalloc", lib().moe_route_noalloc(
+        _ptr(x), T, d, _ptr(Wr), _ptr(br), E, k, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
+        _ptr(offsets), _ptr(sorted_assign), _ptr(assign_pos), _stream(stream)))
 
 
 def moe_permute(topk_idx, E, counts, offsets, sorted_assign, assign_pos, ws, stream=None):

@@ -100,6 +100,9 @@ ExpertGroup to_group(const moe_expert_weights_t& w) {
 }
 
 }  // namespace
+
+void set_last_error(const std::string& msg) { t_last_error = msg; }
+
 }  // namespace moe
 
 using namespace moe;

@@ -5,7 +5,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <string>
+
 namespace moe {
+
+// per-thread detail string returned by moe_last_error()
+void set_last_error(const std::string& msg);
 
 // Device-side view of one expert group (natural NVFP4 layout, see moe_nvfp4.h).
 struct ExpertGroup {
