@@ -100,11 +100,11 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- GPU arm
-def build_layers(T: int, device, n_layers: int):
+def build_layers(T: int, device, n_layers: int, workload: str = "decode"):
     from nvfp4_expert_ffn_b200 import binding as B
     from nvfp4_expert_ffn_b200 import layer as L
     from nvfp4_expert_ffn_b200 import synth
-    cfg = synth.CONFIGS["decode"]
+    cfg = synth.CONFIGS[workload]
     layers = []
     for li in range(n_layers):
         routed = L.quantize_weights_gpu(SEED, cfg, layer=li, device=device)
@@ -141,8 +141,10 @@ def run_gpu(args):
     torch.cuda.set_device(device)
     global N_LAYER_COPIES
     N_LAYER_COPIES = args.layers
-    T, K, W = args.T, args.steps, args.warmup
-    cfg, layers = build_layers(T, device, N_LAYER_COPIES)
+    from nvfp4_expert_ffn_b200 import synth
+    T = args.T if args.T else synth.CONFIGS[args.workload].T_list[-1]
+    K, W = args.steps, args.warmup
+    cfg, layers = build_layers(T, device, N_LAYER_COPIES, args.workload)
     stream = torch.cuda.Stream(device)
     sampler = ClockSampler(local)
     sampler.start()
@@ -243,36 +245,50 @@ def run_gpu(args):
     ms_step = ms_total / K
     tokens_per_s = world * T * K / (ms_total / 1e3)
     e2e_tps = world * T * e2e_steps / (ms_e2e / 1e3) if e2e_steps else None
-    hbm_peak, _, peak_kind = _peaks()
+    hbm_peak, bf16_peak, peak_kind = _peaks()
     U_avg = float(np.mean([b[0] for b in bytes_info]))
     ffn_bytes = float(np.mean([b[1] for b in bytes_info]))
     ffn_ms = ms_ffn / K
     achieved = ffn_bytes / (ffn_ms * 1e-3) / 1e9
+    ffn_flops = 2.0 * T * (cfg.k + 1) * 3 * cfg.d * cfg.I
+    if args.workload == "decode":
+        roof = {"kernel": "moe_expert_ffn (schedule + gather + tcgen05 FFN)", "bound": "hbm",
+                "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
+                "bytes_per_launch": int(ffn_bytes), "avg_launch_us": round(ffn_ms * 1e3, 3),
+                "traffic": None}
+    else:
+        fp4_peak = bf16_peak * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio 9 / 2.25)
+        tf = ffn_flops / (ffn_ms * 1e-3) / 1e12
+        roof = {"kernel": "moe_expert_ffn (schedule + gather + tcgen05 FFN)", "bound": "tensor",
+                "achieved": round(tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                "frac": round(tf / fp4_peak, 4),
+                "peak_kind": f"{peak_kind} bf16 x 4 (nominal fp4/bf16 ratio)",
+                "flops_per_launch": ffn_flops, "bytes_per_launch": int(ffn_bytes),
+                "avg_launch_us": round(ffn_ms * 1e3, 3), "traffic": None}
     launches_per_step = 1 + 3 + 2 + 1 + 1  # quant, route(gemv,topk,perm), ffn(2), combine, hist
     out = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp32", "data": "synthetic",
-        "config": {"workload": f"decode MoE layer: d=2048, 512 experts, top-10 + 1 shared, "
-                               f"I=512, NVFP4 weights, T={T} tokens per step",
+        "config": {"workload": f"{args.workload} MoE layer: d={cfg.d}, {cfg.E} experts, "
+                               f"top-{cfg.k} + {int(cfg.shared)} shared, I={cfg.I}, NVFP4 weights, "
+                               f"T={T} tokens per step",
                    "T": T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I,
                    "zipf_s": cfg.zipf_s, "parallelism": f"replicas x{world}",
                    "l2": f"{N_LAYER_COPIES} distinct layer copies "
-                         f"({N_LAYER_COPIES * 0.91:.1f} GB) rotated every step: inputs > L2",
+                         f"({N_LAYER_COPIES * cfg.E * 3 * cfg.d * cfg.I * 0.5625 / 1e9:.1f} GB) "
+                         f"rotated every step: inputs > L2",
                    "touched_experts_avg": U_avg},
-        "roofline": {"kernel": "moe_expert_ffn (gate/up + down)", "bound": "hbm",
-                     "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
-                     "bytes_per_launch": int(ffn_bytes), "avg_launch_us": round(ffn_ms * 1e3, 3),
-                     "traffic": None},
+        "roofline": roof,
         "e2e": {"value": None if e2e_tps is None else round(e2e_tps, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2,
                 "steps": e2e_steps},
         "gpu_launches": launches_per_step * K,
         "clocks": sampler.summary([win1, win2, win3]),
     }
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and not args.no_cpu_baseline and args.workload == "decode":
         out["cpu_baseline"] = cpu_baseline(T, args.cpu_steps)
     if dist is not None:
         del g_step, g_ffn
@@ -319,7 +335,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    T = args.T
+    T = args.T or 8
     K = max(1, min(args.steps, args.cpu_steps))
     W = max(0, min(args.warmup, 1))
     cb = cpu_baseline(T, K + W)
@@ -339,7 +355,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=40)
-    ap.add_argument("--T", type=int, default=8)
+    ap.add_argument("--T", type=int, default=0, help="tokens per step (default: the workload's)")
+    ap.add_argument("--workload", choices=["decode", "prefill", "wide"], default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
