@@ -15,13 +15,15 @@
 //      expert-major buffer (codes row-major, scales re-tiled into 512-byte scale atoms)
 //      and records (token, weight, output slot) per row; zeroes y in accumulate mode.
 //   3. tc_ffn_kernel (persistent, one CTA per SM, warp-specialised):
-//        warp 0   TMA producer (A rows, B weight tiles, scale atoms) into a 5-stage ring
-//        warp 1   TMEM allocation and the MMA issuer (single thread)
-//        warps 2-5 epilogue: TMEM -> registers
+//        warp 0    TMA producer (A rows, B weight tiles, scale atoms) into a 4-stage ring
+//        warp 1    TMEM allocation and the MMA issuer (single thread)
+//        warps 2-9 epilogue: TMEM -> registers; two warps per TMEM lane quarter, each
+//                  taking half of the tile's columns
 //      phase-1 tiles (m-tile, 64 gate + 64 up rows): SwiGLU and NVFP4 h quantisation in
 //      the epilogue, h written to the workspace; phase-2 tiles (m-tile, 128 output rows)
 //      wait until all phase-1 tiles of their m-tile are done (bounded wait), then the down
-//      GEMM, whose epilogue adds w * o into y (red.global.add.v4.f32) or stores o.
+//      GEMM, whose epilogue stages each token row of w * o in shared memory and adds it
+//      into y with a bulk reduction (cp.reduce.async.bulk .add.f32), or stores o.
 //      Accumulators are double-buffered in TMEM so an epilogue overlaps the next tile.
 #include <cudaTypedefs.h>
 
@@ -31,7 +33,7 @@
 
 namespace moe {
 
-constexpr int kTcStages = 5;
+constexpr int kTcStages = 4;
 constexpr int kTileM = 128;                // tokens per m-tile (MMA M)
 constexpr int kTileN = 128;                // weight rows per tile (MMA N)
 constexpr int kStageK = 256;               // elements of K per pipeline stage (4 MMAs)
@@ -40,7 +42,11 @@ constexpr int kABytes = kTileM * kStageK / 2;   // 16 KB
 constexpr int kBBytes = kTileN * kStageK / 2;   // 16 KB
 constexpr int kSfBytes = 4 * kAtom;             // 2 KB per operand per stage
 constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
-constexpr int kTcThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kTcThreads = 64 + 32 * kEpiWarps;
+constexpr int kEpiRowFloats = 36;              // staged row stride: 144 B keeps rows 16 B aligned and
+                                               // spreads 8 consecutive rows over all 32 banks
+constexpr int kEpiStageBytes = 32 * kEpiRowFloats * 4;  // one warp's 32 rows x 32 float32 columns
 constexpr int kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_mxf4nvf4(kTileM, kTileN);
 
@@ -246,7 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], kEpiWarps);
     }
     mbar_init(&final_bar, 1);
     fence_barrier_init();
@@ -373,15 +379,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     // one thread waits for the accumulator; a named barrier publishes data and decision
     __shared__ int s_epi_go[2];  // by tile parity: a slow warp never reads the next tile's value
     const int q = warp & 3;            // TMEM lane quarter of this warp
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns this warp takes
     const int row = 32 * q + lane;     // accumulator row = token row of the m-tile
     const float ts_x = *p.xq_ts;
-    uint32_t tc = 0;
+    // two 4 KB staging buffers per warp for the bulk reductions of phase 2
+    float* stage_f = reinterpret_cast<float*>(smem + (size_t)kTcStages * kStageBytes) +
+                     (size_t)(warp - 2) * 2 * (kEpiStageBytes / 4);
+    uint32_t tc = 0, nbulk = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tc) {
       const TileInfo ti = decode_tile(t, n_m, nt1, nt2);
       const int buf = tc & 1;
       if (warp == 2 && lane == 0)
         s_epi_go[buf] = mbar_wait(&acc_full[buf], (tc >> 1) & 1, &s_abort, p.status) ? 1 : 0;
-      named_bar_sync(2, 128);
+      named_bar_sync(2, 32 * kEpiWarps);
       if (!s_epi_go[buf]) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kTileN;
@@ -392,39 +402,52 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
       const bool valid = row < p.mt_valid[ti.m];
       const size_t prow = (size_t)ti.m * kTileM + row;
       if (ti.phase == 1) {
+        // columns 32*half .. +31 of gate (0..63) and of up (64..127): 32 h values
         const float sg = G.gu_ts[2 * eloc] * ts_x, su = G.gu_ts[2 * eloc + 1] * ts_x;
-        uint32_t sfbytes = 0;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(taddr + 32 * c, g);
-          tmem_ld32(taddr + 64 + 32 * c, u);
-          tmem_ld_wait();
-          float h[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gv = __uint_as_float(g[i]) * sg, uv = __uint_as_float(u[i]) * su;
-            h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
-          }
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            uint2 codes;
-            const uint32_t sb = quantize_block16(h + 16 * b, 1.0f, &codes);
-            sfbytes |= sb << (8 * (2 * c + b));
-            if (valid)
-              *reinterpret_cast<uint2*>(p.h_codes + prow * (I / 2) + 32 * ti.j + 16 * c + 8 * b) = codes;
-          }
-        }
-        if (valid)
-          *reinterpret_cast<uint32_t*>(p.sfa2 + ((size_t)ti.m * (I / 64) + ti.j) * kAtom + (row % 32) * 16 +
-                                       (row / 32) * 4) = sfbytes;
+        uint32_t g[32], u[32];
+        tmem_ld32(taddr + 32 * half, g);
+        tmem_ld32(taddr + 64 + 32 * half, u);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        float h[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float gv = __uint_as_float(g[i]) * sg, uv = __uint_as_float(u[i]) * su;
+          h[i] = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
+        }
+        uint32_t packed[8];
+        uint32_t sbytes = 0;
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(h[16 * b + i]));
+          const uint32_t sb = f32_to_e4m3_sat(__fdiv_rn(amax, kE2M1Max));  // tensor scale of h is 1
+          const float sval = e4m3_to_f32(sb);
+          const float rs = sval != 0.0f ? __frcp_rn(sval) : 0.0f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t lo = f32x2_to_e2m1x2(h[16 * b + 2 * i] * rs, h[16 * b + 2 * i + 1] * rs);
+            const uint32_t hi = f32x2_to_e2m1x2(h[16 * b + 8 + 2 * i] * rs, h[16 * b + 9 + 2 * i] * rs);
+            if (i == 0) packed[4 * b] = lo, packed[4 * b + 2] = hi;
+            else packed[4 * b] |= lo << (8 * i), packed[4 * b + 2] |= hi << (8 * i);
+          }
+          if (sval == 0.0f) packed[4 * b] = packed[4 * b + 2] = 0;
+          sbytes |= sb << (8 * b);
+        }
+        if (valid) {
+          // 32 codes = 16 bytes at h columns 64j + 32*half
+          *reinterpret_cast<uint4*>(p.h_codes + prow * (I / 2) + 32 * ti.j + 16 * half) =
+              make_uint4(packed[0], packed[2], packed[4], packed[6]);
+          *reinterpret_cast<uint16_t*>(p.sfa2 + ((size_t)ti.m * (I / 64) + ti.j) * kAtom + (row % 32) * 16 +
+                                       (row / 32) * 4 + 2 * half) = (uint16_t)sbytes;
+        }
         // publish h of this tile: generic writes -> visible to other CTAs' TMA reads
         fence_proxy_async_global();
         __threadfence();
-        named_bar_sync(2, 128);
+        named_bar_sync(2, 32 * kEpiWarps);
         if (warp == 2 && lane == 0) atomicAdd(p.done1 + ti.m, 1);
       } else {
         const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
@@ -435,35 +458,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           wgt = p.row_weight[prow];
           slot = p.row_slot[prow];
         }
-#pragma unroll 1
-        for (int c = 0; c < kTileN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(taddr + 32 * c, v);
-          tmem_ld_wait();
-          if (valid) {
-            const int n0 = kTileN * ti.j + 32 * c;
-            if (p.mode == 0) {
-              float* dst = p.out + (size_t)tok * d + n0;
-              const float f = wgt * ts_o;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                red_add_v4(dst + 4 * i, __uint_as_float(v[4 * i]) * f, __uint_as_float(v[4 * i + 1]) * f,
-                           __uint_as_float(v[4 * i + 2]) * f, __uint_as_float(v[4 * i + 3]) * f);
-            } else {
-              float* dst = sh ? p.shared_out + (size_t)tok * d + n0 : p.out + (size_t)slot * d + n0;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                reinterpret_cast<float4*>(dst)[i] =
-                    make_float4(__uint_as_float(v[4 * i]) * ts_o, __uint_as_float(v[4 * i + 1]) * ts_o,
-                                __uint_as_float(v[4 * i + 2]) * ts_o, __uint_as_float(v[4 * i + 3]) * ts_o);
-            }
-          }
-        }
+        const float f = p.mode == 0 ? wgt * ts_o : ts_o;
+        uint32_t v[2][32];
+        tmem_ld32(taddr + 64 * half, v[0]);
+        tmem_ld32(taddr + 64 * half + 32, v[1]);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
+#pragma unroll
+        for (int c = 0; c < 2; ++c, ++nbulk) {
+          float* sb = stage_f + (nbulk & 1) * (kEpiStageBytes / 4);
+          bulk_wait_read<1>();  // the buffer used two chunks ago has been read
+          __syncwarp();
+          float4* rowp = reinterpret_cast<float4*>(sb + kEpiRowFloats * lane);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            rowp[i] = make_float4(__uint_as_float(v[c][4 * i]) * f, __uint_as_float(v[c][4 * i + 1]) * f,
+                                  __uint_as_float(v[c][4 * i + 2]) * f, __uint_as_float(v[c][4 * i + 3]) * f);
+          fence_proxy_async_smem();
+          if (valid) {
+            const int n0 = kTileN * ti.j + 64 * half + 32 * c;
+            if (p.mode == 0)
+              bulk_reduce_add_f32(p.out + (size_t)tok * d + n0, rowp, 128);
+            else
+              bulk_s2g((sh ? p.shared_out + (size_t)tok * d : p.out + (size_t)slot * d) + n0, rowp, 128);
+          }
+          bulk_commit();
+        }
       }
     }
+    bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -538,7 +563,7 @@ size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I) {
 
 bool ffn_tc_supported(int d, int I) { return d % kStageK == 0 && I % kStageK == 0 && d <= 16384 && I <= 16384; }
 
-size_t ffn_tc_smem_bytes() { return (size_t)kTcStages * kStageBytes + 1024; }
+size_t ffn_tc_smem_bytes() { return (size_t)kTcStages * kStageBytes + (size_t)kEpiWarps * 2 * kEpiStageBytes + 1024; }
 
 cudaError_t init_ffn_tc_attributes() {
   return cudaFuncSetAttribute(tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ffn_tc_smem_bytes());

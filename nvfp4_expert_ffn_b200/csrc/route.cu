@@ -7,10 +7,12 @@
 // the lower expert id, weights = softmax restricted to the top-k and renormalised; the
 // permutation is a stable counting sort of assignments a = t*k + j by expert.
 //
-// Precision: a float32 sum over d = 2048 products accumulates ~1e-6 of rounding error,
-// the size of the top-k tie margin. Dot products therefore use float64 accumulation
-// (decode GEMV: exact float64 FMAs; prefill GEMM: float32 partial sums over 32 products
-// folded into float64 totals), and each logit is rounded to float32 once.
+// Precision: a float32 sum of d = 2048 products accumulated in one running total carries
+// ~1e-6 of rounding error, the size of the top-k tie margin. Sums are therefore blocked:
+// the decode GEMV adds 64 products per lane and then reduces the 32 lane sums in a tree;
+// the prefill GEMM sums 32 products per K tile and folds the tile sums into a compensated
+// (Kahan) total. Both leave ~1e-7 of error. Float64 arithmetic is avoided on purpose: the
+// B200 CUDA cores run it at a small fraction of the float32 rate.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,9 +34,9 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   for (int e = blockIdx.x * warps + (threadIdx.x >> 5); e < E; e += gridDim.x * warps) {
-    double acc[kGemvMaxT];
+    float acc[kGemvMaxT];
 #pragma unroll
-    for (int t = 0; t < kGemvMaxT; ++t) acc[t] = 0.0;
+    for (int t = 0; t < kGemvMaxT; ++t) acc[t] = 0.0f;
     const float4* w4 = reinterpret_cast<const float4*>(Wr + (size_t)e * d);
     for (int c = lane; c < d / 4; c += 32) {
       const float4 w = __ldg(w4 + c);
@@ -42,19 +44,19 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
       for (int t = 0; t < kGemvMaxT; ++t) {
         if (t < T) {
           const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * d + 4 * c);
-          acc[t] = fma((double)bf16_to_f32(xv.x & 0xFFFFu), (double)w.x, acc[t]);
-          acc[t] = fma((double)bf16_to_f32(xv.x >> 16), (double)w.y, acc[t]);
-          acc[t] = fma((double)bf16_to_f32(xv.y & 0xFFFFu), (double)w.z, acc[t]);
-          acc[t] = fma((double)bf16_to_f32(xv.y >> 16), (double)w.w, acc[t]);
+          acc[t] = fmaf(bf16_to_f32(xv.x & 0xFFFFu), w.x, acc[t]);
+          acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w.y, acc[t]);
+          acc[t] = fmaf(bf16_to_f32(xv.y & 0xFFFFu), w.z, acc[t]);
+          acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w.w, acc[t]);
         }
       }
     }
-    const double b = br ? (double)__ldg(br + e) : 0.0;
+    const float b = br ? __ldg(br + e) : 0.0f;
 #pragma unroll
     for (int t = 0; t < kGemvMaxT; ++t) {
       if (t < T) {
-        double s = warp_sum_f64(acc[t]);
-        if (lane == 0) logits[(size_t)t * E + e] = (float)(s + b);
+        const float s = warp_sum(acc[t]);
+        if (lane == 0) logits[(size_t)t * E + e] = s + b;
       }
     }
   }
@@ -72,12 +74,11 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __rest
   __shared__ float ws[kRgBK][kRgBN + 4];
   const int m0 = blockIdx.y * kRgBM, n0 = blockIdx.x * kRgBN;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  double tot[4][4];
-  float acc[4][4];
+  float tot[4][4], cmp[4][4], acc[4][4];  // compensated total, its error term, tile sum
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) tot[i][j] = 0.0, acc[i][j] = 0.0f;
+    for (int j = 0; j < 4; ++j) tot[i][j] = 0.0f, cmp[i][j] = 0.0f, acc[i][j] = 0.0f;
   for (int k0 = 0; k0 < d; k0 += kRgBK) {
     // x tile: 64 rows x 32 cols bf16 = 256 x 8 elements
     {
@@ -117,7 +118,13 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __rest
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) tot[i][j] += (double)acc[i][j], acc[i][j] = 0.0f;
+      for (int j = 0; j < 4; ++j) {
+        const float y = __fsub_rn(acc[i][j], cmp[i][j]);
+        const float t = __fadd_rn(tot[i][j], y);
+        cmp[i][j] = __fsub_rn(__fsub_rn(t, tot[i][j]), y);
+        tot[i][j] = t;
+        acc[i][j] = 0.0f;
+      }
     __syncthreads();
   }
 #pragma unroll
@@ -127,60 +134,76 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __rest
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
-      if (n < E) logits[(size_t)m * E + n] = (float)(tot[i][j] + (br ? (double)br[n] : 0.0));
+      if (n < E) logits[(size_t)m * E + n] = __fsub_rn(tot[i][j], cmp[i][j]) + (br ? br[n] : 0.0f);
     }
   }
 }
 
 // ---------------------------------------------------------------- top-k + weights
-// One warp per token. Lane L holds logits L, L+32, ...; k rounds of a warp arg-max with
-// ties to the lower index. Weights: exp(l_j - l_max) / sum over the chosen k.
-constexpr int kTopkMaxPerLane = 32;  // E <= 1024
-
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                   int32_t* __restrict__ topk_idx,
-                                                   float* __restrict__ topk_w) {
+// One warp per token. Lane L holds logits L, L+32, ... and keeps its own best remaining
+// entry; each of the k rounds takes the warp arg-max (ties to the lower index) and only the
+// winning lane rescans. Weights: exp(l_j - l_max) / sum over the chosen k (float32).
+template <int NPER>
+MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
+                        float* __restrict__ w_out) {
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  const float* row = logits + (size_t)t * E;
-  float v[kTopkMaxPerLane];
-  const int nper = (E + 31) >> 5;
+  float v[NPER];
 #pragma unroll
-  for (int j = 0; j < kTopkMaxPerLane; ++j) {
+  for (int j = 0; j < NPER; ++j) {
     const int e = lane + 32 * j;
-    v[j] = (j < nper && e < E) ? row[e] : -INFINITY;
+    v[j] = e < E ? row[e] : -INFINITY;
   }
   uint32_t taken = 0;
+  auto local_best = [&](float& bv, int& be) {
+    bv = -INFINITY;
+    be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NPER; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < be))) bv = v[j], be = e;
+    }
+  };
+  float lbv;
+  int lbe;
+  local_best(lbv, lbe);
   float top0 = 0.0f, mysel_l = 0.0f;
   int mysel_e = 0;
   for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < kTopkMaxPerLane; ++j) {
-      const int e = lane + 32 * j;
-      if (j < nper && e < E && !((taken >> j) & 1u)) {
-        if (v[j] > bv || (v[j] == bv && e < be)) bv = v[j], be = e;
-      }
-    }
+    float bv = lbv;
+    int be = lbe;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
     if (r == 0) top0 = bv;
     if (lane == r) mysel_l = bv, mysel_e = be;
+    if ((be & 31) == lane) {
+      taken |= 1u << (be >> 5);
+      local_best(lbv, lbe);
+    }
   }
-  // lane j < k holds the j-th selection
   const float ex = (lane < k) ? expf(mysel_l - top0) : 0.0f;
   const float sum = warp_sum(ex);
   if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = mysel_e;
-    topk_w[(size_t)t * k + lane] = ex / sum;
+    idx_out[lane] = mysel_e;
+    w_out[lane] = ex / sum;
   }
+}
+
+MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w) {
+  if (E <= 256) topk_token<8>(row, E, k, idx, w);
+  else if (E <= 512) topk_token<16>(row, E, k, idx, w);
+  else topk_token<32>(row, E, k, idx, w);
+}
+
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                   int32_t* __restrict__ topk_idx,
+                                                   float* __restrict__ topk_w) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_dispatch(logits + (size_t)t * E, E, k, topk_idx + (size_t)t * k, topk_w + (size_t)t * k);
 }
 
 // ---------------------------------------------------------------- permutation
@@ -311,6 +334,45 @@ __global__ void __launch_bounds__(kPermThreads) perm_small_kernel(const int32_t*
   chunk_scatter(idx, n, 0, sh, sorted_assign, assign_pos);
 }
 
+// Decode-sized calls (T <= 32 tokens, T*k <= 4096): top-k of every token (one warp each)
+// and the whole permutation in one CTA.
+__global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __restrict__ logits, int T,
+                                                               int E, int k, int32_t* __restrict__ topk_idx,
+                                                               float* __restrict__ topk_w,
+                                                               int32_t* __restrict__ counts,
+                                                               int32_t* __restrict__ offsets,
+                                                               int32_t* __restrict__ sorted_assign,
+                                                               int32_t* __restrict__ assign_pos) {
+  extern __shared__ int sh[];  // [E]
+  __shared__ int tmp[32];
+  __shared__ int carry;
+  const int warp = threadIdx.x >> 5;
+  if (warp < T)
+    topk_dispatch(logits + (size_t)warp * E, E, k, topk_idx + (size_t)warp * k, topk_w + (size_t)warp * k);
+  __syncthreads();  // this CTA's global writes of topk_idx are now visible to all its threads
+  const int n = T * k;
+  chunk_histogram(topk_idx, n, 0, E, sh);
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    const int h = e < E ? sh[e] : 0;
+    int total;
+    const int excl = block_exclusive_scan(h, tmp, &total) + carry;
+    if (e < E) {
+      counts[e] = h;
+      offsets[e] = excl;
+      sh[e] = excl;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) carry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offsets[E] = carry;
+  __syncthreads();
+  chunk_scatter(topk_idx, n, 0, sh, sorted_assign, assign_pos);
+}
+
 __global__ void zero_counts_kernel(int E, int32_t* counts, int32_t* offsets) {
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {
     if (e < E) counts[e] = 0;
@@ -371,6 +433,11 @@ cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
+  if (T <= 32 && T * k <= kPermChunk) {
+    topk_perm_small_kernel<<<1, 1024, (size_t)E * sizeof(int), st>>>(logits, T, E, k, topk_idx, topk_w, counts,
+                                                                      offsets, sorted_assign, assign_pos);
+    return cudaGetLastError();
+  }
   topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
@@ -378,28 +445,51 @@ cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const
 }
 
 // ---------------------------------------------------------------- cumulative histogram
-// One CTA: cum[e] += counts[e] (or = on reset); rank position of e is the number of experts
-// that are hotter, or equally hot with a lower id.
+// One CTA: cum[e] += counts[e] (or = on reset); then a bitonic sort in shared memory of
+// keys (cum descending, id ascending) packed into 64 bits: key = (2^51-1-cum) << 12 | e.
+constexpr int kHistMaxE = 4096;
+
 __global__ void __launch_bounds__(1024) hist_kernel(const int32_t* __restrict__ counts, int E,
                                                     int64_t* __restrict__ cum,
                                                     int32_t* __restrict__ rank_out, int reset) {
-  extern __shared__ long long sc[];  // [E]
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const long long v = (reset ? 0 : cum[e]) + counts[e];
-    sc[e] = v;
-    cum[e] = v;
+  extern __shared__ unsigned long long keys[];  // [n], n = next power of two >= E
+  int n = 1;
+  while (n < E) n <<= 1;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    if (e < E) {
+      const long long v = (reset ? 0 : cum[e]) + counts[e];
+      cum[e] = v;
+      keys[e] = ((((1ull << 51) - 1ull) - (unsigned long long)v) << 12) | (unsigned long long)e;
+    } else {
+      keys[e] = ~0ull;
+    }
   }
   __syncthreads();
   if (!rank_out) return;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const long long v = sc[e];
-    int r = 0;
-    for (int f = 0; f < E; ++f) {
-      const long long w = sc[f];
-      r += (w > v) || (w == v && f < e);
+  for (int size = 2; size <= n; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < n / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const unsigned long long a = keys[lo], b = keys[hi];
+        if ((a > b) == up) {
+          keys[lo] = b;
+          keys[hi] = a;
+        }
+      }
+      __syncthreads();
     }
-    rank_out[r] = e;
   }
+  for (int r = threadIdx.x; r < E; r += blockDim.x) rank_out[r] = (int32_t)(keys[r] & 0xFFFull);
+}
+
+cudaError_t launch_hist(const int32_t* counts, int E, int64_t* cum, int32_t* rank_out, int reset,
+                        cudaStream_t st) {
+  int n = 1;
+  while (n < E) n <<= 1;
+  hist_kernel<<<1, 1024, (size_t)n * sizeof(unsigned long long), st>>>(counts, E, cum, rank_out, reset);
+  return cudaGetLastError();
 }
 
 cudaError_t init_route_attributes() {
@@ -407,10 +497,5 @@ cudaError_t init_route_attributes() {
                               kGemvMaxT * 8192 * (int)sizeof(uint16_t));
 }
 
-cudaError_t launch_hist(const int32_t* counts, int E, int64_t* cum, int32_t* rank_out, int reset,
-                        cudaStream_t st) {
-  hist_kernel<<<1, 1024, (size_t)E * sizeof(long long), st>>>(counts, E, cum, rank_out, reset);
-  return cudaGetLastError();
-}
 
 }  // namespace moe
