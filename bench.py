@@ -126,17 +126,47 @@ def layer_bytes(cfg, lay, T):
     return U, ffn, total
 
 
+# ---------------------------------------------------------------------------- ranks
+def rank_env():
+    """(rank, world size, local rank) from the torchrun environment (1 process: 0, 1, 0)."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_init(backend: str):
+    """Join the process group when launched with more than one rank (else None). The
+    replicas exchange nothing on the data path: the group carries only the barriers and the
+    max-over-ranks of the timings."""
+    _, world, _ = rank_env()
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(dist, ms: float, device) -> float:
+    """The slowest rank's time: every rank takes part, every rank gets the maximum."""
+    if dist is None:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, T: int, steps: int, ms: float) -> float:
+    """Tokens/s of the whole job: each of `world` replicas ran `steps` steps of T tokens in
+    (at most) `ms` milliseconds."""
+    return world * T * steps / (ms / 1e3)
+
+
 def run_gpu(args):
     from nvfp4_expert_ffn_b200 import binding as B
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = None
+    rank, world, local = rank_env()
     if world > 1:
-        import datetime
-        import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dist = dist_init("nccl")
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     global N_LAYER_COPIES
@@ -157,9 +187,12 @@ def run_gpu(args):
     torch.cuda.synchronize()
     bytes_info = [layer_bytes(cfg, lay, T) for lay in layers]
     g_step = torch.cuda.CUDAGraph()
+    n0 = B.moe_launch_count()
     with torch.cuda.graph(g_step, stream=stream):
         for lay in layers:
             lay.forward(lay.x_static)
+    # this library's kernels in one step, counted by the library as the graph was captured
+    launches_per_step = (B.moe_launch_count() - n0) / N_LAYER_COPIES
     g_ffn = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_ffn, stream=stream):
         for lay in layers:
@@ -185,12 +218,7 @@ def run_gpu(args):
             e1.record(stream)
         torch.cuda.synchronize()
         t1h = time.time()
-        ms = e0.elapsed_time(e1)
-        if dist is not None:
-            t = torch.tensor([ms], device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms, (t0h, t1h)
+        return max_over_ranks(dist, e0.elapsed_time(e1), device), (t0h, t1h)
 
     with torch.cuda.stream(stream):
         for _ in range(wreps):
@@ -210,41 +238,37 @@ def run_gpu(args):
     ms_ffn, win2 = timed(g_ffn, reps)
     torch.cuda.nvtx.range_pop()
 
-    # end to end through the public API: pinned host x -> device, forward, y -> pinned host
+    # end to end through the public API (a graphed layer step): pinned host x -> device,
+    # the layer forward, y -> pinned host, every step
+    e2e_steps = 0 if args.no_e2e else min(K, 2000)
+    runners = [lay.graphed(T) for lay in layers] if e2e_steps else []
     xs_host = [lay.x_static.cpu().pin_memory() for lay in layers]
     y_host = torch.empty(T, cfg.d, dtype=torch.int16).pin_memory()
-    x_dev = [torch.empty_like(lay.x_static) for lay in layers]
-    e2e_steps = 0 if args.no_e2e else min(K, 2000)
-    with torch.cuda.stream(stream):
-        for i in range(min(W, 8)):
-            li = i % N_LAYER_COPIES
-            x_dev[li].copy_(xs_host[li], non_blocking=True)
-            y_host.copy_(layers[li].forward(x_dev[li]), non_blocking=True)
+    est = runners[0].stream if runners else stream
+    for i in range(min(W, 8) if runners else 0):
+        runners[i % N_LAYER_COPIES].step(xs_host[i % N_LAYER_COPIES], y_host)
+        est.wait_stream(runners[i % N_LAYER_COPIES].stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     t0h = time.time()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for i in range(e2e_steps):
-            li = i % N_LAYER_COPIES
-            x_dev[li].copy_(xs_host[li], non_blocking=True)
-            y_host.copy_(layers[li].forward(x_dev[li]), non_blocking=True)
-        e1.record(stream)
+    e0.record(est)
+    for i in range(e2e_steps):
+        r = runners[i % N_LAYER_COPIES]
+        r.stream.wait_stream(est)
+        r.step(xs_host[i % N_LAYER_COPIES], y_host)
+        est.wait_stream(r.stream)
+    e1.record(est)
     torch.cuda.synchronize()
     win3 = (t0h, time.time())
-    ms_e2e = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms_e2e], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(dist, e0.elapsed_time(e1), device)
     sampler.stop()
 
     ms_step = ms_total / K
-    tokens_per_s = world * T * K / (ms_total / 1e3)
-    e2e_tps = world * T * e2e_steps / (ms_e2e / 1e3) if e2e_steps else None
+    tokens_per_s = whole_job_rate(world, T, K, ms_total)
+    e2e_tps = whole_job_rate(world, T, e2e_steps, ms_e2e) if e2e_steps else None
     hbm_peak, bf16_peak, peak_kind = _peaks()
     U_avg = float(np.mean([b[0] for b in bytes_info]))
     ffn_bytes = float(np.mean([b[1] for b in bytes_info]))
@@ -266,26 +290,19 @@ def run_gpu(args):
                 "peak_kind": f"{peak_kind} bf16 x 4 (nominal fp4/bf16 ratio)",
                 "flops_per_launch": ffn_flops, "bytes_per_launch": int(ffn_bytes),
                 "avg_launch_us": round(ffn_ms * 1e3, 3), "traffic": None}
-    launches_per_step = 1 + 3 + 2 + 1 + 1  # quant, route(gemv,topk,perm), ffn(2), combine, hist
     out = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(ms_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp32", "data": "synthetic",
-        "config": {"workload": f"{args.workload} MoE layer: d={cfg.d}, {cfg.E} experts, "
-                               f"top-{cfg.k} + {int(cfg.shared)} shared, I={cfg.I}, NVFP4 weights, "
-                               f"T={T} tokens per step",
-                   "T": T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I,
-                   "zipf_s": cfg.zipf_s, "parallelism": f"replicas x{world}",
-                   "l2": f"{N_LAYER_COPIES} distinct layer copies "
-                         f"({N_LAYER_COPIES * cfg.E * 3 * cfg.d * cfg.I * 0.5625 / 1e9:.1f} GB) "
-                         f"rotated every step: inputs > L2",
-                   "touched_experts_avg": U_avg},
+        "config": dict(workload_config(args.workload, T, world, N_LAYER_COPIES),
+                       touched_experts_avg=U_avg),
         "roofline": roof,
         "e2e": {"value": None if e2e_tps is None else round(e2e_tps, 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2,
                 "steps": e2e_steps},
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": int(round(launches_per_step * K)),
+        "gpu_launches_per_step": launches_per_step,
         "clocks": sampler.summary([win1, win2, win3]),
     }
     if rank == 0 and not args.no_cpu_baseline and args.workload == "decode":
@@ -298,56 +315,97 @@ def run_gpu(args):
 
 
 # ---------------------------------------------------------------------------- CPU oracle
+class OracleDecode:
+    """The float64 CPU oracle running decode layer forwards of T tokens (the touched
+    experts' weights are quantised when prepared, like a resident model, and not timed)."""
+
+    def __init__(self, T: int, n_inputs: int):
+        from oracle import moe as omoe
+        from nvfp4_expert_ffn_b200 import synth
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from helpers import OracleWeights
+        self.omoe = omoe
+        self.cfg = cfg = synth.CONFIGS["decode"]
+        self.T = T
+        self.ow = OracleWeights(SEED, cfg)
+        Wr, br = synth.make_router(SEED, cfg)
+        self.Wr, self.br = Wr.numpy(), br.numpy()
+        self.xs = [synth.make_x(SEED, cfg, T, step=100 + s).numpy() for s in range(n_inputs)]
+        for x in self.xs:
+            xf = (x.astype(np.uint16).astype(np.uint32) << 16).view(np.float32)
+            idx = omoe.topk_fast(omoe.router_logits(xf, self.Wr, self.br), cfg.k)
+            for e in np.unique(idx):
+                self.ow[int(e)]
+        self.ow.shared
+
+    def step(self, i: int):
+        return self.omoe.layer_forward(self.xs[i % len(self.xs)], self.Wr, self.br, self.cfg.k,
+                                       self.ow, self.ow.shared)
+
+    @staticmethod
+    def cores() -> int:
+        try:
+            from threadpoolctl import threadpool_info
+            return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            return os.cpu_count() or 1
+
+    def timed(self, steps: int, warmup: int = 0) -> float:
+        """Seconds for `steps` forwards after `warmup` untimed ones."""
+        for i in range(warmup):
+            self.step(i)
+        t0 = time.perf_counter()
+        for i in range(steps):
+            self.step(warmup + i)
+        return time.perf_counter() - t0
+
+
 def cpu_baseline(T: int, steps: int):
-    """Time the float64 CPU oracle on `steps` decode layer forwards of T tokens (weights of
-    the touched experts quantised before timing, like a resident model)."""
-    from oracle import moe as omoe
-    from nvfp4_expert_ffn_b200 import synth
-    sys.path.insert(0, os.path.join(ROOT, "tests"))
-    from helpers import OracleWeights
-    cfg = synth.CONFIGS["decode"]
-    ow = OracleWeights(SEED, cfg)
-    Wr, br = synth.make_router(SEED, cfg)
-    Wr, br = Wr.numpy(), br.numpy()
-    xs = [synth.make_x(SEED, cfg, T, step=100 + s).numpy() for s in range(steps)]
-    from oracle import nvfp4 as onv
-    for x in xs:  # materialise the touched experts (model load, not timed)
-        xf = (x.astype(np.uint16).astype(np.uint32) << 16).view(np.float32)
-        idx = omoe.topk_fast(omoe.router_logits(xf, Wr, br), cfg.k)
-        for e in np.unique(idx):
-            ow[int(e)]
-        ow.shared
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count()
-    t0 = time.perf_counter()
-    for x in xs:
-        omoe.layer_forward(x, Wr, br, cfg.k, ow, ow.shared)
-    dt = time.perf_counter() - t0
-    return {"value": round(T * steps / dt, 3), "unit": "tokens/s", "cores": cores,
+    """The oracle timed on `steps` decode layer forwards of T tokens on the host cores."""
+    o = OracleDecode(T, steps)
+    dt = o.timed(steps)
+    return {"value": round(T * steps / dt, 3), "unit": "tokens/s", "cores": o.cores(),
             "kind": "oracle",
             "sample": f"{steps} decode layer forwards of T={T} tokens (full layer, float64 numpy)"}
 
 
+def workload_config(workload: str, T: int, world: int, n_copies: int) -> dict:
+    from nvfp4_expert_ffn_b200 import synth
+    cfg = synth.CONFIGS[workload]
+    return {"workload": f"{workload} MoE layer: d={cfg.d}, {cfg.E} experts, "
+                        f"top-{cfg.k} + {int(cfg.shared)} shared, I={cfg.I}, NVFP4 weights, "
+                        f"T={T} tokens per step",
+            "T": T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "I": cfg.I,
+            "zipf_s": cfg.zipf_s, "parallelism": f"replicas x{world}",
+            "l2": f"{n_copies} distinct layer copies "
+                  f"({n_copies * cfg.E * 3 * cfg.d * cfg.I * 0.5625 / 1e9:.1f} GB) "
+                  f"rotated every step: inputs > L2"}
+
+
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    """The oracle as the reference arm: rank 0 alone runs W untimed and K timed decode layer
+    forwards (K and W capped so the run stays within minutes); other ranks exit at once."""
+    rank, world, _ = rank_env()
     if rank != 0:
-        return
+        return None
     T = args.T or 8
     K = max(1, min(args.steps, args.cpu_steps))
     W = max(0, min(args.warmup, 1))
-    cb = cpu_baseline(T, K + W)
-    out = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "tokens/s",
-           "n_gpus": 1, "steps": K, "warmup": W, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": f"decode MoE layer: d=2048, 512 experts, top-10 + 1 shared, "
-                                  f"I=512, NVFP4 weights, T={T} tokens per step", "T": T},
-           "cpu_baseline": cb,
-           "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+    o = OracleDecode(T, K + W)
+    dt = o.timed(K, W)
+    value = round(T * K / dt, 3)
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+           "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": round(dt * 1e3 / K, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": workload_config("decode", T, world, args.layers),
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": o.cores(),
+                            "kind": "oracle",
+                            "sample": f"{K} decode layer forwards of T={T} tokens after {W} "
+                                      f"warm-up (full layer, float64 numpy, rank 0 only)"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out))
+    return out
 
 
 def main():

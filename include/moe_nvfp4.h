@@ -221,6 +221,12 @@ const char* moe_last_error(void);
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int32_t moe_version(void);
 
+/* Number of kernels this library has enqueued in this process, counted on the host when
+ * each launch is issued (all devices and streams). A launch recorded into a CUDA graph
+ * counts once at capture; replays of the graph do not add to it. Instrumentation for
+ * launch accounting; the Basalt pages have no counterpart. */
+uint64_t moe_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

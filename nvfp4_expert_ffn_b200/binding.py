@@ -39,6 +39,7 @@ EXPORTS = {
     "moe_status_string": (ctypes.c_char_p, [_I32]),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_version": (_I32, []),
+    "moe_launch_count": (ctypes.c_uint64, []),
 }
 
 
@@ -219,6 +220,11 @@ def moe_expert_hist(counts, cum, rank_out=None, reset=False, stream=None):
     _check("moe_expert_hist", lib().moe_expert_hist(
         _ptr(counts), counts.numel(), _ptr(cum), _ptr(rank_out), 1 if reset else 0,
         _stream(stream)))
+
+
+def moe_launch_count() -> int:
+    """Kernels this library has enqueued in this process (graph replays not counted)."""
+    return int(lib().moe_launch_count())
 
 
 def moe_get_device_status(clear=True, stream=None) -> int:

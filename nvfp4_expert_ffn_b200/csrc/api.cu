@@ -103,6 +103,8 @@ ExpertGroup to_group(const moe_expert_weights_t& w) {
 
 void set_last_error(const std::string& msg) { t_last_error = msg; }
 
+std::atomic<uint64_t> g_launch_count{0};
+
 }  // namespace moe
 
 using namespace moe;
@@ -110,6 +112,8 @@ using namespace moe;
 extern "C" {
 
 int32_t moe_version(void) { return 100; }
+
+uint64_t moe_launch_count(void) { return g_launch_count.load(std::memory_order_relaxed); }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {

@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(256) combine_kernel(int T, int d, int k, const
                                                       const float* __restrict__ w,
                                                       const int32_t* __restrict__ pos, int rms,
                                                       uint16_t* __restrict__ y) {
+  MOE_PDL_PROLOGUE();
   const int t = blockIdx.x;
   float scale = 1.0f;
   if (rms) {
@@ -67,10 +68,9 @@ cudaError_t launch_combine(int T, int d, int k, int mode, const float* eo, const
                            cudaStream_t st) {
   if (T == 0) return cudaSuccess;
   if (mode == 0)
-    combine_kernel<0><<<T, 256, 0, st>>>(T, d, k, eo, so, w, pos, rms, y);
+    return launch_pdl(combine_kernel<0>, dim3(T), dim3(256), 0, st, T, d, k, eo, so, w, pos, rms, y);
   else
-    combine_kernel<1><<<T, 256, 0, st>>>(T, d, k, eo, so, w, pos, rms, y);
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<1>, dim3(T), dim3(256), 0, st, T, d, k, eo, so, w, pos, rms, y);
 }
 
 }  // namespace moe

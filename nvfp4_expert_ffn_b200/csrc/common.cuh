@@ -13,6 +13,16 @@ constexpr float kE2M1Max = 6.0f;
 constexpr float kE4M3Max = 448.0f;
 constexpr int kMaxPartials = 1024;  // per-CTA partial amax values kept in the workspace
 
+// Programmatic dependent launch: let the next kernel on the stream start launching, and
+// wait until the previous kernel's writes are visible (no-ops without the launch attribute).
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+MOE_DEV void pdl_grid_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+#define MOE_PDL_PROLOGUE() \
+  do {                     \
+    pdl_trigger();         \
+    pdl_grid_wait();       \
+  } while (0)
+
 MOE_DEV float bf16_to_f32(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
 // E4M3 ("fn") byte -> float; exact. (Byte 0x7F is NaN in the format; never produced here.)

@@ -501,6 +501,7 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, int32_t* status, cu
   const int units = max_act * (a.I / kBlock);
   const int grid = units < num_sms ? (units > 0 ? units : 1) : num_sms;
   const size_t smem = ffn_decode_smem_fused(a.d, a.I, a.E, c.stage_bytes, nst);
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
   ffn_decode_fused_kernel<<<grid, kFusedThreads, smem, st>>>(a, c);
   return cudaGetLastError();
 }

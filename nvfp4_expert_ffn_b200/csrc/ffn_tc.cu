@@ -8,22 +8,24 @@
 // E4M3 block scales staged into tensor memory: the tensor core consumes E2M1 codes and
 // scales directly, nothing is decoded on the CUDA cores.
 //
-// Three launches per call:
-//   1. tc_schedule_kernel (1 CTA): 128-row m-tiles over each expert's tokens (the shared
-//      expert is slot E); zeroes the per-m-tile completion counters.
-//   2. tc_gather_kernel: copies the activation rows of every m-tile into a padded,
-//      expert-major buffer (codes row-major, scales re-tiled into 512-byte scale atoms)
-//      and records (token, weight, output slot) per row; zeroes y in accumulate mode.
-//   3. tc_ffn_kernel (persistent, one CTA per SM, warp-specialised):
-//        warp 0    TMA producer (A rows, B weight tiles, scale atoms) into a 4-stage ring
+// Two launches per call:
+//   1. tc_schedule_kernel: CTA 0 lays out 128-row m-tiles over each expert's tokens (the
+//      shared expert is slot E) and zeroes the per-m-tile completion counters; the other
+//      CTAs zero y in accumulate mode.
+//   2. tc_ffn_kernel (persistent, one CTA per SM, warp-specialised):
+//        warp 0    producer: gathers each m-tile's activation rows straight from the
+//                  quantised activations with TMA tile::gather4 (and their scale bytes
+//                  with cp.async into 128x4 scale atoms), TMA-loads weight tiles and their
+//                  pre-tiled scale atoms, into a 4-stage shared-memory ring
 //        warp 1    TMEM allocation and the MMA issuer (single thread)
 //        warps 2-9 epilogue: TMEM -> registers; two warps per TMEM lane quarter, each
 //                  taking half of the tile's columns
 //      phase-1 tiles (m-tile, 64 gate + 64 up rows): SwiGLU and NVFP4 h quantisation in
 //      the epilogue, h written to the workspace; phase-2 tiles (m-tile, 128 output rows)
-//      wait until all phase-1 tiles of their m-tile are done (bounded wait), then the down
-//      GEMM, whose epilogue stages each token row of w * o in shared memory and adds it
-//      into y with a bulk reduction (cp.reduce.async.bulk .add.f32), or stores o.
+//      wait until all phase-1 tiles of their m-tile are done (bounded wait; their weights
+//      are already streaming), then the down GEMM, whose epilogue stages each token row of
+//      w * o in shared memory and adds it into y with a bulk reduction
+//      (cp.reduce.async.bulk .add.f32), or stores o.
 //      Accumulators are double-buffered in TMEM so an epilogue overlaps the next tile.
 #include <cudaTypedefs.h>
 
@@ -49,6 +51,7 @@ constexpr int kEpiRowFloats = 36;              // staged row stride: 144 B keeps
 constexpr int kEpiStageBytes = 32 * kEpiRowFloats * 4;  // one warp's 32 rows x 32 float32 columns
 constexpr int kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_mxf4nvf4(kTileM, kTileN);
+constexpr int kSmallT = 64;  // up to this many tokens the producer copies activation scales itself
 
 MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
@@ -68,8 +71,7 @@ struct TcParams {
   int32_t* row_token;
   float* row_weight;
   int32_t* row_slot;
-  uint8_t* a1_codes;  // [rows_cap][d/2]
-  uint8_t* sfa1;      // [m][d/64][512]
+  uint8_t* sfa1;      // [m][d/64][512] x scale atoms gathered per m-tile (large T), or NULL
   uint8_t* h_codes;   // [rows_cap][I/2]
   uint8_t* sfa2;      // [m][I/64][512]
   int max_m;
@@ -89,7 +91,7 @@ struct TcParams {
 };
 
 // ---------------------------------------------------------------- 1. schedule
-__global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
+MOE_DEV void schedule_body(const TcParams& p) {
   __shared__ int tmp[32];
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
@@ -119,49 +121,50 @@ __global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
   if (threadIdx.x == 0) *p.n_mtiles = min(carry, p.max_m);
 }
 
-// ---------------------------------------------------------------- 2. gather
-// One warp per padded row; row r of m-tile m is local token index mt_first[m] + r of its
-// expert.
-__global__ void __launch_bounds__(256) tc_gather_kernel(TcParams p) {
+__global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
+  MOE_PDL_PROLOGUE();
+  if (blockIdx.x == 0) {
+    schedule_body(p);
+    return;
+  }
+  // accumulate mode: y is summed into by the FFN kernel, so it starts at zero
+  const size_t n4 = (size_t)p.T * p.d / 4;
+  float4* o4 = reinterpret_cast<float4*>(p.out);
+  for (size_t i = (blockIdx.x - 1) * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)(gridDim.x - 1) * blockDim.x)
+    o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// ---------------------------------------------------------------- 1b. scale gather (large T)
+// With many rows per m-tile, the producer bulk-copies the activation scale atoms instead of
+// issuing 4-byte copies per row: one warp per row writes the row's d/16 scale bytes into
+// the atoms of its m-tile, and the row's (token, weight, output slot).
+__global__ void __launch_bounds__(256) tc_sf_gather_kernel(TcParams p) {
+  MOE_PDL_PROLOGUE();
   const int n_m = *p.n_mtiles;
   const int lane = threadIdx.x & 31;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int d = p.d;
-  if (p.mode == 0) {
-    const size_t n4 = (size_t)p.T * d / 4;
-    float4* o4 = reinterpret_cast<float4*>(p.out);
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x)
-      o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  for (int w = gw; w < n_m * kTileM; w += nw) {
+  for (int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < n_m * kTileM; w += nw) {
     const int m = w / kTileM, r = w % kTileM;
     if (r >= p.mt_valid[m]) continue;
     const int e = p.mt_expert[m];
     const int i = p.mt_first[m] + r;
-    int t, slot;
-    float wgt;
+    int t = i, slot = -1;
+    float wgt = 1.0f;
     if (e < p.E) {
       const int q = p.offsets[e] + i;
       const int a = p.sorted_assign[q];
       t = a / p.k;
       wgt = p.topk_w[a];
       slot = q;
-    } else {
-      t = i;
-      wgt = 1.0f;
-      slot = -1;
     }
-    const size_t prow = (size_t)m * kTileM + r;
-    const uint4* src = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
-    uint4* dst = reinterpret_cast<uint4*>(p.a1_codes + prow * (d / 2));
-    for (int c = lane; c < d / 32; c += 32) dst[c] = __ldg(src + c);
     const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
-    for (int kc = lane; kc < d / 64; kc += 32) {
-      uint8_t* atom = p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom;
-      *reinterpret_cast<uint32_t*>(atom + (r % 32) * 16 + (r / 32) * 4) = __ldg(ssrc + kc);
-    }
+    for (int kc = lane; kc < d / 64; kc += 32)
+      *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (r % 32) * 16 + (r / 32) * 4) =
+          __ldg(ssrc + kc);
     if (lane == 0) {
+      const size_t prow = (size_t)m * kTileM + r;
       p.row_token[prow] = t;
       p.row_weight[prow] = wgt;
       p.row_slot[prow] = slot;
@@ -206,7 +209,7 @@ __global__ void pack_sf_kernel(const uint8_t* __restrict__ gu_scales, const uint
 
 // ---------------------------------------------------------------- 3. persistent FFN kernel
 struct TcMaps {
-  CUtensorMap a1;    // gathered x codes  [rows_cap][d/2]
+  CUtensorMap xg;    // x codes [T][d/2], one-row boxes for tile::gather4
   CUtensorMap a2;    // h codes           [rows_cap][I/2]
   CUtensorMap b1;    // routed gate/up    {d/2, I, 2, E}
   CUtensorMap b1s;   // shared gate/up    {d/2, I, 2, 1}
@@ -234,6 +237,7 @@ MOE_DEV TileInfo decode_tile(int t, int n_m, int nt1, int nt2) {
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
+  MOE_PDL_PROLOGUE();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t full[kTcStages], empty[kTcStages], acc_full[2], acc_empty[2], final_bar;
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 1 + 32);  // producer lane 0 (expect_tx) + 32 cp.async arrivals
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     mbar_init(&final_bar, 1);
     fence_barrier_init();
     s_abort = 0;
-    prefetch_tensormap(&maps.a1);
+    prefetch_tensormap(&maps.xg);
     prefetch_tensormap(&maps.a2);
     prefetch_tensormap(&maps.b1);
     prefetch_tensormap(&maps.b2);
@@ -272,64 +276,150 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int t = blockIdx.x; t < total && !s_abort; t += gridDim.x) {
-        const TileInfo ti = decode_tile(t, n_m, nt1, nt2);
-        const int e = p.mt_expert[ti.m];
-        const bool sh = (e == p.E);
-        const int eloc = sh ? 0 : e;
-        const int nq = (p.mt_valid[ti.m] + 31) / 32;
-        if (ti.phase == 2) {
-          // h of this m-tile is produced by phase-1 tiles of any CTA
+    // All 32 lanes: lane 0 waits on barriers, arms them and issues weight / h copies; each
+    // lane gathers 4 activation rows (rows 4*lane .. 4*lane+3 of the m-tile) and copies
+    // their scale bytes, then signals the stage's barrier when its cp.async copies land.
+    uint32_t it = 0;
+    bool alive = true;
+    // Token ids of the 4 rows this lane gathers, for a phase-1 tile; the loads for the next
+    // tile are started before the current tile's copies are issued, so their latency hides.
+    auto load_rowtok = [&](int tt, int (&rt)[4]) {
+      const TileInfo tn = decode_tile(tt, n_m, nt1, nt2);
+      if (tt >= total || tn.phase != 1) return;
+      const int en = p.mt_expert[tn.m];
+      const int vn = p.mt_valid[tn.m];
+      const int first = p.mt_first[tn.m];
+      const int off = en == p.E ? 0 : p.offsets[en];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        rt[i] = r < vn ? (en == p.E ? first + r : p.sorted_assign[off + first + r]) : -1;
+      }
+    };
+    int next_tok[4] = {-1, -1, -1, -1};
+    load_rowtok(blockIdx.x, next_tok);
+    for (int t = blockIdx.x; t < total && alive; t += gridDim.x) {
+      const TileInfo ti = decode_tile(t, n_m, nt1, nt2);
+      const int e = p.mt_expert[ti.m];
+      const bool sh = (e == p.E);
+      const int eloc = sh ? 0 : e;
+      const int valid = p.mt_valid[ti.m];
+      const ExpertGroup& G = sh ? p.shared : p.routed;
+      const int nks = ti.phase == 1 ? nks1 : nks2;
+      int rowtok[4] = {0, 0, 0, 0};
+      int ngather = 0;
+      if (ti.phase == 1) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)  // assignment ids -> token ids (the shared expert's are tokens)
+          rowtok[i] = next_tok[i] < 0 ? -1 : (sh ? next_tok[i] : next_tok[i] / p.k);
+        const int tok0 = __shfl_sync(0xffffffffu, rowtok[0], 0);  // row 0 always exists
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (rowtok[i] < 0) rowtok[i] = tok0;  // padding rows of a gather group repeat a real row
+        ngather = (valid + 3) / 4;
+      }
+      load_rowtok(t + gridDim.x, next_tok);
+      const int nq = (valid + 31) / 32;
+      const uint32_t stage_tx =
+          ti.phase == 1 ? (uint32_t)(ngather * 512 + kBBytes + (p.sfa1 ? 2 : 1) * kSfBytes)
+                        : (uint32_t)(nq * 4096 + kBBytes + 2 * kSfBytes);
+      auto wait_empty = [&](uint32_t itx) -> bool {
+        int ok = 1;
+        if (lane == 0)
+          ok = mbar_wait(&empty[itx % kTcStages], ((itx / kTcStages) & 1) ^ 1, &s_abort, p.status) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
+      };
+      auto arm_and_issue_b = [&](int ks, uint32_t s) {
+        if (lane != 0) return;
+        uint8_t* st = smem + (size_t)s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], stage_tx);
+        if (ti.phase == 1) {
+          tma_load_4d(st + kABytes, sh ? &maps.b1s : &maps.b1, &full[s], ks * 128, 64 * ti.j, 0, eloc);
+          bulk_g2s(st + kABytes + kBBytes + kSfBytes,
+                   G.gu_sf_tiled + (((size_t)eloc * nt1 + ti.j) * (d / 64) + 4 * ks) * kAtom, kSfBytes, &full[s]);
+        } else {
+          tma_load_3d(st + kABytes, sh ? &maps.b2s : &maps.b2, &full[s], ks * 128, kTileN * ti.j, eloc);
+          bulk_g2s(st + kABytes + kBBytes + kSfBytes,
+                   G.dn_sf_tiled + (((size_t)eloc * nt2 + ti.j) * (I / 64) + 4 * ks) * kAtom, kSfBytes, &full[s]);
+        }
+      };
+      auto issue_a = [&](int ks, uint32_t s) {
+        uint8_t* st = smem + (size_t)s * kStageBytes;
+        uint8_t* sSFA = st + kABytes + kBBytes;
+        if (ti.phase == 1) {
+          if (p.sfa1 && lane == 0)
+            bulk_g2s(sSFA, p.sfa1 + ((size_t)ti.m * (d / 64) + 4 * ks) * kAtom, kSfBytes, &full[s]);
+          if (4 * lane < valid) {
+            tma_gather4(st + 4 * lane * 128, &maps.xg, &full[s], ks * 128, rowtok[0], rowtok[1], rowtok[2],
+                        rowtok[3]);
+#pragma unroll
+            for (int i = 0; i < 4 && !p.sfa1; ++i) {
+              const int r = 4 * lane + i;
+              if (r < valid) {
+                const uint8_t* src = p.xq_scales + (size_t)rowtok[i] * (d / kBlock) + 16 * ks;
+#pragma unroll
+                for (int kc = 0; kc < 4; ++kc)
+                  cp_async4(sSFA + kc * kAtom + (r % 32) * 16 + (r / 32) * 4, src + 4 * kc);
+              }
+            }
+          }
+        } else if (lane == 0) {
+          for (int q = 0; q < nq; ++q)
+            tma_load_2d(st + q * 4096, &maps.a2, &full[s], ks * 128, ti.m * kTileM + 32 * q);
+          bulk_g2s(sSFA, p.sfa2 + ((size_t)ti.m * (I / 64) + 4 * ks) * kAtom, kSfBytes, &full[s]);
+        }
+        cp_async_arrive(&full[s]);
+      };
+      int ks0 = 0;
+      if (ti.phase == 2) {
+        // the down weights do not depend on phase 1: start streaming them, then wait
+        // until every phase-1 tile of this m-tile has written its h rows
+        const int npre = nks < kTcStages ? nks : kTcStages;
+        for (int ks = 0; ks < npre && alive; ++ks) {
+          if (!wait_empty(it + ks)) alive = false;
+          else arm_and_issue_b(ks, (it + ks) % kTcStages);
+        }
+        if (!alive) break;
+        int ok = 1;
+        if (lane == 0) {
           const uint64_t t0 = globaltimer_ns();
           while (ld_acquire_gpu(p.done1 + ti.m) < nt1) {
-            if (s_abort) break;
+            if (s_abort) {
+              ok = 0;
+              break;
+            }
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
               s_abort = 1;
               atomicExch(p.status, kStatusTimeout);
+              ok = 0;
               break;
             }
           }
-          if (s_abort) break;
           fence_proxy_async_global();
         }
-        const int nks = ti.phase == 1 ? nks1 : nks2;
-        for (int ks = 0; ks < nks; ++ks, ++it) {
-          const int s = it % kTcStages;
-          if (!mbar_wait(&empty[s], ((it / kTcStages) & 1) ^ 1, &s_abort, p.status)) break;
-          uint8_t* st = smem + (size_t)s * kStageBytes;
-          uint8_t* sA = st;
-          uint8_t* sB = st + kABytes;
-          uint8_t* sSFA = sB + kBBytes;
-          uint8_t* sSFB = sSFA + kSfBytes;
-          mbar_arrive_expect_tx(&full[s], (uint32_t)(nq * 4096 + kBBytes + 2 * kSfBytes));
-          const CUtensorMap* ma = ti.phase == 1 ? &maps.a1 : &maps.a2;
-          for (int q = 0; q < nq; ++q)
-            tma_load_2d(sA + q * 4096, ma, &full[s], ks * 128, ti.m * kTileM + 32 * q);
-          const uint8_t* sfa;
-          const uint8_t* sfb;
-          if (ti.phase == 1) {
-            tma_load_4d(sB, sh ? &maps.b1s : &maps.b1, &full[s], ks * 128, 64 * ti.j, 0, eloc);
-            sfa = p.sfa1 + ((size_t)ti.m * (d / 64) + 4 * ks) * kAtom;
-            const ExpertGroup& G = sh ? p.shared : p.routed;
-            sfb = G.gu_sf_tiled + (((size_t)eloc * nt1 + ti.j) * (d / 64) + 4 * ks) * kAtom;
-          } else {
-            tma_load_3d(sB, sh ? &maps.b2s : &maps.b2, &full[s], ks * 128, kTileN * ti.j, eloc);
-            sfa = p.sfa2 + ((size_t)ti.m * (I / 64) + 4 * ks) * kAtom;
-            const ExpertGroup& G = sh ? p.shared : p.routed;
-            sfb = G.dn_sf_tiled + (((size_t)eloc * nt2 + ti.j) * (I / 64) + 4 * ks) * kAtom;
-          }
-          bulk_g2s(sSFA, sfa, kSfBytes, &full[s]);
-          bulk_g2s(sSFB, sfb, kSfBytes, &full[s]);
-        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        for (int ks = 0; ks < npre; ++ks) issue_a(ks, (it + ks) % kTcStages);
+        it += npre;
+        ks0 = npre;
       }
-      // no copies left in flight: the last issued stage of each slot has landed
+      for (int ks = ks0; ks < nks; ++ks, ++it) {
+        const uint32_t s = it % kTcStages;
+        if (!wait_empty(it)) {
+          alive = false;
+          break;
+        }
+        arm_and_issue_b(ks, s);
+        issue_a(ks, s);
+      }
+    }
+    // no copies left in flight: the last issued stage of each slot has landed
+    if (lane == 0) {
       for (uint32_t j = (it > (uint32_t)kTcStages ? it - kTcStages : 0); j < it; ++j) {
         volatile int no_abort = 0;
         mbar_wait(&full[j % kTcStages], (j / kTcStages) & 1, &no_abort, p.status);
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -349,6 +439,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             break;
           }
           tc_fence_after();
+          fence_proxy_async_smem();  // scale bytes arrived through cp.async (generic proxy)
           const uint8_t* st = smem + (size_t)s * kStageBytes;
           const uint32_t aA = smem_u32(st), aB = smem_u32(st + kABytes);
           const uint32_t aSFA = smem_u32(st + kABytes + kBBytes), aSFB = aSFA + kSfBytes;
@@ -444,6 +535,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           *reinterpret_cast<uint16_t*>(p.sfa2 + ((size_t)ti.m * (I / 64) + ti.j) * kAtom + (row % 32) * 16 +
                                        (row / 32) * 4 + 2 * half) = (uint16_t)sbytes;
         }
+        if (!p.sfa1 && ti.j == 0 && half == 0 && valid) {
+          // token, routing weight and output slot of this row, for the phase-2 epilogue
+          const int i = p.mt_first[ti.m] + row;
+          int tokr = i, slotr = -1;
+          float wr = 1.0f;
+          if (!sh) {
+            const int q = p.offsets[e] + i;
+            const int asg = p.sorted_assign[q];
+            tokr = asg / p.k;
+            wr = p.topk_w[asg];
+            slotr = q;
+          }
+          p.row_token[prow] = tokr;
+          p.row_weight[prow] = wr;
+          p.row_slot[prow] = slotr;
+        }
         // publish h of this tile: generic writes -> visible to other CTAs' TMA reads
         fence_proxy_async_global();
         __threadfence();
@@ -453,10 +560,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
         int tok = 0, slot = 0;
         float wgt = 0.0f;
-        if (valid) {
-          tok = p.row_token[prow];
-          wgt = p.row_weight[prow];
-          slot = p.row_slot[prow];
+        if (valid) {  // written by another CTA's phase-1 epilogue: read through L2
+          tok = __ldcg(p.row_token + prow);
+          wgt = __ldcg(p.row_weight + prow);
+          slot = __ldcg(p.row_slot + prow);
         }
         const float f = p.mode == 0 ? wgt * ts_o : ts_o;
         uint32_t v[2][32];
@@ -528,7 +635,7 @@ size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
 struct TcLayout {
   int max_m;
   size_t rows_cap;
-  size_t off_hdr, off_expert, off_valid, off_first, off_done, off_tok, off_w, off_slot, off_a1, off_sfa1, off_h, off_sfa2,
+  size_t off_hdr, off_expert, off_valid, off_first, off_done, off_tok, off_w, off_slot, off_sfa1, off_h, off_sfa2,
       total;
 };
 
@@ -546,7 +653,6 @@ TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   L.off_tok = o; o += a256(L.rows_cap * 4);
   L.off_w = o; o += a256(L.rows_cap * 4);
   L.off_slot = o; o += a256(L.rows_cap * 4);
-  L.off_a1 = o; o += a256(L.rows_cap * (d / 2));
   L.off_sfa1 = o; o += a256(L.rows_cap * (d / kBlock));
   L.off_h = o; o += a256(L.rows_cap * (I / 2));
   L.off_sfa2 = o; o += a256(L.rows_cap * (I / kBlock));
@@ -571,6 +677,7 @@ cudaError_t init_ffn_tc_attributes() {
 
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t, int num_sms,
                            cudaStream_t st) {
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
   pack_sf_kernel<<<num_sms * 4, 256, 0, st>>>(g.gu_scales, g.dn_scales, E, d, I, gu_t, dn_t);
   return cudaGetLastError();
 }
@@ -589,8 +696,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.row_token = reinterpret_cast<int32_t*>(w + L.off_tok);
   p.row_weight = reinterpret_cast<float*>(w + L.off_w);
   p.row_slot = reinterpret_cast<int32_t*>(w + L.off_slot);
-  p.a1_codes = w + L.off_a1;
-  p.sfa1 = w + L.off_sfa1;
+  p.sfa1 = a.T > kSmallT ? w + L.off_sfa1 : nullptr;
   p.h_codes = w + L.off_h;
   p.sfa2 = w + L.off_sfa2;
   p.max_m = L.max_m;
@@ -611,10 +717,10 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   TcMaps maps;
   const int d = a.d, I = a.I;
   {
-    cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)L.rows_cap};
+    cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)a.T};
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
-    cuuint32_t box[2] = {128, 32};
-    if ((e = encode_u8(&maps.a1, p.a1_codes, 2, dims, strides, box)) != cudaSuccess) return e;
+    cuuint32_t box[2] = {128, 1};
+    if ((e = encode_u8(&maps.xg, a.xq_codes, 2, dims, strides, box)) != cudaSuccess) return e;
   }
   {
     cuuint64_t dims[2] = {(cuuint64_t)(I / 2), (cuuint64_t)L.rows_cap};
@@ -641,12 +747,16 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     cuuint32_t box2[3] = {128, 128, 1};
     if ((e = encode_u8(m2, g.dn_codes, 3, dims2, str2, box2)) != cudaSuccess) return e;
   }
-  tc_schedule_kernel<<<1, 1024, 0, st>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_gather_kernel<<<num_sms * 4, 256, 0, st>>>(p);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  tc_ffn_kernel<<<num_sms, kTcThreads, ffn_tc_smem_bytes(), st>>>(maps, p);
-  return cudaGetLastError();
+  int zc = 0;
+  if (a.mode == 0) {
+    const size_t n4 = (size_t)a.T * a.d / 4;
+    zc = (int)((n4 + 4095) / 4096);
+    if (zc > num_sms) zc = num_sms;
+  }
+  if ((e = launch_pdl(tc_schedule_kernel, dim3(1 + zc), dim3(1024), 0, st, p)) != cudaSuccess) return e;
+  if (p.sfa1 && (e = launch_pdl(tc_sf_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess)
+    return e;
+  return launch_pdl(tc_ffn_kernel, dim3(num_sms), dim3(kTcThreads), ffn_tc_smem_bytes(), st, maps, p);
 }
 
 }  // namespace moe

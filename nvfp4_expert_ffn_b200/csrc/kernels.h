@@ -5,9 +5,33 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 
 namespace moe {
+
+// Kernels enqueued by this library in this process (host side; see moe_launch_count).
+extern std::atomic<uint64_t> g_launch_count;
+
+// Launch with programmatic dependent launch allowed: the kernel may start while the
+// previous kernel on the stream drains; every kernel of this library calls
+// griddepcontrol.wait before it reads anything a predecessor wrote.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 
 // per-thread detail string returned by moe_last_error()
 void set_last_error(const std::string& msg);

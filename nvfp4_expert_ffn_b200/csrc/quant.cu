@@ -16,6 +16,7 @@ MOE_DEV uint32_t bf16x2_absmax(uint32_t m, uint32_t w) { return __vmaxu2(m, w & 
 
 __global__ void __launch_bounds__(256) amax_partial_kernel(const uint4* __restrict__ x, int64_t nvec,
                                                            float* __restrict__ partials) {
+  MOE_PDL_PROLOGUE();
   uint32_t m = 0;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -54,6 +55,7 @@ __global__ void __launch_bounds__(256) quant_blocks_kernel(const uint4* __restri
                                                            int npart, uint2* __restrict__ codes,
                                                            uint8_t* __restrict__ scales,
                                                            float* __restrict__ ts_out) {
+  MOE_PDL_PROLOGUE();
   __shared__ float s_ts;
   if (threadIdx.x < 32) {
     float ts = resolve_ts(ts_in, partials, npart);
@@ -84,6 +86,7 @@ __global__ void __launch_bounds__(1024) quant_small_kernel(const uint4* __restri
                                                            uint2* __restrict__ codes,
                                                            uint8_t* __restrict__ scales,
                                                            float* __restrict__ ts_out) {
+  MOE_PDL_PROLOGUE();
   __shared__ float red[32];
   __shared__ float s_ts;
   if (!ts_in) {
@@ -124,6 +127,7 @@ __global__ void __launch_bounds__(1024) quant_small_kernel(const uint4* __restri
 }
 
 __global__ void write_ts_kernel(const float* ts_in, float* ts_out) {
+  MOE_PDL_PROLOGUE();
   if (threadIdx.x == 0 && ts_out) *ts_out = ts_in ? *ts_in : 1.0f;
 }
 
@@ -132,14 +136,12 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int cols, const flo
                             int num_sms, cudaStream_t st) {
   const int64_t nblk = rows * (int64_t)(cols / kBlock);
   if (nblk == 0) {
-    write_ts_kernel<<<1, 32, 0, st>>>(ts_in, ts_out);
-    return cudaGetLastError();
+    return launch_pdl(write_ts_kernel, dim3(1), dim3(32), 0, st, ts_in, ts_out);
   }
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   if (nblk <= 4096) {
-    quant_small_kernel<<<1, 1024, 0, st>>>(xv, nblk, ts_in, reinterpret_cast<uint2*>(codes),
-                                           scales, ts_out);
-    return cudaGetLastError();
+    return launch_pdl(quant_small_kernel, dim3(1), dim3(1024), 0, st, xv, nblk, ts_in,
+                      reinterpret_cast<uint2*>(codes), scales, ts_out);
   }
   float* partials = reinterpret_cast<float*>(ws);
   int npart = 0;
@@ -148,13 +150,13 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int cols, const flo
     int64_t want = (nvec + 255) / 256;
     npart = (int)(want < (int64_t)num_sms * 4 ? want : (int64_t)num_sms * 4);
     if (npart > kMaxPartials) npart = kMaxPartials;
-    amax_partial_kernel<<<npart, 256, 0, st>>>(xv, nvec, partials);
+    cudaError_t e = launch_pdl(amax_partial_kernel, dim3(npart), dim3(256), 0, st, xv, nvec, partials);
+    if (e != cudaSuccess) return e;
   }
   int64_t want = (nblk + 255) / 256;
   int grid = (int)(want < (int64_t)num_sms * 8 ? want : (int64_t)num_sms * 8);
-  quant_blocks_kernel<<<grid, 256, 0, st>>>(xv, nblk, ts_in, partials, npart,
-                                            reinterpret_cast<uint2*>(codes), scales, ts_out);
-  return cudaGetLastError();
+  return launch_pdl(quant_blocks_kernel, dim3(grid), dim3(256), 0, st, xv, nblk, ts_in,
+                    (const float*)partials, npart, reinterpret_cast<uint2*>(codes), scales, ts_out);
 }
 
 }  // namespace moe

@@ -19,35 +19,55 @@
 namespace moe {
 
 // ---------------------------------------------------------------- router GEMV (T <= 8)
-// One warp per expert row of Wr; x (T x d bf16) staged in shared memory.
+// x (T x d bf16) is staged in shared memory; each warp owns expert rows of Wr and keeps
+// 16 float4 loads per lane in flight (a full 8 KB row at d = 2048) before using them.
 constexpr int kGemvMaxT = 8;
+constexpr int kGemvUnroll = 16;
 
 __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __restrict__ x, int T, int d,
                                                           const float* __restrict__ Wr,
                                                           const float* __restrict__ br, int E,
                                                           float* __restrict__ logits) {
+  MOE_PDL_PROLOGUE();
   extern __shared__ __align__(16) uint16_t xs[];  // [T][d]
-  const int nvec = T * d / 8;
-  for (int i = threadIdx.x; i < nvec; i += blockDim.x)
-    reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
-  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
-  for (int e = blockIdx.x * warps + (threadIdx.x >> 5); e < E; e += gridDim.x * warps) {
+  const int nvec = d / 4;
+  int e = blockIdx.x * warps + (threadIdx.x >> 5);
+  // first row's weights in flight while x is staged
+  float4 w[kGemvUnroll];
+  auto load_w = [&](int row, int c0) {
+    const float4* w4 = reinterpret_cast<const float4*>(Wr + (size_t)row * d);
+#pragma unroll
+    for (int u = 0; u < kGemvUnroll; ++u) {
+      const int c = c0 + 32 * u;
+      w[u] = c < nvec ? __ldg(w4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  if (e < E) load_w(e, lane);
+  for (int i = threadIdx.x; i < T * d / 8; i += blockDim.x)
+    reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
+  __syncthreads();
+  for (; e < E; e += gridDim.x * warps) {
     float acc[kGemvMaxT];
 #pragma unroll
     for (int t = 0; t < kGemvMaxT; ++t) acc[t] = 0.0f;
-    const float4* w4 = reinterpret_cast<const float4*>(Wr + (size_t)e * d);
-    for (int c = lane; c < d / 4; c += 32) {
-      const float4 w = __ldg(w4 + c);
+    for (int c0 = lane; c0 < nvec; c0 += 32 * kGemvUnroll) {
+      if (c0 != lane) load_w(e, c0);
 #pragma unroll
-      for (int t = 0; t < kGemvMaxT; ++t) {
-        if (t < T) {
-          const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * d + 4 * c);
-          acc[t] = fmaf(bf16_to_f32(xv.x & 0xFFFFu), w.x, acc[t]);
-          acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w.y, acc[t]);
-          acc[t] = fmaf(bf16_to_f32(xv.y & 0xFFFFu), w.z, acc[t]);
-          acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w.w, acc[t]);
+      for (int u = 0; u < kGemvUnroll; ++u) {
+        const int c = c0 + 32 * u;
+        if (c < nvec) {
+#pragma unroll
+          for (int t = 0; t < kGemvMaxT; ++t) {
+            if (t < T) {
+              const uint2 xv = *reinterpret_cast<const uint2*>(xs + t * d + 4 * c);
+              acc[t] = fmaf(bf16_to_f32(xv.x & 0xFFFFu), w[u].x, acc[t]);
+              acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w[u].y, acc[t]);
+              acc[t] = fmaf(bf16_to_f32(xv.y & 0xFFFFu), w[u].z, acc[t]);
+              acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w[u].w, acc[t]);
+            }
+          }
         }
       }
     }
@@ -59,6 +79,8 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
         if (lane == 0) logits[(size_t)t * E + e] = s + b;
       }
     }
+    const int en = e + gridDim.x * warps;
+    if (en < E) load_w(en, lane);
   }
 }
 
@@ -70,6 +92,7 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __rest
                                                           const float* __restrict__ Wr,
                                                           const float* __restrict__ br, int E,
                                                           float* __restrict__ logits) {
+  MOE_PDL_PROLOGUE();
   __shared__ float xs[kRgBK][kRgBM + 4];
   __shared__ float ws[kRgBK][kRgBN + 4];
   const int m0 = blockIdx.y * kRgBM, n0 = blockIdx.x * kRgBN;
@@ -143,51 +166,55 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __rest
 // One warp per token. Lane L holds logits L, L+32, ... and keeps its own best remaining
 // entry; each of the k rounds takes the warp arg-max (ties to the lower index) and only the
 // winning lane rescans. Weights: exp(l_j - l_max) / sum over the chosen k (float32).
+// float -> unsigned key with the same order
+MOE_DEV uint32_t ordered_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 template <int NPER>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
                         float* __restrict__ w_out) {
   const int lane = threadIdx.x & 31;
-  float v[NPER];
+  uint32_t key[NPER];
 #pragma unroll
   for (int j = 0; j < NPER; ++j) {
     const int e = lane + 32 * j;
-    v[j] = e < E ? row[e] : -INFINITY;
+    key[j] = e < E ? ordered_key(row[e]) : 0u;  // 0 is below every finite float's key
   }
   uint32_t taken = 0;
-  auto local_best = [&](float& bv, int& be) {
-    bv = -INFINITY;
+  // this lane's best remaining entry: largest key, lowest index among equal keys
+  auto local_best = [&](uint32_t& bk, int& be) {
+    bk = 0u;
     be = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < NPER; ++j) {
       const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u) && (v[j] > bv || (v[j] == bv && e < be))) bv = v[j], be = e;
+      if (e < E && !((taken >> j) & 1u) && (key[j] > bk || (key[j] == bk && e < be))) bk = key[j], be = e;
     }
   };
-  float lbv;
+  uint32_t lbk;
   int lbe;
-  local_best(lbv, lbe);
-  float top0 = 0.0f, mysel_l = 0.0f;
-  int mysel_e = 0;
+  local_best(lbk, lbe);
+  uint32_t top_key = 0, my_key = 0;
+  int my_e = 0;
   for (int r = 0; r < k; ++r) {
-    float bv = lbv;
-    int be = lbe;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) bv = ov, be = oe;
-    }
-    if (r == 0) top0 = bv;
-    if (lane == r) mysel_l = bv, mysel_e = be;
-    if ((be & 31) == lane) {
-      taken |= 1u << (be >> 5);
-      local_best(lbv, lbe);
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, lbk);
+    const int me = (int)__reduce_min_sync(0xffffffffu, lbk == mk ? (uint32_t)lbe : 0x7fffffffu);
+    if (r == 0) top_key = mk;
+    if (lane == r) my_key = mk, my_e = me;
+    if ((me & 31) == lane) {
+      taken |= 1u << (me >> 5);
+      local_best(lbk, lbe);
     }
   }
-  const float ex = (lane < k) ? expf(mysel_l - top0) : 0.0f;
+  auto key_to_float = [](uint32_t kk) {
+    return __uint_as_float((kk & 0x80000000u) ? (kk & 0x7fffffffu) : ~kk);
+  };
+  const float ex = (lane < k) ? expf(key_to_float(my_key) - key_to_float(top_key)) : 0.0f;
   const float sum = warp_sum(ex);
   if (lane < k) {
-    idx_out[lane] = mysel_e;
+    idx_out[lane] = my_e;
     w_out[lane] = ex / sum;
   }
 }
@@ -201,6 +228,7 @@ MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* 
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int32_t* __restrict__ topk_idx,
                                                    float* __restrict__ topk_w) {
+  MOE_PDL_PROLOGUE();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   topk_dispatch(logits + (size_t)t * E, E, k, topk_idx + (size_t)t * k, topk_w + (size_t)t * k);
@@ -255,6 +283,8 @@ MOE_DEV void chunk_scatter(const int32_t* idx, int n, int c, int* run, int32_t* 
 
 __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* __restrict__ idx, int n,
                                                                  int E, int32_t* __restrict__ chunk_hist) {
+  MOE_PDL_PROLOGUE();
+  MOE_PDL_PROLOGUE();
   extern __shared__ int sh[];
   chunk_histogram(idx, n, blockIdx.x, E, sh);
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = sh[e];
@@ -264,6 +294,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* 
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_hist, int nchunk,
                                                          int E, int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets) {
+  MOE_PDL_PROLOGUE();
   __shared__ int tmp[32];
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
@@ -297,6 +328,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_scatter_kernel(const int32_
                                                                     const int32_t* __restrict__ chunk_base,
                                                                     int32_t* __restrict__ sorted_assign,
                                                                     int32_t* __restrict__ assign_pos) {
+  MOE_PDL_PROLOGUE();
   extern __shared__ int run[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = chunk_base[(size_t)blockIdx.x * E + e];
   __syncthreads();
@@ -309,6 +341,7 @@ __global__ void __launch_bounds__(kPermThreads) perm_small_kernel(const int32_t*
                                                                   int32_t* __restrict__ offsets,
                                                                   int32_t* __restrict__ sorted_assign,
                                                                   int32_t* __restrict__ assign_pos) {
+  MOE_PDL_PROLOGUE();
   extern __shared__ int sh[];  // [E]
   __shared__ int tmp[32];
   __shared__ int carry;
@@ -343,6 +376,7 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
                                                                int32_t* __restrict__ offsets,
                                                                int32_t* __restrict__ sorted_assign,
                                                                int32_t* __restrict__ assign_pos) {
+  MOE_PDL_PROLOGUE();
   extern __shared__ int sh[];  // [E]
   __shared__ int tmp[32];
   __shared__ int carry;
@@ -350,30 +384,65 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
   if (warp < T)
     topk_dispatch(logits + (size_t)warp * E, E, k, topk_idx + (size_t)warp * k, topk_w + (size_t)warp * k);
   __syncthreads();  // this CTA's global writes of topk_idx are now visible to all its threads
+  if (warp != 0) return;
+  // the permutation of <= 32*k assignments by one warp, without block-wide barriers:
+  // histogram (match_any leaders), warp scan of the counts, then a stable scatter in
+  // assignment order, 32 at a time
+  const int lane = threadIdx.x & 31;
   const int n = T * k;
-  chunk_histogram(topk_idx, n, 0, E, sh);
-  if (threadIdx.x == 0) carry = 0;
-  __syncthreads();
-  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
-    const int e = e0 + threadIdx.x;
-    const int h = e < E ? sh[e] : 0;
-    int total;
-    const int excl = block_exclusive_scan(h, tmp, &total) + carry;
-    if (e < E) {
-      counts[e] = h;
-      offsets[e] = excl;
-      sh[e] = excl;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) carry += total;
-    __syncthreads();
+  for (int e = lane; e < E; e += 32) sh[e] = 0;
+  __syncwarp();
+  for (int base = 0; base < n; base += 32) {
+    const int a = base + lane;
+    const int e = a < n ? topk_idx[a] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (a < n && (peers & ((1u << lane) - 1u)) == 0) sh[e] += __popc(peers);
+    __syncwarp();
   }
-  if (threadIdx.x == 0) offsets[E] = carry;
-  __syncthreads();
-  chunk_scatter(topk_idx, n, 0, sh, sorted_assign, assign_pos);
+  // exclusive scan of sh[0..E): lane L owns the contiguous range [L*per, (L+1)*per)
+  const int per = (E + 31) / 32;
+  int local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < E) local += sh[e];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - local;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < E) {
+      const int c = sh[e];
+      counts[e] = c;
+      offsets[e] = run;
+      sh[e] = run;
+      run += c;
+    }
+  }
+  if (lane == 31) offsets[E] = incl;
+  __syncwarp();
+  for (int base = 0; base < n; base += 32) {
+    const int a = base + lane;
+    const int e = a < n ? topk_idx[a] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (a < n) {
+      const int pos = sh[e] + rank;
+      sorted_assign[pos] = a;
+      assign_pos[a] = pos;
+    }
+    __syncwarp();
+    if (a < n && (peers >> lane) == 1u) sh[e] += __popc(peers);  // highest lane of its group
+    __syncwarp();
+  }
 }
 
 __global__ void zero_counts_kernel(int E, int32_t* counts, int32_t* offsets) {
+  MOE_PDL_PROLOGUE();
   for (int e = threadIdx.x; e <= E; e += blockDim.x) {
     if (e < E) counts[e] = 0;
     offsets[e] = 0;
@@ -385,22 +454,21 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* cou
                            void* ws, cudaStream_t st) {
   const int n = T * k;
   if (n == 0) {
-    zero_counts_kernel<<<1, 1024, 0, st>>>(E, counts, offsets);
-    return cudaGetLastError();
+    return launch_pdl(zero_counts_kernel, dim3(1), dim3(1024), 0, st, E, counts, offsets);
   }
   const size_t smem = (size_t)E * sizeof(int);
   if (n <= kPermChunk) {
-    perm_small_kernel<<<1, kPermThreads, smem, st>>>(idx, n, E, counts, offsets, sorted_assign,
-                                                     assign_pos);
-    return cudaGetLastError();
+    return launch_pdl(perm_small_kernel, dim3(1), dim3(kPermThreads), smem, st, idx, n, E, counts, offsets,
+                      sorted_assign, assign_pos);
   }
   const int nchunk = (n + kPermChunk - 1) / kPermChunk;
   int32_t* chunk_hist = reinterpret_cast<int32_t*>(ws);
-  perm_hist_kernel<<<nchunk, kPermThreads, smem, st>>>(idx, n, E, chunk_hist);
-  perm_scan_kernel<<<1, 1024, 0, st>>>(chunk_hist, nchunk, E, counts, offsets);
-  perm_scatter_kernel<<<nchunk, kPermThreads, smem, st>>>(idx, n, E, chunk_hist, sorted_assign,
-                                                          assign_pos);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(perm_hist_kernel, dim3(nchunk), dim3(kPermThreads), smem, st, idx, n, E, chunk_hist);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, st, chunk_hist, nchunk, E, counts, offsets);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(perm_scatter_kernel, dim3(nchunk), dim3(kPermThreads), smem, st, idx, n, E,
+                    (const int32_t*)chunk_hist, sorted_assign, assign_pos);
 }
 
 size_t permute_ws_bytes(int64_t T, int k, int E) {
@@ -424,22 +492,23 @@ cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const
   const size_t logits_bytes = ((size_t)T * E * sizeof(float) + 255) & ~(size_t)255;
   void* perm_ws = reinterpret_cast<char*>(ws) + logits_bytes;
   if (T <= kGemvMaxT) {
-    const size_t smem = (size_t)T * d * sizeof(uint16_t);
-    const int grid = (E + 7) / 8;
-    router_gemv_kernel<<<grid, 256, smem, st>>>(x, T, d, Wr, br, E, logits);
+    const int grid = (E + 7) / 8;  // 8 warps (experts) per CTA
+    cudaError_t e0 = launch_pdl(router_gemv_kernel, dim3(grid), dim3(256), (size_t)T * d * sizeof(uint16_t), st,
+                                x, T, d, Wr, br, E, logits);
+    if (e0 != cudaSuccess) return e0;
   } else {
     dim3 grid((E + kRgBN - 1) / kRgBN, (T + kRgBM - 1) / kRgBM);
-    router_gemm_kernel<<<grid, 256, 0, st>>>(x, T, d, Wr, br, E, logits);
+    cudaError_t e0 = launch_pdl(router_gemm_kernel, grid, dim3(256), 0, st, x, T, d, Wr, br, E, logits);
+    if (e0 != cudaSuccess) return e0;
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (T <= 32 && T * k <= kPermChunk) {
-    topk_perm_small_kernel<<<1, 1024, (size_t)E * sizeof(int), st>>>(logits, T, E, k, topk_idx, topk_w, counts,
-                                                                      offsets, sorted_assign, assign_pos);
-    return cudaGetLastError();
+    return launch_pdl(topk_perm_small_kernel, dim3(1), dim3(1024), (size_t)E * sizeof(int), st,
+                      (const float*)logits, T, E, k, topk_idx, topk_w, counts, offsets, sorted_assign, assign_pos);
   }
-  topk_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
-  err = cudaGetLastError();
+  err = launch_pdl(topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, (const float*)logits, T, E, k, topk_idx,
+                   topk_w);
   if (err != cudaSuccess) return err;
   return launch_permute(topk_idx, T, k, E, counts, offsets, sorted_assign, assign_pos, perm_ws, st);
 }
@@ -488,8 +557,8 @@ cudaError_t launch_hist(const int32_t* counts, int E, int64_t* cum, int32_t* ran
                         cudaStream_t st) {
   int n = 1;
   while (n < E) n <<= 1;
-  hist_kernel<<<1, 1024, (size_t)n * sizeof(unsigned long long), st>>>(counts, E, cum, rank_out, reset);
-  return cudaGetLastError();
+  return launch_pdl(hist_kernel, dim3(1), dim3(1024), (size_t)n * sizeof(unsigned long long), st, counts, E,
+                    cum, rank_out, reset);
 }
 
 cudaError_t init_route_attributes() {

@@ -70,23 +70,69 @@ class MoeLayer:
         self.rank = torch.empty(E, dtype=torch.int32, device=dev)
         ws = B.moe_workspace_size(B.MOE_OP_LAYER, T_max, d, E, k, I)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+        # the quantiser runs concurrently with the router, so it gets its own workspace
+        self.ws_q = torch.empty(B.moe_workspace_size(B.MOE_OP_QUANT, T_max, d, E, k, I),
+                                dtype=torch.uint8, device=dev)
         self.path = B.MOE_PATH_AUTO
+        self._side = torch.cuda.Stream(device=dev)
+        self._ev = [torch.cuda.Event() for _ in range(4)]
 
     def forward(self, x: torch.Tensor, rms_renorm: bool = False, stream=None) -> torch.Tensor:
         """x: bf16 bits (int16 or bfloat16) [T][d] on the GPU. Returns y bf16 bits [T][d]
-        (a view into this layer's output buffer)."""
+        (a view into this layer's output buffer). Enqueued on `stream` (default: current);
+        the quantiser and the expert histogram run on a side stream that forks from and
+        joins back into it, so the call is capturable in a CUDA graph."""
         T, k = x.shape[0], self.k
         assert T <= self.T_max
+        main = torch.cuda.current_stream() if stream is None else stream
+        side, ev = self._side, self._ev
+        ev[0].record(main)
+        side.wait_event(ev[0])
         B.nvfp4_quantize_act(x, self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
-                             ts_in=self.static_ts, ws=self.ws, stream=stream)
+                             ts_in=self.static_ts, ws=self.ws_q, stream=side)
+        ev[1].record(side)
         B.moe_route(x, self.Wr, self.br, k, self.topk_idx[:T], self.topk_w[:T], self.counts,
                     self.offsets, self.sorted_assign[:T * k], self.assign_pos[:T * k], self.ws,
-                    stream=stream)
+                    stream=main)
+        ev[2].record(main)
+        main.wait_event(ev[1])
         B.moe_expert_ffn(self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1], self.experts, k,
                          self.offsets, self.sorted_assign[:T * k], self.topk_w[:T],
                          B.MOE_FFN_ACCUMULATE, self.path, self.y_acc[:T], None, self.ws,
-                         stream=stream)
+                         stream=main)
+        side.wait_event(ev[2])
+        B.moe_expert_hist(self.counts, self.cum, self.rank, stream=side)
+        ev[3].record(side)
         B.moe_combine(T, self.d, k, B.MOE_FFN_ACCUMULATE, self.y_acc[:T], None, self.topk_w[:T],
-                      self.assign_pos[:T * k], rms_renorm, self.y[:T], stream=stream)
-        B.moe_expert_hist(self.counts, self.cum, self.rank, stream=stream)
+                      self.assign_pos[:T * k], rms_renorm, self.y[:T], stream=main)
+        main.wait_event(ev[3])
         return self.y[:T]
+
+    def graphed(self, T: int) -> "GraphedMoeLayer":
+        """A replayable CUDA graph of forward() for a fixed token count (decode loops)."""
+        return GraphedMoeLayer(self, T)
+
+
+class GraphedMoeLayer:
+    """forward() of one layer captured once as a CUDA graph; step() copies a pinned host
+    batch in, replays the graph and copies the result back (all on one stream)."""
+
+    def __init__(self, layer: MoeLayer, T: int, rms_renorm: bool = False):
+        self.layer, self.T = layer, T
+        dev = layer.xq_codes.device
+        self.x = torch.zeros(T, layer.d, dtype=torch.int16, device=dev)
+        self.stream = torch.cuda.Stream(device=dev)
+        with torch.cuda.stream(self.stream):
+            layer.forward(self.x, rms_renorm)  # first calls do per-device set-up
+        self.stream.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            self.y = layer.forward(self.x, rms_renorm)
+
+    def step(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
+        """x_host, y_host: pinned host tensors [T][d] of bf16 bits. Asynchronous on
+        self.stream; synchronise (or read y_host after self.stream.synchronize())."""
+        with torch.cuda.stream(self.stream):
+            self.x.copy_(x_host, non_blocking=True)
+            self.graph.replay()
+            y_host.copy_(self.y, non_blocking=True)

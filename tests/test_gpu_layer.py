@@ -83,3 +83,20 @@ def test_stack_chaining_with_rms_renorm():
         xr = synth.f32_to_bf16_bits(torch.from_numpy(yr.astype(np.float32))).numpy()
     # bf16 re-rounding between layers can flip an h code; compare loosely on the final layer
     assert_close_layer(bits_to_f32(h.cpu().numpy()), yr, "2-layer stack")
+
+
+def test_graphed_layer_step_matches_forward():
+    """GraphedMoeLayer.step (pinned host in/out around a captured forward) gives the same
+    output as an eager forward on the same input, over several different inputs."""
+    cfg, lay, Wr, br = _layer("decode", T_max=8)
+    runner = lay.graphed(8)
+    y_host = torch.empty(8, cfg.d, dtype=torch.int16).pin_memory()
+    for step in range(3):
+        x = synth.make_x(5, cfg, 8, step=step)
+        runner.step(x.pin_memory(), y_host)
+        runner.stream.synchronize()
+        got = y_host.clone()
+        want = lay.forward(x.cuda()).cpu()
+        torch.cuda.synchronize()
+        assert torch.equal(got, want) or np.allclose(
+            bits_to_f32(got.numpy()), bits_to_f32(want.numpy()), rtol=1e-2, atol=1e-3)
