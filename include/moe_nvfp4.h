@@ -137,9 +137,11 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
 
 /*
  * moe_pack_experts - re-tile the E4M3 scale bytes of an expert group for the tensor-core
- * (PREFILL) path. gu_sf_tiled needs E*2I*d/16 bytes, dn_sf_tiled E*d*I/16 bytes. Run once
- * per weight load; the natural-layout weights stay in use by the DECODE path.
- * Requires d % 128 == 0 and I % 64 == 0.
+ * path: 512-byte atoms of 128 weight rows x 4 scale blocks, the layout the tensor core
+ * reads its scales in. gu_sf_tiled needs E*2I*d/16 bytes, dn_sf_tiled E*d*I/16 bytes
+ * (caller-owned, set in W->gu_sf_tiled / dn_sf_tiled afterwards). Run once per weight
+ * load; the codes and the natural-layout scales stay as they are and remain in use by the
+ * CUDA-core path. Requires d % 128 == 0 and I % 64 == 0.
  */
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
                             uint8_t* dn_sf_tiled, void* stream);
@@ -149,12 +151,20 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
  * expert (A8).
  *   xq_codes [T][d/2], xq_scales [T][d/16], xq_ts float32[1]: the NVFP4 activation.
  *   offsets [E+1], sorted_assign [T*k], topk_w [T][k]: from moe_route / moe_permute.
- *   mode MOE_FFN_ACCUMULATE: out = float32 [T][d] (overwritten), shared_out unused.
+ *   mode MOE_FFN_ACCUMULATE: out = float32 [T][d], set by the call to
+ *        sum_j topk_w[t,j] * o[t,j] + o_shared[t] (the call zeroes it first); shared_out
+ *        unused. The order of the float32 additions is not fixed.
  *   mode MOE_FFN_PER_ASSIGN: out = float32 [T*k][d] in sorted order (unweighted);
  *        shared_out = float32 [T][d] when the layer has a shared expert, else NULL.
- *   path: MOE_PATH_AUTO / DECODE / PREFILL.
- * Limits: d % 16 == 0, I % 16 == 0, d <= 8192, I <= 8192 (PREFILL: d % 256 == 0,
- * I % 64 == 0, scales packed). Accumulation order in ACCUMULATE mode is not fixed.
+ *   path: MOE_PATH_PREFILL = tcgen05 block-scaled tensor-core kernels (any T; needs
+ *        d % 256 == 0, I % 256 == 0 and both groups packed by moe_pack_experts);
+ *        MOE_PATH_DECODE = the CUDA-core kernel on the natural layout (d % 16 == 0,
+ *        I % 16 == 0); MOE_PATH_AUTO = the tensor-core kernels whenever their
+ *        requirements hold, else the CUDA-core kernel.
+ * Limits: d <= 8192, I <= 8192. The workspace (moe_workspace_size(MOE_OP_FFN, ...)) holds
+ * the tile schedule, the NVFP4 intermediate h and, above 64 tokens, the gathered
+ * activation rows. Device waits that exceed 2 s end the kernel and set the device status
+ * to MOE_ERR_TIMEOUT (read it with moe_get_device_status).
  */
 moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales,
                           const float* xq_ts, int32_t T, const moe_experts_t* W, int32_t k,

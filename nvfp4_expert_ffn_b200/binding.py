@@ -15,7 +15,8 @@ from typing import Optional
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "lib", "libmoe_nvfp4.so")
+# MOE_NVFP4_LIB selects another build of the same library (e.g. the timeline-trace build)
+LIB_PATH = os.environ.get("MOE_NVFP4_LIB") or os.path.join(_PKG, "lib", "libmoe_nvfp4.so")
 
 MOE_OK = 0
 MOE_FFN_ACCUMULATE, MOE_FFN_PER_ASSIGN = 0, 1

@@ -8,14 +8,17 @@
 // E4M3 block scales staged into tensor memory: the tensor core consumes E2M1 codes and
 // scales directly, nothing is decoded on the CUDA cores.
 //
-// Two launches per call:
+// Two launches per call (three for more than 64 tokens):
 //   1. tc_schedule_kernel: CTA 0 lays out 128-row m-tiles over each expert's tokens (the
 //      shared expert is slot E) and zeroes the per-m-tile completion counters; the other
 //      CTAs zero y in accumulate mode.
+//   1b. (more than 64 tokens) tc_row_gather_kernel: copies each m-tile's activation rows
+//      and scale bytes into contiguous per-m-tile buffers, read once per phase-1 tile.
 //   2. tc_ffn_kernel (persistent, one CTA per SM, warp-specialised):
-//        warp 0    producer: gathers each m-tile's activation rows straight from the
-//                  quantised activations with TMA tile::gather4 (and their scale bytes
-//                  with cp.async into 128x4 scale atoms), TMA-loads weight tiles and their
+//        warp 0    producer: for few tokens, gathers each m-tile's activation rows
+//                  straight from the quantised activations with TMA tile::gather4 (their
+//                  scale bytes with cp.async into 128x4 scale atoms); for many, one TMA
+//                  box of the gathered rows per stage; TMA-loads weight tiles and their
 //                  pre-tiled scale atoms, into a 4-stage shared-memory ring
 //        warp 1    TMEM allocation and the MMA issuer (single thread)
 //        warps 2-9 epilogue: TMEM -> registers; two warps per TMEM lane quarter, each
@@ -53,6 +56,49 @@ constexpr int kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_mxf4nvf4(kTileM, kTileN);
 constexpr int kSmallT = 64;  // up to this many tokens the producer copies activation scales itself
 
+// ---------------------------------------------------------------- optional timeline trace
+// Built with -DMOE_TRACE (python -m nvfp4_expert_ffn_b200.build --trace), the FFN kernel
+// records per-CTA events into g_tc_trace: record 0 = globaltimer at entry, record 1 =
+// clock64 at entry, then (SM cycles since entry << 32) | event << 24 | tile. Read back with
+// moe_trace_fetch(). Without the flag every hook compiles to nothing.
+enum TraceEvent : uint32_t {
+  kEvSetupDone = 1,   // barriers, TMEM and tensor maps ready
+  kEvProdTile = 2,    // producer starts a tile
+  kEvProdDone1 = 3,   // producer: phase-1 results of the m-tile are complete (phase-2 tile)
+  kEvMmaFirst = 4,    // first stage of a tile landed
+  kEvMmaLast = 5,     // last MMA of a tile issued
+  kEvEpiStart = 6,    // accumulator ready for the epilogue
+  kEvEpiEnd = 7,      // epilogue of a tile done
+  kEvExit = 8,
+};
+#ifdef MOE_TRACE
+constexpr int kTraceCtas = 160, kTraceCap = 254;
+__device__ unsigned long long g_tc_trace[kTraceCtas][kTraceCap + 2];
+#define TC_TRACE_DECL __shared__ unsigned int s_trace_n; __shared__ long long s_trace_clk0;
+#define TC_TRACE_BEGIN()                                                            \
+  do {                                                                              \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) {                              \
+      s_trace_n = 0;                                                                \
+      s_trace_clk0 = clock64();                                                     \
+      g_tc_trace[blockIdx.x][0] = globaltimer_ns();                                 \
+      g_tc_trace[blockIdx.x][1] = (unsigned long long)s_trace_clk0;                 \
+    }                                                                               \
+  } while (0)
+#define TC_TRACE(ev, tile)                                                                       \
+  do {                                                                                           \
+    if (blockIdx.x < kTraceCtas) {                                                               \
+      const unsigned int i_ = atomicAdd(&s_trace_n, 1u);                                         \
+      if (i_ < (unsigned)kTraceCap)                                                              \
+        g_tc_trace[blockIdx.x][2 + i_] = ((unsigned long long)(clock64() - s_trace_clk0) << 32) | \
+                                         ((unsigned long long)(ev) << 24) | ((tile) & 0xFFFFFF);   \
+    }                                                                                            \
+  } while (0)
+#else
+#define TC_TRACE_DECL
+#define TC_TRACE_BEGIN() do { } while (0)
+#define TC_TRACE(ev, tile) do { } while (0)
+#endif
+
 MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 MOE_DEV int32_t ld_acquire_gpu(const int32_t* p) {
@@ -71,6 +117,7 @@ struct TcParams {
   int32_t* row_token;
   float* row_weight;
   int32_t* row_slot;
+  uint8_t* a1;        // [rows_cap][d/2] x codes gathered per m-tile row (large T), or NULL
   uint8_t* sfa1;      // [m][d/64][512] x scale atoms gathered per m-tile (large T), or NULL
   uint8_t* h_codes;   // [rows_cap][I/2]
   uint8_t* sfa2;      // [m][I/64][512]
@@ -135,11 +182,12 @@ __global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
     o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// ---------------------------------------------------------------- 1b. scale gather (large T)
-// With many rows per m-tile, the producer bulk-copies the activation scale atoms instead of
-// issuing 4-byte copies per row: one warp per row writes the row's d/16 scale bytes into
-// the atoms of its m-tile, and the row's (token, weight, output slot).
-__global__ void __launch_bounds__(256) tc_sf_gather_kernel(TcParams p) {
+// ---------------------------------------------------------------- 1b. row gather (large T)
+// With many rows per m-tile, every phase-1 tile of an m-tile would gather the same rows
+// again, 4 rows per TMA request; instead one warp per row copies the row's d/2 code bytes
+// into a contiguous [m-tile row][d/2] buffer (one TMA box per stage then), its d/16 scale
+// bytes into the m-tile's scale atoms, and writes the row's (token, weight, output slot).
+__global__ void __launch_bounds__(256) tc_row_gather_kernel(TcParams p) {
   MOE_PDL_PROLOGUE();
   const int n_m = *p.n_mtiles;
   const int lane = threadIdx.x & 31;
@@ -159,6 +207,9 @@ __global__ void __launch_bounds__(256) tc_sf_gather_kernel(TcParams p) {
       wgt = p.topk_w[a];
       slot = q;
     }
+    const uint4* csrc = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
+    uint4* cdst = reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
+    for (int c = lane; c < d / 32; c += 32) cdst[c] = __ldg(csrc + c);
     const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
     for (int kc = lane; kc < d / 64; kc += 32)
       *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (r % 32) * 16 + (r / 32) * 4) =
@@ -210,6 +261,7 @@ __global__ void pack_sf_kernel(const uint8_t* __restrict__ gu_scales, const uint
 // ---------------------------------------------------------------- 3. persistent FFN kernel
 struct TcMaps {
   CUtensorMap xg;    // x codes [T][d/2], one-row boxes for tile::gather4
+  CUtensorMap a1;    // gathered x codes [rows_cap][d/2] (large T)
   CUtensorMap a2;    // h codes           [rows_cap][I/2]
   CUtensorMap b1;    // routed gate/up    {d/2, I, 2, E}
   CUtensorMap b1s;   // shared gate/up    {d/2, I, 2, 1}
@@ -237,7 +289,9 @@ MOE_DEV TileInfo decode_tile(int t, int n_m, int nt1, int nt2) {
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
+  TC_TRACE_DECL
   MOE_PDL_PROLOGUE();
+  TC_TRACE_BEGIN();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t full[kTcStages], empty[kTcStages], acc_full[2], acc_empty[2], final_bar;
@@ -261,7 +315,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     mbar_init(&final_bar, 1);
     fence_barrier_init();
     s_abort = 0;
-    prefetch_tensormap(&maps.xg);
+    prefetch_tensormap(p.a1 ? &maps.a1 : &maps.xg);
     prefetch_tensormap(&maps.a2);
     prefetch_tensormap(&maps.b1);
     prefetch_tensormap(&maps.b2);
@@ -273,6 +327,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
   const uint32_t tmem = s_tmem;
   const int n_m = *p.n_mtiles;
   const int total = n_m * (nt1 + nt2);
+  if (threadIdx.x == 0) TC_TRACE(kEvSetupDone, n_m);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -285,7 +340,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     // tile are started before the current tile's copies are issued, so their latency hides.
     auto load_rowtok = [&](int tt, int (&rt)[4]) {
       const TileInfo tn = decode_tile(tt, n_m, nt1, nt2);
-      if (tt >= total || tn.phase != 1) return;
+      if (tt >= total || tn.phase != 1 || p.a1) return;
       const int en = p.mt_expert[tn.m];
       const int vn = p.mt_valid[tn.m];
       const int first = p.mt_first[tn.m];
@@ -306,6 +361,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
       const int valid = p.mt_valid[ti.m];
       const ExpertGroup& G = sh ? p.shared : p.routed;
       const int nks = ti.phase == 1 ? nks1 : nks2;
+      if (lane == 0) TC_TRACE(kEvProdTile, t);
       int rowtok[4] = {0, 0, 0, 0};
       int ngather = 0;
       if (ti.phase == 1) {
@@ -321,7 +377,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
       load_rowtok(t + gridDim.x, next_tok);
       const int nq = (valid + 31) / 32;
       const uint32_t stage_tx =
-          ti.phase == 1 ? (uint32_t)(ngather * 512 + kBBytes + (p.sfa1 ? 2 : 1) * kSfBytes)
+          ti.phase == 1 ? (p.a1 ? (uint32_t)(kABytes + kBBytes + 2 * kSfBytes)
+                                : (uint32_t)(ngather * 512 + kBBytes + kSfBytes))
                         : (uint32_t)(nq * 4096 + kBBytes + 2 * kSfBytes);
       auto wait_empty = [&](uint32_t itx) -> bool {
         int ok = 1;
@@ -346,14 +403,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
       auto issue_a = [&](int ks, uint32_t s) {
         uint8_t* st = smem + (size_t)s * kStageBytes;
         uint8_t* sSFA = st + kABytes + kBBytes;
-        if (ti.phase == 1) {
-          if (p.sfa1 && lane == 0)
+        if (ti.phase == 1 && p.a1) {
+          if (lane == 0) {
+            tma_load_2d(st, &maps.a1, &full[s], ks * 128, ti.m * kTileM);
             bulk_g2s(sSFA, p.sfa1 + ((size_t)ti.m * (d / 64) + 4 * ks) * kAtom, kSfBytes, &full[s]);
+          }
+        } else if (ti.phase == 1) {
           if (4 * lane < valid) {
             tma_gather4(st + 4 * lane * 128, &maps.xg, &full[s], ks * 128, rowtok[0], rowtok[1], rowtok[2],
                         rowtok[3]);
 #pragma unroll
-            for (int i = 0; i < 4 && !p.sfa1; ++i) {
+            for (int i = 0; i < 4; ++i) {
               const int r = 4 * lane + i;
               if (r < valid) {
                 const uint8_t* src = p.xq_scales + (size_t)rowtok[i] * (d / kBlock) + 16 * ks;
@@ -396,6 +456,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             }
           }
           fence_proxy_async_global();
+          TC_TRACE(kEvProdDone1, t);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         for (int ks = 0; ks < npre; ++ks) issue_a(ks, (it + ks) % kTcStages);
@@ -439,6 +500,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             break;
           }
           tc_fence_after();
+          if (ks == 0) TC_TRACE(kEvMmaFirst, t);
           fence_proxy_async_smem();  // scale bytes arrived through cp.async (generic proxy)
           const uint8_t* st = smem + (size_t)s * kStageBytes;
           const uint32_t aA = smem_u32(st), aB = smem_u32(st + kABytes);
@@ -457,6 +519,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           mma_commit(&empty[s]);
         }
         if (!ok) break;
+        TC_TRACE(kEvMmaLast, t);
         mma_commit(&acc_full[buf]);
       }
       // all issued tensor-core work has completed before TMEM is released
@@ -484,6 +547,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         s_epi_go[buf] = mbar_wait(&acc_full[buf], (tc >> 1) & 1, &s_abort, p.status) ? 1 : 0;
       named_bar_sync(2, 32 * kEpiWarps);
       if (!s_epi_go[buf]) break;
+      if (warp == 2 && lane == 0) TC_TRACE(kEvEpiStart, t);
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kTileN;
       const int e = p.mt_expert[ti.m];
@@ -535,7 +599,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           *reinterpret_cast<uint16_t*>(p.sfa2 + ((size_t)ti.m * (I / 64) + ti.j) * kAtom + (row % 32) * 16 +
                                        (row / 32) * 4 + 2 * half) = (uint16_t)sbytes;
         }
-        if (!p.sfa1 && ti.j == 0 && half == 0 && valid) {
+        if (!p.a1 && ti.j == 0 && half == 0 && valid) {
           // token, routing weight and output slot of this row, for the phase-2 epilogue
           const int i = p.mt_first[ti.m] + row;
           int tokr = i, slotr = -1;
@@ -555,7 +619,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         fence_proxy_async_global();
         __threadfence();
         named_bar_sync(2, 32 * kEpiWarps);
-        if (warp == 2 && lane == 0) atomicAdd(p.done1 + ti.m, 1);
+        if (warp == 2 && lane == 0) {
+          atomicAdd(p.done1 + ti.m, 1);
+          TC_TRACE(kEvEpiEnd, t);
+        }
       } else {
         const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
         int tok = 0, slot = 0;
@@ -593,6 +660,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           }
           bulk_commit();
         }
+        if (warp == 2 && lane == 0) TC_TRACE(kEvEpiEnd, t);
       }
     }
     bulk_wait_all();
@@ -603,6 +671,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (threadIdx.x == 0) TC_TRACE(kEvExit, 0);
 }
 
 // ---------------------------------------------------------------- host side
@@ -635,8 +704,8 @@ size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
 struct TcLayout {
   int max_m;
   size_t rows_cap;
-  size_t off_hdr, off_expert, off_valid, off_first, off_done, off_tok, off_w, off_slot, off_sfa1, off_h, off_sfa2,
-      total;
+  size_t off_hdr, off_expert, off_valid, off_first, off_done, off_tok, off_w, off_slot, off_a1, off_sfa1, off_h,
+      off_sfa2, total;
 };
 
 TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
@@ -653,7 +722,9 @@ TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   L.off_tok = o; o += a256(L.rows_cap * 4);
   L.off_w = o; o += a256(L.rows_cap * 4);
   L.off_slot = o; o += a256(L.rows_cap * 4);
-  L.off_sfa1 = o; o += a256(L.rows_cap * (d / kBlock));
+  const bool big = T > kSmallT;  // large T: activation rows gathered before the FFN kernel
+  L.off_a1 = o; o += big ? a256(L.rows_cap * (d / 2)) : 0;
+  L.off_sfa1 = o; o += big ? a256(L.rows_cap * (d / kBlock)) : 0;
   L.off_h = o; o += a256(L.rows_cap * (I / 2));
   L.off_sfa2 = o; o += a256(L.rows_cap * (I / kBlock));
   L.total = o;
@@ -696,6 +767,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.row_token = reinterpret_cast<int32_t*>(w + L.off_tok);
   p.row_weight = reinterpret_cast<float*>(w + L.off_w);
   p.row_slot = reinterpret_cast<int32_t*>(w + L.off_slot);
+  p.a1 = a.T > kSmallT ? w + L.off_a1 : nullptr;
   p.sfa1 = a.T > kSmallT ? w + L.off_sfa1 : nullptr;
   p.h_codes = w + L.off_h;
   p.sfa2 = w + L.off_sfa2;
@@ -721,6 +793,14 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
     cuuint32_t box[2] = {128, 1};
     if ((e = encode_u8(&maps.xg, a.xq_codes, 2, dims, strides, box)) != cudaSuccess) return e;
+  }
+  if (p.a1) {
+    cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)L.rows_cap};
+    cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
+    cuuint32_t box[2] = {128, 128};
+    if ((e = encode_u8(&maps.a1, p.a1, 2, dims, strides, box)) != cudaSuccess) return e;
+  } else {
+    maps.a1 = maps.xg;
   }
   {
     cuuint64_t dims[2] = {(cuuint64_t)(I / 2), (cuuint64_t)L.rows_cap};
@@ -754,9 +834,23 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     if (zc > num_sms) zc = num_sms;
   }
   if ((e = launch_pdl(tc_schedule_kernel, dim3(1 + zc), dim3(1024), 0, st, p)) != cudaSuccess) return e;
-  if (p.sfa1 && (e = launch_pdl(tc_sf_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess)
+  if (p.a1 && (e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess)
     return e;
   return launch_pdl(tc_ffn_kernel, dim3(num_sms), dim3(kTcThreads), ffn_tc_smem_bytes(), st, maps, p);
 }
 
 }  // namespace moe
+
+#ifdef MOE_TRACE
+// Trace builds only: copy the FFN kernel's timeline records to `host` (at most `bytes`)
+// and clear them. Returns the number of bytes copied, or -1 on a CUDA error.
+extern "C" int64_t moe_trace_fetch(void* host, size_t bytes) {
+  const size_t n = sizeof(moe::g_tc_trace) < bytes ? sizeof(moe::g_tc_trace) : bytes;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(host, moe::g_tc_trace, n) != cudaSuccess) return -1;
+  constexpr size_t kWords = (size_t)moe::kTraceCtas * (moe::kTraceCap + 2);
+  static const unsigned long long zeros[kWords] = {};
+  if (cudaMemcpyToSymbol(moe::g_tc_trace, zeros, sizeof(zeros)) != cudaSuccess) return -1;
+  return (int64_t)n;
+}
+#endif

@@ -284,7 +284,6 @@ MOE_DEV void chunk_scatter(const int32_t* idx, int n, int c, int* run, int32_t* 
 __global__ void __launch_bounds__(kPermThreads) perm_hist_kernel(const int32_t* __restrict__ idx, int n,
                                                                  int E, int32_t* __restrict__ chunk_hist) {
   MOE_PDL_PROLOGUE();
-  MOE_PDL_PROLOGUE();
   extern __shared__ int sh[];
   chunk_histogram(idx, n, blockIdx.x, E, sh);
   for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = sh[e];
