@@ -58,9 +58,10 @@ typedef enum moe_status {
 #define MOE_FFN_PER_ASSIGN 1  /* out = float32 [T*k][d], row p = o of sorted_assign[p];
                                  shared_out = float32 [T][d] (unweighted) */
 /* FFN kernel paths */
-#define MOE_PATH_AUTO 0       /* PREFILL when available and T is large, else DECODE */
-#define MOE_PATH_DECODE 1     /* CUDA-core GEMV path (any T; meant for 1-64 tokens) */
-#define MOE_PATH_PREFILL 2    /* tcgen05 block-scaled grouped GEMM path */
+#define MOE_PATH_AUTO 0       /* the fastest path whose requirements hold */
+#define MOE_PATH_DECODE 1     /* tcgen05 split-over-I decode kernel (T <= 8) */
+#define MOE_PATH_PREFILL 2    /* tcgen05 block-scaled grouped GEMM path (any T) */
+#define MOE_PATH_CUDA_CORE 3  /* CUDA-core kernel on the natural layout (any shape) */
 
 /* workspace query operations */
 #define MOE_OP_LAYER 0        /* enough for every call of one layer forward */
@@ -156,11 +157,15 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
  *        unused. The order of the float32 additions is not fixed.
  *   mode MOE_FFN_PER_ASSIGN: out = float32 [T*k][d] in sorted order (unweighted);
  *        shared_out = float32 [T][d] when the layer has a shared expert, else NULL.
- *   path: MOE_PATH_PREFILL = tcgen05 block-scaled tensor-core kernels (any T; needs
- *        d % 256 == 0, I % 256 == 0 and both groups packed by moe_pack_experts);
- *        MOE_PATH_DECODE = the CUDA-core kernel on the natural layout (d % 16 == 0,
- *        I % 16 == 0); MOE_PATH_AUTO = the tensor-core kernels whenever their
- *        requirements hold, else the CUDA-core kernel.
+ *   path: MOE_PATH_DECODE = tcgen05 kernel for at most 8 tokens, one CTA per (expert,
+ *        64-column slice of I) computing gate/up, SwiGLU, h and that slice's share of
+ *        the down projection (needs T <= 8, MOE_FFN_ACCUMULATE, d % 512 == 0,
+ *        I % 64 == 0 and both groups packed by moe_pack_experts);
+ *        MOE_PATH_PREFILL = tcgen05 block-scaled grouped GEMMs over 128-token tiles
+ *        (any T; needs d % 256 == 0, I % 256 == 0 and packed scales);
+ *        MOE_PATH_CUDA_CORE = the CUDA-core kernel on the natural layout (d % 16 == 0,
+ *        I % 16 == 0); MOE_PATH_AUTO = DECODE when its requirements hold, else PREFILL
+ *        when its requirements hold, else CUDA_CORE.
  * Limits: d <= 8192, I <= 8192. The workspace (moe_workspace_size(MOE_OP_FFN, ...)) holds
  * the tile schedule, the NVFP4 intermediate h and, above 64 tokens, the gathered
  * activation rows. Device waits that exceed 2 s end the kernel and set the device status

@@ -20,7 +20,7 @@ LIB_PATH = os.environ.get("MOE_NVFP4_LIB") or os.path.join(_PKG, "lib", "libmoe_
 
 MOE_OK = 0
 MOE_FFN_ACCUMULATE, MOE_FFN_PER_ASSIGN = 0, 1
-MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL = 0, 1, 2
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_CUDA_CORE = 0, 1, 2, 3
 MOE_OP_LAYER, MOE_OP_ROUTE, MOE_OP_QUANT, MOE_OP_FFN = 0, 1, 2, 3
 
 # (name, restype, argtypes) of every C export; tests check the header declares the same set

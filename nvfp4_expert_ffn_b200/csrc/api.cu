@@ -71,7 +71,9 @@ size_t quant_ws_bytes() { return align256(kMaxPartials * sizeof(float)); }
 size_t ffn_ws_bytes(int64_t T, int d, int E, int k, int I) {
   const size_t a = ffn_decode_ws_bytes(T, d, E, k, I);
   const size_t b = ffn_tc_ws_bytes(T, d, E, k, I);
-  return a > b ? a : b;
+  const size_t c = ffn_dec_ws_bytes(E);
+  const size_t ab = a > b ? a : b;
+  return ab > c ? ab : c;
 }
 
 moe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
@@ -249,7 +251,7 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   if (d <= 0 || I <= 0 || d % kBlock || I % kBlock || d > 8192 || I > 8192)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE, "d and I must be multiples of 16 in [16, 8192]");
   if (mode != MOE_FFN_ACCUMULATE && mode != MOE_FFN_PER_ASSIGN) return fail(MOE_ERR_INVALID_ARG, "bad mode");
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL)
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL && path != MOE_PATH_CUDA_CORE)
     return fail(MOE_ERR_INVALID_ARG, "bad path");
   moe_status s = check_weights(W->routed, "routed", E, d, I);
   if (s != MOE_OK) return s;
@@ -266,11 +268,18 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
   const bool tc_ok = ffn_tc_supported(d, I) && packed;
+  const bool dec_ok = ffn_dec_supported(T, d, I, mode) && packed;
   if (path == MOE_PATH_PREFILL && !tc_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "tensor-core path needs d % 256 == 0, I % 256 == 0 and scales packed by moe_pack_experts");
-  const bool use_tc = (path == MOE_PATH_PREFILL) || (path == MOE_PATH_AUTO && tc_ok);
-  const size_t need = use_tc ? ffn_tc_ws_bytes(T, d, E, k, I) : ffn_decode_ws_bytes(T, d, E, k, I);
+  if (path == MOE_PATH_DECODE && !dec_ok)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                "decode path needs T <= 8, ACCUMULATE mode, d % 512 == 0, I % 64 == 0 and packed scales");
+  const int kind = path == MOE_PATH_AUTO ? (dec_ok ? MOE_PATH_DECODE : tc_ok ? MOE_PATH_PREFILL : MOE_PATH_CUDA_CORE)
+                                         : path;
+  const size_t need = kind == MOE_PATH_DECODE    ? ffn_dec_ws_bytes(E)
+                      : kind == MOE_PATH_PREFILL ? ffn_tc_ws_bytes(T, d, E, k, I)
+                                                 : ffn_decode_ws_bytes(T, d, E, k, I);
   s = check_ws(ws, ws_bytes, need);
   if (s != MOE_OK) return s;
   int sms = 0;
@@ -294,8 +303,9 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const size_t slots = (size_t)T * k + T;
   a.h_codes = reinterpret_cast<uint8_t*>(ws);
   a.h_scales = reinterpret_cast<uint8_t*>(ws) + align256(slots * (I / 2));
-  cudaError_t e = use_tc ? launch_ffn_tc(a, ws, sms, dstatus, (cudaStream_t)stream)
-                         : launch_ffn_decode(a, sms, dstatus, (cudaStream_t)stream);
+  cudaError_t e = kind == MOE_PATH_DECODE    ? launch_ffn_dec(a, ws, sms, dstatus, (cudaStream_t)stream)
+                  : kind == MOE_PATH_PREFILL ? launch_ffn_tc(a, ws, sms, dstatus, (cudaStream_t)stream)
+                                             : launch_ffn_decode(a, sms, dstatus, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
 }
 
@@ -342,3 +352,15 @@ moe_status moe_get_device_status(void* stream, int32_t clear, int32_t* status_ou
 }
 
 }  // extern "C"
+
+#ifdef MOE_TRACE
+namespace moe {
+int64_t trace_fetch_tc(void* host, size_t bytes);
+int64_t trace_fetch_dec(void* host, size_t bytes);
+}  // namespace moe
+// Trace builds only: timeline records of the last runs of the tensor-core FFN kernel
+// (kernel 0: the grouped-GEMM path, 1: the decode path), copied to `host` and cleared.
+extern "C" int64_t moe_trace_fetch(int32_t kernel, void* host, size_t bytes) {
+  return kernel == 0 ? moe::trace_fetch_tc(host, bytes) : moe::trace_fetch_dec(host, bytes);
+}
+#endif

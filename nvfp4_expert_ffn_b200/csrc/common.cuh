@@ -103,6 +103,18 @@ MOE_DEV uint32_t quantize_block16(const float v[16], float ts, uint2* codes) {
   return s;
 }
 
+// h = silu(g) * u for 16 consecutive columns (g, u: float32 sums, scaled by sg and su), then
+// the NVFP4 quantisation of that block of h with tensor scale 1. Returns the scale byte.
+MOE_DEV uint32_t swiglu_quant16(const uint32_t (&g)[16], const uint32_t (&u)[16], float sg, float su, uint2* codes) {
+  float h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float gv = __uint_as_float(g[i]) * sg, uv = __uint_as_float(u[i]) * su;
+    h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
+  }
+  return quantize_block16(h, 1.0f, codes);
+}
+
 // ---------------------------------------------------------------- warp / block reductions
 MOE_DEV float warp_max(float v) {
 #pragma unroll

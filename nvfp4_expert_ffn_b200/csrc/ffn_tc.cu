@@ -30,11 +30,11 @@
 //      w * o in shared memory and adds it into y with a bulk reduction
 //      (cp.reduce.async.bulk .add.f32), or stores o.
 //      Accumulators are double-buffered in TMEM so an epilogue overlaps the next tile.
-#include <cudaTypedefs.h>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "tmap.h"
+#include "trace.cuh"
 
 namespace moe {
 
@@ -56,56 +56,9 @@ constexpr int kTmemCols = 512;
 constexpr uint32_t kIdesc = idesc_mxf4nvf4(kTileM, kTileN);
 constexpr int kSmallT = 64;  // up to this many tokens the producer copies activation scales itself
 
-// ---------------------------------------------------------------- optional timeline trace
-// Built with -DMOE_TRACE (python -m nvfp4_expert_ffn_b200.build --trace), the FFN kernel
-// records per-CTA events into g_tc_trace: record 0 = globaltimer at entry, record 1 =
-// clock64 at entry, then (SM cycles since entry << 32) | event << 24 | tile. Read back with
-// moe_trace_fetch(). Without the flag every hook compiles to nothing.
-enum TraceEvent : uint32_t {
-  kEvSetupDone = 1,   // barriers, TMEM and tensor maps ready
-  kEvProdTile = 2,    // producer starts a tile
-  kEvProdDone1 = 3,   // producer: phase-1 results of the m-tile are complete (phase-2 tile)
-  kEvMmaFirst = 4,    // first stage of a tile landed
-  kEvMmaLast = 5,     // last MMA of a tile issued
-  kEvEpiStart = 6,    // accumulator ready for the epilogue
-  kEvEpiEnd = 7,      // epilogue of a tile done
-  kEvExit = 8,
-};
-#ifdef MOE_TRACE
-constexpr int kTraceCtas = 160, kTraceCap = 254;
-__device__ unsigned long long g_tc_trace[kTraceCtas][kTraceCap + 2];
-#define TC_TRACE_DECL __shared__ unsigned int s_trace_n; __shared__ long long s_trace_clk0;
-#define TC_TRACE_BEGIN()                                                            \
-  do {                                                                              \
-    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) {                              \
-      s_trace_n = 0;                                                                \
-      s_trace_clk0 = clock64();                                                     \
-      g_tc_trace[blockIdx.x][0] = globaltimer_ns();                                 \
-      g_tc_trace[blockIdx.x][1] = (unsigned long long)s_trace_clk0;                 \
-    }                                                                               \
-  } while (0)
-#define TC_TRACE(ev, tile)                                                                       \
-  do {                                                                                           \
-    if (blockIdx.x < kTraceCtas) {                                                               \
-      const unsigned int i_ = atomicAdd(&s_trace_n, 1u);                                         \
-      if (i_ < (unsigned)kTraceCap)                                                              \
-        g_tc_trace[blockIdx.x][2 + i_] = ((unsigned long long)(clock64() - s_trace_clk0) << 32) | \
-                                         ((unsigned long long)(ev) << 24) | ((tile) & 0xFFFFFF);   \
-    }                                                                                            \
-  } while (0)
-#else
-#define TC_TRACE_DECL
-#define TC_TRACE_BEGIN() do { } while (0)
-#define TC_TRACE(ev, tile) do { } while (0)
-#endif
 
-MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
-MOE_DEV int32_t ld_acquire_gpu(const int32_t* p) {
-  int32_t v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
+TC_TRACE_ARRAY(g_tc_trace)
 
 struct TcParams {
   // schedule and gathered rows (workspace)
@@ -291,7 +244,7 @@ MOE_DEV TileInfo decode_tile(int t, int n_m, int nt1, int nt2) {
 __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
   TC_TRACE_DECL
   MOE_PDL_PROLOGUE();
-  TC_TRACE_BEGIN();
+  TC_TRACE_BEGIN(g_tc_trace);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t full[kTcStages], empty[kTcStages], acc_full[2], acc_empty[2], final_bar;
@@ -327,7 +280,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
   const uint32_t tmem = s_tmem;
   const int n_m = *p.n_mtiles;
   const int total = n_m * (nt1 + nt2);
-  if (threadIdx.x == 0) TC_TRACE(kEvSetupDone, n_m);
+  if (threadIdx.x == 0) TC_TRACE_AT(g_tc_trace, kEvSetupDone, n_m);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -361,7 +314,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
       const int valid = p.mt_valid[ti.m];
       const ExpertGroup& G = sh ? p.shared : p.routed;
       const int nks = ti.phase == 1 ? nks1 : nks2;
-      if (lane == 0) TC_TRACE(kEvProdTile, t);
+      if (lane == 0) TC_TRACE_AT(g_tc_trace, kEvProdTile, t);
       int rowtok[4] = {0, 0, 0, 0};
       int ngather = 0;
       if (ti.phase == 1) {
@@ -456,7 +409,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             }
           }
           fence_proxy_async_global();
-          TC_TRACE(kEvProdDone1, t);
+          TC_TRACE_AT(g_tc_trace, kEvProdDone1, t);
         }
         if (!__shfl_sync(0xffffffffu, ok, 0)) break;
         for (int ks = 0; ks < npre; ++ks) issue_a(ks, (it + ks) % kTcStages);
@@ -500,7 +453,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
             break;
           }
           tc_fence_after();
-          if (ks == 0) TC_TRACE(kEvMmaFirst, t);
+          if (ks == 0) TC_TRACE_AT(g_tc_trace, kEvMmaFirst, t);
           fence_proxy_async_smem();  // scale bytes arrived through cp.async (generic proxy)
           const uint8_t* st = smem + (size_t)s * kStageBytes;
           const uint32_t aA = smem_u32(st), aB = smem_u32(st + kABytes);
@@ -519,7 +472,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           mma_commit(&empty[s]);
         }
         if (!ok) break;
-        TC_TRACE(kEvMmaLast, t);
+        TC_TRACE_AT(g_tc_trace, kEvMmaLast, t);
         mma_commit(&acc_full[buf]);
       }
       // all issued tensor-core work has completed before TMEM is released
@@ -547,7 +500,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         s_epi_go[buf] = mbar_wait(&acc_full[buf], (tc >> 1) & 1, &s_abort, p.status) ? 1 : 0;
       named_bar_sync(2, 32 * kEpiWarps);
       if (!s_epi_go[buf]) break;
-      if (warp == 2 && lane == 0) TC_TRACE(kEvEpiStart, t);
+      if (warp == 2 && lane == 0) TC_TRACE_AT(g_tc_trace, kEvEpiStart, t);
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + buf * kTileN;
       const int e = p.mt_expert[ti.m];
@@ -621,7 +574,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         named_bar_sync(2, 32 * kEpiWarps);
         if (warp == 2 && lane == 0) {
           atomicAdd(p.done1 + ti.m, 1);
-          TC_TRACE(kEvEpiEnd, t);
+          TC_TRACE_AT(g_tc_trace, kEvEpiEnd, t);
         }
       } else {
         const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
@@ -660,7 +613,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
           }
           bulk_commit();
         }
-        if (warp == 2 && lane == 0) TC_TRACE(kEvEpiEnd, t);
+        if (warp == 2 && lane == 0) TC_TRACE_AT(g_tc_trace, kEvEpiEnd, t);
       }
     }
     bulk_wait_all();
@@ -671,33 +624,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0) TC_TRACE(kEvExit, 0);
+  if (threadIdx.x == 0) TC_TRACE_AT(g_tc_trace, kEvExit, 0);
 }
 
 // ---------------------------------------------------------------- host side
 namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-cudaError_t get_encode() {
-  if (g_encode) return cudaSuccess;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
-  if (e != cudaSuccess) return e;
-  if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  return cudaSuccess;
-}
-
-cudaError_t encode_u8(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-                      const cuuint64_t* strides, const cuuint32_t* box) {
-  cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, (cuuint32_t)rank, const_cast<void*>(base), dims,
-                        strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
 
 size_t a256(size_t v) { return (v + 255) & ~(size_t)255; }
 
@@ -792,13 +723,13 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)a.T};
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
     cuuint32_t box[2] = {128, 1};
-    if ((e = encode_u8(&maps.xg, a.xq_codes, 2, dims, strides, box)) != cudaSuccess) return e;
+    if ((e = encode_u8(&maps.xg, a.xq_codes, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   }
   if (p.a1) {
     cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)L.rows_cap};
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
     cuuint32_t box[2] = {128, 128};
-    if ((e = encode_u8(&maps.a1, p.a1, 2, dims, strides, box)) != cudaSuccess) return e;
+    if ((e = encode_u8(&maps.a1, p.a1, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   } else {
     maps.a1 = maps.xg;
   }
@@ -806,7 +737,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     cuuint64_t dims[2] = {(cuuint64_t)(I / 2), (cuuint64_t)L.rows_cap};
     cuuint64_t strides[1] = {(cuuint64_t)(I / 2)};
     cuuint32_t box[2] = {128, 32};
-    if ((e = encode_u8(&maps.a2, p.h_codes, 2, dims, strides, box)) != cudaSuccess) return e;
+    if ((e = encode_u8(&maps.a2, p.h_codes, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   }
   for (int which = 0; which < 2; ++which) {
     const ExpertGroup& g = which ? a.shared : a.routed;
@@ -821,11 +752,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     cuuint64_t dims1[4] = {(cuuint64_t)(d / 2), (cuuint64_t)I, 2, (cuuint64_t)E};
     cuuint64_t str1[3] = {(cuuint64_t)(d / 2), (cuuint64_t)I * (d / 2), (cuuint64_t)2 * I * (d / 2)};
     cuuint32_t box1[4] = {128, 64, 2, 1};
-    if ((e = encode_u8(m1, g.gu_codes, 4, dims1, str1, box1)) != cudaSuccess) return e;
+    if ((e = encode_u8(m1, g.gu_codes, 4, dims1, str1, box1, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
     cuuint64_t dims2[3] = {(cuuint64_t)(I / 2), (cuuint64_t)d, (cuuint64_t)E};
     cuuint64_t str2[2] = {(cuuint64_t)(I / 2), (cuuint64_t)d * (I / 2)};
     cuuint32_t box2[3] = {128, 128, 1};
-    if ((e = encode_u8(m2, g.dn_codes, 3, dims2, str2, box2)) != cudaSuccess) return e;
+    if ((e = encode_u8(m2, g.dn_codes, 3, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
   }
   int zc = 0;
   if (a.mode == 0) {
@@ -842,15 +773,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
 }  // namespace moe
 
 #ifdef MOE_TRACE
-// Trace builds only: copy the FFN kernel's timeline records to `host` (at most `bytes`)
-// and clear them. Returns the number of bytes copied, or -1 on a CUDA error.
-extern "C" int64_t moe_trace_fetch(void* host, size_t bytes) {
-  const size_t n = sizeof(moe::g_tc_trace) < bytes ? sizeof(moe::g_tc_trace) : bytes;
-  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
-  if (cudaMemcpyFromSymbol(host, moe::g_tc_trace, n) != cudaSuccess) return -1;
-  constexpr size_t kWords = (size_t)moe::kTraceCtas * (moe::kTraceCap + 2);
-  static const unsigned long long zeros[kWords] = {};
-  if (cudaMemcpyToSymbol(moe::g_tc_trace, zeros, sizeof(zeros)) != cudaSuccess) return -1;
-  return (int64_t)n;
-}
+namespace moe {
+int64_t trace_fetch_tc(void* host, size_t bytes) { return trace_fetch(g_tc_trace, host, bytes); }
+}  // namespace moe
 #endif

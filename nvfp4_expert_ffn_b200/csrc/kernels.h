@@ -96,6 +96,10 @@ cudaError_t launch_combine(int T, int d, int k, int mode, const float* expert_ou
 bool ffn_tc_supported(int d, int I);
 size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I);
 cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
+// tcgen05 decode FFN (at most 8 tokens)
+bool ffn_dec_supported(int64_t T, int d, int I, int mode);
+size_t ffn_dec_ws_bytes(int E);
+cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
                            int num_sms, cudaStream_t st);
 
@@ -103,12 +107,15 @@ cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* g
 cudaError_t init_route_attributes();
 cudaError_t init_ffn_decode_attributes();
 cudaError_t init_ffn_tc_attributes();
+cudaError_t init_ffn_dec_attributes();
 inline cudaError_t init_kernel_attributes() {
   cudaError_t e = init_route_attributes();
   if (e != cudaSuccess) return e;
   e = init_ffn_decode_attributes();
   if (e != cudaSuccess) return e;
-  return init_ffn_tc_attributes();
+  e = init_ffn_tc_attributes();
+  if (e != cudaSuccess) return e;
+  return init_ffn_dec_attributes();
 }
 
 }  // namespace moe

@@ -45,8 +45,21 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
     }
   };
   if (e < E) load_w(e, lane);
-  for (int i = threadIdx.x; i < T * d / 8; i += blockDim.x)
-    reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(x) + i);
+  // stage x with every load of a round in flight before the stores (one round trip per 8)
+  const int nx = T * d / 8;
+  for (int i0 = threadIdx.x; i0 < nx; i0 += 8 * blockDim.x) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < nx) v[u] = __ldg(reinterpret_cast<const uint4*>(x) + i);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < nx) reinterpret_cast<uint4*>(xs)[i] = v[u];
+    }
+  }
   __syncthreads();
   for (; e < E; e += gridDim.x * warps) {
     float acc[kGemvMaxT];
@@ -174,7 +187,7 @@ MOE_DEV uint32_t ordered_key(float v) {
 
 template <int NPER>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* __restrict__ idx_out,
-                        float* __restrict__ w_out) {
+                        float* __restrict__ w_out, int* idx_smem = nullptr) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NPER];
 #pragma unroll
@@ -216,13 +229,14 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* __
   if (lane < k) {
     idx_out[lane] = my_e;
     w_out[lane] = ex / sum;
+    if (idx_smem) idx_smem[lane] = my_e;
   }
 }
 
-MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w) {
-  if (E <= 256) topk_token<8>(row, E, k, idx, w);
-  else if (E <= 512) topk_token<16>(row, E, k, idx, w);
-  else topk_token<32>(row, E, k, idx, w);
+MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w, int* idx_smem = nullptr) {
+  if (E <= 256) topk_token<8>(row, E, k, idx, w, idx_smem);
+  else if (E <= 512) topk_token<16>(row, E, k, idx, w, idx_smem);
+  else topk_token<32>(row, E, k, idx, w, idx_smem);
 }
 
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
@@ -376,13 +390,13 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
                                                                int32_t* __restrict__ sorted_assign,
                                                                int32_t* __restrict__ assign_pos) {
   MOE_PDL_PROLOGUE();
-  extern __shared__ int sh[];  // [E]
-  __shared__ int tmp[32];
-  __shared__ int carry;
+  extern __shared__ int sh[];  // [E] counts / running positions, then [T*k] chosen experts
+  int* sidx = sh + E;
   const int warp = threadIdx.x >> 5;
   if (warp < T)
-    topk_dispatch(logits + (size_t)warp * E, E, k, topk_idx + (size_t)warp * k, topk_w + (size_t)warp * k);
-  __syncthreads();  // this CTA's global writes of topk_idx are now visible to all its threads
+    topk_dispatch(logits + (size_t)warp * E, E, k, topk_idx + (size_t)warp * k, topk_w + (size_t)warp * k,
+                  sidx + warp * k);
+  __syncthreads();
   if (warp != 0) return;
   // the permutation of <= 32*k assignments by one warp, without block-wide barriers:
   // histogram (match_any leaders), warp scan of the counts, then a stable scatter in
@@ -393,7 +407,7 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
   __syncwarp();
   for (int base = 0; base < n; base += 32) {
     const int a = base + lane;
-    const int e = a < n ? topk_idx[a] : -1;
+    const int e = a < n ? sidx[a] : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     if (a < n && (peers & ((1u << lane) - 1u)) == 0) sh[e] += __popc(peers);
     __syncwarp();
@@ -426,7 +440,7 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
   __syncwarp();
   for (int base = 0; base < n; base += 32) {
     const int a = base + lane;
-    const int e = a < n ? topk_idx[a] : -1;
+    const int e = a < n ? sidx[a] : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     if (a < n) {
@@ -503,7 +517,7 @@ cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (T <= 32 && T * k <= kPermChunk) {
-    return launch_pdl(topk_perm_small_kernel, dim3(1), dim3(1024), (size_t)E * sizeof(int), st,
+    return launch_pdl(topk_perm_small_kernel, dim3(1), dim3(1024), (size_t)(E + T * k) * sizeof(int), st,
                       (const float*)logits, T, E, k, topk_idx, topk_w, counts, offsets, sorted_assign, assign_pos);
   }
   err = launch_pdl(topk_kernel, dim3((T + 7) / 8), dim3(256), 0, st, (const float*)logits, T, E, k, topk_idx,

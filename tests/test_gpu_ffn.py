@@ -88,9 +88,9 @@ def _tiny_case(seed, d, E, k, I, T, shared, zipf=0.0, pack=False):
     (2048, 16, 2, 512, 5, True),      # decode-like widths
     (48, 8, 2, 32, 9, True),          # d not a multiple of 32
 ])
-def test_ffn_decode_path_matches_oracle(mode, d, E, k, I, T, shared):
+def test_ffn_cuda_core_path_matches_oracle(mode, d, E, k, I, T, shared):
     experts, sh, xq, routing, gpu = _tiny_case(11, d, E, k, I, T, shared)
-    o_g, os_g, y_g = _run_ffn(xq, routing, gpu, k, mode, B.MOE_PATH_DECODE, T, d)
+    o_g, os_g, y_g = _run_ffn(xq, routing, gpu, k, mode, B.MOE_PATH_CUDA_CORE, T, d)
     o_r, os_r, y_r = _oracle_outputs(xq, routing, experts, sh, T, d, k)
     idx, w, offsets, sa, pos = routing
     if mode == B.MOE_FFN_PER_ASSIGN:
@@ -125,6 +125,33 @@ def test_ffn_tensor_core_path_matches_oracle(mode, d, E, k, I, T, shared, zipf):
     assert_close_layer(bits_to_f32(y_g), y_r, "y bf16")
 
 
+@pytest.mark.parametrize("d,E,k,I,T,shared,zipf", [
+    (512, 8, 2, 64, 1, False, 0.0),       # one token, one unit per expert, one down stage
+    (512, 16, 4, 128, 3, True, 0.0),      # odd T, shared expert
+    (1024, 32, 4, 192, 8, True, 1.0),     # full 8 tokens, Zipf: several tokens per expert
+    (2048, 64, 8, 512, 5, True, 0.0),     # decode widths, T not a power of two
+    (512, 4, 4, 256, 8, False, 0.0),      # every token uses every expert
+    (4096, 8, 2, 64, 2, True, 0.0),       # wide d: 16 gate/up stages, 8 down stages
+])
+def test_ffn_decode_path_matches_oracle(d, E, k, I, T, shared, zipf):
+    experts, sh, xq, routing, gpu = _tiny_case(13, d, E, k, I, T, shared, zipf=zipf, pack=True)
+    o_g, _, y_g = _run_ffn(xq, routing, gpu, k, B.MOE_FFN_ACCUMULATE, B.MOE_PATH_DECODE, T, d)
+    _, _, y_r = _oracle_outputs(xq, routing, experts, sh, T, d, k)
+    assert_close_layer(o_g, y_r, "y_acc")
+    assert_close_layer(bits_to_f32(y_g), y_r, "y bf16")
+
+
+def test_ffn_decode_path_repeated_calls_and_unsupported():
+    """The decode path leaves its workspace ready for the next call (same result twice), and
+    rejects what it does not cover instead of falling back."""
+    experts, sh, xq, routing, gpu = _tiny_case(14, 512, 16, 4, 128, 6, True, pack=True)
+    _, _, y1 = _run_ffn(xq, routing, gpu, 4, B.MOE_FFN_ACCUMULATE, B.MOE_PATH_DECODE, 6, 512)
+    _, _, y2 = _run_ffn(xq, routing, gpu, 4, B.MOE_FFN_ACCUMULATE, B.MOE_PATH_DECODE, 6, 512)
+    assert np.allclose(bits_to_f32(y1), bits_to_f32(y2), rtol=1e-2, atol=1e-3)
+    with pytest.raises(B.MoeError):
+        _run_ffn(xq, routing, gpu, 4, B.MOE_FFN_PER_ASSIGN, B.MOE_PATH_DECODE, 6, 512)
+
+
 @pytest.fixture(scope="module")
 def decode_layer():
     cfg = synth.CONFIGS["decode"]
@@ -133,7 +160,7 @@ def decode_layer():
     return cfg, B.Experts(routed, shared), OracleWeights(0, cfg)
 
 
-@pytest.mark.parametrize("path", [B.MOE_PATH_DECODE, B.MOE_PATH_PREFILL])
+@pytest.mark.parametrize("path", [B.MOE_PATH_DECODE, B.MOE_PATH_PREFILL, B.MOE_PATH_CUDA_CORE])
 @pytest.mark.parametrize("T", [1, 4, 8])
 def test_ffn_decode_config_full_size(decode_layer, T, path):
     cfg, gpu, ow = decode_layer
