@@ -80,6 +80,9 @@ typedef enum moe_status {
  *   dn_ts     [E]            float32
  *   gu_sf_tiled, dn_sf_tiled: the same scale bytes re-tiled for the tensor-core path by
  *            moe_pack_experts (NULL if not packed; the PREFILL path then refuses).
+ *   dn_codes_slice [E][I/64][d][32], dn_sf_slice [E][I/64][d/128][512]: the down matrix
+ *            regrouped by 64-column slices of I (each slice's codes, and its scale atoms,
+ *            contiguous), written by moe_pack_experts for the DECODE path (NULL if absent).
  */
 typedef struct moe_expert_weights {
   int32_t E, d, I;
@@ -91,6 +94,8 @@ typedef struct moe_expert_weights {
   const float* dn_ts;
   const uint8_t* gu_sf_tiled;
   const uint8_t* dn_sf_tiled;
+  const uint8_t* dn_codes_slice;
+  const uint8_t* dn_sf_slice;
 } moe_expert_weights_t;
 
 typedef struct moe_experts {
@@ -137,15 +142,21 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
                        int32_t* assign_pos, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * moe_pack_experts - re-tile the E4M3 scale bytes of an expert group for the tensor-core
- * path: 512-byte atoms of 128 weight rows x 4 scale blocks, the layout the tensor core
- * reads its scales in. gu_sf_tiled needs E*2I*d/16 bytes, dn_sf_tiled E*d*I/16 bytes
- * (caller-owned, set in W->gu_sf_tiled / dn_sf_tiled afterwards). Run once per weight
- * load; the codes and the natural-layout scales stay as they are and remain in use by the
- * CUDA-core path. Requires d % 128 == 0 and I % 64 == 0.
+ * moe_pack_experts - derived layouts of an expert group for the tensor-core paths, written
+ * once per weight load into caller-owned buffers (set them in W afterwards):
+ *   gu_sf_tiled (E*2I*d/16 bytes), dn_sf_tiled (E*d*I/16 bytes): the E4M3 scale bytes in
+ *     512-byte atoms of 128 weight rows x 4 scale blocks, the layout the tensor core reads
+ *     its scales in (gate/up atoms [E][I/64][d/64], atom rows 0-63 gate, 64-127 up; down
+ *     atoms [E][d/128][I/64]);
+ *   dn_codes_slice (E*d*I/2 bytes), dn_sf_slice (E*d*I/16 bytes), both optional (NULL to
+ *     skip): the down codes and scale atoms regrouped per 64-column slice of I, so that
+ *     the DECODE path reads each slice as contiguous bytes.
+ * The natural-layout arrays stay as they are and remain in use by the CUDA-core path.
+ * Requires d % 128 == 0 and I % 64 == 0.
  */
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
-                            uint8_t* dn_sf_tiled, void* stream);
+                            uint8_t* dn_sf_tiled, uint8_t* dn_codes_slice, uint8_t* dn_sf_slice,
+                            void* stream);
 
 /*
  * moe_expert_ffn - expert SwiGLU FFN for all routed assignments (A5-A7) and the shared
@@ -160,7 +171,7 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
  *   path: MOE_PATH_DECODE = tcgen05 kernel for at most 8 tokens, one CTA per (expert,
  *        64-column slice of I) computing gate/up, SwiGLU, h and that slice's share of
  *        the down projection (needs T <= 8, MOE_FFN_ACCUMULATE, d % 512 == 0,
- *        I % 64 == 0 and both groups packed by moe_pack_experts);
+ *        I % 64 == 0 and both groups packed by moe_pack_experts, slices included);
  *        MOE_PATH_PREFILL = tcgen05 block-scaled grouped GEMMs over 128-token tiles
  *        (any T; needs d % 256 == 0, I % 256 == 0 and packed scales);
  *        MOE_PATH_CUDA_CORE = the CUDA-core kernel on the natural layout (d % 16 == 0,

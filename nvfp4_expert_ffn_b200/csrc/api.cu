@@ -97,8 +97,8 @@ moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E,
 }
 
 ExpertGroup to_group(const moe_expert_weights_t& w) {
-  return ExpertGroup{w.gu_codes, w.gu_scales, w.gu_ts, w.dn_codes, w.dn_scales, w.dn_ts,
-                     w.gu_sf_tiled, w.dn_sf_tiled};
+  return ExpertGroup{w.gu_codes,    w.gu_scales,   w.gu_ts,          w.dn_codes,      w.dn_scales,
+                     w.dn_ts,       w.gu_sf_tiled, w.dn_sf_tiled, w.dn_codes_slice, w.dn_sf_slice};
 }
 
 }  // namespace
@@ -224,8 +224,14 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t d, const float* Wr, c
 }
 
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
-                            uint8_t* dn_sf_tiled, void* stream) {
+                            uint8_t* dn_sf_tiled, uint8_t* dn_codes_slice, uint8_t* dn_sf_slice,
+                            void* stream) {
   if (!W || !gu_sf_tiled || !dn_sf_tiled) return fail(MOE_ERR_INVALID_ARG, "null argument");
+  if ((dn_codes_slice == nullptr) != (dn_sf_slice == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "dn_codes_slice and dn_sf_slice are given together");
+  if ((dn_codes_slice && !aligned16(dn_codes_slice)) || (dn_sf_slice && !aligned16(dn_sf_slice)) ||
+      (dn_codes_slice && (!W->dn_codes || !aligned16(W->dn_codes))))
+    return fail(MOE_ERR_INVALID_ARG, "slice buffers and dn_codes must be 16-byte aligned");
   if (W->E < 1 || W->d <= 0 || W->I <= 0) return fail(MOE_ERR_INVALID_ARG, "bad E/d/I");
   if (W->d % 128 || W->I % 64) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "packing needs d % 128 == 0 and I % 64 == 0");
   if (!W->gu_scales || !W->dn_scales) return fail(MOE_ERR_INVALID_ARG, "null scales");
@@ -236,6 +242,8 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
   if (s != MOE_OK) return s;
   cudaError_t e = launch_pack_sf(to_group(*W), W->E, W->d, W->I, gu_sf_tiled, dn_sf_tiled, sms,
                                  (cudaStream_t)stream);
+  if (e == cudaSuccess && dn_codes_slice)
+    e = launch_pack_slices(to_group(*W), W->E, W->d, W->I, dn_codes_slice, dn_sf_slice, sms, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_pack_experts launch");
 }
 
@@ -268,13 +276,15 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
   const bool tc_ok = ffn_tc_supported(d, I) && packed;
-  const bool dec_ok = ffn_dec_supported(T, d, I, mode) && packed;
+  const bool sliced = W->routed.dn_codes_slice && W->routed.dn_sf_slice &&
+                      (!W->has_shared || (W->shared.dn_codes_slice && W->shared.dn_sf_slice));
+  const bool dec_ok = ffn_dec_supported(T, d, I, mode) && packed && sliced;
   if (path == MOE_PATH_PREFILL && !tc_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "tensor-core path needs d % 256 == 0, I % 256 == 0 and scales packed by moe_pack_experts");
   if (path == MOE_PATH_DECODE && !dec_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
-                "decode path needs T <= 8, ACCUMULATE mode, d % 512 == 0, I % 64 == 0 and packed scales");
+                "decode path needs T <= 8, ACCUMULATE mode, d % 512 == 0, I % 64 == 0 and packed scales and slices");
   const int kind = path == MOE_PATH_AUTO ? (dec_ok ? MOE_PATH_DECODE : tc_ok ? MOE_PATH_PREFILL : MOE_PATH_CUDA_CORE)
                                          : path;
   const size_t need = kind == MOE_PATH_DECODE    ? ffn_dec_ws_bytes(E)

@@ -23,7 +23,10 @@
 //   * the ring of shared-memory stages therefore carries only weights: one stage is either
 //     a 64-gate + 64-up row x 256-column tile of the stacked gate/up matrix (TMA, 128-byte
 //     swizzle) or four 128-row x 64-column tiles of the down matrix (TMA, 32-byte swizzle),
-//     each with its pre-tiled scale atoms (bulk copies).
+//     each with its scale atoms (one bulk copy). The down tiles come from the slice-grouped
+//     copy of the down matrix (moe_pack_experts), where a slice's 32-byte rows are
+//     contiguous: read from the natural layout, each row's 32 bytes sit 256 bytes apart and
+//     the stream runs at about half the HBM bandwidth.
 //
 // Warp roles (320 threads, one CTA per SM): warp 0 lane 0 issues the copies; warp 1 owns
 // TMEM and lane 0 issues tcgen05.cp / tcgen05.mma; warps 2-9 run the epilogue. The MMA
@@ -79,48 +82,48 @@ struct DecParams {
 
 struct DecMaps {
   CUtensorMap b1, b1s;  // gate/up codes {d/2, I, 2, E}, boxes {128, 64, 2, 1}, 128-byte swizzle
-  CUtensorMap b2, b2s;  // down codes {I/2, d, E}, boxes {32, 128, 1}, 32-byte swizzle
+  CUtensorMap b2, b2s;  // down codes by I-slice {32, 128, d/128, E*I/64}, boxes {32, 128, 4, 1}, 32-byte swizzle
 };
 
 // ---------------------------------------------------------------- preparation (one CTA)
+// One pass over the experts (E <= 1024 = blockDim) lists those in use after the shared
+// expert; then one thread per routed assignment writes its token's weight into its
+// expert's row of slot_w (rows cleared first).
 __global__ void __launch_bounds__(1024) ffn_dec_prep_kernel(DecParams p) {
   MOE_PDL_PROLOGUE();
   __shared__ int tmp[32];
-  __shared__ int carry;
+  __shared__ int s_off[1025];
+  __shared__ int s_slot[1024];
   const size_t n4 = (size_t)p.T * p.d / 4;
   float4* y4 = reinterpret_cast<float4*>(p.out);
   for (size_t i = threadIdx.x; i < n4; i += blockDim.x) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (threadIdx.x == 0) carry = p.has_shared;
-  if (p.has_shared && threadIdx.x < kDecMaxT) {
-    if (threadIdx.x == 0) p.slots[0] = p.E;
-    p.slot_w[threadIdx.x] = threadIdx.x < p.T ? 1.0f : 0.0f;
-  }
+  for (int e = threadIdx.x; e <= p.E; e += blockDim.x) s_off[e] = p.offsets[e];
   __syncthreads();
-  for (int e0 = 0; e0 < p.E; e0 += blockDim.x) {
-    const int e = e0 + threadIdx.x;
-    const int beg = e < p.E ? p.offsets[e] : 0, end = e < p.E ? p.offsets[e + 1] : 0;
-    int total;
-    const int slot = block_exclusive_scan(end > beg ? 1 : 0, tmp, &total) + carry;
-    if (end > beg) {
-      p.slots[slot] = e;
-      float w[kDecMaxT];
-#pragma unroll
-      for (int t = 0; t < kDecMaxT; ++t) w[t] = 0.0f;
-      for (int q = beg; q < end; ++q) {
-        const int a = p.sorted_assign[q];
-        const int t = a / p.k;
-#pragma unroll
-        for (int tt = 0; tt < kDecMaxT; ++tt)
-          if (tt == t) w[tt] = p.topk_w[a];
-      }
-#pragma unroll
-      for (int t = 0; t < kDecMaxT; ++t) p.slot_w[(size_t)slot * kDecMaxT + t] = w[t];
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) carry += total;
-    __syncthreads();
+  const int e = threadIdx.x;
+  const bool active = e < p.E && s_off[e + 1] > s_off[e];
+  int total;
+  const int slot = block_exclusive_scan(active ? 1 : 0, tmp, &total) + p.has_shared;
+  if (e < p.E) s_slot[e] = active ? slot : -1;
+  if (active) p.slots[slot] = e;
+  const int nslots = total + p.has_shared;
+  if (threadIdx.x == 0) {
+    *p.nslots = nslots;
+    if (p.has_shared) p.slots[0] = p.E;
   }
-  if (threadIdx.x == 0) *p.nslots = carry;
+  for (int i = threadIdx.x; i < nslots * kDecMaxT; i += blockDim.x)
+    p.slot_w[i] = (p.has_shared && i < kDecMaxT && i < p.T) ? 1.0f : 0.0f;
+  __syncthreads();
+  const int n = p.T * p.k;
+  for (int q = threadIdx.x; q < n; q += blockDim.x) {
+    int lo = 0, hi = p.E - 1;  // the expert e with s_off[e] <= q < s_off[e + 1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= q) lo = mid;
+      else hi = mid - 1;
+    }
+    const int a = p.sorted_assign[q];
+    p.slot_w[(size_t)s_slot[lo] * kDecMaxT + a / p.k] = p.topk_w[a];
+  }
 }
 
 // ---------------------------------------------------------------- the FFN kernel
@@ -205,6 +208,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
     j = ug % nt1;
     e = p.slots[slot];
   };
+  // Gate/up K blocks are visited in an order rotated per CTA and unit: CTAs that start
+  // together then read different 128-byte columns of their 1 KB weight rows at any moment,
+  // instead of all reading the same column (which loads a fraction of the HBM channels).
+  auto unit_rot = [&](int u) { return (int)((blockIdx.x + 3 * u) % nks1); };
   if (threadIdx.x == 0) TC_TRACE_AT(g_dec_trace, kEvSetupDone, nu);
 
   if (warp == 0) {
@@ -220,6 +227,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
         const int el = sh ? 0 : e;
         const ExpertGroup& G = sh ? p.shared : p.routed;
         TC_TRACE_AT(g_dec_trace, kEvProdTile, u);
+        const int rot = unit_rot(u);
         for (int q = 0; q < nks1 + nks2; ++q, ++it) {
           const int st = (int)(it % (uint32_t)NST);
           if (!mbar_wait(&empty[st], ((it / NST) & 1) ^ 1, &s_abort, p.status)) {
@@ -230,18 +238,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
           if (it < 40) TC_TRACE_AT(g_dec_trace, kEvProdIssue, it);
           mbar_arrive_expect_tx(&full[st], kDecStageBytes);
           if (q < nks1) {
-            tma_load_4d(sb, sh ? &maps.b1s : &maps.b1, &full[st], q * 128, 64 * j, 0, el);
-            bulk_g2s(sb + kDecBBytes, G.gu_sf_tiled + (((size_t)el * nt1 + j) * (d / 64) + 4 * q) * kDecAtom,
+            const int kq = (q + rot) % nks1;  // K block of this stage
+            tma_load_4d(sb, sh ? &maps.b1s : &maps.b1, &full[st], kq * 128, 64 * j, 0, el);
+            bulk_g2s(sb + kDecBBytes, G.gu_sf_tiled + (((size_t)el * nt1 + j) * (d / 64) + 4 * kq) * kDecAtom,
                      4 * kDecAtom, &full[st]);
           } else {
+            // four 128-row chunks of slice j (16 KB contiguous) and their scale atoms (2 KB)
             const int q2 = q - nks1;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int c = 4 * q2 + i;
-              tma_load_3d(sb + 4096 * i, sh ? &maps.b2s : &maps.b2, &full[st], 32 * j, 128 * c, el);
-              bulk_g2s(sb + kDecBBytes + kDecAtom * i,
-                       G.dn_sf_tiled + (((size_t)el * nch + c) * (I / 64) + j) * kDecAtom, kDecAtom, &full[st]);
-            }
+            tma_load_4d(sb, sh ? &maps.b2s : &maps.b2, &full[st], 0, 0, 4 * q2, el * nt1 + j);
+            bulk_g2s(sb + kDecBBytes, G.dn_sf_slice + (((size_t)el * nt1 + j) * nch + 4 * q2) * kDecAtom,
+                     4 * kDecAtom, &full[st]);
           }
         }
       }
@@ -274,7 +280,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
         // gate/up of unit u into D1: tokens (broadcast 8-row A) x 64 gate + 64 up rows
         if (!mbar_wait(&acc1_empty, (u & 1) ^ 1, &s_abort, p.status)) break;
         tc_fence_after();
+        const int rot = unit_rot(u);
         for (int q = 0; q < nks1; ++q, ++it) {
+          const int kq = (q + rot) % nks1;  // K block of this stage
           if (!stage_in(it)) {
             ok = false;
             break;
@@ -284,12 +292,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
           const uint32_t sf = tmem + kColSf + 32 * (it % kDecSfSlots);
 #pragma unroll
           for (int kc = 0; kc < 4; ++kc) {
-            tmem_cp_sf(sf + 4 * kc, sdesc_sf(smem_u32(xsf + (size_t)(4 * q + kc) * kDecAtom)));
+            tmem_cp_sf(sf + 4 * kc, sdesc_sf(smem_u32(xsf + (size_t)(4 * kq + kc) * kDecAtom)));
             tmem_cp_sf(sf + 16 + 4 * kc, sdesc_sf(smem_u32(sb + kDecBBytes + kc * kDecAtom)));
           }
+          if (it < 40) TC_TRACE_AT(g_dec_trace, kEvMmaCps, it);
 #pragma unroll
           for (int kc = 0; kc < 4; ++kc)
-            mma_mxf4nvf4(tmem + kColD1, sdesc_kmajor(smem_u32(xs + q * 1024 + 32 * kc), 0, kSwizzle128B),
+            mma_mxf4nvf4(tmem + kColD1, sdesc_kmajor(smem_u32(xs + kq * 1024 + 32 * kc), 0, kSwizzle128B),
                          sdesc_kmajor(smem_u32(sb + 32 * kc), 1024, kSwizzle128B), kDecIdesc, sf + 4 * kc,
                          sf + 16 + 4 * kc, (q | kc) ? 1u : 0u);
           mma_commit(&empty[it % NST]);
@@ -525,10 +534,10 @@ cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* sta
     cuuint64_t str1[3] = {(cuuint64_t)(d / 2), (cuuint64_t)I * (d / 2), (cuuint64_t)2 * I * (d / 2)};
     cuuint32_t box1[4] = {128, 64, 2, 1};
     if ((e = encode_u8(m1, g.gu_codes, 4, dims1, str1, box1, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
-    cuuint64_t dims2[3] = {(cuuint64_t)(I / 2), (cuuint64_t)d, (cuuint64_t)E};
-    cuuint64_t str2[2] = {(cuuint64_t)(I / 2), (cuuint64_t)d * (I / 2)};
-    cuuint32_t box2[3] = {32, 128, 1};
-    if ((e = encode_u8(m2, g.dn_codes, 3, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
+    cuuint64_t dims2[4] = {32, 128, (cuuint64_t)(d / 128), (cuuint64_t)E * (I / 64)};
+    cuuint64_t str2[3] = {32, 128 * 32, (cuuint64_t)d * 32};
+    cuuint32_t box2[4] = {32, 128, 4, 1};
+    if ((e = encode_u8(m2, g.dn_codes_slice, 4, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess) return e;
   }
   if ((e = launch_pdl(ffn_dec_prep_kernel, dim3(1), dim3(1024), 0, st, p)) != cudaSuccess) return e;
   return launch_pdl(ffn_dec_kernel, dim3(num_sms), dim3(kDecThreads), dec_smem_bytes(d), st, maps, p);

@@ -46,6 +46,8 @@ struct ExpertGroup {
   const float* dn_ts;
   const uint8_t* gu_sf_tiled;
   const uint8_t* dn_sf_tiled;
+  const uint8_t* dn_codes_slice;  // [E][I/64][d][32]
+  const uint8_t* dn_sf_slice;     // [E][I/64][d/128][512]
 };
 
 struct FfnArgs {
@@ -100,6 +102,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
 bool ffn_dec_supported(int64_t T, int d, int I, int mode);
 size_t ffn_dec_ws_bytes(int E);
 cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
+cudaError_t launch_pack_slices(const ExpertGroup& g, int E, int d, int I, uint8_t* dn_codes_slice,
+                               uint8_t* dn_sf_slice, int num_sms, cudaStream_t st);
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
                            int num_sms, cudaStream_t st);
 

@@ -505,8 +505,9 @@ cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const
   const size_t logits_bytes = ((size_t)T * E * sizeof(float) + 255) & ~(size_t)255;
   void* perm_ws = reinterpret_cast<char*>(ws) + logits_bytes;
   if (T <= kGemvMaxT) {
-    const int grid = (E + 7) / 8;  // 8 warps (experts) per CTA
-    cudaError_t e0 = launch_pdl(router_gemv_kernel, dim3(grid), dim3(256), (size_t)T * d * sizeof(uint16_t), st,
+    // 4 warps (one expert row each) per CTA: E = 512 spreads the router matrix over 128 SMs
+    const int grid = (E + 3) / 4;
+    cudaError_t e0 = launch_pdl(router_gemv_kernel, dim3(grid), dim3(128), (size_t)T * d * sizeof(uint16_t), st,
                                 x, T, d, Wr, br, E, logits);
     if (e0 != cudaSuccess) return e0;
   } else {

@@ -27,6 +27,7 @@ enum TraceEvent : uint32_t {
   kEvMmaFull = 13,    // MMA issuer: stage `tile` landed
   kEvMmaSlot = 14,    // MMA issuer: its scale slot is free
   kEvMmaIssued = 15,  // MMA issuer: the stage's MMAs are issued
+  kEvMmaCps = 16,     // MMA issuer: the stage's scale-factor copies are issued
 };
 
 constexpr int kTraceCtas = 160, kTraceCap = 254;
