@@ -276,7 +276,7 @@ def run_gpu(args):
     achieved = ffn_bytes / (ffn_ms * 1e-3) / 1e9
     ffn_flops = 2.0 * T * (cfg.k + 1) * 3 * cfg.d * cfg.I
     if args.workload == "decode":
-        roof = {"kernel": "moe_expert_ffn (schedule + gather + tcgen05 FFN)", "bound": "hbm",
+        roof = {"kernel": "moe_expert_ffn (decode: preparation + tcgen05 split-I kernel)", "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
                 "bytes_per_launch": int(ffn_bytes), "avg_launch_us": round(ffn_ms * 1e3, 3),
@@ -284,7 +284,7 @@ def run_gpu(args):
     else:
         fp4_peak = bf16_peak * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio 9 / 2.25)
         tf = ffn_flops / (ffn_ms * 1e-3) / 1e12
-        roof = {"kernel": "moe_expert_ffn (schedule + gather + tcgen05 FFN)", "bound": "tensor",
+        roof = {"kernel": "moe_expert_ffn (schedule + row gather + tcgen05 grouped GEMMs)", "bound": "tensor",
                 "achieved": round(tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                 "frac": round(tf / fp4_peak, 4),
                 "peak_kind": f"{peak_kind} bf16 x 4 (nominal fp4/bf16 ratio)",

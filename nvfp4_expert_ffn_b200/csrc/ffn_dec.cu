@@ -45,7 +45,7 @@
 namespace moe {
 
 constexpr int kDecMaxT = 8;
-constexpr int kDecThreads = 320;
+constexpr int kDecThreads = 352;  // producer, two MMA issuers, 8 epilogue warps
 constexpr int kDecEpiWarps = 8;
 constexpr int kDecMaxStages = 12;
 constexpr int kDecMinStages = 4;
@@ -53,11 +53,8 @@ constexpr int kDecAtom = 512;                          // scale atom: 128 rows x
 constexpr int kDecBBytes = 16384;                      // weight bytes of one stage
 constexpr int kDecStageBytes = kDecBBytes + 4 * kDecAtom;
 constexpr int kDecSfSlots = 4;
-constexpr uint32_t kDecIdesc = idesc_mxf4nvf4(128, 128);  // gate/up: 128 token rows x 128 weight rows
-constexpr int kDecDnN = 16;                                 // down: 128 output rows x 16 token columns
-constexpr uint32_t kDecIdescDn = idesc_mxf4nvf4(128, kDecDnN);
-constexpr int kDecGroupChunks = 16;                         // 128-row down chunks per accumulator group
-constexpr uint32_t kColD1 = 0, kColD2 = 128, kColSf = 384;
+constexpr int kDecDnN = 16;                                // 16 token columns (8 tokens read twice)
+constexpr uint32_t kDecIdescT = idesc_mxf4nvf4(128, kDecDnN);  // 128 weight rows x 16 token columns
 constexpr int kDecHBytes = 1024;                       // h codes (8 rows x 32 B) + its atom at +512
 
 TC_TRACE_ARRAY(g_dec_trace)
@@ -73,6 +70,7 @@ struct DecParams {
   int has_shared;
   int E, d, I, T, k;
   int nstages;
+  int group_chunks;    // down chunks accumulated in TMEM at a time
   float* out;          // y [T][d] float32
   int32_t* nslots;     // workspace: experts in use (shared expert included)
   int32_t* slots;      // [E + 1] expert ids (E = the shared expert)
@@ -89,8 +87,12 @@ struct DecMaps {
 // One pass over the experts (E <= 1024 = blockDim) lists those in use after the shared
 // expert; then one thread per routed assignment writes its token's weight into its
 // expert's row of slot_w (rows cleared first).
+RT_TRACE_ARRAY(g_prep_trace)
+
 __global__ void __launch_bounds__(1024) ffn_dec_prep_kernel(DecParams p) {
+  RT_TRACE(g_prep_trace, 0, 0);
   MOE_PDL_PROLOGUE();
+  RT_TRACE(g_prep_trace, 0, 1);
   __shared__ int tmp[32];
   __shared__ int s_off[1025];
   __shared__ int s_slot[1024];
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(1024) ffn_dec_prep_kernel(DecParams p) {
     const int a = p.sorted_assign[q];
     p.slot_w[(size_t)s_slot[lo] * kDecMaxT + a / p.k] = p.topk_w[a];
   }
+  RT_TRACE(g_prep_trace, 0, 2);
 }
 
 // ---------------------------------------------------------------- the FFN kernel
@@ -131,13 +134,19 @@ MOE_DEV uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~(uintptr_t)1023);
 }
 
+// TMEM columns (512 allocated): gate/up accumulators of the two MMA issuers, h scale slots
+// (per issuer, per unit parity), the weight-scale ring, the resident activation scales
+// (d/16 columns), then the down accumulators (16 columns per 128-row chunk).
+constexpr uint32_t kColD1 = 0, kColH = 32, kColSf = 48, kColX = 112;
+__host__ __device__ inline uint32_t dec_col_d2(int d) { return (kColX + (uint32_t)d / 16 + 15u) & ~15u; }
+
 __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_constant__ DecMaps maps, DecParams p) {
   TC_TRACE_DECL
   TC_TRACE_BEGIN(g_dec_trace);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   __shared__ uint64_t full[kDecMaxStages], empty[kDecMaxStages];
-  __shared__ uint64_t acc1_full, acc1_empty, h_full[2], acc2_full, acc2_empty, final_bar;
+  __shared__ uint64_t xsf_ready, acc1_full, acc1_empty, h_full[2], acc2_full, acc2_empty, final_bar;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_go;
@@ -148,11 +157,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
   const int nks1 = d / 256;  // gate/up stages per unit
   const int nch = d / 128;   // down chunks per unit
   const int nks2 = nch / 4;  // down stages per unit
+  const int gch = p.group_chunks;  // down chunks accumulated in TMEM at a time (multiple of 4)
+  const int gst = gch / 4;         // down stages per group
+  const uint32_t col_d2 = dec_col_d2(d);
 
   uint8_t* ring = smem;                                    // NST x 18 KB
   uint8_t* xs = ring + (size_t)NST * kDecStageBytes;       // [d/256][8 rows x 128 B], swizzled
   uint8_t* xsf = xs + (size_t)nks1 * 1024;                 // [d/64] scale atoms of x
-  uint8_t* hb = xsf + (size_t)(d / 64) * kDecAtom;         // [2] h buffers
+  uint8_t* hb = xsf + (size_t)(d / 64) * kDecAtom;         // [2] h tiles (codes + scale atom)
+  float* s_gu = reinterpret_cast<float*>(hb + 2 * kDecHBytes);  // [128][8] gate/up sums of a unit
 
   // setup, overlapping the previous kernel's tail
   if (threadIdx.x == 0) {
@@ -160,13 +173,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(&acc1_full, 1);
+    mbar_init(&xsf_ready, 2);
+    mbar_init(&acc1_full, 2);
     mbar_init(&acc1_empty, kDecEpiWarps);
     mbar_init(&h_full[0], 1);
     mbar_init(&h_full[1], 1);
-    mbar_init(&acc2_full, 1);
+    mbar_init(&acc2_full, 2);
     mbar_init(&acc2_empty, kDecEpiWarps);
-    mbar_init(&final_bar, 1);
+    mbar_init(&final_bar, 2);
     fence_barrier_init();
     s_abort = 0;
     prefetch_tensormap(&maps.b1);
@@ -177,7 +191,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
     }
   }
   if (warp == 1) tmem_alloc(&s_tmem, 512);
+  RT_TRACE(g_prep_trace, 1, 0);
   MOE_PDL_PROLOGUE();
+  RT_TRACE(g_prep_trace, 1, 1);
 
   // x codes -> 8-row 128-byte-swizzled tiles (rows >= T are zero); chunk c of a row goes to
   // 16-byte slot c ^ row within its 128-byte line
@@ -208,27 +224,37 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
     j = ug % nt1;
     e = p.slots[slot];
   };
-  // Gate/up K blocks are visited in an order rotated per CTA and unit: CTAs that start
-  // together then read different 128-byte columns of their 1 KB weight rows at any moment,
-  // instead of all reading the same column (which loads a fraction of the HBM channels).
+  // Gate/up K blocks are visited in an order rotated per CTA and unit (the sum does not
+  // depend on the order).
   auto unit_rot = [&](int u) { return (int)((blockIdx.x + 3 * u) % nks1); };
+  // job jb of 2*nu: gu(0), then pairs (gu(s), dn(s-1)) for s = 1..nu-1, then dn(nu-1), so the
+  // SwiGLU of unit s overlaps the gate/up product of unit s+1
+  auto job_is_gu = [&](int jb) { return jb == 0 || (jb < 2 * nu - 1 && (jb & 1)); };
+  auto job_unit = [&](int jb) {
+    if (jb == 0) return 0;
+    if (jb == 2 * nu - 1) return nu - 1;
+    return (jb & 1) ? (jb + 1) / 2 : jb / 2 - 1;
+  };
   if (threadIdx.x == 0) TC_TRACE_AT(g_dec_trace, kEvSetupDone, nu);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    // per unit: nks1 gate/up stages, then nks2 down stages (the order the MMA consumes them)
+    // jobs in the order the MMAs consume them: gu(0), gu(1), dn(0), gu(2), dn(1), ..., dn(n-1)
     if (lane == 0) {
       uint32_t it = 0;
       bool alive = true;
-      for (int u = 0; u < nu && alive; ++u) {
+      for (int jb = 0; jb < 2 * nu && alive; ++jb) {
+        const bool gu = job_is_gu(jb);
+        const int u = job_unit(jb);
         int slot, e, j;
         unit(u, slot, e, j);
         const bool sh = e == p.E;
         const int el = sh ? 0 : e;
         const ExpertGroup& G = sh ? p.shared : p.routed;
-        TC_TRACE_AT(g_dec_trace, kEvProdTile, u);
+        if (gu) TC_TRACE_AT(g_dec_trace, kEvProdTile, u);
         const int rot = unit_rot(u);
-        for (int q = 0; q < nks1 + nks2; ++q, ++it) {
+        const int q0 = gu ? 0 : nks1, q1 = gu ? nks1 : nks1 + nks2;
+        for (int q = q0; q < q1; ++q, ++it) {
           const int st = (int)(it % (uint32_t)NST);
           if (!mbar_wait(&empty[st], ((it / NST) & 1) ^ 1, &s_abort, p.status)) {
             alive = false;
@@ -258,13 +284,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------------ MMA issuers
+    // Two threads issue tcgen05 work, each for the ring stages of its parity: issuing a
+    // scale copy or an MMA takes tens of nanoseconds, and one thread alone would pace the
+    // weight stream. Gate/up is computed transposed, D1[weight row][token] (weights are the
+    // 128-row A operand, the tokens a 16-column B operand whose two 8-row groups both read
+    // the 8 tokens), each issuer into its own 16 columns; the epilogue adds the two.
+    const int who = warp - 1;
     if (lane == 0) {
+      // the activation scale atoms stay in TMEM for the whole kernel (each issuer copies
+      // half of them; both wait for all)
+      for (int a = who; a < d / 64; a += 2) tmem_cp_sf(tmem + kColX + 4 * a, sdesc_sf(smem_u32(xsf + (size_t)a * kDecAtom)));
+      mma_commit(&xsf_ready);
+      bool ok = mbar_wait(&xsf_ready, 0, &s_abort, p.status);
+      tc_fence_after();
       uint32_t it = 0, gc = 0;
-      bool ok = true;
-      // stage `itx` has landed and the scale slot it reuses (last used by stage itx - 4)
-      // is no longer read by an MMA in flight
+      // stage `itx` has landed and the scale slot it reuses (last used by stage itx - 4, of
+      // the same issuer) is no longer read by an MMA in flight
       auto stage_in = [&](uint32_t itx) -> bool {
         if (!mbar_wait(&full[itx % NST], (itx / NST) & 1, &s_abort, p.status)) return false;
         if (itx < 40) TC_TRACE_AT(g_dec_trace, kEvMmaFull, itx);
@@ -272,79 +309,85 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
           const uint32_t pv = itx - kDecSfSlots;
           if (!mbar_wait(&empty[pv % NST], (pv / NST) & 1, &s_abort, p.status)) return false;
         }
-        if (itx < 40) TC_TRACE_AT(g_dec_trace, kEvMmaSlot, itx);
         tc_fence_after();
         return true;
       };
-      for (int u = 0; u < nu && ok; ++u) {
-        // gate/up of unit u into D1: tokens (broadcast 8-row A) x 64 gate + 64 up rows
+      const uint32_t d1 = tmem + kColD1 + 16 * who;
+      for (int jb = 0; jb < 2 * nu && ok; ++jb) {
+        const int u = job_unit(jb);
+        if (job_is_gu(jb)) {
         if (!mbar_wait(&acc1_empty, (u & 1) ^ 1, &s_abort, p.status)) break;
         tc_fence_after();
         const int rot = unit_rot(u);
+        bool first = true;
         for (int q = 0; q < nks1; ++q, ++it) {
-          const int kq = (q + rot) % nks1;  // K block of this stage
+          if ((int)(it & 1) != who) continue;
           if (!stage_in(it)) {
             ok = false;
             break;
           }
-          if (q == 0) TC_TRACE_AT(g_dec_trace, kEvMmaFirst, u);
+          if (who == 0 && first) TC_TRACE_AT(g_dec_trace, kEvMmaFirst, u);
+          const int kq = (q + rot) % nks1;
           const uint8_t* sb = ring + (size_t)(it % NST) * kDecStageBytes;
-          const uint32_t sf = tmem + kColSf + 32 * (it % kDecSfSlots);
+          const uint32_t sf = tmem + kColSf + 16 * (it % kDecSfSlots);
 #pragma unroll
-          for (int kc = 0; kc < 4; ++kc) {
-            tmem_cp_sf(sf + 4 * kc, sdesc_sf(smem_u32(xsf + (size_t)(4 * kq + kc) * kDecAtom)));
-            tmem_cp_sf(sf + 16 + 4 * kc, sdesc_sf(smem_u32(sb + kDecBBytes + kc * kDecAtom)));
-          }
+          for (int kc = 0; kc < 4; ++kc) tmem_cp_sf(sf + 4 * kc, sdesc_sf(smem_u32(sb + kDecBBytes + kc * kDecAtom)));
           if (it < 40) TC_TRACE_AT(g_dec_trace, kEvMmaCps, it);
 #pragma unroll
           for (int kc = 0; kc < 4; ++kc)
-            mma_mxf4nvf4(tmem + kColD1, sdesc_kmajor(smem_u32(xs + kq * 1024 + 32 * kc), 0, kSwizzle128B),
-                         sdesc_kmajor(smem_u32(sb + 32 * kc), 1024, kSwizzle128B), kDecIdesc, sf + 4 * kc,
-                         sf + 16 + 4 * kc, (q | kc) ? 1u : 0u);
+            mma_mxf4nvf4(d1, sdesc_kmajor(smem_u32(sb + 32 * kc), 1024, kSwizzle128B),
+                         sdesc_kmajor(smem_u32(xs + kq * 1024 + 32 * kc), 0, kSwizzle128B), kDecIdescT, sf + 4 * kc,
+                         tmem + kColX + 4 * (4 * kq + kc), (!first || kc) ? 1u : 0u);
+          first = false;
           mma_commit(&empty[it % NST]);
           if (it < 40) TC_TRACE_AT(g_dec_trace, kEvMmaIssued, it);
         }
         if (!ok) break;
-        TC_TRACE_AT(g_dec_trace, kEvMmaLast, u);
+        if (who == 0) TC_TRACE_AT(g_dec_trace, kEvMmaLast, u);
         mma_commit(&acc1_full);
+        continue;
+        }
         // down projection of unit u, transposed: D2[output row][token] = Wd chunk x h^T, one
-        // 16-column accumulator per 128-row chunk, up to 16 chunks (one group) at a time
+        // 16-column accumulator per 128-row chunk, gch chunks (one group) at a time
         const uint8_t* hbuf = hb + (u & 1) * kDecHBytes;
         if (!mbar_wait(&h_full[u & 1], (u >> 1) & 1, &s_abort, p.status)) break;
         tc_fence_after();
+        const uint32_t hsf = tmem + kColH + 8 * who + 4 * (u & 1);
+        tmem_cp_sf(hsf, sdesc_sf(smem_u32(hbuf + 512)));
         for (int q = 0; q < nks2; ++q, ++it) {
-          if (q % 4 == 0) {  // a new group: the epilogue has read the previous one
+          if (q % gst == 0) {  // a new group: the epilogue has read the previous one
             if (!mbar_wait(&acc2_empty, (gc & 1) ^ 1, &s_abort, p.status)) {
               ok = false;
               break;
             }
             tc_fence_after();
           }
-          if (!stage_in(it)) {
-            ok = false;
-            break;
-          }
-          if (q == 0) TC_TRACE_AT(g_dec_trace, kEvDnFirst, u);
-          const uint8_t* sb = ring + (size_t)(it % NST) * kDecStageBytes;
-          const uint32_t sf = tmem + kColSf + 32 * (it % kDecSfSlots);
+          if ((int)(it & 1) == who) {
+            if (!stage_in(it)) {
+              ok = false;
+              break;
+            }
+            if (who == 0 && q == 0) TC_TRACE_AT(g_dec_trace, kEvDnFirst, u);
+            const uint8_t* sb = ring + (size_t)(it % NST) * kDecStageBytes;
+            const uint32_t sf = tmem + kColSf + 16 * (it % kDecSfSlots);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) tmem_cp_sf(sf + 4 * i, sdesc_sf(smem_u32(sb + kDecBBytes + i * kDecAtom)));
-          tmem_cp_sf(sf + 16, sdesc_sf(smem_u32(hbuf + 512)));
+            for (int i = 0; i < 4; ++i) tmem_cp_sf(sf + 4 * i, sdesc_sf(smem_u32(sb + kDecBBytes + i * kDecAtom)));
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int cl = (4 * q + i) % kDecGroupChunks;
-            mma_mxf4nvf4(tmem + kColD2 + kDecDnN * cl, sdesc_kmajor(smem_u32(sb + 4096 * i), 256, kSwizzle32B),
-                         sdesc_kmajor(smem_u32(hbuf), 0, kSwizzle32B), kDecIdescDn, sf + 4 * i, sf + 16, 0u);
+            for (int i = 0; i < 4; ++i) {
+              const int cl = (4 * q + i) % gch;
+              mma_mxf4nvf4(tmem + col_d2 + kDecDnN * cl, sdesc_kmajor(smem_u32(sb + 4096 * i), 256, kSwizzle32B),
+                           sdesc_kmajor(smem_u32(hbuf), 0, kSwizzle32B), kDecIdescT, sf + 4 * i, hsf, 0u);
+            }
+            mma_commit(&empty[it % NST]);
+            if (it < 40) TC_TRACE_AT(g_dec_trace, kEvMmaIssued, it);
           }
-          mma_commit(&empty[it % NST]);
-          if (it < 40) TC_TRACE_AT(g_dec_trace, kEvMmaIssued, it);
-          if (q % 4 == 3 || q == nks2 - 1) {
+          if (q % gst == gst - 1 || q == nks2 - 1) {
             mma_commit(&acc2_full);
             ++gc;
           }
         }
         if (!ok) break;
-        TC_TRACE_AT(g_dec_trace, kEvDnLast, u);
+        if (who == 0) TC_TRACE_AT(g_dec_trace, kEvDnLast, u);
       }
       // every issued tensor-core operation has completed before TMEM is released
       mma_commit(&final_bar);
@@ -357,99 +400,113 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
     // Warp w reads TMEM lane quarter q4 = w % 4. Every epilogue warp runs the same sequence
     // of named barriers whatever happens (after an abort the waits return at once and
     // nothing is written), so none can be left behind.
-    const int ew = warp - 2;
+    const int ew = warp - 3;
     const int q4 = warp & 3;
     const int half = ew >> 2;
     const float ts_x = *p.xq_ts;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
     uint32_t gc = 0;
-    for (int u = 0; u < nu; ++u) {
+    for (int jb = 0; jb < 2 * nu; ++jb) {
+      const int u = job_unit(jb);
       int slot, e, j;
       unit(u, slot, e, j);
       const bool sh = e == p.E;
       const int el = sh ? 0 : e;
       const ExpertGroup& G = sh ? p.shared : p.routed;
-      // ---- SwiGLU of unit u. D1 lane 32*q4 + l holds token l % 8; warp (q4, half) takes h
-      // block q4 (16 columns) of tokens 4*half .. 4*half+3, lane l the 4 columns 4*(l/8)..
-      if (ew == 0 && lane == 0) s_go = mbar_wait(&acc1_full, u & 1, &s_abort, p.status) ? 1 : 0;
-      named_bar_sync(2, 32 * kDecEpiWarps);
-      const bool go = s_go != 0;
-      if (ew == 0 && lane == 0) TC_TRACE_AT(g_dec_trace, kEvEpiStart, u);
-      tc_fence_after();
-      uint32_t g[16], uu[16];
-      tmem_ld16(lane_base + kColD1 + 16 * q4, g);
-      tmem_ld16(lane_base + kColD1 + 64 + 16 * q4, uu);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc1_empty);
-      {
-        const int t = lane & 7, r = lane >> 3;
-        const float sg = G.gu_ts[2 * el] * ts_x, su = G.gu_ts[2 * el + 1] * ts_x;
-        float h[4];
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          // this lane's 4 columns (selects, so the arrays stay in registers)
-          const uint32_t gi = r == 0 ? g[i] : r == 1 ? g[4 + i] : r == 2 ? g[8 + i] : g[12 + i];
-          const uint32_t ui = r == 0 ? uu[i] : r == 1 ? uu[4 + i] : r == 2 ? uu[8 + i] : uu[12 + i];
-          const float gv = __uint_as_float(gi) * sg, uv = __uint_as_float(ui) * su;
-          h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
-          amax = fmaxf(amax, fabsf(h[i]));
-        }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 8));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 16));
-        const uint32_t sbyte = f32_to_e4m3_sat(__fdiv_rn(amax, kE2M1Max));  // tensor scale of h is 1
-        const float sval = e4m3_to_f32(sbyte);
-        uint32_t code2 = 0;
-        if (sval != 0.0f)
-          code2 = f32x2_to_e2m1x2(__fdiv_rn(h[0], sval), __fdiv_rn(h[1], sval)) |
-                  (f32x2_to_e2m1x2(__fdiv_rn(h[2], sval), __fdiv_rn(h[3], sval)) << 8);
-        uint8_t* hbuf = hb + (u & 1) * kDecHBytes;
-        if (go && (t >> 2) == half) {
-          // row t of the 32-byte swizzled h tile: 16-byte half (q4 >> 1) ^ (t >> 2), byte 8*(q4&1) + 2r
-          *reinterpret_cast<uint16_t*>(hbuf + t * 32 + ((((q4 >> 1) ^ (t >> 2)) & 1) << 4) + (q4 & 1) * 8 + 2 * r) =
-              (uint16_t)code2;
-          // h scale atom: row r0 = t + 8r (token t) for all four r1, block q4
-#pragma unroll
-          for (int r1 = 0; r1 < 4; ++r1) hbuf[512 + (t + 8 * r) * 16 + r1 * 4 + q4] = (uint8_t)sbyte;
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(2, 32 * kDecEpiWarps);
-      if (ew == 0 && lane == 0) {
-        mbar_arrive(&h_full[u & 1]);
-        TC_TRACE_AT(g_dec_trace, kEvEpiEnd, u);
-      }
-      // ---- down projection of unit u: D2 lane 32*q4 + l is output row 128c + 32*q4 + l of
-      // chunk c; column 16*(c % 16) + t is token t. Warp (q4, half) takes the chunks of
-      // parity `half`.
-      const float ts_o = G.dn_ts[el];
-      float wf[kDecMaxT];
-#pragma unroll
-      for (int t = 0; t < kDecMaxT; ++t) wf[t] = p.slot_w[(size_t)slot * kDecMaxT + t] * ts_o;
-      for (int g0 = 0; g0 < nch; g0 += kDecGroupChunks, ++gc) {
-        const int ng = nch - g0 < kDecGroupChunks ? nch - g0 : kDecGroupChunks;
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(&acc2_full, gc & 1, &s_abort, p.status) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (job_is_gu(jb)) {
+        // ---- SwiGLU of unit u. D1 lane r < 64 holds gate row r of the slice, lane 64 + r up
+        // row r (h column r); columns 0..7 are the tokens, each issuer's sums 16 columns apart.
+        // Every warp copies its quarter's sums to shared memory (one warp of each quarter), then
+        // warp ew computes token ew: lane l takes h columns l and l + 32.
+        if (ew == 0 && lane == 0) s_go = mbar_wait(&acc1_full, u & 1, &s_abort, p.status) ? 1 : 0;
+        named_bar_sync(2, 32 * kDecEpiWarps);
+        const bool go = s_go != 0;
+        if (ew == 0 && lane == 0) TC_TRACE_AT(g_dec_trace, kEvEpiStart, u);
         tc_fence_after();
-        for (int cl = half; cl < ng; cl += 2) {
-          uint32_t v[16];
-          tmem_ld16(lane_base + kColD2 + kDecDnN * cl, v);
-          tmem_ld_wait();
-          if (ok) {
-            float* dst = p.out + (size_t)128 * (g0 + cl) + 32 * q4 + lane;
-#pragma unroll
-            for (int t = 0; t < kDecMaxT; ++t)
-              if (t < T && wf[t] != 0.0f) red_add_f32(dst + (size_t)t * d, __uint_as_float(v[t]) * wf[t]);
-          }
-        }
+        uint32_t va[8], vb[8];
+        tmem_ld8(lane_base + kColD1, va);
+        tmem_ld8(lane_base + kColD1 + 16, vb);
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&acc2_empty);
+        if (lane == 0) mbar_arrive(&acc1_empty);
+        if (half == 0) {
+          float4* dst = reinterpret_cast<float4*>(s_gu + (32 * q4 + lane) * 8);
+          dst[0] = make_float4(__uint_as_float(va[0]) + __uint_as_float(vb[0]), __uint_as_float(va[1]) + __uint_as_float(vb[1]),
+                               __uint_as_float(va[2]) + __uint_as_float(vb[2]), __uint_as_float(va[3]) + __uint_as_float(vb[3]));
+          dst[1] = make_float4(__uint_as_float(va[4]) + __uint_as_float(vb[4]), __uint_as_float(va[5]) + __uint_as_float(vb[5]),
+                               __uint_as_float(va[6]) + __uint_as_float(vb[6]), __uint_as_float(va[7]) + __uint_as_float(vb[7]));
+        }
+        named_bar_sync(2, 32 * kDecEpiWarps);
+        uint8_t* hbuf = hb + (u & 1) * kDecHBytes;
+        const int t = ew;  // token of this warp
+        const float sg = G.gu_ts[2 * el] * ts_x, su = G.gu_ts[2 * el + 1] * ts_x;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int i = lane + 32 * hh;  // h column within the slice
+          const float gv = s_gu[i * 8 + t] * sg, uv = s_gu[(64 + i) * 8 + t] * su;
+          const float h = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
+          // NVFP4 block of 16 h columns (16 lanes), tensor scale 1
+          float amax = fabsf(h);
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          const uint32_t sbyte = f32_to_e4m3_sat(__fdiv_rn(amax, kE2M1Max));
+          const float sval = e4m3_to_f32(sbyte);
+          const uint32_t nib = sval != 0.0f ? (f32x2_to_e2m1x2(__fdiv_rn(h, sval), 0.0f) & 0xFu) : 0u;
+          // byte of columns (i, i+1) on even lanes, then 4 bytes (8 columns) on lanes i % 8 == 0
+          const uint32_t b = nib | (__shfl_down_sync(0xffffffffu, nib, 1) << 4);
+          const uint32_t b1 = __shfl_down_sync(0xffffffffu, b, 2), b2 = __shfl_down_sync(0xffffffffu, b, 4),
+                         b3 = __shfl_down_sync(0xffffffffu, b, 6);
+          if (go && (lane & 7) == 0) {
+            const uint32_t word = (b & 0xFFu) | ((b1 & 0xFFu) << 8) | ((b2 & 0xFFu) << 16) | ((b3 & 0xFFu) << 24);
+            // row t of the 32-byte swizzled h tile: bytes i/2 .. i/2+3 in 16-byte half (i >> 5)
+            *reinterpret_cast<uint32_t*>(hbuf + t * 32 + ((hh ^ (t >> 2)) & 1) * 16 + ((i >> 1) & 15)) = word;
+          }
+          if (go && (lane & 15) < 4) {
+            // h scale atom: rows r0 = t + 8r (token t), all four r1, block i / 16 (lanes
+            // 0..3 and 16..19 each write one r)
+            const int r = lane & 3;
+#pragma unroll
+            for (int r1 = 0; r1 < 4; ++r1) hbuf[512 + (t + 8 * r) * 16 + r1 * 4 + (i >> 4)] = (uint8_t)sbyte;
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(2, 32 * kDecEpiWarps);
+        if (ew == 0 && lane == 0) {
+          mbar_arrive(&h_full[u & 1]);
+          TC_TRACE_AT(g_dec_trace, kEvEpiEnd, u);
+        }
+      } else {
+        // ---- down projection of unit u: D2 lane 32*q4 + l is output row 128c + 32*q4 + l of
+        // chunk c; column 16*(c % gch) + t is token t. Warp (q4, half) takes the chunks of
+        // parity `half`.
+        const float ts_o = G.dn_ts[el];
+        float wf[kDecMaxT];
+#pragma unroll
+        for (int t = 0; t < kDecMaxT; ++t) wf[t] = p.slot_w[(size_t)slot * kDecMaxT + t] * ts_o;
+        for (int g0 = 0; g0 < nch; g0 += gch, ++gc) {
+          const int ng = nch - g0 < gch ? nch - g0 : gch;
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait(&acc2_full, gc & 1, &s_abort, p.status) ? 1 : 0;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          tc_fence_after();
+          for (int cl = half; cl < ng; cl += 2) {
+            uint32_t v[8];
+            tmem_ld8(lane_base + col_d2 + kDecDnN * cl, v);
+            tmem_ld_wait();
+            if (ok) {
+              float* dst = p.out + (size_t)128 * (g0 + cl) + 32 * q4 + lane;
+#pragma unroll
+              for (int t = 0; t < kDecMaxT; ++t)
+                if (t < T && wf[t] != 0.0f) red_add_f32(dst + (size_t)t * d, __uint_as_float(v[t]) * wf[t]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc2_empty);
+        }
+        if (ew == 0 && lane == 0) TC_TRACE_AT(g_dec_trace, kEvDrainEnd, u);
       }
-      if (ew == 0 && lane == 0) TC_TRACE_AT(g_dec_trace, kEvDrainEnd, u);
     }
   }
   tc_fence_before();
@@ -459,6 +516,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
     tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0) TC_TRACE_AT(g_dec_trace, kEvExit, 0);
+  RT_TRACE(g_prep_trace, 1, 2);
 }
 
 // ---------------------------------------------------------------- host side
@@ -467,7 +525,15 @@ namespace {
 constexpr size_t kDecSmemBudget = 226 * 1024;  // dynamic shared memory; the rest of 227 KB is static
 
 size_t dec_fixed_smem(int d) {
-  return (size_t)(d / 256) * 1024 + (size_t)(d / 64) * kDecAtom + 2 * kDecHBytes + 1024;  // + alignment slack
+  // x tiles, x scale atoms, two h tiles, the gate/up sums exchange, alignment slack
+  return (size_t)(d / 256) * 1024 + (size_t)(d / 64) * kDecAtom + 2 * kDecHBytes + 128 * 8 * 4 + 1024;
+}
+
+// down chunks whose 16-column accumulators fit in TMEM next to everything else
+int dec_group_chunks(int d) {
+  const int avail = (512 - (int)dec_col_d2(d)) / kDecDnN;
+  const int g = avail & ~3;
+  return g < d / 128 ? g : d / 128;
 }
 
 int dec_stages(int d) {
@@ -485,8 +551,8 @@ size_t a256d(size_t v) { return (v + 255) & ~(size_t)255; }
 }  // namespace
 
 bool ffn_dec_supported(int64_t T, int d, int I, int mode) {
-  return T >= 1 && T <= kDecMaxT && mode == 0 && d % 512 == 0 && I % 64 == 0 && d <= 8192 && I <= 16384 &&
-         dec_stages(d) >= kDecMinStages;
+  return T >= 1 && T <= kDecMaxT && mode == 0 && d % 512 == 0 && I % 64 == 0 && d <= 4096 && I <= 16384 &&
+         dec_stages(d) >= kDecMinStages && dec_group_chunks(d) >= 4;
 }
 
 size_t ffn_dec_ws_bytes(int E) { return 256 + a256d((size_t)(E + 1) * 4) + a256d((size_t)(E + 1) * kDecMaxT * 4); }
@@ -512,6 +578,7 @@ cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* sta
   p.has_shared = a.has_shared;
   p.E = a.E; p.d = a.d; p.I = a.I; p.T = (int)a.T; p.k = a.k;
   p.nstages = dec_stages(a.d);
+  p.group_chunks = dec_group_chunks(a.d);
   p.out = a.out;
   p.nslots = reinterpret_cast<int32_t*>(w);
   p.slots = reinterpret_cast<int32_t*>(w + 256);
@@ -548,5 +615,6 @@ cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* sta
 #ifdef MOE_TRACE
 namespace moe {
 int64_t trace_fetch_dec(void* host, size_t bytes) { return trace_fetch(g_dec_trace, host, bytes); }
+int64_t trace_fetch_prep(void* host, size_t bytes) { return trace_fetch(g_prep_trace, host, bytes); }
 }  // namespace moe
 #endif

@@ -15,12 +15,16 @@
 // B200 CUDA cores run it at a small fraction of the float32 rate.
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
+#include "trace.cuh"
 
 namespace moe {
 
 // ---------------------------------------------------------------- router GEMV (T <= 8)
 // x (T x d bf16) is staged in shared memory; each warp owns expert rows of Wr and keeps
 // 16 float4 loads per lane in flight (a full 8 KB row at d = 2048) before using them.
+RT_TRACE_ARRAY(g_route_trace)
+
 constexpr int kGemvMaxT = 8;
 constexpr int kGemvUnroll = 16;
 
@@ -28,7 +32,9 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
                                                           const float* __restrict__ Wr,
                                                           const float* __restrict__ br, int E,
                                                           float* __restrict__ logits) {
+  RT_TRACE(g_route_trace, 0, 0);
   MOE_PDL_PROLOGUE();
+  RT_TRACE(g_route_trace, 0, 1);
   extern __shared__ __align__(16) uint16_t xs[];  // [T][d]
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
@@ -61,6 +67,7 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
     }
   }
   __syncthreads();
+  RT_TRACE(g_route_trace, 0, 2);
   for (; e < E; e += gridDim.x * warps) {
     float acc[kGemvMaxT];
 #pragma unroll
@@ -95,6 +102,7 @@ __global__ void __launch_bounds__(256) router_gemv_kernel(const uint16_t* __rest
     const int en = e + gridDim.x * warps;
     if (en < E) load_w(en, lane);
   }
+  RT_TRACE(g_route_trace, 0, 3);
 }
 
 // ---------------------------------------------------------------- router GEMM (large T)
@@ -389,7 +397,9 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
                                                                int32_t* __restrict__ offsets,
                                                                int32_t* __restrict__ sorted_assign,
                                                                int32_t* __restrict__ assign_pos) {
+  RT_TRACE(g_route_trace, 1, 0);
   MOE_PDL_PROLOGUE();
+  RT_TRACE(g_route_trace, 1, 1);
   extern __shared__ int sh[];  // [E] counts / running positions, then [T*k] chosen experts
   int* sidx = sh + E;
   const int warp = threadIdx.x >> 5;
@@ -397,6 +407,7 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
     topk_dispatch(logits + (size_t)warp * E, E, k, topk_idx + (size_t)warp * k, topk_w + (size_t)warp * k,
                   sidx + warp * k);
   __syncthreads();
+  RT_TRACE(g_route_trace, 1, 2);
   if (warp != 0) return;
   // the permutation of <= 32*k assignments by one warp, without block-wide barriers:
   // histogram (match_any leaders), warp scan of the counts, then a stable scatter in
@@ -452,6 +463,7 @@ __global__ void __launch_bounds__(1024) topk_perm_small_kernel(const float* __re
     if (a < n && (peers >> lane) == 1u) sh[e] += __popc(peers);  // highest lane of its group
     __syncwarp();
   }
+  RT_TRACE(g_route_trace, 1, 3);
 }
 
 __global__ void zero_counts_kernel(int E, int32_t* counts, int32_t* offsets) {
@@ -582,3 +594,9 @@ cudaError_t init_route_attributes() {
 
 
 }  // namespace moe
+
+#ifdef MOE_TRACE
+namespace moe {
+int64_t trace_fetch_route(void* host, size_t bytes) { return trace_fetch(g_route_trace, host, bytes); }
+}  // namespace moe
+#endif

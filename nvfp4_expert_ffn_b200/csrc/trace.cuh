@@ -61,10 +61,20 @@ int64_t trace_fetch(A& arr, void* host, size_t bytes) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;
   if (cudaMemcpyFromSymbol(host, arr, n) != cudaSuccess) return -1;
   static const unsigned long long zeros[(size_t)kTraceCtas * (kTraceCap + 2)] = {};
-  if (cudaMemcpyToSymbol(arr, zeros, sizeof(zeros)) != cudaSuccess) return -1;
+  static_assert(sizeof(arr) <= sizeof(zeros), "trace array larger than the zero buffer");
+  if (cudaMemcpyToSymbol(arr, zeros, sizeof(arr)) != cudaSuccess) return -1;
   return (int64_t)n;
 }
+// short kernels: globaltimer stamps [kernel][cta][event] (event 0 = entry)
+constexpr int kRtKernels = 8, kRtEvents = 8;
+#define RT_TRACE_ARRAY(name) __device__ unsigned long long name[kRtKernels][kTraceCtas][kRtEvents];
+#define RT_TRACE(arr, kern, ev)                                                                   \
+  do {                                                                                           \
+    if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) arr[kern][blockIdx.x][ev] = globaltimer_ns(); \
+  } while (0)
 #else
+#define RT_TRACE_ARRAY(name)
+#define RT_TRACE(arr, kern, ev) do { } while (0)
 #define TC_TRACE_ARRAY(name)
 #define TC_TRACE_DECL
 #define TC_TRACE_BEGIN(arr) do { } while (0)
