@@ -68,6 +68,7 @@ typedef enum moe_status {
 #define MOE_OP_ROUTE 1
 #define MOE_OP_QUANT 2
 #define MOE_OP_FFN 3
+#define MOE_OP_LAYER_DECODE 4 /* moe_layer_decode (zero-filled before its first use) */
 
 /*
  * Expert weights of one expert group (E routed experts, or E = 1 for the shared expert),
@@ -201,6 +202,35 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
                        const float* shared_out, const float* topk_w,
                        const int32_t* assign_pos, int32_t rms_renorm, uint16_t* y_bf16,
                        void* stream);
+
+/*
+ * moe_layer_decode - one whole MoE layer forward for at most 8 tokens in one kernel launch:
+ * activation quantisation (as nvfp4_quantize_act), router, top-k and weights, permutation
+ * and per-call histogram (as moe_route), the expert FFN with the shared expert (as
+ * moe_expert_ffn, MOE_FFN_ACCUMULATE, DECODE path) and the combine into bf16 (as
+ * moe_combine). The same steps as those calls in that order, with the same outputs, for
+ * the decode case where each of them is a few microseconds of work and their launches and
+ * memory round trips would cost more than the work (Basalt pages: "What Basalt changes in a
+ * Blackwell local inference stack", section "Experts can move without becoming free").
+ *   x_bf16 [T][d]; ts_in float32[1] static activation scale or NULL (dynamic amax);
+ *   Wr float32 [E][d]; br float32 [E] or NULL; W: both groups packed by moe_pack_experts,
+ *   slices included.
+ *   Outputs: xq_codes [T][d/2], xq_scales [T][d/16], xq_ts [1]; topk_idx [T][k],
+ *   topk_w [T][k]; counts [E], offsets [E+1], sorted_assign [T*k], assign_pos [T*k];
+ *   y_acc float32 [T][d] (the unrounded output); y_bf16 [T][d]; rms_renorm as moe_combine.
+ *   ws: moe_workspace_size(MOE_OP_LAYER_DECODE, ...) bytes, zero-filled before the first
+ *   call (it holds the counter of the kernel's grid-wide barrier, which every call leaves
+ *   at zero; after a MOE_ERR_TIMEOUT from moe_get_device_status, zero it again).
+ * Limits: 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024.
+ * The kernel uses all SMs but one and waits at grid-wide barriers, so it must not share the
+ * GPU with a kernel that occupies more than one SM until this one ends.
+ */
+moe_status moe_layer_decode(const uint16_t* x_bf16, int32_t T, const float* ts_in, const float* Wr,
+                            const float* br, const moe_experts_t* W, int32_t k, uint8_t* xq_codes,
+                            uint8_t* xq_scales, float* xq_ts, int32_t* topk_idx, float* topk_w,
+                            int32_t* counts, int32_t* offsets, int32_t* sorted_assign,
+                            int32_t* assign_pos, float* y_acc, uint16_t* y_bf16, int32_t rms_renorm,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /*
  * moe_expert_hist - cumulative routing counts and hot-to-cold ranking (A10).

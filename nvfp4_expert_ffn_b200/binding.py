@@ -21,7 +21,7 @@ LIB_PATH = os.environ.get("MOE_NVFP4_LIB") or os.path.join(_PKG, "lib", "libmoe_
 MOE_OK = 0
 MOE_FFN_ACCUMULATE, MOE_FFN_PER_ASSIGN = 0, 1
 MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_CUDA_CORE = 0, 1, 2, 3
-MOE_OP_LAYER, MOE_OP_ROUTE, MOE_OP_QUANT, MOE_OP_FFN = 0, 1, 2, 3
+MOE_OP_LAYER, MOE_OP_ROUTE, MOE_OP_QUANT, MOE_OP_FFN, MOE_OP_LAYER_DECODE = 0, 1, 2, 3, 4
 
 # (name, restype, argtypes) of every C export; tests check the header declares the same set
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -35,6 +35,8 @@ EXPORTS = {
                               _SZ, _P]),
     "moe_combine": (_I32, [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _I32, _P, _P]),
     "moe_expert_hist": (_I32, [_P, _I32, _P, _P, _I32, _P]),
+    "moe_layer_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                _P, _P, _I32, _P, _SZ, _P]),
     "moe_workspace_size": (_SZ, [_I32, _I64, _I32, _I32, _I32, _I32]),
     "moe_get_device_status": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
@@ -172,6 +174,20 @@ def moe_route(x, Wr, br, k, topk_idx, topk_w, counts, offsets, sorted_assign, as
         _ptr(x), T, d, _ptr(Wr), _ptr(br), E, k, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
         _ptr(offsets), _ptr(sorted_assign), _ptr(assign_pos), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_layer_decode(x, ts_in, Wr, br, experts: "Experts", k, xq_codes, xq_scales, xq_ts, topk_idx,
+                     topk_w, counts, offsets, sorted_assign, assign_pos, y_acc, y, rms_renorm, ws,
+                     stream=None):
+    """The whole layer for at most 8 tokens in one kernel (see include/moe_nvfp4.h); ws must
+    be zero-filled before its first use."""
+    T = x.shape[0]
+    s = experts.struct()
+    _check("moe_layer_decode", lib().moe_layer_decode(
+        _ptr(x), T, _ptr(ts_in), _ptr(Wr), _ptr(br), ctypes.byref(s), k, _ptr(xq_codes),
+        _ptr(xq_scales), _ptr(xq_ts), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(offsets),
+        _ptr(sorted_assign), _ptr(assign_pos), _ptr(y_acc), _ptr(y), 1 if rms_renorm else 0,
+        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def moe_route_noalloc(x, Wr, br, k, topk_idx, topk_w, counts, offsets, sorted_assign, assign_pos,

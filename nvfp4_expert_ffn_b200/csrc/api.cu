@@ -144,6 +144,7 @@ size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k
       size_t m = q > r ? q : r;
       return m > f ? m : f;
     }
+    case MOE_OP_LAYER_DECODE: return layer_dec_ws_bytes(T, E);
   }
   return 0;
 }
@@ -273,12 +274,16 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   if (!aligned16(xq_codes) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "xq_codes/out must be 16-byte aligned");
   if (mode == MOE_FFN_PER_ASSIGN && W->has_shared && !shared_out)
     return fail(MOE_ERR_INVALID_ARG, "shared_out needed in PER_ASSIGN mode with a shared expert");
+  int sms = 0;
+  int32_t* dstatus = nullptr;
+  s = device_info(&sms, &dstatus);
+  if (s != MOE_OK) return s;
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
   const bool tc_ok = ffn_tc_supported(d, I) && packed;
   const bool sliced = W->routed.dn_codes_slice && W->routed.dn_sf_slice &&
                       (!W->has_shared || (W->shared.dn_codes_slice && W->shared.dn_sf_slice));
-  const bool dec_ok = ffn_dec_supported(T, d, I, mode) && packed && sliced;
+  const bool dec_ok = ffn_dec_supported(T, d, I, mode, E, k, W->has_shared ? 1 : 0, sms) && packed && sliced;
   if (path == MOE_PATH_PREFILL && !tc_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "tensor-core path needs d % 256 == 0, I % 256 == 0 and scales packed by moe_pack_experts");
@@ -291,10 +296,6 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
                       : kind == MOE_PATH_PREFILL ? ffn_tc_ws_bytes(T, d, E, k, I)
                                                  : ffn_decode_ws_bytes(T, d, E, k, I);
   s = check_ws(ws, ws_bytes, need);
-  if (s != MOE_OK) return s;
-  int sms = 0;
-  int32_t* dstatus = nullptr;
-  s = device_info(&sms, &dstatus);
   if (s != MOE_OK) return s;
   FfnArgs a;
   a.xq_codes = xq_codes;
@@ -317,6 +318,58 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
                   : kind == MOE_PATH_PREFILL ? launch_ffn_tc(a, ws, sms, dstatus, (cudaStream_t)stream)
                                              : launch_ffn_decode(a, sms, dstatus, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn launch");
+}
+
+moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, const float* Wr, const float* br,
+                            const moe_experts_t* W, int32_t k, uint8_t* xq_codes, uint8_t* xq_scales,
+                            float* xq_ts, int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
+                            int32_t* sorted_assign, int32_t* assign_pos, float* y_acc, uint16_t* y,
+                            int32_t rms_renorm, void* ws, size_t ws_bytes, void* stream) {
+  if (!W) return fail(MOE_ERR_INVALID_ARG, "null weights");
+  const int E = W->routed.E, d = W->routed.d, I = W->routed.I;
+  moe_status s = check_weights(W->routed, "routed", E, d, I);
+  if (s != MOE_OK) return s;
+  if (W->has_shared && (s = check_weights(W->shared, "shared", 1, d, I)) != MOE_OK) return s;
+  if (!x || !Wr || !xq_codes || !xq_scales || !xq_ts || !topk_idx || !topk_w || !counts || !offsets ||
+      !sorted_assign || !assign_pos || !y_acc || !y)
+    return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(x) || !aligned16(Wr) || !aligned16(xq_codes) || !aligned16(y_acc) || !aligned16(y))
+    return fail(MOE_ERR_INVALID_ARG, "x, Wr, xq_codes, y_acc and y must be 16-byte aligned");
+  const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled && W->routed.dn_codes_slice &&
+                      W->routed.dn_sf_slice &&
+                      (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled &&
+                                          W->shared.dn_codes_slice && W->shared.dn_sf_slice));
+  if (!packed) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "weights must be packed by moe_pack_experts, slices included");
+  int sms = 0;
+  int32_t* dstatus = nullptr;
+  if ((s = device_info(&sms, &dstatus)) != MOE_OK) return s;
+  if (!layer_dec_supported(T, d, I, E, k, W->has_shared ? 1 : 0, sms))
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                "moe_layer_decode needs 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024");
+  if ((s = check_ws(ws, ws_bytes, layer_dec_ws_bytes(T, E))) != MOE_OK) return s;
+  LayerDecArgs a;
+  a.x = x;
+  a.ts_in = ts_in;
+  a.Wr = Wr;
+  a.br = br;
+  a.routed = to_group(W->routed);
+  a.shared = W->has_shared ? to_group(W->shared) : ExpertGroup{};
+  a.has_shared = W->has_shared ? 1 : 0;
+  a.E = E; a.d = d; a.I = I; a.T = T; a.k = k;
+  a.rms = rms_renorm ? 1 : 0;
+  a.xq_codes = xq_codes;
+  a.xq_scales = xq_scales;
+  a.xq_ts = xq_ts;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.sorted_assign = sorted_assign;
+  a.assign_pos = assign_pos;
+  a.y_acc = y_acc;
+  a.y = y;
+  cudaError_t e = launch_layer_dec(a, ws, sms, dstatus, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer_decode launch");
 }
 
 moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const float* expert_out,

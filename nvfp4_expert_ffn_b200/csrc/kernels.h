@@ -99,9 +99,34 @@ bool ffn_tc_supported(int d, int I);
 size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I);
 cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
 // tcgen05 decode FFN (at most 8 tokens)
-bool ffn_dec_supported(int64_t T, int d, int I, int mode);
+bool ffn_dec_supported(int64_t T, int d, int I, int mode, int E, int k, int has_shared, int grid);
 size_t ffn_dec_ws_bytes(int E);
 cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
+// fused decode layer (at most 8 tokens): quantise, route, expert FFN and combine in one kernel
+struct LayerDecArgs {
+  const uint16_t* x;
+  const float* ts_in;
+  const float* Wr;
+  const float* br;
+  ExpertGroup routed, shared;
+  int has_shared;
+  int E, d, I, T, k;
+  int rms;
+  uint8_t* xq_codes;
+  uint8_t* xq_scales;
+  float* xq_ts;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_assign;
+  int32_t* assign_pos;
+  float* y_acc;
+  uint16_t* y;
+};
+bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms);
+size_t layer_dec_ws_bytes(int64_t T, int E);
+cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
 cudaError_t launch_pack_slices(const ExpertGroup& g, int E, int d, int I, uint8_t* dn_codes_slice,
                                uint8_t* dn_sf_slice, int num_sms, cudaStream_t st);
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
@@ -112,6 +137,7 @@ cudaError_t init_route_attributes();
 cudaError_t init_ffn_decode_attributes();
 cudaError_t init_ffn_tc_attributes();
 cudaError_t init_ffn_dec_attributes();
+cudaError_t init_layer_dec_attributes();
 inline cudaError_t init_kernel_attributes() {
   cudaError_t e = init_route_attributes();
   if (e != cudaSuccess) return e;
@@ -119,7 +145,9 @@ inline cudaError_t init_kernel_attributes() {
   if (e != cudaSuccess) return e;
   e = init_ffn_tc_attributes();
   if (e != cudaSuccess) return e;
-  return init_ffn_dec_attributes();
+  e = init_ffn_dec_attributes();
+  if (e != cudaSuccess) return e;
+  return init_layer_dec_attributes();
 }
 
 }  // namespace moe

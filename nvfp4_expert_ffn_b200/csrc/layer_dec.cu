@@ -1,0 +1,455 @@
+// One MoE layer forward for at most 8 tokens in one persistent kernel: activation
+// quantisation (A4), router (A1), top-k and weights (A2), permutation and per-call
+// histogram (A3), the expert FFN with the shared expert (A5-A8, the unit core of
+// dec_core.cuh) and the combine into bf16 (A9).
+//
+// With a handful of tokens every step but the expert FFN is a few microseconds of work,
+// and as separate kernels each costs a launch and a chain of dependent memory round trips.
+// Here one CTA per SM (all but one SM, left to a side-stream kernel such as the cumulative
+// histogram) runs:
+//   phase 1  every CTA loads x, takes the global amax itself (the NVFP4 tensor scale),
+//            quantises its share of the 16-element blocks into the xq output buffers, and
+//            computes the router logits of its expert rows (E / grid rows, the router
+//            weights loaded before the kernel waits on its predecessor); CTA 0 zeroes y_acc.
+//   barrier
+//   phase 2  every CTA reads all tokens' codes into its shared-memory tiles, runs the
+//            top-k of all tokens itself and derives its own units; the last CTA also
+//            writes the routing outputs (top-k, counts, offsets, permutation).
+//   phase 3  the units (expert, 64-column slice of I), adding into y_acc.
+//   barrier
+//   phase 4  CTA t < T converts row t of y_acc to bf16 (optionally RMS-renormalised).
+// The grid barrier counts arrivals in a workspace word that must be zero before the first
+// call; every barrier leaves it at zero.
+#include <cuda_bf16.h>
+
+#include "dec_core.cuh"
+#include "route_core.cuh"
+
+namespace moe {
+
+constexpr int kLayerMaxK = 32;
+
+struct LayerArgs {
+  const uint16_t* x;   // [T][d] bf16
+  const float* ts_in;  // static activation tensor scale, or NULL
+  const float* Wr;     // [E][d]
+  const float* br;     // [E] or NULL
+  ExpertGroup routed, shared;
+  int has_shared;
+  int E, d, I, T, k;
+  int nstages, group_chunks;
+  int rms;
+  // outputs
+  uint8_t* xq_codes;   // [T][d/2]
+  uint8_t* xq_scales;  // [T][d/16]
+  float* xq_ts;        // [1]
+  int32_t* topk_idx;   // [T][k]
+  float* topk_w;       // [T][k]
+  int32_t* counts;     // [E]
+  int32_t* offsets;    // [E+1]
+  int32_t* sorted_assign;  // [T*k]
+  int32_t* assign_pos;     // [T*k]
+  float* y_acc;        // [T][d]
+  uint16_t* y;         // [T][d] bf16
+  // workspace
+  float* logits;       // [T][E]
+  int32_t* sync;       // [2]: arrival count (zero between barriers), generation
+  int32_t* status;
+};
+
+// Grid-wide barrier: thread 0 of each CTA reads the generation, then counts itself in; the
+// last to arrive resets the count and advances the generation, the others wait (bounded)
+// for it to change. Writes before the barrier are visible to every CTA after it.
+MOE_DEV bool grid_sync(int32_t* sync, volatile int* abort, int32_t* status) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = *abort ? 0 : 1;
+    if (ok) {
+      const int32_t g0 = ld_acquire_gpu(sync + 1);
+      __threadfence();
+      if (atomicAdd(sync, 1) == (int)gridDim.x - 1) {
+        atomicExch(sync, 0);
+        __threadfence();
+        atomicAdd(sync + 1, 1);
+      } else {
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(sync + 1) == g0) {
+          if (*abort) {
+            ok = 0;
+            break;
+          }
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicExch(status, kStatusTimeout);
+            ok = 0;
+            break;
+          }
+          __nanosleep(32);
+        }
+      }
+      __threadfence();
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+// Shared-memory scratch of phases 1 and 2, on the weight ring (not in use before phase 3):
+// the bf16 activations (phase 1), then at the same place the logits (phase 2); the top-k of
+// each token, the expert-use flags and list, and the permutation's counters.
+struct LayerScratch {
+  uint16_t* xb;   // [8][d] (phase 1)
+  float* logits;  // [8][E] (phase 2, over xb)
+  int* tidx;      // [8][32] expert ids of each token's top-k
+  float* tw;      // [8][32] their weights
+  int* flag;      // [1024] expert used by some token
+  int* list;      // [1025] experts in use, in id order after the shared expert
+  int* perm;      // [1024] counters of the permutation
+  int* sidx;      // [256] top-k expert ids, assignment order
+};
+
+__host__ __device__ inline size_t layer_scratch_head(int d) {
+  const size_t xb = 16 * (size_t)d, lg = (size_t)kDecMaxT * 1024 * 4;
+  return xb > lg ? xb : lg;
+}
+
+MOE_DEV LayerScratch layer_scratch(uint8_t* ring, int d) {
+  LayerScratch s;
+  s.xb = reinterpret_cast<uint16_t*>(ring);
+  s.logits = reinterpret_cast<float*>(ring);
+  s.tidx = reinterpret_cast<int*>(ring + layer_scratch_head(d));
+  s.tw = reinterpret_cast<float*>(s.tidx + kDecMaxT * kLayerMaxK);
+  s.flag = reinterpret_cast<int*>(s.tw + kDecMaxT * kLayerMaxK);
+  s.list = s.flag + 1024;
+  s.perm = s.list + 1040;
+  s.sidx = s.perm + 1024;
+  return s;
+}
+// bytes of scratch past the head
+constexpr size_t kLayerScratchTail = 2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 1040 + 1024 + 256) * 4;
+
+__global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_constant__ DecMaps maps, LayerArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ DecBars bar;
+  __shared__ int s_ue[kDecMaxUnits], s_uj[kDecMaxUnits];
+  __shared__ float s_uw[kDecMaxUnits * kDecMaxT];
+  __shared__ float s_red[32];
+  __shared__ int s_tmp[32];
+  const DecSmem sm = dec_smem(align1024(smem_raw), p.d, p.nstages);
+  const LayerScratch sc = layer_scratch(sm.ring, p.d);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = p.d, T = p.T, E = p.E, k = p.k;
+  const int G = (int)gridDim.x, b = (int)blockIdx.x;
+  const int nvec = d / 4;  // float4 per router row
+  volatile int* abort = reinterpret_cast<volatile int*>(&bar.abort);
+
+  dec_init(bar, p.nstages, maps, p.has_shared);
+  // this warp's router row; its first 512 float4 (d <= 2048: all of it) are loaded before
+  // the kernel waits on its predecessor (the router weights are not written by anything)
+  const int er = b + warp * G;
+  const bool has_row = er < E;
+  const float4* wrow = reinterpret_cast<const float4*>(p.Wr) + (size_t)(has_row ? er : 0) * nvec;
+  float4 w[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int c = lane + 32 * u;
+    w[u] = (has_row && c < nvec) ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  MOE_PDL_PROLOGUE();
+
+  // ---------------------------------------------------------------- phase 1
+  // x -> shared memory (every load of a round in flight before the stores)
+  {
+    const int nx = T * d / 8;
+    const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
+    uint4* xb4 = reinterpret_cast<uint4*>(sc.xb);
+    for (int i0 = threadIdx.x; i0 < nx; i0 += 8 * blockDim.x) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < nx) v[u] = __ldg(x4 + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < nx) xb4[i] = v[u];
+      }
+    }
+  }
+  __syncthreads();
+  // NVFP4 tensor scale: amax / (6 * 448) over all T tokens (every CTA computes the same), or
+  // the static scale
+  float ts;
+  if (p.ts_in) {
+    ts = *p.ts_in;
+  } else {
+    uint32_t m = 0;
+    const uint4* xb4 = reinterpret_cast<const uint4*>(sc.xb);
+    for (int i = threadIdx.x; i < T * d / 8; i += blockDim.x) {
+      const uint4 v = xb4[i];
+      m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    }
+    float f = warp_max(fmaxf(bf16_to_f32(m & 0xFFFFu), bf16_to_f32(m >> 16)));
+    if (lane == 0) s_red[warp] = f;
+    __syncthreads();
+    f = lane < (int)(blockDim.x >> 5) ? s_red[lane] : 0.0f;
+    f = warp_max(f);
+    ts = f > 0.0f ? __fdiv_rn(f, kE2M1Max * kE4M3Max) : 1.0f;
+  }
+  // this CTA's share of the 16-element blocks: codes and scales into the xq outputs
+  {
+    const int nblk = T * (d / kBlock);
+    for (int q = b + G * (int)threadIdx.x; q < nblk; q += G * (int)blockDim.x) {
+      const int t = q / (d / kBlock), blk = q % (d / kBlock);
+      const uint4* src = reinterpret_cast<const uint4*>(sc.xb + (size_t)t * d + kBlock * blk);
+      const uint4 p0 = src[0], p1 = src[1];
+      const uint32_t wd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_to_f32(wd[i] & 0xFFFFu);
+        v[2 * i + 1] = bf16_to_f32(wd[i] >> 16);
+      }
+      uint2 codes;
+      p.xq_scales[q] = (uint8_t)quantize_block16(v, ts, &codes);
+      reinterpret_cast<uint2*>(p.xq_codes)[q] = codes;
+    }
+    if (b == G - 1 && threadIdx.x == 0) *p.xq_ts = ts;
+  }
+  // router logits of this warp's row: 64-term lane partials, then a lane tree per token
+  if (has_row) {
+    float acc[kDecMaxT];
+#pragma unroll
+    for (int t = 0; t < kDecMaxT; ++t) acc[t] = 0.0f;
+    for (int c0 = 0; c0 < nvec; c0 += 512) {
+      if (c0 > 0) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int c = c0 + lane + 32 * u;
+          w[u] = c < nvec ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int c = c0 + lane + 32 * u;
+        if (c < nvec) {
+#pragma unroll
+          for (int t = 0; t < kDecMaxT; ++t) {
+            if (t < T) {
+              const uint2 xv = *reinterpret_cast<const uint2*>(sc.xb + (size_t)t * d + 4 * c);
+              acc[t] = fmaf(bf16_to_f32(xv.x & 0xFFFFu), w[u].x, acc[t]);
+              acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w[u].y, acc[t]);
+              acc[t] = fmaf(bf16_to_f32(xv.y & 0xFFFFu), w[u].z, acc[t]);
+              acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w[u].w, acc[t]);
+            }
+          }
+        }
+      }
+    }
+    const float bias = p.br ? __ldg(p.br + er) : 0.0f;
+#pragma unroll
+    for (int t = 0; t < kDecMaxT; ++t) {
+      if (t < T) {
+        const float s = warp_sum(acc[t]);
+        if (lane == 0) p.logits[(size_t)t * E + er] = s + bias;
+      }
+    }
+  }
+  // y_acc starts at zero: the units add into it after the barrier
+  if (b == 0) {
+    float4* y4 = reinterpret_cast<float4*>(p.y_acc);
+    for (int i = threadIdx.x; i < T * d / 4; i += blockDim.x) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  bool ok = grid_sync(p.sync, abort, p.status);
+
+  // ---------------------------------------------------------------- phase 2
+  // Data written by other CTAs before the barrier is read through L2 (ld.global.cg).
+  const int nt1 = p.I / 64;
+  const bool writer = b == G - 1;  // the CTA with the fewest units writes the routing outputs
+  int nu = 0;
+  if (ok) {
+    // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms
+    for (int i = threadIdx.x; i < kDecMaxT * (d / 32); i += blockDim.x) {
+      const int t = i / (d / 32), c = i % (d / 32);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (t < T) v = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
+      *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(t, c)) = v;
+    }
+    for (int i = threadIdx.x; i < (d / 64) * 32; i += blockDim.x) {
+      const int kc = i / 32, r0 = i % 32, t = r0 & 7;
+      uint32_t wd = 0u;
+      if (t < T) wd = __ldcg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock)) + kc);
+      dec_xsf_store(sm.xsf, kc, r0, wd);
+    }
+    for (int i = threadIdx.x; i < T * E; i += blockDim.x) sc.logits[i] = __ldcg(p.logits + i);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) sc.flag[e] = 0;
+    __syncthreads();
+    // top-k of every token (one warp each)
+    if (warp < T)
+      topk_dispatch(sc.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
+                    writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
+                    sc.tw + warp * kLayerMaxK);
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+      const int e = sc.tidx[(i / k) * kLayerMaxK + i % k];
+      sc.flag[e] = 1;
+      sc.sidx[i] = e;
+    }
+    __syncthreads();
+    // experts in use, in id order after the shared expert (contiguous ranges per thread)
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per;
+    int cnt = 0;
+    for (int e = e0; e < E && e < e0 + per; ++e) cnt += sc.flag[e];
+    int total;
+    int slot = block_exclusive_scan(cnt, s_tmp, &total) + p.has_shared;
+    for (int e = e0; e < E && e < e0 + per; ++e)
+      if (sc.flag[e]) sc.list[slot++] = e;
+    if (threadIdx.x == 0 && p.has_shared) sc.list[0] = E;
+    const int nslots = total + p.has_shared;
+    __syncthreads();
+    if (writer && warp == 0)
+      perm_small_warp(sc.sidx, T * k, E, sc.perm, p.counts, p.offsets, p.sorted_assign, p.assign_pos);
+    // this CTA's units: blockIdx.x, blockIdx.x + gridDim.x, ... of nslots * nt1
+    const int nunits = nslots * nt1;
+    nu = b < nunits ? (nunits - 1 - b) / G + 1 : 0;
+    if (nu > kDecMaxUnits) {  // the host checks the worst case, so this does not happen
+      if (threadIdx.x == 0) atomicExch(p.status, kStatusUnsupported);
+      nu = kDecMaxUnits;
+    }
+    for (int i = threadIdx.x; i < nu * (kDecMaxT + 1); i += blockDim.x) {
+      const int u = i / (kDecMaxT + 1), f = i % (kDecMaxT + 1);
+      const int ug = b + u * G;
+      const int e = sc.list[ug / nt1];
+      if (f == kDecMaxT) {
+        s_ue[u] = e;
+        s_uj[u] = ug % nt1;
+      } else {
+        float wt = 0.0f;
+        if (f < T) {
+          if (e == E) {
+            wt = 1.0f;
+          } else {
+            for (int j = 0; j < k; ++j)
+              if (sc.tidx[f * kLayerMaxK + j] == e) wt = sc.tw[f * kLayerMaxK + j];
+          }
+        }
+        s_uw[u * kDecMaxT + f] = wt;
+      }
+    }
+  }
+  fence_proxy_async_smem();  // the tiles and atoms above are read by tcgen05 (async proxy)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---------------------------------------------------------------- phase 3
+  DecArgs a;
+  a.routed = p.routed;
+  a.shared = p.shared;
+  a.has_shared = p.has_shared;
+  a.E = E; a.d = d; a.I = p.I; a.T = T;
+  a.nstages = p.nstages;
+  a.group_chunks = p.group_chunks;
+  a.ts_x = ts;
+  a.out = p.y_acc;
+  a.status = p.status;
+  dec_run(maps, a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw});
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(bar.tmem, 512);
+  }
+
+  // ---------------------------------------------------------------- phase 4
+  ok = grid_sync(p.sync, abort, p.status) && ok;
+  if (ok && b < T) {
+    // row t = b of y_acc -> bf16, optionally scaled to unit root-mean-square
+    const int t = b;
+    const float* row = p.y_acc + (size_t)t * d;
+    float scale = 1.0f;
+    if (p.rms) {
+      float ss = 0.0f;
+      for (int n = threadIdx.x; n < d; n += blockDim.x) {
+        const float v = __ldcg(row + n);
+        ss = fmaf(v, v, ss);
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) s_red[warp] = ss;
+      __syncthreads();
+      float tot = lane < (int)(blockDim.x >> 5) ? s_red[lane] : 0.0f;
+      tot = warp_sum(tot);
+      const float ms = tot / (float)d;
+      scale = ms > 0.0f ? rsqrtf(ms) : 0.0f;
+    }
+    for (int n2 = threadIdx.x; n2 < d / 2; n2 += blockDim.x) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(row) + n2);
+      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v.x * scale));
+      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v.y * scale));
+      reinterpret_cast<uint32_t*>(p.y + (size_t)t * d)[n2] = lo | (hi << 16);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+size_t a256l(size_t v) { return (v + 255) & ~(size_t)255; }
+int layer_grid(int num_sms) { return num_sms > 1 ? num_sms - 1 : 1; }
+}  // namespace
+
+size_t layer_dec_ws_bytes(int64_t T, int E) { return 256 + a256l((size_t)T * E * 4); }
+
+bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms) {
+  const int G = layer_grid(num_sms);
+  if (!dec_shape_ok(T, d, I) || k < 1 || k > kLayerMaxK || E < k || E > 1024) return false;
+  if (E > G * (kDecThreads / 32)) return false;  // router rows: one per warp
+  const int nst = dec_stages(d);
+  if ((size_t)nst * kDecStageBytes < layer_scratch_head(d) + kLayerScratchTail) return false;
+  const int64_t slots = (T * k < E ? T * k : E) + has_shared;
+  return (slots * (I / 64) + G - 1) / G <= kDecMaxUnits;
+}
+
+cudaError_t init_layer_dec_attributes() {
+  return cudaFuncSetAttribute(layer_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmemBudget);
+}
+
+cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st) {
+  uint8_t* w = reinterpret_cast<uint8_t*>(ws);
+  LayerArgs p;
+  p.x = a.x;
+  p.ts_in = a.ts_in;
+  p.Wr = a.Wr;
+  p.br = a.br;
+  p.routed = a.routed;
+  p.shared = a.shared;
+  p.has_shared = a.has_shared;
+  p.E = a.E; p.d = a.d; p.I = a.I; p.T = a.T; p.k = a.k;
+  p.nstages = dec_stages(a.d);
+  p.group_chunks = dec_group_chunks(a.d);
+  p.rms = a.rms;
+  p.xq_codes = a.xq_codes;
+  p.xq_scales = a.xq_scales;
+  p.xq_ts = a.xq_ts;
+  p.topk_idx = a.topk_idx;
+  p.topk_w = a.topk_w;
+  p.counts = a.counts;
+  p.offsets = a.offsets;
+  p.sorted_assign = a.sorted_assign;
+  p.assign_pos = a.assign_pos;
+  p.y_acc = a.y_acc;
+  p.y = a.y;
+  p.sync = reinterpret_cast<int32_t*>(w);
+  p.logits = reinterpret_cast<float*>(w + 256);
+  p.status = status;
+  DecMaps maps;
+  cudaError_t e = dec_encode_maps(&maps, a.routed, a.shared, a.has_shared, a.E, a.d, a.I);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st, maps, p);
+}
+
+}  // namespace moe

@@ -1,0 +1,140 @@
+// Device routines of the routing step shared by the routing kernels and the fused decode
+// layer kernel: per-token top-k with renormalised weights, and the stable counting sort of a
+// few hundred assignments by one warp.
+//
+// Basalt pages: "What Basalt changes in a Blackwell local inference stack", section
+// "Experts can move without becoming free" (each token selects a subset of experts).
+// Reading: top-k by logit with ties to the lower expert id; weights = softmax restricted to
+// the top-k and renormalised, exp(l_j - l_max) / sum over the chosen k; the permutation is a
+// stable counting sort of assignments a = t*k + j by expert.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// float -> unsigned key with the same order
+MOE_DEV uint32_t ordered_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One warp per token. Lane L holds logits L, L+32, ... and keeps its own best remaining
+// entry; each of the k rounds takes the warp arg-max (ties to the lower index) and only the
+// winning lane rescans. Outputs (each may be NULL): idx_out / w_out in global memory,
+// idx_smem / w_smem in shared memory, k entries each, in descending logit order.
+template <int NPER>
+MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* idx_out, float* w_out,
+                        int* idx_smem = nullptr, float* w_smem = nullptr) {
+  const int lane = threadIdx.x & 31;
+  uint32_t key[NPER];
+#pragma unroll
+  for (int j = 0; j < NPER; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = e < E ? ordered_key(row[e]) : 0u;  // 0 is below every finite float's key
+  }
+  uint32_t taken = 0;
+  // this lane's best remaining entry: largest key, lowest index among equal keys
+  auto local_best = [&](uint32_t& bk, int& be) {
+    bk = 0u;
+    be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NPER; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u) && (key[j] > bk || (key[j] == bk && e < be))) bk = key[j], be = e;
+    }
+  };
+  uint32_t lbk;
+  int lbe;
+  local_best(lbk, lbe);
+  uint32_t top_key = 0, my_key = 0;
+  int my_e = 0;
+  for (int r = 0; r < k; ++r) {
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, lbk);
+    const int me = (int)__reduce_min_sync(0xffffffffu, lbk == mk ? (uint32_t)lbe : 0x7fffffffu);
+    if (r == 0) top_key = mk;
+    if (lane == r) my_key = mk, my_e = me;
+    if ((me & 31) == lane) {
+      taken |= 1u << (me >> 5);
+      local_best(lbk, lbe);
+    }
+  }
+  auto key_to_float = [](uint32_t kk) {
+    return __uint_as_float((kk & 0x80000000u) ? (kk & 0x7fffffffu) : ~kk);
+  };
+  const float ex = (lane < k) ? expf(key_to_float(my_key) - key_to_float(top_key)) : 0.0f;
+  const float sum = warp_sum(ex);
+  if (lane < k) {
+    const float w = ex / sum;
+    if (idx_out) idx_out[lane] = my_e;
+    if (w_out) w_out[lane] = w;
+    if (idx_smem) idx_smem[lane] = my_e;
+    if (w_smem) w_smem[lane] = w;
+  }
+}
+
+MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w, int* idx_smem = nullptr,
+                           float* w_smem = nullptr) {
+  if (E <= 256) topk_token<8>(row, E, k, idx, w, idx_smem, w_smem);
+  else if (E <= 512) topk_token<16>(row, E, k, idx, w, idx_smem, w_smem);
+  else topk_token<32>(row, E, k, idx, w, idx_smem, w_smem);
+}
+
+// The permutation of n <= 32*k assignments by one warp, without block-wide barriers:
+// histogram of sidx[0..n) (match_any leaders), warp scan of the counts, then a stable
+// scatter in assignment order, 32 at a time. sh: E ints of shared scratch.
+MOE_DEV void perm_small_warp(const int* sidx, int n, int E, int* sh, int32_t* counts, int32_t* offsets,
+                             int32_t* sorted_assign, int32_t* assign_pos) {
+  const int lane = threadIdx.x & 31;
+  for (int e = lane; e < E; e += 32) sh[e] = 0;
+  __syncwarp();
+  for (int base = 0; base < n; base += 32) {
+    const int a = base + lane;
+    const int e = a < n ? sidx[a] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    if (a < n && (peers & ((1u << lane) - 1u)) == 0) sh[e] += __popc(peers);
+    __syncwarp();
+  }
+  // exclusive scan of sh[0..E): lane L owns the contiguous range [L*per, (L+1)*per)
+  const int per = (E + 31) / 32;
+  int local = 0;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < E) local += sh[e];
+  }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - local;
+  for (int i = 0; i < per; ++i) {
+    const int e = lane * per + i;
+    if (e < E) {
+      const int c = sh[e];
+      counts[e] = c;
+      offsets[e] = run;
+      sh[e] = run;
+      run += c;
+    }
+  }
+  if (lane == 31) offsets[E] = incl;
+  __syncwarp();
+  for (int base = 0; base < n; base += 32) {
+    const int a = base + lane;
+    const int e = a < n ? sidx[a] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (a < n) {
+      const int pos = sh[e] + rank;
+      sorted_assign[pos] = a;
+      assign_pos[a] = pos;
+    }
+    __syncwarp();
+    if (a < n && (peers >> lane) == 1u) sh[e] += __popc(peers);  // highest lane of its group
+    __syncwarp();
+  }
+}
+
+}  // namespace moe

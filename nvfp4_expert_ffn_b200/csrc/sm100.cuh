@@ -11,6 +11,7 @@
 namespace moe {
 
 constexpr int32_t kStatusTimeout = 4;                   // MOE_ERR_TIMEOUT
+constexpr int32_t kStatusUnsupported = 2;               // MOE_ERR_UNSUPPORTED_SHAPE
 constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;  // 2 s
 
 MOE_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }

@@ -33,7 +33,7 @@ enum TraceEvent : uint32_t {
 constexpr int kTraceCtas = 160, kTraceCap = 254;
 
 #ifdef MOE_TRACE
-#define TC_TRACE_ARRAY(name) __device__ unsigned long long name[kTraceCtas][kTraceCap + 2];
+#define TC_TRACE_ARRAY(name) static __device__ unsigned long long name[kTraceCtas][kTraceCap + 2];
 #define TC_TRACE_DECL __shared__ unsigned int s_trace_n; __shared__ long long s_trace_clk0;
 #define TC_TRACE_BEGIN(arr)                                                         \
   do {                                                                              \
@@ -67,7 +67,7 @@ int64_t trace_fetch(A& arr, void* host, size_t bytes) {
 }
 // short kernels: globaltimer stamps [kernel][cta][event] (event 0 = entry)
 constexpr int kRtKernels = 8, kRtEvents = 8;
-#define RT_TRACE_ARRAY(name) __device__ unsigned long long name[kRtKernels][kTraceCtas][kRtEvents];
+#define RT_TRACE_ARRAY(name) static __device__ unsigned long long name[kRtKernels][kTraceCtas][kRtEvents];
 #define RT_TRACE(arr, kern, ev)                                                                   \
   do {                                                                                           \
     if (threadIdx.x == 0 && blockIdx.x < kTraceCtas) arr[kern][blockIdx.x][ev] = globaltimer_ns(); \

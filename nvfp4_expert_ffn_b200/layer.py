@@ -47,7 +47,8 @@ class MoeLayer:
     """Device buffers for one layer and up to T_max tokens per call."""
 
     def __init__(self, experts: B.Experts, Wr: torch.Tensor, br: Optional[torch.Tensor], k: int,
-                 T_max: int, static_ts: Optional[torch.Tensor] = None, device="cuda"):
+                 T_max: int, static_ts: Optional[torch.Tensor] = None, device="cuda",
+                 fused: Optional[bool] = None):
         self.experts, self.Wr, self.br, self.k = experts, Wr, br, k
         r = experts.routed
         self.E, self.d, self.I = r.E, r.d, r.I
@@ -76,16 +77,40 @@ class MoeLayer:
         self.path = B.MOE_PATH_AUTO
         self._side = torch.cuda.Stream(device=dev)
         self._ev = [torch.cuda.Event() for _ in range(4)]
+        # calls of at most 8 tokens go through the one-kernel decode layer when the shapes allow;
+        # its workspace holds a barrier counter and must start zeroed
+        can_fuse = (d % 512 == 0 and d <= 4096 and I % 64 == 0 and k <= 32 and E <= 1024
+                    and experts.routed.dn_codes_slice is not None
+                    and (experts.shared is None or experts.shared.dn_codes_slice is not None))
+        self.fused = can_fuse if fused is None else (fused and can_fuse)
+        self.ws_dec = torch.zeros(
+            max(256, B.moe_workspace_size(B.MOE_OP_LAYER_DECODE, min(T_max, 8), d, E, k, I)),
+            dtype=torch.uint8, device=dev) if self.fused else None
 
-    def forward(self, x: torch.Tensor, rms_renorm: bool = False, stream=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, rms_renorm: bool = False, stream=None,
+                join: bool = True) -> torch.Tensor:
         """x: bf16 bits (int16 or bfloat16) [T][d] on the GPU. Returns y bf16 bits [T][d]
         (a view into this layer's output buffer). Enqueued on `stream` (default: current);
-        the quantiser and the expert histogram run on a side stream that forks from and
-        joins back into it, so the call is capturable in a CUDA graph."""
+        work on the side stream (the quantiser, the expert histogram) forks from it and, with
+        join=True, joins back at the end, so the call is capturable in a CUDA graph. With
+        join=False the histogram may still run when the call returns; join(stream) later."""
         T, k = x.shape[0], self.k
         assert T <= self.T_max
         main = torch.cuda.current_stream() if stream is None else stream
         side, ev = self._side, self._ev
+        if self.fused and T <= 8:
+            B.moe_layer_decode(x, self.static_ts, self.Wr, self.br, self.experts, k,
+                               self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
+                               self.topk_idx[:T], self.topk_w[:T], self.counts, self.offsets,
+                               self.sorted_assign[:T * k], self.assign_pos[:T * k],
+                               self.y_acc[:T], self.y[:T], rms_renorm, self.ws_dec, stream=main)
+            ev[2].record(main)
+            side.wait_event(ev[2])
+            B.moe_expert_hist(self.counts, self.cum, self.rank, stream=side)
+            ev[3].record(side)
+            if join:
+                main.wait_event(ev[3])
+            return self.y[:T]
         ev[0].record(main)
         side.wait_event(ev[0])
         B.nvfp4_quantize_act(x, self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
@@ -105,8 +130,13 @@ class MoeLayer:
         ev[3].record(side)
         B.moe_combine(T, self.d, k, B.MOE_FFN_ACCUMULATE, self.y_acc[:T], None, self.topk_w[:T],
                       self.assign_pos[:T * k], rms_renorm, self.y[:T], stream=main)
-        main.wait_event(ev[3])
+        if join:
+            main.wait_event(ev[3])
         return self.y[:T]
+
+    def join(self, stream=None) -> None:
+        """Make `stream` (default: current) wait for this layer's side-stream work."""
+        (torch.cuda.current_stream() if stream is None else stream).wait_event(self._ev[3])
 
     def graphed(self, T: int) -> "GraphedMoeLayer":
         """A replayable CUDA graph of forward() for a fixed token count (decode loops)."""

@@ -15,18 +15,21 @@ from helpers import (OracleWeights, assert_close_layer, bits_to_f32, compare_top
 pytestmark = pytest.mark.gpu
 
 
-def _layer(cfg_name, seed=0, T_max=64):
+def _layer(cfg_name, seed=0, T_max=64, fused=None):
     cfg = synth.CONFIGS[cfg_name]
     routed = L.quantize_weights_gpu(seed, cfg)
     shared = L.quantize_weights_gpu(seed, cfg, shared=True) if cfg.shared else None
     Wr, br = synth.make_router(seed, cfg)
-    lay = L.MoeLayer(B.Experts(routed, shared), Wr.cuda(), br.cuda(), cfg.k, T_max)
+    lay = L.MoeLayer(B.Experts(routed, shared), Wr.cuda(), br.cuda(), cfg.k, T_max, fused=fused)
     return cfg, lay, Wr.numpy(), br.numpy()
 
 
-@pytest.mark.parametrize("cfg_name,T", [("tiny", 16), ("decode", 1), ("decode", 8)])
-def test_layer_matches_oracle(cfg_name, T):
-    cfg, lay, Wr, br = _layer(cfg_name)
+@pytest.mark.parametrize("cfg_name,T,fused", [("tiny", 16, None), ("decode", 1, False), ("decode", 8, False),
+                                              ("decode", 1, True), ("decode", 4, True), ("decode", 8, True)])
+def test_layer_matches_oracle(cfg_name, T, fused):
+    cfg, lay, Wr, br = _layer(cfg_name, fused=fused)
+    if fused:
+        assert lay.fused
     ow = OracleWeights(0, cfg)
     x = synth.make_x(0, cfg, T, step=3)
     y = lay.forward(x.cuda())
@@ -36,8 +39,11 @@ def test_layer_matches_oracle(cfg_name, T):
     keep = [t for t in range(T) if t not in set(excused)]
     assert_close_layer(bits_to_f32(y.cpu().numpy())[keep], ref["y"][keep], cfg_name)
     assert np.array_equal(lay.xq_codes[:T].cpu().numpy(), ref["x_codes"])
+    assert np.array_equal(lay.xq_scales[:T].cpu().numpy(), ref["x_scales"])
     if not excused:
         assert np.array_equal(lay.counts.cpu().numpy(), ref["counts"])
+        assert np.array_equal(lay.offsets.cpu().numpy(), ref["offsets"])
+        assert np.array_equal(lay.sorted_assign[:T * cfg.k].cpu().numpy(), ref["sorted_assign"])
         cum, rank = omoe.hist_update(ref["counts"])
         assert np.array_equal(lay.cum.cpu().numpy(), cum)
         assert np.array_equal(lay.rank.cpu().numpy(), rank)
@@ -100,3 +106,26 @@ def test_graphed_layer_step_matches_forward():
         torch.cuda.synchronize()
         assert torch.equal(got, want) or np.allclose(
             bits_to_f32(got.numpy()), bits_to_f32(want.numpy()), rtol=1e-2, atol=1e-3)
+
+
+def test_fused_decode_layer_repeated_calls():
+    """The one-kernel decode layer leaves its barrier counter at zero, gives the same result on
+    repeated calls, and agrees with the five-call path on the same inputs."""
+    cfg, lay, Wr, br = _layer("decode", T_max=8, fused=True)
+    _, lay5, _, _ = _layer("decode", T_max=8, fused=False)
+    outs = []
+    for step in range(3):
+        x = synth.make_x(7, cfg, 8, step=step).cuda()
+        y = lay.forward(x).clone()
+        y5 = lay5.forward(x).clone()
+        torch.cuda.synchronize()
+        assert B.moe_get_device_status() == 0
+        assert int(lay.ws_dec[:4].view(torch.int32)[0]) == 0
+        a, b5 = bits_to_f32(y.cpu().numpy()), bits_to_f32(y5.cpu().numpy())
+        assert np.abs(a - b5).max() <= 2e-2 * np.sqrt((b5 ** 2).mean())
+        assert np.array_equal(lay.topk_idx.cpu().numpy(), lay5.topk_idx.cpu().numpy())
+        outs.append(y.cpu())
+    x = synth.make_x(7, cfg, 8, step=0).cuda()
+    y = lay.forward(x).clone()
+    torch.cuda.synchronize()
+    assert np.allclose(bits_to_f32(y.cpu().numpy()), bits_to_f32(outs[0].numpy()), rtol=1e-2, atol=1e-3)
