@@ -219,8 +219,9 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
  *   topk_w [T][k]; counts [E], offsets [E+1], sorted_assign [T*k], assign_pos [T*k];
  *   y_acc float32 [T][d] (the unrounded output); y_bf16 [T][d]; rms_renorm as moe_combine.
  *   ws: moe_workspace_size(MOE_OP_LAYER_DECODE, ...) bytes, zero-filled before the first
- *   call (it holds the counter of the kernel's grid-wide barrier, which every call leaves
- *   at zero; after a MOE_ERR_TIMEOUT from moe_get_device_status, zero it again).
+ *   call (it holds the arrival counter of the kernel's grid-wide barrier, which every call
+ *   leaves at a multiple of the grid size; after a MOE_ERR_TIMEOUT from
+ *   moe_get_device_status, zero it again).
  * Limits: 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024.
  * The kernel uses all SMs but one and waits at grid-wide barriers, so it must not share the
  * GPU with a kernel that occupies more than one SM until this one ends.

@@ -422,15 +422,18 @@ int64_t trace_fetch_tc(void* host, size_t bytes);
 int64_t trace_fetch_dec(void* host, size_t bytes);
 int64_t trace_fetch_route(void* host, size_t bytes);
 int64_t trace_fetch_prep(void* host, size_t bytes);
+int64_t trace_fetch_layer(void* host, size_t bytes);
 }  // namespace moe
 // Trace builds only: timeline records of the last runs of the tensor-core FFN kernel
 // (kernel 0: the grouped-GEMM path, 1: the decode path; 2: entry/wait/exit stamps of the
-// routing kernels, 3: of the decode preparation and FFN kernels), copied to `host` and cleared.
+// routing kernels, 3: of the decode preparation and FFN kernels, 4: phase stamps of the
+// one-kernel decode layer), copied to `host` and cleared.
 extern "C" int64_t moe_trace_fetch(int32_t kernel, void* host, size_t bytes) {
   switch (kernel) {
     case 0: return moe::trace_fetch_tc(host, bytes);
     case 1: return moe::trace_fetch_dec(host, bytes);
     case 2: return moe::trace_fetch_route(host, bytes);
+    case 4: return moe::trace_fetch_layer(host, bytes);
     default: return moe::trace_fetch_prep(host, bytes);
   }
 }

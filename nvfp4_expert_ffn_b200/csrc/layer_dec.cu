@@ -19,7 +19,7 @@
 //   barrier
 //   phase 4  CTA t < T converts row t of y_acc to bf16 (optionally RMS-renormalised).
 // The grid barrier counts arrivals in a workspace word that must be zero before the first
-// call; every barrier leaves it at zero.
+// call; every call leaves it at a multiple of the grid size.
 #include <cuda_bf16.h>
 
 #include "dec_core.cuh"
@@ -28,6 +28,8 @@
 namespace moe {
 
 constexpr int kLayerMaxK = 32;
+
+RT_TRACE_ARRAY(g_layer_trace)
 
 struct LayerArgs {
   const uint16_t* x;   // [T][d] bf16
@@ -53,39 +55,38 @@ struct LayerArgs {
   uint16_t* y;         // [T][d] bf16
   // workspace
   float* logits;       // [T][E]
-  int32_t* sync;       // [2]: arrival count (zero between barriers), generation
+  unsigned long long* sync;  // arrival counter of the grid barrier (zero before the first call)
   int32_t* status;
 };
 
-// Grid-wide barrier: thread 0 of each CTA reads the generation, then counts itself in; the
-// last to arrive resets the count and advances the generation, the others wait (bounded)
-// for it to change. Writes before the barrier are visible to every CTA after it.
-MOE_DEV bool grid_sync(int32_t* sync, volatile int* abort, int32_t* status) {
+// Grid-wide barrier on a 64-bit arrival counter that only grows: thread 0 of each CTA adds
+// one and waits (bounded) until the count reaches the next multiple of the grid size. The
+// counter starts at zero and every call adds two multiples, so it stays aligned. Writes
+// before the barrier are visible to every CTA after it.
+MOE_DEV bool grid_sync(unsigned long long* count, volatile int* abort, int32_t* status) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = *abort ? 0 : 1;
     if (ok) {
-      const int32_t g0 = ld_acquire_gpu(sync + 1);
+      const unsigned long long G = gridDim.x;
       __threadfence();
-      if (atomicAdd(sync, 1) == (int)gridDim.x - 1) {
-        atomicExch(sync, 0);
-        __threadfence();
-        atomicAdd(sync + 1, 1);
-      } else {
-        const uint64_t t0 = globaltimer_ns();
-        while (ld_acquire_gpu(sync + 1) == g0) {
-          if (*abort) {
-            ok = 0;
-            break;
-          }
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicExch(status, kStatusTimeout);
-            ok = 0;
-            break;
-          }
-          __nanosleep(32);
+      const unsigned long long old = atomicAdd(count, 1ull);
+      const unsigned long long target = (old / G + 1) * G;
+      const uint64_t t0 = globaltimer_ns();
+      while (true) {
+        unsigned long long c;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count) : "memory");
+        if (c >= target) break;
+        if (*abort) {
+          ok = 0;
+          break;
+        }
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+          *abort = 1;
+          atomicExch(status, kStatusTimeout);
+          ok = 0;
+          break;
         }
       }
       __threadfence();
@@ -145,6 +146,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   const int nvec = d / 4;  // float4 per router row
   volatile int* abort = reinterpret_cast<volatile int*>(&bar.abort);
 
+  RT_TRACE(g_layer_trace, 0, 0);
   dec_init(bar, p.nstages, maps, p.has_shared);
   // this warp's router row; its first 512 float4 (d <= 2048: all of it) are loaded before
   // the kernel waits on its predecessor (the router weights are not written by anything)
@@ -158,6 +160,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     w[u] = (has_row && c < nvec) ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   MOE_PDL_PROLOGUE();
+  RT_TRACE(g_layer_trace, 0, 1);
 
   // ---------------------------------------------------------------- phase 1
   // x -> shared memory (every load of a round in flight before the stores)
@@ -180,6 +183,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     }
   }
   __syncthreads();
+  RT_TRACE(g_layer_trace, 0, 2);
   // NVFP4 tensor scale: amax / (6 * 448) over all T tokens (every CTA computes the same), or
   // the static scale
   float ts;
@@ -202,26 +206,35 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     f = warp_max(f);
     ts = f > 0.0f ? __fdiv_rn(f, kE2M1Max * kE4M3Max) : 1.0f;
   }
-  // this CTA's share of the 16-element blocks: codes and scales into the xq outputs
+  RT_TRACE(g_layer_trace, 2, 0);
+  // this CTA's share of the 16-element blocks (b, b + G, ...): codes and scales into the xq
+  // outputs, one block per 16 lanes (the steps of quantize_block16, one element per lane)
   {
     const int nblk = T * (d / kBlock);
-    for (int q = b + G * (int)threadIdx.x; q < nblk; q += G * (int)blockDim.x) {
-      const int t = q / (d / kBlock), blk = q % (d / kBlock);
-      const uint4* src = reinterpret_cast<const uint4*>(sc.xb + (size_t)t * d + kBlock * blk);
-      const uint4 p0 = src[0], p1 = src[1];
-      const uint32_t wd[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-      float v[16];
+    const int h = lane >> 4, e16 = lane & 15;
+    for (int i0 = 0; b + G * i0 < nblk; i0 += 2 * (int)(blockDim.x >> 5)) {
+      const int q = b + G * (i0 + 2 * warp + h);
+      const bool valid = q < nblk;
+      float v = 0.0f;
+      if (valid) v = bf16_to_f32(sc.xb[(size_t)(q / (d / kBlock)) * d + kBlock * (q % (d / kBlock)) + e16]);
+      float amax = fabsf(v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[2 * i] = bf16_to_f32(wd[i] & 0xFFFFu);
-        v[2 * i + 1] = bf16_to_f32(wd[i] >> 16);
-      }
-      uint2 codes;
-      p.xq_scales[q] = (uint8_t)quantize_block16(v, ts, &codes);
-      reinterpret_cast<uint2*>(p.xq_codes)[q] = codes;
+      for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const uint32_t sbyte = f32_to_e4m3_sat(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), ts));
+      const float sval = e4m3_to_f32(sbyte);
+      uint32_t nib = 0u;
+      if (sval != 0.0f) nib = f32x2_to_e2m1x2(__fdiv_rn(v, __fmul_rn(sval, ts)), 0.0f) & 0xFu;
+      const uint32_t pr = nib | (__shfl_down_sync(0xffffffffu, nib, 1) << 4);
+      const uint32_t p1 = __shfl_down_sync(0xffffffffu, pr, 2), p2 = __shfl_down_sync(0xffffffffu, pr, 4),
+                     p3 = __shfl_down_sync(0xffffffffu, pr, 6);
+      if (valid && (e16 & 7) == 0)
+        reinterpret_cast<uint32_t*>(p.xq_codes)[2 * q + (e16 >> 3)] =
+            (pr & 0xFFu) | ((p1 & 0xFFu) << 8) | ((p2 & 0xFFu) << 16) | ((p3 & 0xFFu) << 24);
+      if (valid && e16 == 0) p.xq_scales[q] = (uint8_t)sbyte;
     }
     if (b == G - 1 && threadIdx.x == 0) *p.xq_ts = ts;
   }
+  RT_TRACE(g_layer_trace, 2, 1);
   // router logits of this warp's row: 64-term lane partials, then a lane tree per token
   if (has_row) {
     float acc[kDecMaxT];
@@ -261,12 +274,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
       }
     }
   }
+  RT_TRACE(g_layer_trace, 2, 2);
   // y_acc starts at zero: the units add into it after the barrier
   if (b == 0) {
     float4* y4 = reinterpret_cast<float4*>(p.y_acc);
     for (int i = threadIdx.x; i < T * d / 4; i += blockDim.x) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  RT_TRACE(g_layer_trace, 0, 3);
   bool ok = grid_sync(p.sync, abort, p.status);
+  RT_TRACE(g_layer_trace, 0, 4);
 
   // ---------------------------------------------------------------- phase 2
   // Data written by other CTAs before the barrier is read through L2 (ld.global.cg).
@@ -274,28 +290,51 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   const bool writer = b == G - 1;  // the CTA with the fewest units writes the routing outputs
   int nu = 0;
   if (ok) {
-    // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms
-    for (int i = threadIdx.x; i < kDecMaxT * (d / 32); i += blockDim.x) {
-      const int t = i / (d / 32), c = i % (d / 32);
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (t < T) v = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
-      *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(t, c)) = v;
+    // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms; each thread's
+    // loads of a round go out together
+    {
+      const int nc = kDecMaxT * (d / 32);
+      for (int i0 = threadIdx.x; i0 < nc; i0 += 4 * blockDim.x) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * blockDim.x, t = i / (d / 32), c = i % (d / 32);
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (i < nc && t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * blockDim.x;
+          if (i < nc) *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(i / (d / 32), i % (d / 32))) = v[u];
+        }
+      }
+      const int ns = (d / 64) * 32;
+      for (int i0 = threadIdx.x; i0 < ns; i0 += 4 * blockDim.x) {
+        uint32_t wd[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * blockDim.x, kc = i / 32, t = (i % 32) & 7;
+          wd[u] = 0u;
+          if (i < ns && t < T)
+            wd[u] = __ldcg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock)) + kc);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * blockDim.x;
+          if (i < ns) dec_xsf_store(sm.xsf, i / 32, i % 32, wd[u]);
+        }
+      }
     }
-    for (int i = threadIdx.x; i < (d / 64) * 32; i += blockDim.x) {
-      const int kc = i / 32, r0 = i % 32, t = r0 & 7;
-      uint32_t wd = 0u;
-      if (t < T) wd = __ldcg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock)) + kc);
-      dec_xsf_store(sm.xsf, kc, r0, wd);
-    }
-    for (int i = threadIdx.x; i < T * E; i += blockDim.x) sc.logits[i] = __ldcg(p.logits + i);
     for (int e = threadIdx.x; e < E; e += blockDim.x) sc.flag[e] = 0;
     __syncthreads();
+    RT_TRACE(g_layer_trace, 3, 0);
     // top-k of every token (one warp each)
     if (warp < T)
-      topk_dispatch(sc.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
-                    writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
-                    sc.tw + warp * kLayerMaxK);
+      topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
+                          writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
+                          sc.tw + warp * kLayerMaxK);
     __syncthreads();
+    RT_TRACE(g_layer_trace, 3, 1);
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
       const int e = sc.tidx[(i / k) * kLayerMaxK + i % k];
       sc.flag[e] = 1;
@@ -314,6 +353,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     if (threadIdx.x == 0 && p.has_shared) sc.list[0] = E;
     const int nslots = total + p.has_shared;
     __syncthreads();
+    RT_TRACE(g_layer_trace, 3, 2);
     if (writer && warp == 0)
       perm_small_warp(sc.sidx, T * k, E, sc.perm, p.counts, p.offsets, p.sorted_assign, p.assign_pos);
     // this CTA's units: blockIdx.x, blockIdx.x + gridDim.x, ... of nslots * nt1
@@ -349,6 +389,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
 
+  RT_TRACE(g_layer_trace, 0, 5);
   // ---------------------------------------------------------------- phase 3
   DecArgs a;
   a.routed = p.routed;
@@ -366,8 +407,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     tmem_dealloc(bar.tmem, 512);
   }
 
+  RT_TRACE(g_layer_trace, 0, 6);
   // ---------------------------------------------------------------- phase 4
   ok = grid_sync(p.sync, abort, p.status) && ok;
+  RT_TRACE(g_layer_trace, 1, 0);
   if (ok && b < T) {
     // row t = b of y_acc -> bf16, optionally scaled to unit root-mean-square
     const int t = b;
@@ -394,6 +437,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
       reinterpret_cast<uint32_t*>(p.y + (size_t)t * d)[n2] = lo | (hi << 16);
     }
   }
+  RT_TRACE(g_layer_trace, 1, 1);
 }
 
 // ---------------------------------------------------------------- host side
@@ -443,7 +487,7 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
   p.assign_pos = a.assign_pos;
   p.y_acc = a.y_acc;
   p.y = a.y;
-  p.sync = reinterpret_cast<int32_t*>(w);
+  p.sync = reinterpret_cast<unsigned long long*>(w);
   p.logits = reinterpret_cast<float*>(w + 256);
   p.status = status;
   DecMaps maps;
@@ -453,3 +497,9 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
 }
 
 }  // namespace moe
+
+#ifdef MOE_TRACE
+namespace moe {
+int64_t trace_fetch_layer(void* host, size_t bytes) { return trace_fetch(g_layer_trace, host, bytes); }
+}  // namespace moe
+#endif

@@ -22,8 +22,10 @@ MOE_DEV uint32_t ordered_key(float v) {
 // One warp per token. Lane L holds logits L, L+32, ... and keeps its own best remaining
 // entry; each of the k rounds takes the warp arg-max (ties to the lower index) and only the
 // winning lane rescans. Outputs (each may be NULL): idx_out / w_out in global memory,
-// idx_smem / w_smem in shared memory, k entries each, in descending logit order.
-template <int NPER>
+// idx_smem / w_smem in shared memory, k entries each, in descending logit order. With
+// kL2 = true the logits are read through L2 (ld.global.cg: written by other CTAs of the
+// same kernel).
+template <int NPER, bool kL2 = false>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* idx_out, float* w_out,
                         int* idx_smem = nullptr, float* w_smem = nullptr) {
   const int lane = threadIdx.x & 31;
@@ -31,7 +33,9 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
 #pragma unroll
   for (int j = 0; j < NPER; ++j) {
     const int e = lane + 32 * j;
-    key[j] = e < E ? ordered_key(row[e]) : 0u;  // 0 is below every finite float's key
+    float v = 0.0f;
+    if (e < E) v = kL2 ? __ldcg(row + e) : row[e];
+    key[j] = e < E ? ordered_key(v) : 0u;  // 0 is below every finite float's key
   }
   uint32_t taken = 0;
   // this lane's best remaining entry: largest key, lowest index among equal keys
@@ -73,11 +77,12 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
   }
 }
 
+template <bool kL2 = false>
 MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w, int* idx_smem = nullptr,
                            float* w_smem = nullptr) {
-  if (E <= 256) topk_token<8>(row, E, k, idx, w, idx_smem, w_smem);
-  else if (E <= 512) topk_token<16>(row, E, k, idx, w, idx_smem, w_smem);
-  else topk_token<32>(row, E, k, idx, w, idx_smem, w_smem);
+  if (E <= 256) topk_token<8, kL2>(row, E, k, idx, w, idx_smem, w_smem);
+  else if (E <= 512) topk_token<16, kL2>(row, E, k, idx, w, idx_smem, w_smem);
+  else topk_token<32, kL2>(row, E, k, idx, w, idx_smem, w_smem);
 }
 
 // The permutation of n <= 32*k assignments by one warp, without block-wide barriers:

@@ -109,8 +109,8 @@ def test_graphed_layer_step_matches_forward():
 
 
 def test_fused_decode_layer_repeated_calls():
-    """The one-kernel decode layer leaves its barrier counter at zero, gives the same result on
-    repeated calls, and agrees with the five-call path on the same inputs."""
+    """The one-kernel decode layer leaves its barrier counter aligned to the grid, gives the same
+    result on repeated calls, and agrees with the five-call path on the same inputs."""
     cfg, lay, Wr, br = _layer("decode", T_max=8, fused=True)
     _, lay5, _, _ = _layer("decode", T_max=8, fused=False)
     outs = []
@@ -120,7 +120,10 @@ def test_fused_decode_layer_repeated_calls():
         y5 = lay5.forward(x).clone()
         torch.cuda.synchronize()
         assert B.moe_get_device_status() == 0
-        assert int(lay.ws_dec[:4].view(torch.int32)[0]) == 0
+        # the barrier's arrival counter ends every call at a multiple of the grid size
+        grid = torch.cuda.get_device_properties(0).multi_processor_count - 1
+        count = int(lay.ws_dec[:8].view(torch.int64)[0])
+        assert count > 0 and count % grid == 0
         a, b5 = bits_to_f32(y.cpu().numpy()), bits_to_f32(y5.cpu().numpy())
         assert np.abs(a - b5).max() <= 2e-2 * np.sqrt((b5 ** 2).mean())
         assert np.array_equal(lay.topk_idx.cpu().numpy(), lay5.topk_idx.cpu().numpy())
