@@ -84,6 +84,9 @@ typedef enum moe_status {
  *   dn_codes_slice [E][I/64][d][32], dn_sf_slice [E][I/64][d/128][512]: the down matrix
  *            regrouped by 64-column slices of I (each slice's codes, and its scale atoms,
  *            contiguous), written by moe_pack_experts for the DECODE path (NULL if absent).
+ *   gu_codes_slice [E][I/64][d/256][128][128]: the gate/up codes regrouped the same way:
+ *            per 64-row slice of I and 256-column block of d, one 16 KB tile of the slice's
+ *            64 gate rows then its 64 up rows, 128 bytes each (DECODE path; NULL if absent).
  */
 typedef struct moe_expert_weights {
   int32_t E, d, I;
@@ -97,6 +100,7 @@ typedef struct moe_expert_weights {
   const uint8_t* dn_sf_tiled;
   const uint8_t* dn_codes_slice;
   const uint8_t* dn_sf_slice;
+  const uint8_t* gu_codes_slice;
 } moe_expert_weights_t;
 
 typedef struct moe_experts {
@@ -149,15 +153,17 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
  *     512-byte atoms of 128 weight rows x 4 scale blocks, the layout the tensor core reads
  *     its scales in (gate/up atoms [E][I/64][d/64], atom rows 0-63 gate, 64-127 up; down
  *     atoms [E][d/128][I/64]);
- *   dn_codes_slice (E*d*I/2 bytes), dn_sf_slice (E*d*I/16 bytes), both optional (NULL to
- *     skip): the down codes and scale atoms regrouped per 64-column slice of I, so that
- *     the DECODE path reads each slice as contiguous bytes.
+ *   dn_codes_slice (E*d*I/2 bytes), dn_sf_slice (E*d*I/16 bytes), gu_codes_slice
+ *     (E*2I*d/2 bytes), all three or none (NULL to skip): the down codes and scale atoms
+ *     regrouped per 64-column slice of I, and the gate/up codes per 64-row slice of I and
+ *     256-column block of d, so that the DECODE path reads every weight tile as contiguous
+ *     bytes (the gate/up scale atoms above are already grouped that way).
  * The natural-layout arrays stay as they are and remain in use by the CUDA-core path.
- * Requires d % 128 == 0 and I % 64 == 0.
+ * Requires d % 128 == 0 and I % 64 == 0 (and d % 256 == 0 with the slices).
  */
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
                             uint8_t* dn_sf_tiled, uint8_t* dn_codes_slice, uint8_t* dn_sf_slice,
-                            void* stream);
+                            uint8_t* gu_codes_slice, void* stream);
 
 /*
  * moe_expert_ffn - expert SwiGLU FFN for all routed assignments (A5-A7) and the shared

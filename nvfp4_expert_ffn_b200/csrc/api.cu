@@ -98,7 +98,8 @@ moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E,
 
 ExpertGroup to_group(const moe_expert_weights_t& w) {
   return ExpertGroup{w.gu_codes,    w.gu_scales,   w.gu_ts,          w.dn_codes,      w.dn_scales,
-                     w.dn_ts,       w.gu_sf_tiled, w.dn_sf_tiled, w.dn_codes_slice, w.dn_sf_slice};
+                     w.dn_ts,       w.gu_sf_tiled, w.dn_sf_tiled, w.dn_codes_slice, w.dn_sf_slice,
+                     w.gu_codes_slice};
 }
 
 }  // namespace
@@ -226,15 +227,17 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t d, const float* Wr, c
 
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
                             uint8_t* dn_sf_tiled, uint8_t* dn_codes_slice, uint8_t* dn_sf_slice,
-                            void* stream) {
+                            uint8_t* gu_codes_slice, void* stream) {
   if (!W || !gu_sf_tiled || !dn_sf_tiled) return fail(MOE_ERR_INVALID_ARG, "null argument");
-  if ((dn_codes_slice == nullptr) != (dn_sf_slice == nullptr))
-    return fail(MOE_ERR_INVALID_ARG, "dn_codes_slice and dn_sf_slice are given together");
+  if ((dn_codes_slice == nullptr) != (dn_sf_slice == nullptr) || (dn_codes_slice == nullptr) != (gu_codes_slice == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "dn_codes_slice, dn_sf_slice and gu_codes_slice are given together");
   if ((dn_codes_slice && !aligned16(dn_codes_slice)) || (dn_sf_slice && !aligned16(dn_sf_slice)) ||
-      (dn_codes_slice && (!W->dn_codes || !aligned16(W->dn_codes))))
-    return fail(MOE_ERR_INVALID_ARG, "slice buffers and dn_codes must be 16-byte aligned");
+      (gu_codes_slice && !aligned16(gu_codes_slice)) ||
+      (dn_codes_slice && (!W->dn_codes || !aligned16(W->dn_codes) || !W->gu_codes || !aligned16(W->gu_codes))))
+    return fail(MOE_ERR_INVALID_ARG, "slice buffers, dn_codes and gu_codes must be 16-byte aligned");
   if (W->E < 1 || W->d <= 0 || W->I <= 0) return fail(MOE_ERR_INVALID_ARG, "bad E/d/I");
   if (W->d % 128 || W->I % 64) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "packing needs d % 128 == 0 and I % 64 == 0");
+  if (dn_codes_slice && W->d % 256) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "the slices need d % 256 == 0");
   if (!W->gu_scales || !W->dn_scales) return fail(MOE_ERR_INVALID_ARG, "null scales");
   if (!aligned16(W->gu_scales) || !aligned16(W->dn_scales) || !aligned16(gu_sf_tiled) || !aligned16(dn_sf_tiled))
     return fail(MOE_ERR_INVALID_ARG, "scale pointers must be 16-byte aligned");
@@ -244,7 +247,8 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
   cudaError_t e = launch_pack_sf(to_group(*W), W->E, W->d, W->I, gu_sf_tiled, dn_sf_tiled, sms,
                                  (cudaStream_t)stream);
   if (e == cudaSuccess && dn_codes_slice)
-    e = launch_pack_slices(to_group(*W), W->E, W->d, W->I, dn_codes_slice, dn_sf_slice, sms, (cudaStream_t)stream);
+    e = launch_pack_slices(to_group(*W), W->E, W->d, W->I, dn_codes_slice, dn_sf_slice, gu_codes_slice, sms,
+                           (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_pack_experts launch");
 }
 
@@ -271,7 +275,8 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   if (T == 0) return MOE_OK;
   if (!xq_codes || !xq_scales || !xq_ts || !offsets || !sorted_assign || !topk_w || !out)
     return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned16(xq_codes) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "xq_codes/out must be 16-byte aligned");
+  if (!aligned16(xq_codes) || !aligned16(xq_scales) || !aligned16(out))
+    return fail(MOE_ERR_INVALID_ARG, "xq_codes, xq_scales and out must be 16-byte aligned");
   if (mode == MOE_FFN_PER_ASSIGN && W->has_shared && !shared_out)
     return fail(MOE_ERR_INVALID_ARG, "shared_out needed in PER_ASSIGN mode with a shared expert");
   int sms = 0;
@@ -281,8 +286,9 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
   const bool tc_ok = ffn_tc_supported(d, I) && packed;
-  const bool sliced = W->routed.dn_codes_slice && W->routed.dn_sf_slice &&
-                      (!W->has_shared || (W->shared.dn_codes_slice && W->shared.dn_sf_slice));
+  const bool sliced = W->routed.dn_codes_slice && W->routed.dn_sf_slice && W->routed.gu_codes_slice &&
+                      (!W->has_shared ||
+                       (W->shared.dn_codes_slice && W->shared.dn_sf_slice && W->shared.gu_codes_slice));
   const bool dec_ok = ffn_dec_supported(T, d, I, mode, E, k, W->has_shared ? 1 : 0, sms) && packed && sliced;
   if (path == MOE_PATH_PREFILL && !tc_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
@@ -333,12 +339,14 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
   if (!x || !Wr || !xq_codes || !xq_scales || !xq_ts || !topk_idx || !topk_w || !counts || !offsets ||
       !sorted_assign || !assign_pos || !y_acc || !y)
     return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
-  if (!aligned16(x) || !aligned16(Wr) || !aligned16(xq_codes) || !aligned16(y_acc) || !aligned16(y))
-    return fail(MOE_ERR_INVALID_ARG, "x, Wr, xq_codes, y_acc and y must be 16-byte aligned");
+  if (!aligned16(x) || !aligned16(Wr) || !aligned16(xq_codes) || !aligned16(xq_scales) || !aligned16(y_acc) ||
+      !aligned16(y))
+    return fail(MOE_ERR_INVALID_ARG, "x, Wr, xq_codes, xq_scales, y_acc and y must be 16-byte aligned");
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled && W->routed.dn_codes_slice &&
-                      W->routed.dn_sf_slice &&
+                      W->routed.dn_sf_slice && W->routed.gu_codes_slice &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled &&
-                                          W->shared.dn_codes_slice && W->shared.dn_sf_slice));
+                                          W->shared.dn_codes_slice && W->shared.dn_sf_slice &&
+                                          W->shared.gu_codes_slice));
   if (!packed) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "weights must be packed by moe_pack_experts, slices included");
   int sms = 0;
   int32_t* dstatus = nullptr;

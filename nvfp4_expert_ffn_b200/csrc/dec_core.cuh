@@ -23,9 +23,11 @@
 //     128-row A operand, the tokens a 16-column B operand, so an accumulator takes 16 TMEM
 //     columns and a unit's 16 down chunks accumulate side by side.
 //   * the ring of shared-memory stages carries only weights: a 64-gate + 64-up row x 256-column
-//     tile of the stacked gate/up matrix (TMA, 128-byte swizzle) with its 4 scale atoms, or
-//     four 128-row x 64-column chunks of the slice-grouped down matrix (one TMA box, 32-byte
-//     swizzle) with theirs (one bulk copy).
+//     tile of the slice-grouped gate/up matrix (one contiguous 16 KB TMA box, 128-byte
+//     swizzle) with its 4 scale atoms, or four 128-row x 64-column chunks of the
+//     slice-grouped down matrix (one TMA box, 32-byte swizzle) with theirs (one bulk copy).
+//     Every stage reads contiguous bytes: 128-byte pieces of rows 1 KB apart (the natural
+//     layout) keep HBM well below its streaming rate.
 //
 // Warp roles (352 threads, one CTA per SM): warp 0 lane 0 issues the copies; warps 1 and 2
 // (lane 0) issue tcgen05 copies and MMAs for alternate ring stages (an issued tcgen05
@@ -64,7 +66,7 @@ constexpr uint32_t kColD1 = 0, kColH = 32, kColSf = 48, kColX = 112;
 __host__ __device__ inline uint32_t dec_col_d2(int d) { return (kColX + (uint32_t)d / 16 + 15u) & ~15u; }
 
 struct DecMaps {
-  CUtensorMap b1, b1s;  // gate/up codes {d/2, I, 2, E}, boxes {128, 64, 2, 1}, 128-byte swizzle
+  CUtensorMap b1, b1s;  // gate/up codes by I-slice {128, 128, d/256, E*I/64}, boxes {128, 128, 1, 1}, 128-byte swizzle
   CUtensorMap b2, b2s;  // down codes by I-slice {32, 128, d/128, E*I/64}, boxes {32, 128, 4, 1}, 32-byte swizzle
 };
 
@@ -199,7 +201,6 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
   const int gst = gch / 4;         // down stages per group
   const uint32_t col_d2 = dec_col_d2(d);
   const int nu = U.n;
-  (void)nt1;
   // Gate/up K blocks are visited in an order rotated per CTA and unit (the sum does not
   // depend on the order).
   auto unit_rot = [&](int u) { return (int)((blockIdx.x + 3 * u) % nks1); };
@@ -240,7 +241,7 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
           mbar_arrive_expect_tx(&full[st], kDecStageBytes);
           if (q < nks1) {
             const int kq = (q + rot) % nks1;  // K block of this stage
-            tma_load_4d(sb, sh ? &maps.b1s : &maps.b1, &full[st], kq * 128, 64 * j, 0, el);
+            tma_load_4d(sb, sh ? &maps.b1s : &maps.b1, &full[st], 0, 0, kq, el * nt1 + j);
             bulk_g2s(sb + kDecBBytes, G.gu_sf_tiled + (((size_t)el * nt1 + j) * (d / 64) + 4 * kq) * kDecAtom,
                      4 * kDecAtom, &full[st]);
           } else {
@@ -519,9 +520,10 @@ inline bool dec_shape_ok(int64_t T, int d, int I) {
 }
 
 // Tensor maps of an expert group pair (the shared group, when absent, repeats the routed
-// maps): gate/up codes {d/2, I, 2, E} in {128, 64, 2, 1} boxes (64 gate + 64 up rows x 256
-// columns, 128-byte swizzle); slice-grouped down codes {32, 128, d/128, E*I/64} in
-// {32, 128, 4, 1} boxes (four 128-row chunks of one slice, 32-byte swizzle).
+// maps): slice-grouped gate/up codes {128, 128, d/256, E*I/64} in {128, 128, 1, 1} boxes
+// (one contiguous 16 KB tile: 64 gate + 64 up rows x 256 columns, 128-byte swizzle);
+// slice-grouped down codes {32, 128, d/128, E*I/64} in {32, 128, 4, 1} boxes (four 128-row
+// chunks of one slice, 32-byte swizzle).
 inline cudaError_t dec_encode_maps(DecMaps* maps, const ExpertGroup& routed, const ExpertGroup& shared,
                                    int has_shared, int E_routed, int d, int I) {
   cudaError_t e = get_encode();
@@ -536,10 +538,11 @@ inline cudaError_t dec_encode_maps(DecMaps* maps, const ExpertGroup& routed, con
       *m2 = maps->b2;
       continue;
     }
-    cuuint64_t dims1[4] = {(cuuint64_t)(d / 2), (cuuint64_t)I, 2, (cuuint64_t)E};
-    cuuint64_t str1[3] = {(cuuint64_t)(d / 2), (cuuint64_t)I * (d / 2), (cuuint64_t)2 * I * (d / 2)};
-    cuuint32_t box1[4] = {128, 64, 2, 1};
-    if ((e = encode_u8(m1, g.gu_codes, 4, dims1, str1, box1, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+    cuuint64_t dims1[4] = {128, 128, (cuuint64_t)(d / 256), (cuuint64_t)E * (I / 64)};
+    cuuint64_t str1[3] = {128, 128 * 128, (cuuint64_t)(d / 256) * 128 * 128};
+    cuuint32_t box1[4] = {128, 128, 1, 1};
+    if ((e = encode_u8(m1, g.gu_codes_slice, 4, dims1, str1, box1, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+      return e;
     cuuint64_t dims2[4] = {32, 128, (cuuint64_t)(d / 128), (cuuint64_t)E * (I / 64)};
     cuuint64_t str2[3] = {32, 128 * 32, (cuuint64_t)d * 32};
     cuuint32_t box2[4] = {32, 128, 4, 1};

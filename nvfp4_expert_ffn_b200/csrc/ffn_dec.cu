@@ -96,11 +96,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
     if (t < T) v = __ldg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
     *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(t, c)) = v;
   }
-  for (int i = threadIdx.x; i < (d / 64) * 32; i += blockDim.x) {
-    const int kc = i / 32, r0 = i % 32, t = r0 & 7;
-    uint32_t w = 0u;
-    if (t < T) w = __ldg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock)) + kc);
-    dec_xsf_store(sm.xsf, kc, r0, w);
+  // scale words: token t's row as d/256 16-byte pieces; word kc goes to rows t, t + 8, t + 16,
+  // t + 24 of atom kc (one load per piece: every CTA reads these same few lines)
+  const int q4 = d / 256;
+  if (threadIdx.x < kDecMaxT * q4) {
+    const int t = threadIdx.x / q4, c4 = threadIdx.x % q4;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t < T) v = __ldg(reinterpret_cast<const uint4*>(p.xq_scales + (size_t)t * (d / kBlock)) + c4);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+      for (int r1 = 0; r1 < 4; ++r1) dec_xsf_store(sm.xsf, 4 * c4 + w, t + 8 * r1, wv[w]);
   }
   // this CTA's units (blockIdx.x, blockIdx.x + gridDim.x, ...) from the preparation lists
   const int nunits = *p.nslots * nt1;

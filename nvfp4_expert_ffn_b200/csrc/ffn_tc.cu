@@ -215,12 +215,28 @@ __global__ void pack_sf_kernel(const uint8_t* __restrict__ gu_scales, const uint
 // 32j..32j+31 of row n), scale atoms [E][I/64][d/128][512] (atom (e, j, c) = rows 128c.. of
 // scale blocks 4j..4j+3, laid out as in pack_sf_kernel)
 __global__ void pack_slices_kernel(const uint8_t* __restrict__ dn_codes, const uint8_t* __restrict__ dn_scales,
-                                   int E, int d, int I, uint8_t* __restrict__ cs, uint8_t* __restrict__ ss) {
+                                   const uint8_t* __restrict__ gu_codes, int E, int d, int I,
+                                   uint8_t* __restrict__ cs, uint8_t* __restrict__ ss, uint8_t* __restrict__ gs) {
   const int nj = I / 64;
   const size_t nc = (size_t)E * nj * d * 2;          // 16-byte pieces of codes
   const size_t ns = (size_t)E * nj * (d / 128) * 128;  // 32-bit words of scale atoms
-  for (size_t w = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w < nc + ns; w += (size_t)gridDim.x * blockDim.x) {
-    if (w < nc) {
+  const size_t ng = (size_t)E * I * d / 16;            // 16-byte pieces of gate/up codes
+  for (size_t w = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w < nc + ns + ng;
+       w += (size_t)gridDim.x * blockDim.x) {
+    if (w >= nc + ns) {
+      // gate/up tile (e, j, kb): row r < 64 is gate row 64j + r, row r >= 64 up row 64j + r - 64,
+      // columns 256kb..256kb+255 (128 bytes, 8 pieces)
+      const size_t g = w - nc - ns;
+      const int piece = (int)(g % 8);
+      const int r = (int)((g / 8) % 128);
+      const size_t tile = g / 1024;  // over [E][I/64][d/256]
+      const int kb = (int)(tile % (d / 256));
+      const int j = (int)((tile / (d / 256)) % nj);
+      const size_t e = tile / (d / 256) / nj;
+      const size_t row = e * 2 * I + (r < 64 ? 64 * j + r : I + 64 * j + r - 64);
+      *reinterpret_cast<uint4*>(gs + g * 16) =
+          *reinterpret_cast<const uint4*>(gu_codes + row * (d / 2) + 128 * kb + 16 * piece);
+    } else if (w < nc) {
       const int piece = (int)(w & 1);
       const size_t row = w >> 1;  // over [E][I/64][d]
       const int n = (int)(row % d);
@@ -716,10 +732,10 @@ cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* g
   return cudaGetLastError();
 }
 
-cudaError_t launch_pack_slices(const ExpertGroup& g, int E, int d, int I, uint8_t* cs, uint8_t* ss, int num_sms,
-                               cudaStream_t st) {
+cudaError_t launch_pack_slices(const ExpertGroup& g, int E, int d, int I, uint8_t* cs, uint8_t* ss, uint8_t* gs,
+                               int num_sms, cudaStream_t st) {
   g_launch_count.fetch_add(1, std::memory_order_relaxed);
-  pack_slices_kernel<<<num_sms * 4, 256, 0, st>>>(g.dn_codes, g.dn_scales, E, d, I, cs, ss);
+  pack_slices_kernel<<<num_sms * 4, 256, 0, st>>>(g.dn_codes, g.dn_scales, g.gu_codes, E, d, I, cs, ss, gs);
   return cudaGetLastError();
 }
 

@@ -28,6 +28,7 @@
 namespace moe {
 
 constexpr int kLayerMaxK = 32;
+constexpr int kLayerMaxRows = kDecThreads / 32;  // router rows per CTA (the host checks E <= grid * this)
 
 RT_TRACE_ARRAY(g_layer_trace)
 
@@ -109,6 +110,9 @@ struct LayerScratch {
   int* list;      // [1025] experts in use, in id order after the shared expert
   int* perm;      // [1024] counters of the permutation
   int* sidx;      // [256] top-k expert ids, assignment order
+  float* part;    // [kDecThreads] router partial sums (phase 1)
+  uint32_t* tks;  // [8][64] top-k scratch of each token's warp
+  float* wr;      // [rows][d] this CTA's router rows (phase 1)
 };
 
 __host__ __device__ inline size_t layer_scratch_head(int d) {
@@ -126,10 +130,14 @@ MOE_DEV LayerScratch layer_scratch(uint8_t* ring, int d) {
   s.list = s.flag + 1024;
   s.perm = s.list + 1040;
   s.sidx = s.perm + 1024;
+  s.part = reinterpret_cast<float*>(s.sidx + 256);
+  s.tks = reinterpret_cast<uint32_t*>(s.part + kDecThreads);
+  s.wr = reinterpret_cast<float*>(s.tks + kDecMaxT * 64);
   return s;
 }
 // bytes of scratch past the head
-constexpr size_t kLayerScratchTail = 2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 1040 + 1024 + 256) * 4;
+constexpr size_t kLayerScratchTail = 2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 1040 + 1024 + 256 + kDecThreads + kDecMaxT * 64) * 4;
+static_assert(kLayerScratchTail % 16 == 0, "router rows must start 16-byte aligned");
 
 __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_constant__ DecMaps maps, LayerArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -147,17 +155,18 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   volatile int* abort = reinterpret_cast<volatile int*>(&bar.abort);
 
   RT_TRACE(g_layer_trace, 0, 0);
-  dec_init(bar, p.nstages, maps, p.has_shared);
-  // this warp's router row; its first 512 float4 (d <= 2048: all of it) are loaded before
-  // the kernel waits on its predecessor (the router weights are not written by anything)
-  const int er = b + warp * G;
-  const bool has_row = er < E;
-  const float4* wrow = reinterpret_cast<const float4*>(p.Wr) + (size_t)(has_row ? er : 0) * nvec;
-  float4 w[16];
-#pragma unroll
-  for (int u = 0; u < 16; ++u) {
-    const int c = lane + 32 * u;
-    w[u] = (has_row && c < nvec) ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+  // this CTA's router rows b, b + G, ... are copied into shared memory before the kernel
+  // waits on its predecessor (the router weights are not written by anything)
+  const int nrows = b < E ? (E - 1 - b) / G + 1 : 0;
+  __shared__ uint64_t s_wbar;
+  __shared__ float s_bias[kLayerMaxRows];
+  if (threadIdx.x == 0) mbar_init(&s_wbar, 1);
+  if (threadIdx.x < nrows) s_bias[threadIdx.x] = p.br ? __ldg(p.br + b + threadIdx.x * G) : 0.0f;
+  dec_init(bar, p.nstages, maps, p.has_shared);  // includes the barrier-init fence
+  if (threadIdx.x == 0 && nrows > 0) {
+    mbar_arrive_expect_tx(&s_wbar, (uint32_t)(nrows * d * 4));
+    for (int r = 0; r < nrows; ++r)
+      bulk_g2s(sc.wr + (size_t)r * d, p.Wr + (size_t)(b + r * G) * d, (uint32_t)(d * 4), &s_wbar);
   }
   MOE_PDL_PROLOGUE();
   RT_TRACE(g_layer_trace, 0, 1);
@@ -207,71 +216,95 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     ts = f > 0.0f ? __fdiv_rn(f, kE2M1Max * kE4M3Max) : 1.0f;
   }
   RT_TRACE(g_layer_trace, 2, 0);
-  // this CTA's share of the 16-element blocks (b, b + G, ...): codes and scales into the xq
-  // outputs, one block per 16 lanes (the steps of quantize_block16, one element per lane)
+  // this CTA's share of the 64-element groups (b, b + G, ...), one warp per group of four
+  // 16-element blocks, two elements per lane (the steps of quantize_block16): the group's 32
+  // code bytes and its 4 scale bytes leave as whole 32-bit words
   {
-    const int nblk = T * (d / kBlock);
-    const int h = lane >> 4, e16 = lane & 15;
-    for (int i0 = 0; b + G * i0 < nblk; i0 += 2 * (int)(blockDim.x >> 5)) {
-      const int q = b + G * (i0 + 2 * warp + h);
-      const bool valid = q < nblk;
-      float v = 0.0f;
-      if (valid) v = bf16_to_f32(sc.xb[(size_t)(q / (d / kBlock)) * d + kBlock * (q % (d / kBlock)) + e16]);
-      float amax = fabsf(v);
+    const int gpr = d / 64;  // groups per token row
+    const int ngrp = T * gpr;
+    const int nw = (int)(blockDim.x >> 5);
+    for (int g = b + G * warp; g < ngrp; g += G * nw) {
+      const int t = g / gpr, c = g % gpr;
+      const uint32_t xv = *reinterpret_cast<const uint32_t*>(sc.xb + (size_t)t * d + 64 * c + 2 * lane);
+      const float v0 = bf16_to_f32(xv & 0xFFFFu), v1 = bf16_to_f32(xv >> 16);
+      float amax = fmaxf(fabsf(v0), fabsf(v1));
 #pragma unroll
-      for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const uint32_t sbyte = f32_to_e4m3_sat(__fdiv_rn(__fdiv_rn(amax, kE2M1Max), ts));
       const float sval = e4m3_to_f32(sbyte);
-      uint32_t nib = 0u;
-      if (sval != 0.0f) nib = f32x2_to_e2m1x2(__fdiv_rn(v, __fmul_rn(sval, ts)), 0.0f) & 0xFu;
-      const uint32_t pr = nib | (__shfl_down_sync(0xffffffffu, nib, 1) << 4);
-      const uint32_t p1 = __shfl_down_sync(0xffffffffu, pr, 2), p2 = __shfl_down_sync(0xffffffffu, pr, 4),
-                     p3 = __shfl_down_sync(0xffffffffu, pr, 6);
-      if (valid && (e16 & 7) == 0)
-        reinterpret_cast<uint32_t*>(p.xq_codes)[2 * q + (e16 >> 3)] =
-            (pr & 0xFFu) | ((p1 & 0xFFu) << 8) | ((p2 & 0xFFu) << 16) | ((p3 & 0xFFu) << 24);
-      if (valid && e16 == 0) p.xq_scales[q] = (uint8_t)sbyte;
+      uint32_t cb = 0u;
+      if (sval != 0.0f) {
+        const float den = __fmul_rn(sval, ts);
+        cb = f32x2_to_e2m1x2(__fdiv_rn(v0, den), __fdiv_rn(v1, den)) & 0xFFu;
+      }
+      const uint32_t word = cb | (__shfl_down_sync(0xffffffffu, cb, 1) << 8) |
+                            (__shfl_down_sync(0xffffffffu, cb, 2) << 16) | (__shfl_down_sync(0xffffffffu, cb, 3) << 24);
+      const uint32_t swd = sbyte | (__shfl_down_sync(0xffffffffu, sbyte, 8) << 8) |
+                           (__shfl_down_sync(0xffffffffu, sbyte, 16) << 16) |
+                           (__shfl_down_sync(0xffffffffu, sbyte, 24) << 24);
+      if ((lane & 3) == 0) reinterpret_cast<uint32_t*>(p.xq_codes)[8 * g + (lane >> 2)] = word;
+      if (lane == 0) reinterpret_cast<uint32_t*>(p.xq_scales)[g] = swd;
     }
     if (b == G - 1 && threadIdx.x == 0) *p.xq_ts = ts;
   }
   RT_TRACE(g_layer_trace, 2, 1);
-  // router logits of this warp's row: 64-term lane partials, then a lane tree per token
-  if (has_row) {
-    float acc[kDecMaxT];
+  // router logits of this CTA's rows b + r*G, four rows at a time: thread i takes float4
+  // columns i, i + blockDim.x, ... of every row and token (32 partial sums), a warp
+  // reduce-scatter leaves lane l with the warp's sum of (row l / 8, token l % 8), and warp 0
+  // adds the warps' sums
+  if (nrows > 0) {
+    mbar_wait(&s_wbar, 0, abort, p.status);
+    RT_TRACE(g_layer_trace, 2, 3);
+    for (int r0 = 0; r0 < nrows; r0 += 4) {
+      float v[32];
 #pragma unroll
-    for (int t = 0; t < kDecMaxT; ++t) acc[t] = 0.0f;
-    for (int c0 = 0; c0 < nvec; c0 += 512) {
-      if (c0 > 0) {
+      for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+      for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
+        float xf[kDecMaxT][4];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int c = c0 + lane + 32 * u;
-          w[u] = c < nvec ? __ldg(wrow + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int t = 0; t < kDecMaxT; ++t) {
+          uint2 xv = make_uint2(0u, 0u);
+          if (t < T) xv = *reinterpret_cast<const uint2*>(sc.xb + (size_t)t * d + 4 * c);
+          xf[t][0] = bf16_to_f32(xv.x & 0xFFFFu);
+          xf[t][1] = bf16_to_f32(xv.x >> 16);
+          xf[t][2] = bf16_to_f32(xv.y & 0xFFFFu);
+          xf[t][3] = bf16_to_f32(xv.y >> 16);
         }
-      }
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int c = c0 + lane + 32 * u;
-        if (c < nvec) {
+        for (int r = 0; r < 4; ++r) {
+          if (r0 + r < nrows) {
+            const float4 wv = reinterpret_cast<const float4*>(sc.wr + (size_t)(r0 + r) * d)[c];
 #pragma unroll
-          for (int t = 0; t < kDecMaxT; ++t) {
-            if (t < T) {
-              const uint2 xv = *reinterpret_cast<const uint2*>(sc.xb + (size_t)t * d + 4 * c);
-              acc[t] = fmaf(bf16_to_f32(xv.x & 0xFFFFu), w[u].x, acc[t]);
-              acc[t] = fmaf(bf16_to_f32(xv.x >> 16), w[u].y, acc[t]);
-              acc[t] = fmaf(bf16_to_f32(xv.y & 0xFFFFu), w[u].z, acc[t]);
-              acc[t] = fmaf(bf16_to_f32(xv.y >> 16), w[u].w, acc[t]);
+            for (int t = 0; t < kDecMaxT; ++t) {
+              float a = v[8 * r + t];
+              a = fmaf(xf[t][0], wv.x, a);
+              a = fmaf(xf[t][1], wv.y, a);
+              a = fmaf(xf[t][2], wv.z, a);
+              a = fmaf(xf[t][3], wv.w, a);
+              v[8 * r + t] = a;
             }
           }
         }
       }
-    }
-    const float bias = p.br ? __ldg(p.br + er) : 0.0f;
 #pragma unroll
-    for (int t = 0; t < kDecMaxT; ++t) {
-      if (t < T) {
-        const float s = warp_sum(acc[t]);
-        if (lane == 0) p.logits[(size_t)t * E + er] = s + bias;
+      for (int o = 16; o >= 1; o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+          const float send = upper ? v[i] : v[i + o];
+          const float keep = upper ? v[i + o] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
       }
+      sc.part[threadIdx.x] = v[0];
+      __syncthreads();
+      if (warp == 0) {
+        float sum = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += sc.part[32 * w + lane];
+        const int r = r0 + (lane >> 3), t = lane & 7;
+        if (r < nrows && t < T) p.logits[(size_t)t * E + b + r * G] = sum + s_bias[r];
+      }
+      __syncthreads();
     }
   }
   RT_TRACE(g_layer_trace, 2, 2);
@@ -293,46 +326,72 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
     // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms; each thread's
     // loads of a round go out together
     {
+      const int q4 = d / 256;  // 16-byte pieces of a token's scale row
+      uint4 sv = make_uint4(0u, 0u, 0u, 0u);
+      if (threadIdx.x < kDecMaxT * q4 && (int)threadIdx.x / q4 < T)
+        sv = __ldcg(reinterpret_cast<const uint4*>(p.xq_scales + (size_t)(threadIdx.x / q4) * (d / kBlock)) +
+                    threadIdx.x % q4);
       const int nc = kDecMaxT * (d / 32);
+      // every CTA reads the same few lines right after the barrier: each starts at a different
+      // place so that the requests to one L2 line do not all arrive at once
+      const int rot_c = (b * 37) % nc;
       for (int i0 = threadIdx.x; i0 < nc; i0 += 4 * blockDim.x) {
         uint4 v[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u * blockDim.x, t = i / (d / 32), c = i % (d / 32);
+          const int iu = i0 + u * blockDim.x;
+          const int i = iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc;
+          const int t = i / (d / 32), c = i % (d / 32);
           v[u] = make_uint4(0u, 0u, 0u, 0u);
-          if (i < nc && t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
+          if (iu < nc && t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u * blockDim.x;
-          if (i < nc) *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(i / (d / 32), i % (d / 32))) = v[u];
+          const int iu = i0 + u * blockDim.x;
+          const int i = iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc;
+          if (iu < nc) *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(i / (d / 32), i % (d / 32))) = v[u];
         }
       }
-      const int ns = (d / 64) * 32;
-      for (int i0 = threadIdx.x; i0 < ns; i0 += 4 * blockDim.x) {
-        uint32_t wd[4];
+      RT_TRACE(g_layer_trace, 3, 3);
+      // the scale words of token t arrive as d/256 16-byte pieces (loaded above); word kc of
+      // token t goes to the four rows t, t + 8, t + 16, t + 24 of atom kc
+      if (threadIdx.x < kDecMaxT * q4) {
+        const int t = threadIdx.x / q4, c4 = threadIdx.x % q4;
+        const uint32_t wv[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u * blockDim.x, kc = i / 32, t = (i % 32) & 7;
-          wd[u] = 0u;
-          if (i < ns && t < T)
-            wd[u] = __ldcg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock)) + kc);
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int r1 = 0; r1 < 4; ++r1) dec_xsf_store(sm.xsf, 4 * c4 + w, t + 8 * r1, wv[w]);
+      }
+      RT_TRACE(g_layer_trace, 3, 4);
+      // the logits -> shared memory, the same way
+      const int nl = T * E;
+      const int rot_l = (b * 131) % nl;
+      for (int i0 = threadIdx.x; i0 < nl; i0 += 8 * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int iu = i0 + u * blockDim.x;
+          const int i = iu + rot_l < nl ? iu + rot_l : iu + rot_l - nl;
+          v[u] = iu < nl ? __ldcg(p.logits + i) : 0.0f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = i0 + u * blockDim.x;
-          if (i < ns) dec_xsf_store(sm.xsf, i / 32, i % 32, wd[u]);
+        for (int u = 0; u < 8; ++u) {
+          const int iu = i0 + u * blockDim.x;
+          const int i = iu + rot_l < nl ? iu + rot_l : iu + rot_l - nl;
+          if (iu < nl) sc.logits[i] = v[u];
         }
       }
     }
+    RT_TRACE(g_layer_trace, 3, 5);
     for (int e = threadIdx.x; e < E; e += blockDim.x) sc.flag[e] = 0;
     __syncthreads();
     RT_TRACE(g_layer_trace, 3, 0);
     // top-k of every token (one warp each)
     if (warp < T)
-      topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
-                          writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
-                          sc.tw + warp * kLayerMaxK);
+      topk_dispatch(sc.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
+                    writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
+                    sc.tw + warp * kLayerMaxK, sc.tks + warp * 64);
     __syncthreads();
     RT_TRACE(g_layer_trace, 3, 1);
     for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
@@ -453,7 +512,8 @@ bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, 
   if (!dec_shape_ok(T, d, I) || k < 1 || k > kLayerMaxK || E < k || E > 1024) return false;
   if (E > G * (kDecThreads / 32)) return false;  // router rows: one per warp
   const int nst = dec_stages(d);
-  if ((size_t)nst * kDecStageBytes < layer_scratch_head(d) + kLayerScratchTail) return false;
+  const size_t rows = (size_t)(E + G - 1) / G;  // router rows of one CTA, staged in the ring
+  if ((size_t)nst * kDecStageBytes < layer_scratch_head(d) + kLayerScratchTail + rows * d * 4) return false;
   const int64_t slots = (T * k < E ? T * k : E) + has_shared;
   return (slots * (I / 64) + G - 1) / G <= kDecMaxUnits;
 }

@@ -189,10 +189,12 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(const uint16_t* __rest
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int32_t* __restrict__ topk_idx,
                                                    float* __restrict__ topk_w) {
+  __shared__ uint32_t scratch[8][64];
   MOE_PDL_PROLOGUE();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  topk_dispatch(logits + (size_t)t * E, E, k, topk_idx + (size_t)t * k, topk_w + (size_t)t * k);
+  topk_dispatch(logits + (size_t)t * E, E, k, topk_idx + (size_t)t * k, topk_w + (size_t)t * k, nullptr, nullptr,
+                scratch[threadIdx.x >> 5]);
 }
 
 // ---------------------------------------------------------------- permutation

@@ -19,15 +19,21 @@ MOE_DEV uint32_t ordered_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// One warp per token. Lane L holds logits L, L+32, ... and keeps its own best remaining
-// entry; each of the k rounds takes the warp arg-max (ties to the lower index) and only the
-// winning lane rescans. Outputs (each may be NULL): idx_out / w_out in global memory,
-// idx_smem / w_smem in shared memory, k entries each, in descending logit order. With
-// kL2 = true the logits are read through L2 (ld.global.cg: written by other CTAs of the
-// same kernel).
+// One warp per token. Lane L holds logits L, L+32, ... (keys that order like the floats).
+// Outputs (each may be NULL): idx_out / w_out in global memory, idx_smem / w_smem in shared
+// memory, k entries each, in descending logit order, ties to the lower expert id. With
+// kL2 = true the logits are read through L2 (ld.global.cg: written by other CTAs of the same
+// kernel).
+//
+// With a 64-word shared scratch and k <= 32 the selection first takes a threshold: the k-th
+// largest of the 32 lane maxima. At least k logits reach it (those k maxima), so every logit
+// of the top k is among the candidates at or above it; when there are at most 32 candidates
+// (the usual case: about k + 2 for independent logits) they are gathered one per lane and
+// each candidate's rank is counted against the other 31. Otherwise k rounds of a warp
+// arg-max pick the winners one at a time, and only the winning lane rescans its entries.
 template <int NPER, bool kL2 = false>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* idx_out, float* w_out,
-                        int* idx_smem = nullptr, float* w_smem = nullptr) {
+                        int* idx_smem = nullptr, float* w_smem = nullptr, uint32_t* scratch = nullptr) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NPER];
 #pragma unroll
@@ -35,8 +41,10 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
     const int e = lane + 32 * j;
     float v = 0.0f;
     if (e < E) v = kL2 ? __ldcg(row + e) : row[e];
-    key[j] = e < E ? ordered_key(v) : 0u;  // 0 is below every finite float's key
+    key[j] = e < E ? ordered_key(v) : 0u;  // 0 is below every float's key
   }
+  // does (ka, ea) come before (kb, eb): larger key, or equal key and lower index
+  auto before = [](uint32_t ka, int ea, uint32_t kb, int eb) { return ka > kb || (ka == kb && ea < eb); };
   uint32_t taken = 0;
   // this lane's best remaining entry: largest key, lowest index among equal keys
   auto local_best = [&](uint32_t& bk, int& be) {
@@ -45,22 +53,84 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
 #pragma unroll
     for (int j = 0; j < NPER; ++j) {
       const int e = lane + 32 * j;
-      if (e < E && !((taken >> j) & 1u) && (key[j] > bk || (key[j] == bk && e < be))) bk = key[j], be = e;
+      if (e < E && !((taken >> j) & 1u) && before(key[j], e, bk, be)) bk = key[j], be = e;
     }
   };
   uint32_t lbk;
   int lbe;
   local_best(lbk, lbe);
-  uint32_t top_key = 0, my_key = 0;
+  uint32_t top_key = 0, my_key = 0;  // lane r < k ends with the r-th pick
   int my_e = 0;
-  for (int r = 0; r < k; ++r) {
-    const uint32_t mk = __reduce_max_sync(0xffffffffu, lbk);
-    const int me = (int)__reduce_min_sync(0xffffffffu, lbk == mk ? (uint32_t)lbe : 0x7fffffffu);
-    if (r == 0) top_key = mk;
-    if (lane == r) my_key = mk, my_e = me;
-    if ((me & 31) == lane) {
-      taken |= 1u << (me >> 5);
-      local_best(lbk, lbe);
+  bool done = false;
+  if (scratch != nullptr && k <= 32) {
+    // rank of this lane's maximum among the lanes' maxima (lanes without entries tie at
+    // the bottom, behind min(E, 32) >= k valid maxima)
+    int rank = 0;
+#pragma unroll 8
+    for (int o = 1; o < 32; ++o) {
+      const int src = (lane + o) & 31;
+      const uint32_t ok = __shfl_sync(0xffffffffu, lbk, src);
+      const int oe = __shfl_sync(0xffffffffu, lbe, src);
+      rank += before(ok, oe, lbk, lbe) ? 1 : 0;
+    }
+    const uint32_t th = __shfl_sync(0xffffffffu, lbk, __ffs(__ballot_sync(0xffffffffu, rank == k - 1)) - 1);
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < NPER; ++j) c += (lane + 32 * j < E && key[j] >= th) ? 1 : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total <= 32) {
+      int pos = incl - c;
+#pragma unroll
+      for (int j = 0; j < NPER; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && key[j] >= th) {
+          scratch[pos] = key[j];
+          scratch[32 + pos] = (uint32_t)e;
+          ++pos;
+        }
+      }
+      __syncwarp();
+      const uint32_t ck = lane < total ? scratch[lane] : 0u;
+      const int ce = lane < total ? (int)scratch[32 + lane] : 0x7fffffff;
+      __syncwarp();
+      int r = 0;
+#pragma unroll 8
+      for (int o = 1; o < 32; ++o) {
+        const int src = (lane + o) & 31;
+        const uint32_t ok = __shfl_sync(0xffffffffu, ck, src);
+        const int oe = __shfl_sync(0xffffffffu, ce, src);
+        r += before(ok, oe, ck, ce) ? 1 : 0;
+      }
+      if (lane < total && r < k) {
+        scratch[r] = ck;
+        scratch[32 + r] = (uint32_t)ce;
+      }
+      __syncwarp();
+      if (lane < k) {
+        my_key = scratch[lane];
+        my_e = (int)scratch[32 + lane];
+      }
+      top_key = __shfl_sync(0xffffffffu, my_key, 0);
+      __syncwarp();
+      done = true;
+    }
+  }
+  if (!done) {
+    for (int r = 0; r < k; ++r) {
+      const uint32_t mk = __reduce_max_sync(0xffffffffu, lbk);
+      const int me = (int)__reduce_min_sync(0xffffffffu, lbk == mk ? (uint32_t)lbe : 0x7fffffffu);
+      if (r == 0) top_key = mk;
+      if (lane == r) my_key = mk, my_e = me;
+      if ((me & 31) == lane) {
+        taken |= 1u << (me >> 5);
+        local_best(lbk, lbe);
+      }
     }
   }
   auto key_to_float = [](uint32_t kk) {
@@ -77,12 +147,13 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
   }
 }
 
+// scratch: NULL, or 64 words of shared memory for this warp
 template <bool kL2 = false>
 MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w, int* idx_smem = nullptr,
-                           float* w_smem = nullptr) {
-  if (E <= 256) topk_token<8, kL2>(row, E, k, idx, w, idx_smem, w_smem);
-  else if (E <= 512) topk_token<16, kL2>(row, E, k, idx, w, idx_smem, w_smem);
-  else topk_token<32, kL2>(row, E, k, idx, w, idx_smem, w_smem);
+                           float* w_smem = nullptr, uint32_t* scratch = nullptr) {
+  if (E <= 256) topk_token<8, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch);
+  else if (E <= 512) topk_token<16, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch);
+  else topk_token<32, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch);
 }
 
 // The permutation of n <= 32*k assignments by one warp, without block-wide barriers:

@@ -216,9 +216,10 @@ def test_ffn_prefill_configs_sampled(cfg_name, n_sample):
     assert np.isfinite(yf).all() and (np.abs(yf).sum(1) > 0).all()
 
 
-def test_pack_slices_regroup_the_down_matrix():
-    """moe_pack_experts' slice copies are exact regroupings: codes [E][d][I/2] -> [E][I/64][d][32]
-    and the down scale atoms [E][d/128][I/64] -> [E][I/64][d/128] (integer, bit-exact)."""
+def test_pack_slices_regroup_the_weights():
+    """moe_pack_experts' slice copies are exact regroupings: down codes [E][d][I/2] ->
+    [E][I/64][d][32], the down scale atoms [E][d/128][I/64] -> [E][I/64][d/128], and gate/up codes
+    [E][2I][d/2] -> [E][I/64][d/256][64 gate rows + 64 up rows][128] (integer, bit-exact)."""
     experts, sh, xq, routing, gpu = _tiny_case(15, 512, 4, 2, 192, 3, True, pack=True)
     for w in (gpu.routed, gpu.shared):
         E, d, I = w.E, w.d, w.I
@@ -226,3 +227,6 @@ def test_pack_slices_regroup_the_down_matrix():
         assert np.array_equal(w.dn_codes_slice.cpu().numpy().reshape(E, I // 64, d, 32), nat)
         atoms = w.dn_sf_tiled.cpu().numpy().reshape(E, d // 128, I // 64, 512).transpose(0, 2, 1, 3)
         assert np.array_equal(w.dn_sf_slice.cpu().numpy().reshape(E, I // 64, d // 128, 512), atoms)
+        gu = w.gu_codes.cpu().numpy().reshape(E, 2, I // 64, 64, d // 256, 128)  # [e][g/u][j][r][kb][byte]
+        tiles = gu.transpose(0, 2, 4, 1, 3, 5).reshape(E, I // 64, d // 256, 128, 128)
+        assert np.array_equal(w.gu_codes_slice.cpu().numpy().reshape(E, I // 64, d // 256, 128, 128), tiles)
