@@ -289,11 +289,15 @@ def run_gpu(args):
     if args.workload == "decode":
         name = ("layer_dec_kernel (moe_layer_decode: quantise, route, tcgen05 expert FFN, combine)"
                 if fused else "moe_expert_ffn (decode: preparation + tcgen05 split-I kernel)")
+        # DRAM traffic of layer_dec_kernel from one ncu capture of the same kernel and shapes
+        # (dram__bytes_read.sum + dram__bytes_write.sum = 59,812,864 B on a launch whose run
+        # averaged 60,075,008 algorithmic bytes), scaled to this run's bytes per launch
+        traffic = int(ffn_bytes * (59812864 / 60075008)) if fused else None
         roof = {"kernel": name, "bound": "hbm",
                 "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind,
                 "bytes_per_launch": int(ffn_bytes), "avg_launch_us": round(ffn_ms * 1e3, 3),
-                "traffic": None}
+                "traffic": traffic}
     else:
         fp4_peak = bf16_peak * 4.0  # dense FP4 = 4 x dense bf16 (nominal ratio 9 / 2.25)
         tf = ffn_flops / (ffn_ms * 1e-3) / 1e12

@@ -81,12 +81,9 @@ typedef enum moe_status {
  *   dn_ts     [E]            float32
  *   gu_sf_tiled, dn_sf_tiled: the same scale bytes re-tiled for the tensor-core path by
  *            moe_pack_experts (NULL if not packed; the PREFILL path then refuses).
- *   dn_codes_slice [E][I/64][d][32], dn_sf_slice [E][I/64][d/128][512]: the down matrix
- *            regrouped by 64-column slices of I (each slice's codes, and its scale atoms,
- *            contiguous), written by moe_pack_experts for the DECODE path (NULL if absent).
- *   gu_codes_slice [E][I/64][d/256][128][128]: the gate/up codes regrouped the same way:
- *            per 64-row slice of I and 256-column block of d, one 16 KB tile of the slice's
- *            64 gate rows then its 64 up rows, 128 bytes each (DECODE path; NULL if absent).
+ *   dec_pack  the decode pack written by moe_pack_experts for the DECODE path and
+ *            moe_layer_decode (NULL if absent): every weight byte and scale of the group
+ *            again, as the 18432-byte blocks the decode kernel copies into shared memory.
  */
 typedef struct moe_expert_weights {
   int32_t E, d, I;
@@ -98,9 +95,7 @@ typedef struct moe_expert_weights {
   const float* dn_ts;
   const uint8_t* gu_sf_tiled;
   const uint8_t* dn_sf_tiled;
-  const uint8_t* dn_codes_slice;
-  const uint8_t* dn_sf_slice;
-  const uint8_t* gu_codes_slice;
+  const uint8_t* dec_pack;
 } moe_expert_weights_t;
 
 typedef struct moe_experts {
@@ -153,17 +148,21 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
  *     512-byte atoms of 128 weight rows x 4 scale blocks, the layout the tensor core reads
  *     its scales in (gate/up atoms [E][I/64][d/64], atom rows 0-63 gate, 64-127 up; down
  *     atoms [E][d/128][I/64]);
- *   dn_codes_slice (E*d*I/2 bytes), dn_sf_slice (E*d*I/16 bytes), gu_codes_slice
- *     (E*2I*d/2 bytes), all three or none (NULL to skip): the down codes and scale atoms
- *     regrouped per 64-column slice of I, and the gate/up codes per 64-row slice of I and
- *     256-column block of d, so that the DECODE path reads every weight tile as contiguous
- *     bytes (the gate/up scale atoms above are already grouped that way).
+ *   dec_pack (E*I*d*27/16 bytes; optional, NULL to skip; needs d % 512 == 0): for each
+ *     unit (expert e, 64-wide slice j of I), d/256 gate/up blocks then d/512 down blocks of
+ *     18432 bytes each, in that order. Gate/up block kb: the 128 x 128-byte tile of gate
+ *     rows 64j..64j+63 then up rows 64j..64j+63, bytes 128kb..128kb+127 of each, stored in
+ *     the 128-byte swizzle (16-byte piece c of row r at r*128 + (c ^ (r % 8))*16), then the
+ *     four gate/up scale atoms 4kb..4kb+3 of (e, j). Down block q: chunks c = 4q..4q+3, each
+ *     the 128 x 32-byte tile of rows 128c..128c+127, bytes 32j..32j+31, stored in the 32-byte
+ *     swizzle (piece c' of row r at r*32 + (c' ^ ((r / 4) % 2))*16), then the four down
+ *     scale atoms of those chunks for slice j. A block is exactly what one shared-memory
+ *     stage of the decode kernel holds, so it moves with one bulk copy.
  * The natural-layout arrays stay as they are and remain in use by the CUDA-core path.
- * Requires d % 128 == 0 and I % 64 == 0 (and d % 256 == 0 with the slices).
+ * Requires d % 128 == 0 and I % 64 == 0.
  */
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
-                            uint8_t* dn_sf_tiled, uint8_t* dn_codes_slice, uint8_t* dn_sf_slice,
-                            uint8_t* gu_codes_slice, void* stream);
+                            uint8_t* dn_sf_tiled, uint8_t* dec_pack, void* stream);
 
 /*
  * moe_expert_ffn - expert SwiGLU FFN for all routed assignments (A5-A7) and the shared

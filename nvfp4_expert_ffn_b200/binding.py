@@ -30,7 +30,7 @@ EXPORTS = {
     "moe_route": (_I32, [_P, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_permute": (_I32, [_P, _I32, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "moe_route_noalloc": (_I32, [_P, _I32, _I32, _P, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
-    "moe_pack_experts": (_I32, [_P, _P, _P, _P, _P, _P, _P]),
+    "moe_pack_experts": (_I32, [_P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_I32, [_P, _P, _P, _I32, _P, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P,
                               _SZ, _P]),
     "moe_combine": (_I32, [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _I32, _P, _P]),
@@ -100,7 +100,7 @@ class _WeightsC(ctypes.Structure):
                 ("gu_codes", _P), ("gu_scales", _P), ("gu_ts", _P),
                 ("dn_codes", _P), ("dn_scales", _P), ("dn_ts", _P),
                 ("gu_sf_tiled", _P), ("dn_sf_tiled", _P),
-                ("dn_codes_slice", _P), ("dn_sf_slice", _P), ("gu_codes_slice", _P)]
+                ("dec_pack", _P)]
 
 
 class _ExpertsC(ctypes.Structure):
@@ -118,9 +118,7 @@ class ExpertWeights:
     dn_ts: torch.Tensor      # float32 [E]
     gu_sf_tiled: Optional[torch.Tensor] = None
     dn_sf_tiled: Optional[torch.Tensor] = None
-    dn_codes_slice: Optional[torch.Tensor] = None
-    dn_sf_slice: Optional[torch.Tensor] = None
-    gu_codes_slice: Optional[torch.Tensor] = None
+    dec_pack: Optional[torch.Tensor] = None
 
     @property
     def E(self):
@@ -138,8 +136,7 @@ class ExpertWeights:
         p = lambda t: None if t is None else _ptr(t).value  # noqa: E731
         return _WeightsC(self.E, self.d, self.I, p(self.gu_codes), p(self.gu_scales),
                          p(self.gu_ts), p(self.dn_codes), p(self.dn_scales), p(self.dn_ts),
-                         p(self.gu_sf_tiled), p(self.dn_sf_tiled), p(self.dn_codes_slice),
-                         p(self.dn_sf_slice), p(self.gu_codes_slice))
+                         p(self.gu_sf_tiled), p(self.dn_sf_tiled), p(self.dec_pack))
 
 
 @dataclass
@@ -212,20 +209,24 @@ def moe_permute(topk_idx, E, counts, offsets, sorted_assign, assign_pos, ws, str
 
 def moe_pack_experts(w: ExpertWeights, stream=None, slices: bool = True):
     """Allocate and fill the derived layouts used by the tensor-core paths: re-tiled scales,
-    and (slices=True) the down and gate/up matrices regrouped by 64-wide slices of I for the
-    decode path."""
+    and (slices=True, d % 512 == 0) the decode pack: all weights again as the 18 KB blocks
+    the decode kernel copies into shared memory."""
     if w.gu_sf_tiled is None:
         w.gu_sf_tiled = torch.empty_like(w.gu_scales)
     if w.dn_sf_tiled is None:
         w.dn_sf_tiled = torch.empty_like(w.dn_scales)
-    if slices and w.dn_codes_slice is None and w.d % 256 == 0:
-        w.dn_codes_slice = torch.empty_like(w.dn_codes)
-        w.dn_sf_slice = torch.empty_like(w.dn_scales)
-        w.gu_codes_slice = torch.empty_like(w.gu_codes)
+    if slices and w.dec_pack is None and w.d % 512 == 0:
+        w.dec_pack = torch.empty(dec_pack_bytes(w.E, w.d, w.I), dtype=torch.uint8,
+                                 device=w.gu_codes.device)
     s = w.struct()
     _check("moe_pack_experts", lib().moe_pack_experts(
-        ctypes.byref(s), _ptr(w.gu_sf_tiled), _ptr(w.dn_sf_tiled), _ptr(w.dn_codes_slice),
-        _ptr(w.dn_sf_slice), _ptr(w.gu_codes_slice), _stream(stream)))
+        ctypes.byref(s), _ptr(w.gu_sf_tiled), _ptr(w.dn_sf_tiled), _ptr(w.dec_pack),
+        _stream(stream)))
+
+
+def dec_pack_bytes(E: int, d: int, I: int) -> int:
+    """Bytes of the decode pack of an expert group (d % 512 == 0, I % 64 == 0)."""
+    return E * (I // 64) * (d // 256 + d // 512) * 18432
 
 
 def moe_expert_ffn(xq_codes, xq_scales, xq_ts, experts: Experts, k, offsets, sorted_assign,

@@ -98,8 +98,7 @@ moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E,
 
 ExpertGroup to_group(const moe_expert_weights_t& w) {
   return ExpertGroup{w.gu_codes,    w.gu_scales,   w.gu_ts,          w.dn_codes,      w.dn_scales,
-                     w.dn_ts,       w.gu_sf_tiled, w.dn_sf_tiled, w.dn_codes_slice, w.dn_sf_slice,
-                     w.gu_codes_slice};
+                     w.dn_ts,       w.gu_sf_tiled, w.dn_sf_tiled, w.dec_pack};
 }
 
 }  // namespace
@@ -226,18 +225,14 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t d, const float* Wr, c
 }
 
 moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
-                            uint8_t* dn_sf_tiled, uint8_t* dn_codes_slice, uint8_t* dn_sf_slice,
-                            uint8_t* gu_codes_slice, void* stream) {
+                            uint8_t* dn_sf_tiled, uint8_t* dec_pack, void* stream) {
   if (!W || !gu_sf_tiled || !dn_sf_tiled) return fail(MOE_ERR_INVALID_ARG, "null argument");
-  if ((dn_codes_slice == nullptr) != (dn_sf_slice == nullptr) || (dn_codes_slice == nullptr) != (gu_codes_slice == nullptr))
-    return fail(MOE_ERR_INVALID_ARG, "dn_codes_slice, dn_sf_slice and gu_codes_slice are given together");
-  if ((dn_codes_slice && !aligned16(dn_codes_slice)) || (dn_sf_slice && !aligned16(dn_sf_slice)) ||
-      (gu_codes_slice && !aligned16(gu_codes_slice)) ||
-      (dn_codes_slice && (!W->dn_codes || !aligned16(W->dn_codes) || !W->gu_codes || !aligned16(W->gu_codes))))
-    return fail(MOE_ERR_INVALID_ARG, "slice buffers, dn_codes and gu_codes must be 16-byte aligned");
+  if (dec_pack && (!aligned16(dec_pack) || !W->dn_codes || !aligned16(W->dn_codes) || !W->gu_codes ||
+                   !aligned16(W->gu_codes)))
+    return fail(MOE_ERR_INVALID_ARG, "dec_pack, dn_codes and gu_codes must be 16-byte aligned");
   if (W->E < 1 || W->d <= 0 || W->I <= 0) return fail(MOE_ERR_INVALID_ARG, "bad E/d/I");
   if (W->d % 128 || W->I % 64) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "packing needs d % 128 == 0 and I % 64 == 0");
-  if (dn_codes_slice && W->d % 256) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "the slices need d % 256 == 0");
+  if (dec_pack && W->d % 512) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "the decode pack needs d % 512 == 0");
   if (!W->gu_scales || !W->dn_scales) return fail(MOE_ERR_INVALID_ARG, "null scales");
   if (!aligned16(W->gu_scales) || !aligned16(W->dn_scales) || !aligned16(gu_sf_tiled) || !aligned16(dn_sf_tiled))
     return fail(MOE_ERR_INVALID_ARG, "scale pointers must be 16-byte aligned");
@@ -246,9 +241,9 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
   if (s != MOE_OK) return s;
   cudaError_t e = launch_pack_sf(to_group(*W), W->E, W->d, W->I, gu_sf_tiled, dn_sf_tiled, sms,
                                  (cudaStream_t)stream);
-  if (e == cudaSuccess && dn_codes_slice)
-    e = launch_pack_slices(to_group(*W), W->E, W->d, W->I, dn_codes_slice, dn_sf_slice, gu_codes_slice, sms,
-                           (cudaStream_t)stream);
+  if (e == cudaSuccess && dec_pack)
+    e = launch_pack_dec(to_group(*W), W->E, W->d, W->I, gu_sf_tiled, dn_sf_tiled, dec_pack, sms,
+                        (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_pack_experts launch");
 }
 
@@ -286,16 +281,14 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
   const bool tc_ok = ffn_tc_supported(d, I) && packed;
-  const bool sliced = W->routed.dn_codes_slice && W->routed.dn_sf_slice && W->routed.gu_codes_slice &&
-                      (!W->has_shared ||
-                       (W->shared.dn_codes_slice && W->shared.dn_sf_slice && W->shared.gu_codes_slice));
-  const bool dec_ok = ffn_dec_supported(T, d, I, mode, E, k, W->has_shared ? 1 : 0, sms) && packed && sliced;
+  const bool dec_packed = W->routed.dec_pack && (!W->has_shared || W->shared.dec_pack);
+  const bool dec_ok = ffn_dec_supported(T, d, I, mode, E, k, W->has_shared ? 1 : 0, sms) && dec_packed;
   if (path == MOE_PATH_PREFILL && !tc_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "tensor-core path needs d % 256 == 0, I % 256 == 0 and scales packed by moe_pack_experts");
   if (path == MOE_PATH_DECODE && !dec_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
-                "decode path needs T <= 8, ACCUMULATE mode, d % 512 == 0, I % 64 == 0 and packed scales and slices");
+                "decode path needs T <= 8, ACCUMULATE mode, d % 512 == 0, I % 64 == 0 and the decode pack");
   const int kind = path == MOE_PATH_AUTO ? (dec_ok ? MOE_PATH_DECODE : tc_ok ? MOE_PATH_PREFILL : MOE_PATH_CUDA_CORE)
                                          : path;
   const size_t need = kind == MOE_PATH_DECODE    ? ffn_dec_ws_bytes(E)
@@ -342,12 +335,8 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
   if (!aligned16(x) || !aligned16(Wr) || !aligned16(xq_codes) || !aligned16(xq_scales) || !aligned16(y_acc) ||
       !aligned16(y))
     return fail(MOE_ERR_INVALID_ARG, "x, Wr, xq_codes, xq_scales, y_acc and y must be 16-byte aligned");
-  const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled && W->routed.dn_codes_slice &&
-                      W->routed.dn_sf_slice && W->routed.gu_codes_slice &&
-                      (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled &&
-                                          W->shared.dn_codes_slice && W->shared.dn_sf_slice &&
-                                          W->shared.gu_codes_slice));
-  if (!packed) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "weights must be packed by moe_pack_experts, slices included");
+  const bool packed = W->routed.dec_pack && (!W->has_shared || W->shared.dec_pack);
+  if (!packed) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "weights need the decode pack of moe_pack_experts");
   int sms = 0;
   int32_t* dstatus = nullptr;
   if ((s = device_info(&sms, &dstatus)) != MOE_OK) return s;
@@ -431,17 +420,19 @@ int64_t trace_fetch_dec(void* host, size_t bytes);
 int64_t trace_fetch_route(void* host, size_t bytes);
 int64_t trace_fetch_prep(void* host, size_t bytes);
 int64_t trace_fetch_layer(void* host, size_t bytes);
+int64_t trace_fetch_layer_core(void* host, size_t bytes);
 }  // namespace moe
 // Trace builds only: timeline records of the last runs of the tensor-core FFN kernel
 // (kernel 0: the grouped-GEMM path, 1: the decode path; 2: entry/wait/exit stamps of the
 // routing kernels, 3: of the decode preparation and FFN kernels, 4: phase stamps of the
-// one-kernel decode layer), copied to `host` and cleared.
+// one-kernel decode layer, 5: its unit-core records), copied to `host` and cleared.
 extern "C" int64_t moe_trace_fetch(int32_t kernel, void* host, size_t bytes) {
   switch (kernel) {
     case 0: return moe::trace_fetch_tc(host, bytes);
     case 1: return moe::trace_fetch_dec(host, bytes);
     case 2: return moe::trace_fetch_route(host, bytes);
     case 4: return moe::trace_fetch_layer(host, bytes);
+    case 5: return moe::trace_fetch_layer_core(host, bytes);
     default: return moe::trace_fetch_prep(host, bytes);
   }
 }

@@ -65,10 +65,6 @@ constexpr size_t kDecSmemBudget = 224 * 1024;          // dynamic shared memory;
 constexpr uint32_t kColD1 = 0, kColH = 32, kColSf = 48, kColX = 112;
 __host__ __device__ inline uint32_t dec_col_d2(int d) { return (kColX + (uint32_t)d / 16 + 15u) & ~15u; }
 
-struct DecMaps {
-  CUtensorMap b1, b1s;  // gate/up codes by I-slice {128, 128, d/256, E*I/64}, boxes {128, 128, 1, 1}, 128-byte swizzle
-  CUtensorMap b2, b2s;  // down codes by I-slice {32, 128, d/128, E*I/64}, boxes {32, 128, 4, 1}, 32-byte swizzle
-};
 
 // What the unit loop needs besides its units.
 struct DecArgs {
@@ -78,6 +74,7 @@ struct DecArgs {
   int nstages;       // ring stages
   int group_chunks;  // down chunks accumulated in TMEM at a time (multiple of 4)
   float ts_x;        // tensor scale of the activations
+  int xsf_loaded;    // the activation scale atoms are in TMEM already (xsf_ready completes)
   float* out;        // y [T][d] float32, added into
   int32_t* status;
 };
@@ -93,7 +90,7 @@ struct DecUnits {
 
 struct DecBars {
   uint64_t full[kDecMaxStages], empty[kDecMaxStages];
-  uint64_t xsf_ready, acc1_full, acc1_empty, h_full[2], acc2_full, acc2_empty, final_bar;
+  uint64_t xsf_ready, acc1_full, acc1_empty, h_full[2], acc2_full[2], acc2_empty[2], final_bar;
   uint32_t tmem;
   int abort;
   int go;
@@ -124,7 +121,7 @@ MOE_DEV DecSmem dec_smem(uint8_t* base, int d, int nst) {
 
 // Barriers (thread 0) and TMEM (warp 1); called by every thread before the first
 // __syncthreads of the kernel, so it can run before the kernel waits on its predecessor.
-MOE_DEV void dec_init(DecBars& b, int nst, const DecMaps& maps, int has_shared) {
+MOE_DEV void dec_init(DecBars& b, int nst) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < nst; ++s) {
       mbar_init(&b.full[s], 1);
@@ -135,17 +132,13 @@ MOE_DEV void dec_init(DecBars& b, int nst, const DecMaps& maps, int has_shared) 
     mbar_init(&b.acc1_empty, kDecEpiWarps);
     mbar_init(&b.h_full[0], 1);
     mbar_init(&b.h_full[1], 1);
-    mbar_init(&b.acc2_full, 2);
-    mbar_init(&b.acc2_empty, kDecEpiWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&b.acc2_full[i], 2);
+      mbar_init(&b.acc2_empty[i], kDecEpiWarps);
+    }
     mbar_init(&b.final_bar, 2);
     fence_barrier_init();
     b.abort = 0;
-    prefetch_tensormap(&maps.b1);
-    prefetch_tensormap(&maps.b2);
-    if (has_shared) {
-      prefetch_tensormap(&maps.b1s);
-      prefetch_tensormap(&maps.b2s);
-    }
   }
   if ((threadIdx.x >> 5) == 1) tmem_alloc(&b.tmem, 512);
 }
@@ -163,13 +156,15 @@ MOE_DEV void dec_xsf_store(uint8_t* xsf, int kc, int r0, uint32_t word_of_token)
 }
 
 // Runs this CTA's units. Preconditions: dec_init() done and visible (a __syncthreads), the
-// x tiles and x scale atoms written to shared memory and made visible to the async proxy,
+// x tiles and x scale atoms written to shared memory and made visible to the async proxy
+// (with p.xsf_loaded, the atoms already copied to TMEM by tcgen05.cp with two commits on
+// xsf_ready),
 // y zeroed (or holding what the units should add to). Every thread of the CTA calls it; it
 // returns once every unit's results have been added into p.out and every tensor-core
 // operation has completed. TMEM stays allocated (the caller releases it).
 TC_TRACE_ARRAY(g_dec_trace)
 
-MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, DecBars& bar, const DecUnits& U) {
+MOE_DEV void dec_run(const DecArgs& p, const DecSmem& sm, DecBars& bar, const DecUnits& U) {
   TC_TRACE_DECL
   TC_TRACE_BEGIN(g_dec_trace);
   __syncthreads();
@@ -179,8 +174,8 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
   uint64_t& acc1_full = bar.acc1_full;
   uint64_t& acc1_empty = bar.acc1_empty;
   uint64_t* h_full = bar.h_full;
-  uint64_t& acc2_full = bar.acc2_full;
-  uint64_t& acc2_empty = bar.acc2_empty;
+  uint64_t* acc2_full = bar.acc2_full;    // per down-accumulator buffer
+  uint64_t* acc2_empty = bar.acc2_empty;
   uint64_t& final_bar = bar.final_bar;
   volatile int& s_abort = *reinterpret_cast<volatile int*>(&bar.abort);
   int& s_go = bar.go;
@@ -197,7 +192,9 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
   const int nks1 = d / 256;        // gate/up stages per unit
   const int nch = d / 128;         // down chunks per unit
   const int nks2 = nch / 4;        // down stages per unit
-  const int gch = p.group_chunks;  // down chunks accumulated in TMEM at a time (multiple of 4)
+  // down chunks accumulated in TMEM at a time (multiple of 4); groups alternate between two
+  // accumulator buffers, so the MMAs of one group overlap the epilogue's reading of the last
+  const int gch = p.group_chunks;
   const int gst = gch / 4;         // down stages per group
   const uint32_t col_d2 = dec_col_d2(d);
   const int nu = U.n;
@@ -238,19 +235,12 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
           }
           uint8_t* sb = ring + (size_t)st * kDecStageBytes;
           if (it < 40) TC_TRACE_AT(g_dec_trace, kEvProdIssue, it);
+          // one contiguous 18 KB block of the decode pack: the stage's swizzled codes and its
+          // four scale atoms (gate/up K block (q + rot) % nks1, or down chunks 4(q - nks1)..+3)
+          const int qp = q < nks1 ? (q + rot) % nks1 : q;
           mbar_arrive_expect_tx(&full[st], kDecStageBytes);
-          if (q < nks1) {
-            const int kq = (q + rot) % nks1;  // K block of this stage
-            tma_load_4d(sb, sh ? &maps.b1s : &maps.b1, &full[st], 0, 0, kq, el * nt1 + j);
-            bulk_g2s(sb + kDecBBytes, G.gu_sf_tiled + (((size_t)el * nt1 + j) * (d / 64) + 4 * kq) * kDecAtom,
-                     4 * kDecAtom, &full[st]);
-          } else {
-            // four 128-row chunks of slice j (16 KB contiguous) and their scale atoms (2 KB)
-            const int q2 = q - nks1;
-            tma_load_4d(sb, sh ? &maps.b2s : &maps.b2, &full[st], 0, 0, 4 * q2, el * nt1 + j);
-            bulk_g2s(sb + kDecBBytes, G.dn_sf_slice + (((size_t)el * nt1 + j) * nch + 4 * q2) * kDecAtom,
-                     4 * kDecAtom, &full[st]);
-          }
+          bulk_g2s(sb, G.dec_pack + (((size_t)el * nt1 + j) * (nks1 + nks2) + qp) * kDecStageBytes, kDecStageBytes,
+                   &full[st]);
         }
       }
       // no copy may still be landing when the CTA exits
@@ -271,8 +261,11 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
     if (lane == 0) {
       // the activation scale atoms stay in TMEM for the whole kernel (each issuer copies
       // half of them; both wait for all)
-      for (int a = who; a < d / 64; a += 2) tmem_cp_sf(tmem + kColX + 4 * a, sdesc_sf(smem_u32(xsf + (size_t)a * kDecAtom)));
-      mma_commit(&xsf_ready);
+      if (!p.xsf_loaded) {
+        for (int a = who; a < d / 64; a += 2)
+          tmem_cp_sf(tmem + kColX + 4 * a, sdesc_sf(smem_u32(xsf + (size_t)a * kDecAtom)));
+        mma_commit(&xsf_ready);
+      }
       bool ok = mbar_wait(&xsf_ready, 0, &s_abort, p.status);
       tc_fence_after();
       uint32_t it = 0, gc = 0;
@@ -331,8 +324,8 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
         const uint32_t hsf = tmem + kColH + 8 * who + 4 * (u & 1);
         tmem_cp_sf(hsf, sdesc_sf(smem_u32(hbuf + 512)));
         for (int q = 0; q < nks2; ++q, ++it) {
-          if (q % gst == 0) {  // a new group: the epilogue has read the previous one
-            if (!mbar_wait(&acc2_empty, (gc & 1) ^ 1, &s_abort, p.status)) {
+          if (q % gst == 0) {  // a new group: the epilogue has read this buffer's last group
+            if (!mbar_wait(&acc2_empty[gc & 1], ((gc >> 1) & 1) ^ 1, &s_abort, p.status)) {
               ok = false;
               break;
             }
@@ -351,14 +344,15 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               const int cl = (4 * q + i) % gch;
-              mma_mxf4nvf4(tmem + col_d2 + kDecDnN * cl, sdesc_kmajor(smem_u32(sb + 4096 * i), 256, kSwizzle32B),
+              mma_mxf4nvf4(tmem + col_d2 + (gc & 1) * gch * kDecDnN + kDecDnN * cl,
+                           sdesc_kmajor(smem_u32(sb + 4096 * i), 256, kSwizzle32B),
                            sdesc_kmajor(smem_u32(hbuf), 0, kSwizzle32B), kDecIdescT, sf + 4 * i, hsf, 0u);
             }
             mma_commit(&empty[it % NST]);
             if (it < 40) TC_TRACE_AT(g_dec_trace, kEvMmaIssued, it);
           }
           if (q % gst == gst - 1 || q == nks2 - 1) {
-            mma_commit(&acc2_full);
+            mma_commit(&acc2_full[gc & 1]);
             ++gc;
           }
         }
@@ -462,12 +456,12 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
         for (int g0 = 0; g0 < nch; g0 += gch, ++gc) {
           const int ng = nch - g0 < gch ? nch - g0 : gch;
           int ok = 1;
-          if (lane == 0) ok = mbar_wait(&acc2_full, gc & 1, &s_abort, p.status) ? 1 : 0;
+          if (lane == 0) ok = mbar_wait(&acc2_full[gc & 1], (gc >> 1) & 1, &s_abort, p.status) ? 1 : 0;
           ok = __shfl_sync(0xffffffffu, ok, 0);
           tc_fence_after();
           for (int cl = half; cl < ng; cl += 2) {
             uint32_t v[8];
-            tmem_ld8(lane_base + col_d2 + kDecDnN * cl, v);
+            tmem_ld8(lane_base + col_d2 + (gc & 1) * gch * kDecDnN + kDecDnN * cl, v);
             tmem_ld_wait();
             if (ok) {
               float* dst = p.out + (size_t)128 * (g0 + cl) + 32 * q4 + lane;
@@ -478,7 +472,7 @@ MOE_DEV void dec_run(const DecMaps& maps, const DecArgs& p, const DecSmem& sm, D
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc2_empty);
+          if (lane == 0) mbar_arrive(&acc2_empty[gc & 1]);
         }
         if (ew == 0 && lane == 0) TC_TRACE_AT(g_dec_trace, kEvDrainEnd, u);
       }
@@ -497,7 +491,7 @@ inline size_t dec_fixed_smem(int d) {
 
 // down chunks whose 16-column accumulators fit in TMEM next to everything else
 inline int dec_group_chunks(int d) {
-  const int avail = (512 - (int)dec_col_d2(d)) / kDecDnN;
+  const int avail = (512 - (int)dec_col_d2(d)) / kDecDnN / 2;  // two buffers
   const int g = avail & ~3;
   return g < d / 128 ? g : d / 128;
 }
@@ -517,39 +511,6 @@ inline size_t dec_smem_bytes(int d, size_t extra = 0) {
 inline bool dec_shape_ok(int64_t T, int d, int I) {
   return T >= 1 && T <= kDecMaxT && d % 512 == 0 && I % 64 == 0 && d <= 4096 && I <= 16384 &&
          dec_stages(d) >= kDecMinStages && dec_group_chunks(d) >= 4;
-}
-
-// Tensor maps of an expert group pair (the shared group, when absent, repeats the routed
-// maps): slice-grouped gate/up codes {128, 128, d/256, E*I/64} in {128, 128, 1, 1} boxes
-// (one contiguous 16 KB tile: 64 gate + 64 up rows x 256 columns, 128-byte swizzle);
-// slice-grouped down codes {32, 128, d/128, E*I/64} in {32, 128, 4, 1} boxes (four 128-row
-// chunks of one slice, 32-byte swizzle).
-inline cudaError_t dec_encode_maps(DecMaps* maps, const ExpertGroup& routed, const ExpertGroup& shared,
-                                   int has_shared, int E_routed, int d, int I) {
-  cudaError_t e = get_encode();
-  if (e != cudaSuccess) return e;
-  for (int which = 0; which < 2; ++which) {
-    const ExpertGroup& g = which ? shared : routed;
-    const int E = which ? 1 : E_routed;
-    CUtensorMap* m1 = which ? &maps->b1s : &maps->b1;
-    CUtensorMap* m2 = which ? &maps->b2s : &maps->b2;
-    if (which && !has_shared) {
-      *m1 = maps->b1;
-      *m2 = maps->b2;
-      continue;
-    }
-    cuuint64_t dims1[4] = {128, 128, (cuuint64_t)(d / 256), (cuuint64_t)E * (I / 64)};
-    cuuint64_t str1[3] = {128, 128 * 128, (cuuint64_t)(d / 256) * 128 * 128};
-    cuuint32_t box1[4] = {128, 128, 1, 1};
-    if ((e = encode_u8(m1, g.gu_codes_slice, 4, dims1, str1, box1, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
-      return e;
-    cuuint64_t dims2[4] = {32, 128, (cuuint64_t)(d / 128), (cuuint64_t)E * (I / 64)};
-    cuuint64_t str2[3] = {32, 128 * 32, (cuuint64_t)d * 32};
-    cuuint32_t box2[4] = {32, 128, 4, 1};
-    if ((e = encode_u8(m2, g.dn_codes_slice, 4, dims2, str2, box2, CU_TENSOR_MAP_SWIZZLE_32B)) != cudaSuccess)
-      return e;
-  }
-  return cudaSuccess;
 }
 
 }  // namespace moe

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(1024) ffn_dec_prep_kernel(DecParams p) {
 }
 
 // ---------------------------------------------------------------- the FFN kernel
-__global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_constant__ DecMaps maps, DecParams p) {
+__global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(DecParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ DecBars bar;
   __shared__ int s_ue[kDecMaxUnits], s_uj[kDecMaxUnits];
@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
   const DecSmem sm = dec_smem(align1024(smem_raw), p.d, p.nstages);
   const int d = p.d, T = p.T, nt1 = p.I / 64;
 
-  dec_init(bar, p.nstages, maps, p.has_shared);  // overlaps the previous kernel's tail
+  dec_init(bar, p.nstages);  // overlaps the previous kernel's tail
   RT_TRACE(g_prep_trace, 1, 0);
   MOE_PDL_PROLOGUE();
   RT_TRACE(g_prep_trace, 1, 1);
@@ -140,9 +140,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
   a.nstages = p.nstages;
   a.group_chunks = p.group_chunks;
   a.ts_x = *p.xq_ts;
+  a.xsf_loaded = 0;
   a.out = p.out;
   a.status = p.status;
-  dec_run(maps, a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw});
+  dec_run(a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw});
   if ((threadIdx.x >> 5) == 1) {
     tc_fence_after();
     tmem_dealloc(bar.tmem, 512);
@@ -150,7 +151,61 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_dec_kernel(const __grid_co
   RT_TRACE(g_prep_trace, 1, 2);
 }
 
+// ---------------------------------------------------------------- the decode pack
+// Per unit (expert e, 64-wide slice j of I): d/256 gate/up stages, then d/512 down stages,
+// each an 18 KB block that one bulk copy moves into a ring stage as the MMAs read it:
+//   gate/up stage kb: 128 rows x 128 bytes (rows 0-63 gate rows 64j.., rows 64-127 up rows
+//     64j..; bytes 128kb.. of each row) in the 128-byte swizzle (16-byte piece c of row r at
+//     r*128 + ((c ^ (r % 8)) * 16)), then the 4 scale atoms 4kb..4kb+3 of (e, j);
+//   down stage q: four 128-row chunks c = 4q..4q+3 (rows 128c.. of the down matrix, bytes
+//     32j..32j+31), each 128 x 32 bytes in the 32-byte swizzle (piece c' of row r at
+//     r*32 + ((c' ^ ((r / 4) % 2)) * 16)), then the scale atoms of those chunks for slice j.
+// One thread per 16-byte piece of the output.
+__global__ void pack_dec_kernel(const uint8_t* __restrict__ gu_codes, const uint8_t* __restrict__ dn_codes,
+                                const uint8_t* __restrict__ gu_sf, const uint8_t* __restrict__ dn_sf, int E, int d,
+                                int I, uint8_t* __restrict__ out) {
+  const int nt1 = I / 64, nks1 = d / 256, nks2 = d / 512, nsu = nks1 + nks2;
+  constexpr int kPieces = kDecStageBytes / 16;  // 1152 per stage, 1024 of them codes
+  const size_t n = (size_t)E * nt1 * nsu * kPieces;
+  for (size_t w = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w < n; w += (size_t)gridDim.x * blockDim.x) {
+    const int pc = (int)(w % kPieces);
+    const size_t us = w / kPieces;
+    const int q = (int)(us % nsu);
+    const size_t unit = us / nsu;
+    const int j = (int)(unit % nt1);
+    const size_t e = unit / nt1;
+    const uint8_t* src;
+    if (pc < kDecBBytes / 16) {
+      if (q < nks1) {
+        const int r = pc / 8, c = (pc % 8) ^ (r % 8);
+        const size_t row = e * 2 * I + (r < 64 ? 64 * j + r : I + 64 * j + r - 64);
+        src = gu_codes + row * (d / 2) + 128 * q + 16 * c;
+      } else {
+        const int ch = 4 * (q - nks1) + pc / 256, r = (pc % 256) / 2, c = (pc % 2) ^ ((r / 4) % 2);
+        src = dn_codes + (e * d + 128 * ch + r) * (I / 2) + 32 * j + 16 * c;
+      }
+    } else {
+      const int a = (pc - kDecBBytes / 16) / 32, pa = (pc - kDecBBytes / 16) % 32;
+      const size_t atom = q < nks1 ? (e * nt1 + j) * (d / 64) + 4 * q + a
+                                   : (e * (d / 128) + 4 * (q - nks1) + a) * nt1 + j;
+      src = (q < nks1 ? gu_sf : dn_sf) + atom * kDecAtom + 16 * pa;
+    }
+    *reinterpret_cast<uint4*>(out + w * 16) = *reinterpret_cast<const uint4*>(src);
+  }
+}
+
 // ---------------------------------------------------------------- host side
+size_t dec_pack_bytes(int E, int d, int I) {
+  return (size_t)E * (I / 64) * (d / 256 + d / 512) * kDecStageBytes;
+}
+
+cudaError_t launch_pack_dec(const ExpertGroup& g, int E, int d, int I, const uint8_t* gu_sf_tiled,
+                            const uint8_t* dn_sf_tiled, uint8_t* dec_pack, int num_sms, cudaStream_t st) {
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  pack_dec_kernel<<<num_sms * 4, 256, 0, st>>>(g.gu_codes, g.dn_codes, gu_sf_tiled, dn_sf_tiled, E, d, I, dec_pack);
+  return cudaGetLastError();
+}
+
 namespace {
 size_t a256d(size_t v) { return (v + 255) & ~(size_t)255; }
 }  // namespace
@@ -191,11 +246,9 @@ cudaError_t launch_ffn_dec(const FfnArgs& a, void* ws, int num_sms, int32_t* sta
   p.slots = reinterpret_cast<int32_t*>(w + 256);
   p.slot_w = reinterpret_cast<float*>(w + 256 + a256d((size_t)(a.E + 1) * 4));
   p.status = status;
-  DecMaps maps;
-  cudaError_t e = dec_encode_maps(&maps, a.routed, a.shared, a.has_shared, a.E, a.d, a.I);
+  cudaError_t e = launch_pdl(ffn_dec_prep_kernel, dim3(1), dim3(1024), 0, st, p);
   if (e != cudaSuccess) return e;
-  if ((e = launch_pdl(ffn_dec_prep_kernel, dim3(1), dim3(1024), 0, st, p)) != cudaSuccess) return e;
-  return launch_pdl(ffn_dec_kernel, dim3(num_sms), dim3(kDecThreads), dec_smem_bytes(a.d), st, maps, p);
+  return launch_pdl(ffn_dec_kernel, dim3(num_sms), dim3(kDecThreads), dec_smem_bytes(a.d), st, p);
 }
 
 }  // namespace moe

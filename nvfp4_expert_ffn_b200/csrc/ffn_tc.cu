@@ -211,54 +211,6 @@ __global__ void pack_sf_kernel(const uint8_t* __restrict__ gu_scales, const uint
   }
 }
 
-// down matrix per 64-column slice of I: codes [E][I/64][d][32] (row n of slice j = bytes
-// 32j..32j+31 of row n), scale atoms [E][I/64][d/128][512] (atom (e, j, c) = rows 128c.. of
-// scale blocks 4j..4j+3, laid out as in pack_sf_kernel)
-__global__ void pack_slices_kernel(const uint8_t* __restrict__ dn_codes, const uint8_t* __restrict__ dn_scales,
-                                   const uint8_t* __restrict__ gu_codes, int E, int d, int I,
-                                   uint8_t* __restrict__ cs, uint8_t* __restrict__ ss, uint8_t* __restrict__ gs) {
-  const int nj = I / 64;
-  const size_t nc = (size_t)E * nj * d * 2;          // 16-byte pieces of codes
-  const size_t ns = (size_t)E * nj * (d / 128) * 128;  // 32-bit words of scale atoms
-  const size_t ng = (size_t)E * I * d / 16;            // 16-byte pieces of gate/up codes
-  for (size_t w = blockIdx.x * (size_t)blockDim.x + threadIdx.x; w < nc + ns + ng;
-       w += (size_t)gridDim.x * blockDim.x) {
-    if (w >= nc + ns) {
-      // gate/up tile (e, j, kb): row r < 64 is gate row 64j + r, row r >= 64 up row 64j + r - 64,
-      // columns 256kb..256kb+255 (128 bytes, 8 pieces)
-      const size_t g = w - nc - ns;
-      const int piece = (int)(g % 8);
-      const int r = (int)((g / 8) % 128);
-      const size_t tile = g / 1024;  // over [E][I/64][d/256]
-      const int kb = (int)(tile % (d / 256));
-      const int j = (int)((tile / (d / 256)) % nj);
-      const size_t e = tile / (d / 256) / nj;
-      const size_t row = e * 2 * I + (r < 64 ? 64 * j + r : I + 64 * j + r - 64);
-      *reinterpret_cast<uint4*>(gs + g * 16) =
-          *reinterpret_cast<const uint4*>(gu_codes + row * (d / 2) + 128 * kb + 16 * piece);
-    } else if (w < nc) {
-      const int piece = (int)(w & 1);
-      const size_t row = w >> 1;  // over [E][I/64][d]
-      const int n = (int)(row % d);
-      const int j = (int)((row / d) % nj);
-      const size_t e = row / d / nj;
-      *reinterpret_cast<uint4*>(cs + row * 32 + 16 * piece) =
-          *reinterpret_cast<const uint4*>(dn_codes + (e * d + n) * (I / 2) + 32 * j + 16 * piece);
-    } else {
-      const size_t ww = w - nc;
-      const size_t atom = ww / 128;
-      const int slot = (int)(ww % 128);  // r0 * 4 + r1
-      const int r = (slot % 4) * 32 + slot / 4;
-      const int c = (int)(atom % (d / 128));
-      const int j = (int)((atom / (d / 128)) % nj);
-      const size_t e = atom / (d / 128) / nj;
-      const uint32_t v =
-          *reinterpret_cast<const uint32_t*>(dn_scales + (e * d + 128 * c + r) * (I / kBlock) + 4 * j);
-      *reinterpret_cast<uint32_t*>(ss + atom * kAtom + (slot / 4) * 16 + (slot % 4) * 4) = v;
-    }
-  }
-}
-
 // ---------------------------------------------------------------- 3. persistent FFN kernel
 struct TcMaps {
   CUtensorMap xg;    // x codes [T][d/2], one-row boxes for tile::gather4
@@ -732,12 +684,6 @@ cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* g
   return cudaGetLastError();
 }
 
-cudaError_t launch_pack_slices(const ExpertGroup& g, int E, int d, int I, uint8_t* cs, uint8_t* ss, uint8_t* gs,
-                               int num_sms, cudaStream_t st) {
-  g_launch_count.fetch_add(1, std::memory_order_relaxed);
-  pack_slices_kernel<<<num_sms * 4, 256, 0, st>>>(g.dn_codes, g.dn_scales, g.gu_codes, E, d, I, cs, ss, gs);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st) {
   cudaError_t e = get_encode();

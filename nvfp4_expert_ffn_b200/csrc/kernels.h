@@ -46,9 +46,7 @@ struct ExpertGroup {
   const float* dn_ts;
   const uint8_t* gu_sf_tiled;
   const uint8_t* dn_sf_tiled;
-  const uint8_t* dn_codes_slice;  // [E][I/64][d][32]
-  const uint8_t* dn_sf_slice;     // [E][I/64][d/128][512]
-  const uint8_t* gu_codes_slice;  // [E][I/64][d/256][128][128]
+  const uint8_t* dec_pack;  // [E][I/64][d/256 + d/512][18432]: decode stages (moe_pack_experts)
 };
 
 struct FfnArgs {
@@ -128,8 +126,9 @@ struct LayerDecArgs {
 bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms);
 size_t layer_dec_ws_bytes(int64_t T, int E);
 cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
-cudaError_t launch_pack_slices(const ExpertGroup& g, int E, int d, int I, uint8_t* dn_codes_slice,
-                               uint8_t* dn_sf_slice, uint8_t* gu_codes_slice, int num_sms, cudaStream_t st);
+cudaError_t launch_pack_dec(const ExpertGroup& g, int E, int d, int I, const uint8_t* gu_sf_tiled,
+                            const uint8_t* dn_sf_tiled, uint8_t* dec_pack, int num_sms, cudaStream_t st);
+size_t dec_pack_bytes(int E, int d, int I);
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
                            int num_sms, cudaStream_t st);
 

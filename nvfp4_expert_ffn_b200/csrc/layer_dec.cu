@@ -8,13 +8,16 @@
 // Here one CTA per SM (all but one SM, left to a side-stream kernel such as the cumulative
 // histogram) runs:
 //   phase 1  every CTA loads x, takes the global amax itself (the NVFP4 tensor scale),
-//            quantises its share of the 16-element blocks into the xq output buffers, and
+//            quantises its share of the 64-element groups into the xq output buffers, and
 //            computes the router logits of its expert rows (E / grid rows, the router
-//            weights loaded before the kernel waits on its predecessor); CTA 0 zeroes y_acc.
+//            weights copied in before the kernel waits on its predecessor); CTA 0 zeroes
+//            y_acc.
 //   barrier
-//   phase 2  every CTA reads all tokens' codes into its shared-memory tiles, runs the
-//            top-k of all tokens itself and derives its own units; the last CTA also
-//            writes the routing outputs (top-k, counts, offsets, permutation).
+//   phase 2  every CTA reads all tokens' codes into its MMA operand tiles (their scales go
+//            on to TMEM while the rest of the phase runs) and all logits, runs the top-k of
+//            all tokens itself and derives its own units from the bitmap of chosen experts;
+//            the last CTA also writes the routing outputs (top-k, counts, offsets,
+//            permutation).
 //   phase 3  the units (expert, 64-column slice of I), adding into y_acc.
 //   barrier
 //   phase 4  CTA t < T converts row t of y_acc to bf16 (optionally RMS-renormalised).
@@ -63,51 +66,61 @@ struct LayerArgs {
 // Grid-wide barrier on a 64-bit arrival counter that only grows: thread 0 of each CTA adds
 // one and waits (bounded) until the count reaches the next multiple of the grid size. The
 // counter starts at zero and every call adds two multiples, so it stays aligned. Writes
-// before the barrier are visible to every CTA after it.
-MOE_DEV bool grid_sync(unsigned long long* count, volatile int* abort, int32_t* status) {
-  __shared__ int s_ok;
+// before the arrival are visible to every CTA after the wait; the CTA may work between the
+// two halves.
+//
+// Arrival (every thread calls it): returns, in thread 0, the count to wait for (0 if the
+// kernel is aborting and did not arrive).
+MOE_DEV unsigned long long grid_arrive(unsigned long long* count, volatile int* abort) {
   __syncthreads();
+  unsigned long long target = 0;
+  if (threadIdx.x == 0 && !*abort) {
+    const unsigned long long G = gridDim.x;
+    __threadfence();
+    const unsigned long long old = atomicAdd(count, 1ull);
+    target = (old / G + 1) * G;
+  }
+  return target;
+}
+
+// Wait (every thread calls it, thread 0 with the arrival's target): false after an abort or
+// a timeout.
+MOE_DEV bool grid_wait(unsigned long long* count, unsigned long long target, volatile int* abort, int32_t* status) {
+  __shared__ int s_ok;
   if (threadIdx.x == 0) {
-    int ok = *abort ? 0 : 1;
-    if (ok) {
-      const unsigned long long G = gridDim.x;
-      __threadfence();
-      const unsigned long long old = atomicAdd(count, 1ull);
-      const unsigned long long target = (old / G + 1) * G;
-      const uint64_t t0 = globaltimer_ns();
-      while (true) {
-        unsigned long long c;
-        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count) : "memory");
-        if (c >= target) break;
-        if (*abort) {
-          ok = 0;
-          break;
-        }
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-          *abort = 1;
-          atomicExch(status, kStatusTimeout);
-          ok = 0;
-          break;
-        }
+    int ok = target != 0 && !*abort ? 1 : 0;
+    const uint64_t t0 = globaltimer_ns();
+    while (ok) {
+      unsigned long long c;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count) : "memory");
+      if (c >= target) break;
+      if (*abort) {
+        ok = 0;
+      } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicExch(status, kStatusTimeout);
+        ok = 0;
       }
-      __threadfence();
     }
+    __threadfence();
     s_ok = ok;
   }
   __syncthreads();
   return s_ok != 0;
 }
 
+MOE_DEV bool grid_sync(unsigned long long* count, volatile int* abort, int32_t* status) {
+  return grid_wait(count, grid_arrive(count, abort), abort, status);
+}
+
 // Shared-memory scratch of phases 1 and 2, on the weight ring (not in use before phase 3):
 // the bf16 activations (phase 1), then at the same place the logits (phase 2); the top-k of
-// each token, the expert-use flags and list, and the permutation's counters.
+// each token, the permutation's counters, the router's partial sums and rows.
 struct LayerScratch {
   uint16_t* xb;   // [8][d] (phase 1)
   float* logits;  // [8][E] (phase 2, over xb)
   int* tidx;      // [8][32] expert ids of each token's top-k
   float* tw;      // [8][32] their weights
-  int* flag;      // [1024] expert used by some token
-  int* list;      // [1025] experts in use, in id order after the shared expert
   int* perm;      // [1024] counters of the permutation
   int* sidx;      // [256] top-k expert ids, assignment order
   float* part;    // [kDecThreads] router partial sums (phase 1)
@@ -126,9 +139,7 @@ MOE_DEV LayerScratch layer_scratch(uint8_t* ring, int d) {
   s.logits = reinterpret_cast<float*>(ring);
   s.tidx = reinterpret_cast<int*>(ring + layer_scratch_head(d));
   s.tw = reinterpret_cast<float*>(s.tidx + kDecMaxT * kLayerMaxK);
-  s.flag = reinterpret_cast<int*>(s.tw + kDecMaxT * kLayerMaxK);
-  s.list = s.flag + 1024;
-  s.perm = s.list + 1040;
+  s.perm = reinterpret_cast<int*>(s.tw + kDecMaxT * kLayerMaxK);
   s.sidx = s.perm + 1024;
   s.part = reinterpret_cast<float*>(s.sidx + 256);
   s.tks = reinterpret_cast<uint32_t*>(s.part + kDecThreads);
@@ -136,16 +147,17 @@ MOE_DEV LayerScratch layer_scratch(uint8_t* ring, int d) {
   return s;
 }
 // bytes of scratch past the head
-constexpr size_t kLayerScratchTail = 2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 1040 + 1024 + 256 + kDecThreads + kDecMaxT * 64) * 4;
+constexpr size_t kLayerScratchTail = 2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 256 + kDecThreads + kDecMaxT * 64) * 4;
 static_assert(kLayerScratchTail % 16 == 0, "router rows must start 16-byte aligned");
 
-__global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_constant__ DecMaps maps, LayerArgs p) {
+__global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ DecBars bar;
   __shared__ int s_ue[kDecMaxUnits], s_uj[kDecMaxUnits];
   __shared__ float s_uw[kDecMaxUnits * kDecMaxT];
   __shared__ float s_red[32];
-  __shared__ int s_tmp[32];
+  __shared__ uint32_t s_bits[32];  // experts chosen by some token (E <= 1024)
+  __shared__ int s_nu;
   const DecSmem sm = dec_smem(align1024(smem_raw), p.d, p.nstages);
   const LayerScratch sc = layer_scratch(sm.ring, p.d);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,8 +173,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   __shared__ uint64_t s_wbar;
   __shared__ float s_bias[kLayerMaxRows];
   if (threadIdx.x == 0) mbar_init(&s_wbar, 1);
+  if (threadIdx.x < 32) s_bits[threadIdx.x] = 0u;
   if (threadIdx.x < nrows) s_bias[threadIdx.x] = p.br ? __ldg(p.br + b + threadIdx.x * G) : 0.0f;
-  dec_init(bar, p.nstages, maps, p.has_shared);  // includes the barrier-init fence
+  dec_init(bar, p.nstages);  // includes the barrier-init fence
   if (threadIdx.x == 0 && nrows > 0) {
     mbar_arrive_expect_tx(&s_wbar, (uint32_t)(nrows * d * 4));
     for (int r = 0; r < nrows; ++r)
@@ -323,8 +336,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   const bool writer = b == G - 1;  // the CTA with the fewest units writes the routing outputs
   int nu = 0;
   if (ok) {
-    // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms; each thread's
-    // loads of a round go out together
+    // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms, logits -> shared
+    // memory; each thread's loads of a round go out together
     {
       const int q4 = d / 256;  // 16-byte pieces of a token's scale row
       uint4 sv = make_uint4(0u, 0u, 0u, 0u);
@@ -383,67 +396,97 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
         }
       }
     }
-    RT_TRACE(g_layer_trace, 3, 5);
-    for (int e = threadIdx.x; e < E; e += blockDim.x) sc.flag[e] = 0;
+    fence_proxy_async_smem();  // the tiles and atoms are read by tcgen05 (async proxy)
     __syncthreads();
     RT_TRACE(g_layer_trace, 3, 0);
-    // top-k of every token (one warp each)
-    if (warp < T)
+    // the activation scale atoms -> TMEM for the whole of phase 3, issued by a warp the top-k
+    // leaves idle (both issuers' arrivals on xsf_ready come from here)
+    if (warp == kDecThreads / 32 - 1 && lane == 0) {
+      tc_fence_after();
+      for (int a = 0; a < d / 64; ++a)
+        tmem_cp_sf(bar.tmem + kColX + 4 * a, sdesc_sf(smem_u32(sm.xsf + (size_t)a * kDecAtom)));
+      mma_commit(&bar.xsf_ready);
+      mma_commit(&bar.xsf_ready);
+    }
+    // top-k of every token (one warp each); the chosen experts are marked in s_bits
+    if (warp < T) {
       topk_dispatch(sc.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
                     writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
                     sc.tw + warp * kLayerMaxK, sc.tks + warp * 64);
+      __syncwarp();
+      if (lane < k) {
+        const int e = sc.tidx[warp * kLayerMaxK + lane];
+        atomicOr(&s_bits[e >> 5], 1u << (e & 31));
+      }
+    }
     __syncthreads();
     RT_TRACE(g_layer_trace, 3, 1);
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-      const int e = sc.tidx[(i / k) * kLayerMaxK + i % k];
-      sc.flag[e] = 1;
-      sc.sidx[i] = e;
-    }
-    __syncthreads();
-    // experts in use, in id order after the shared expert (contiguous ranges per thread)
-    const int per = (E + blockDim.x - 1) / blockDim.x;
-    const int e0 = threadIdx.x * per;
-    int cnt = 0;
-    for (int e = e0; e < E && e < e0 + per; ++e) cnt += sc.flag[e];
-    int total;
-    int slot = block_exclusive_scan(cnt, s_tmp, &total) + p.has_shared;
-    for (int e = e0; e < E && e < e0 + per; ++e)
-      if (sc.flag[e]) sc.list[slot++] = e;
-    if (threadIdx.x == 0 && p.has_shared) sc.list[0] = E;
-    const int nslots = total + p.has_shared;
-    __syncthreads();
-    RT_TRACE(g_layer_trace, 3, 2);
-    if (writer && warp == 0)
-      perm_small_warp(sc.sidx, T * k, E, sc.perm, p.counts, p.offsets, p.sorted_assign, p.assign_pos);
-    // this CTA's units: blockIdx.x, blockIdx.x + gridDim.x, ... of nslots * nt1
-    const int nunits = nslots * nt1;
-    nu = b < nunits ? (nunits - 1 - b) / G + 1 : 0;
-    if (nu > kDecMaxUnits) {  // the host checks the worst case, so this does not happen
-      if (threadIdx.x == 0) atomicExch(p.status, kStatusUnsupported);
-      nu = kDecMaxUnits;
-    }
-    for (int i = threadIdx.x; i < nu * (kDecMaxT + 1); i += blockDim.x) {
-      const int u = i / (kDecMaxT + 1), f = i % (kDecMaxT + 1);
-      const int ug = b + u * G;
-      const int e = sc.list[ug / nt1];
-      if (f == kDecMaxT) {
-        s_ue[u] = e;
-        s_uj[u] = ug % nt1;
-      } else {
+    if (warp == 0) {
+      // This CTA's units are b, b + G, ... of nslots * nt1 (slot 0 the shared expert, then the
+      // experts in use in id order; unit ug is slice ug % nt1 of slot ug / nt1). Lane w holds
+      // bitmap word w and the inclusive count of experts in use up to it; lane u finds its
+      // unit's expert as the n-th chosen bit.
+      const int nwd = (E + 31) >> 5;
+      const uint32_t word = lane < nwd ? s_bits[lane] : 0u;
+      int incl = __popc(word);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int nslots = __shfl_sync(0xffffffffu, incl, 31) + p.has_shared;
+      const int nunits = nslots * nt1;
+      int n = b < nunits ? (nunits - 1 - b) / G + 1 : 0;
+      if (n > kDecMaxUnits) {  // the host checks the worst case, so this does not happen
+        if (lane == 0) atomicExch(p.status, kStatusUnsupported);
+        n = kDecMaxUnits;
+      }
+      const int ug = b + lane * G;
+      const int rnk = ug / nt1 - p.has_shared;  // rank among the experts in use (< 0: shared)
+      int lo = 0;                                // the first word whose inclusive count exceeds rnk
+#pragma unroll
+      for (int step = 16; step >= 1; step >>= 1)
+        if (__shfl_sync(0xffffffffu, incl, lo + step - 1) <= rnk) lo += step;
+      // (every lane takes part in every shuffle)
+      uint32_t wd = __shfl_sync(0xffffffffu, word, lo);
+      const int prev = __shfl_sync(0xffffffffu, incl, lo > 0 ? lo - 1 : 0);
+      const int below = lo > 0 ? prev : 0;
+      if (lane < n) {
+        int e = E;
+        if (rnk >= 0) {
+          for (int i = 0; i < rnk - below; ++i) wd &= wd - 1u;
+          e = 32 * lo + __ffs(wd) - 1;
+        }
+        s_ue[lane] = e;
+        s_uj[lane] = ug % nt1;
+      }
+      if (lane == 0) s_nu = n;
+      __syncwarp();
+      for (int i = lane; i < n * kDecMaxT; i += 32) {
+        const int u = i / kDecMaxT, t = i % kDecMaxT;
+        const int e = s_ue[u];
         float wt = 0.0f;
-        if (f < T) {
+        if (t < T) {
           if (e == E) {
             wt = 1.0f;
           } else {
             for (int j = 0; j < k; ++j)
-              if (sc.tidx[f * kLayerMaxK + j] == e) wt = sc.tw[f * kLayerMaxK + j];
+              if (sc.tidx[t * kLayerMaxK + j] == e) wt = sc.tw[t * kLayerMaxK + j];
           }
         }
-        s_uw[u * kDecMaxT + f] = wt;
+        s_uw[u * kDecMaxT + t] = wt;
       }
+    } else if (warp == 1 && writer) {
+      // the routing outputs: assignment a = t*k + j in expert order
+      for (int a = lane; a < T * k; a += 32) sc.sidx[a] = sc.tidx[(a / k) * kLayerMaxK + a % k];
+      __syncwarp();
+      perm_small_warp(sc.sidx, T * k, E, sc.perm, p.counts, p.offsets, p.sorted_assign, p.assign_pos);
     }
+    __syncthreads();
+    nu = s_nu;
+    RT_TRACE(g_layer_trace, 3, 2);
   }
-  fence_proxy_async_smem();  // the tiles and atoms above are read by tcgen05 (async proxy)
+  fence_proxy_async_smem();  // the bulk copies of phase 3 overwrite the scratch written above
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -458,9 +501,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(const __grid_
   a.nstages = p.nstages;
   a.group_chunks = p.group_chunks;
   a.ts_x = ts;
+  a.xsf_loaded = 1;
   a.out = p.y_acc;
   a.status = p.status;
-  dec_run(maps, a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw});
+  dec_run(a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw});
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(bar.tmem, 512);
@@ -550,10 +594,7 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
   p.sync = reinterpret_cast<unsigned long long*>(w);
   p.logits = reinterpret_cast<float*>(w + 256);
   p.status = status;
-  DecMaps maps;
-  cudaError_t e = dec_encode_maps(&maps, a.routed, a.shared, a.has_shared, a.E, a.d, a.I);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st, maps, p);
+  return launch_pdl(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st, p);
 }
 
 }  // namespace moe
@@ -561,5 +602,6 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
 #ifdef MOE_TRACE
 namespace moe {
 int64_t trace_fetch_layer(void* host, size_t bytes) { return trace_fetch(g_layer_trace, host, bytes); }
+int64_t trace_fetch_layer_core(void* host, size_t bytes) { return trace_fetch(g_dec_trace, host, bytes); }
 }  // namespace moe
 #endif

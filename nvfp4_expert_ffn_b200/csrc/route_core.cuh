@@ -31,6 +31,7 @@ MOE_DEV uint32_t ordered_key(float v) {
 // (the usual case: about k + 2 for independent logits) they are gathered one per lane and
 // each candidate's rank is counted against the other 31. Otherwise k rounds of a warp
 // arg-max pick the winners one at a time, and only the winning lane rescans its entries.
+// Both give the same picks in the same order.
 template <int NPER, bool kL2 = false>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* idx_out, float* w_out,
                         int* idx_smem = nullptr, float* w_smem = nullptr, uint32_t* scratch = nullptr) {
@@ -56,24 +57,25 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
       if (e < E && !((taken >> j) & 1u) && before(key[j], e, bk, be)) bk = key[j], be = e;
     }
   };
-  uint32_t lbk;
-  int lbe;
-  local_best(lbk, lbe);
   uint32_t top_key = 0, my_key = 0;  // lane r < k ends with the r-th pick
   int my_e = 0;
   bool done = false;
   if (scratch != nullptr && k <= 32) {
-    // rank of this lane's maximum among the lanes' maxima (lanes without entries tie at
-    // the bottom, behind min(E, 32) >= k valid maxima)
-    int rank = 0;
+    // the lane's largest key (a tree, so the steps do not wait on one another)
+    uint32_t m[NPER];
+#pragma unroll
+    for (int j = 0; j < NPER; ++j) m[j] = key[j];
+#pragma unroll
+    for (int w = NPER / 2; w >= 1; w /= 2)
+#pragma unroll
+      for (int j = 0; j < w; ++j) m[j] = max(m[j], m[j + w]);
+    const uint32_t lmax = m[0];
+    // threshold: the k-th largest lane maximum = the smallest maximum with fewer than k
+    // maxima strictly above it (lanes without entries hold 0, below every key)
+    int above = 0;
 #pragma unroll 8
-    for (int o = 1; o < 32; ++o) {
-      const int src = (lane + o) & 31;
-      const uint32_t ok = __shfl_sync(0xffffffffu, lbk, src);
-      const int oe = __shfl_sync(0xffffffffu, lbe, src);
-      rank += before(ok, oe, lbk, lbe) ? 1 : 0;
-    }
-    const uint32_t th = __shfl_sync(0xffffffffu, lbk, __ffs(__ballot_sync(0xffffffffu, rank == k - 1)) - 1);
+    for (int o = 1; o < 32; ++o) above += __shfl_sync(0xffffffffu, lmax, (lane + o) & 31) > lmax ? 1 : 0;
+    const uint32_t th = __reduce_min_sync(0xffffffffu, above < k ? lmax : 0xffffffffu);
     int c = 0;
 #pragma unroll
     for (int j = 0; j < NPER; ++j) c += (lane + 32 * j < E && key[j] >= th) ? 1 : 0;
@@ -99,13 +101,19 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
       const uint32_t ck = lane < total ? scratch[lane] : 0u;
       const int ce = lane < total ? (int)scratch[32 + lane] : 0x7fffffff;
       __syncwarp();
+      // rank of each candidate: keys strictly above it, then (only when two candidates share
+      // a key) the equal keys of lower expert id
       int r = 0;
 #pragma unroll 8
-      for (int o = 1; o < 32; ++o) {
-        const int src = (lane + o) & 31;
-        const uint32_t ok = __shfl_sync(0xffffffffu, ck, src);
-        const int oe = __shfl_sync(0xffffffffu, ce, src);
-        r += before(ok, oe, ck, ce) ? 1 : 0;
+      for (int o = 1; o < 32; ++o) r += __shfl_sync(0xffffffffu, ck, (lane + o) & 31) > ck ? 1 : 0;
+      const uint32_t same = __match_any_sync(0xffffffffu, ck);
+      if (__any_sync(0xffffffffu, lane < total && __popc(same) > 1)) {
+        for (int o = 1; o < 32; ++o) {
+          const int src = (lane + o) & 31;
+          const uint32_t ok = __shfl_sync(0xffffffffu, ck, src);
+          const int oe = __shfl_sync(0xffffffffu, ce, src);
+          r += (ok == ck && oe < ce) ? 1 : 0;
+        }
       }
       if (lane < total && r < k) {
         scratch[r] = ck;
@@ -122,6 +130,9 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
     }
   }
   if (!done) {
+    uint32_t lbk;
+    int lbe;
+    local_best(lbk, lbe);
     for (int r = 0; r < k; ++r) {
       const uint32_t mk = __reduce_max_sync(0xffffffffu, lbk);
       const int me = (int)__reduce_min_sync(0xffffffffu, lbk == mk ? (uint32_t)lbe : 0x7fffffffu);

@@ -80,8 +80,8 @@ class MoeLayer:
         # calls of at most 8 tokens go through the one-kernel decode layer when the shapes allow;
         # its workspace holds a barrier counter and must start zeroed
         can_fuse = (d % 512 == 0 and d <= 4096 and I % 64 == 0 and k <= 32 and E <= 1024
-                    and experts.routed.gu_codes_slice is not None
-                    and (experts.shared is None or experts.shared.gu_codes_slice is not None))
+                    and experts.routed.dec_pack is not None
+                    and (experts.shared is None or experts.shared.dec_pack is not None))
         self.fused = can_fuse if fused is None else (fused and can_fuse)
         self.ws_dec = torch.zeros(
             max(256, B.moe_workspace_size(B.MOE_OP_LAYER_DECODE, min(T_max, 8), d, E, k, I)),

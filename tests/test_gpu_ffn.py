@@ -216,17 +216,48 @@ def test_ffn_prefill_configs_sampled(cfg_name, n_sample):
     assert np.isfinite(yf).all() and (np.abs(yf).sum(1) > 0).all()
 
 
-def test_pack_slices_regroup_the_weights():
-    """moe_pack_experts' slice copies are exact regroupings: down codes [E][d][I/2] ->
-    [E][I/64][d][32], the down scale atoms [E][d/128][I/64] -> [E][I/64][d/128], and gate/up codes
-    [E][2I][d/2] -> [E][I/64][d/256][64 gate rows + 64 up rows][128] (integer, bit-exact)."""
+def _swizzle_rows(tile, piece_of):
+    """Place 16-byte piece c of row r of a byte tile [rows][16 * n] at piece piece_of(r, c)."""
+    rows, n = tile.shape[0], tile.shape[1] // 16
+    t = tile.reshape(rows, n, 16)
+    out = np.empty_like(t)
+    r = np.arange(rows)[:, None]
+    c = np.arange(n)[None, :]
+    out[r, piece_of(r, c)] = t
+    return out.reshape(-1)
+
+
+def _scale_atom(rows4):
+    """[128 rows][4 scale bytes] -> the 512-byte atom: row 32*r1 + r0, block b at r0*16 + r1*4 + b."""
+    return rows4.reshape(4, 32, 4).transpose(1, 0, 2).reshape(512)
+
+
+def test_pack_dec_layout():
+    """The decode pack of moe_pack_experts holds, per unit (e, slice j) and 18432-byte block,
+    exactly the bytes its header describes, rebuilt here from the natural layout: swizzled
+    gate/up and down tiles and the scale atoms (integer, bit-exact)."""
     experts, sh, xq, routing, gpu = _tiny_case(15, 512, 4, 2, 192, 3, True, pack=True)
     for w in (gpu.routed, gpu.shared):
         E, d, I = w.E, w.d, w.I
-        nat = w.dn_codes.cpu().numpy().reshape(E, d, I // 64, 32).transpose(0, 2, 1, 3)
-        assert np.array_equal(w.dn_codes_slice.cpu().numpy().reshape(E, I // 64, d, 32), nat)
-        atoms = w.dn_sf_tiled.cpu().numpy().reshape(E, d // 128, I // 64, 512).transpose(0, 2, 1, 3)
-        assert np.array_equal(w.dn_sf_slice.cpu().numpy().reshape(E, I // 64, d // 128, 512), atoms)
-        gu = w.gu_codes.cpu().numpy().reshape(E, 2, I // 64, 64, d // 256, 128)  # [e][g/u][j][r][kb][byte]
-        tiles = gu.transpose(0, 2, 4, 1, 3, 5).reshape(E, I // 64, d // 256, 128, 128)
-        assert np.array_equal(w.gu_codes_slice.cpu().numpy().reshape(E, I // 64, d // 256, 128, 128), tiles)
+        guc, gus = w.gu_codes.cpu().numpy(), w.gu_scales.cpu().numpy()
+        dnc, dns = w.dn_codes.cpu().numpy(), w.dn_scales.cpu().numpy()
+        blocks = []
+        for e in range(E):
+            for j in range(I // 64):
+                rows = np.r_[64 * j:64 * j + 64, I + 64 * j:I + 64 * j + 64]
+                for kb in range(d // 256):
+                    tile = guc[e, rows, 128 * kb:128 * kb + 128]
+                    blocks.append(_swizzle_rows(tile, lambda r, c: c ^ (r % 8)))
+                    for a in range(4):
+                        kc = 4 * kb + a
+                        blocks.append(_scale_atom(gus[e, rows, 4 * kc:4 * kc + 4]))
+                for q in range(d // 512):
+                    for c in range(4 * q, 4 * q + 4):
+                        tile = dnc[e, 128 * c:128 * c + 128, 32 * j:32 * j + 32]
+                        blocks.append(_swizzle_rows(tile, lambda r, cc: cc ^ ((r // 4) % 2)))
+                    for c in range(4 * q, 4 * q + 4):
+                        blocks.append(_scale_atom(dns[e, 128 * c:128 * c + 128, 4 * j:4 * j + 4]))
+        want = np.concatenate(blocks)
+        got = w.dec_pack.cpu().numpy()
+        assert got.size == B.dec_pack_bytes(E, d, I) == want.size
+        assert np.array_equal(got, want)
