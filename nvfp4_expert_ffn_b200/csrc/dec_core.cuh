@@ -22,12 +22,14 @@
 //   * both products are computed transposed, D[weight row][token]: the weight tile is the
 //     128-row A operand, the tokens a 16-column B operand, so an accumulator takes 16 TMEM
 //     columns and a unit's 16 down chunks accumulate side by side.
-//   * the ring of shared-memory stages carries only weights: a 64-gate + 64-up row x 256-column
-//     tile of the slice-grouped gate/up matrix (one contiguous 16 KB TMA box, 128-byte
-//     swizzle) with its 4 scale atoms, or four 128-row x 64-column chunks of the
-//     slice-grouped down matrix (one TMA box, 32-byte swizzle) with theirs (one bulk copy).
-//     Every stage reads contiguous bytes: 128-byte pieces of rows 1 KB apart (the natural
-//     layout) keep HBM well below its streaming rate.
+//   * the ring of shared-memory stages carries only weights, each stage one 18 KB block of
+//     the decode pack (moe_pack_experts) moved by one bulk copy: a 64-gate + 64-up row x
+//     256-column tile already in the 128-byte swizzle, or four 128-row x 64-column down
+//     chunks already in the 32-byte swizzle, followed by the stage's 4 scale atoms. A unit's
+//     blocks are contiguous, so HBM streams whole runs, and one copy per stage leaves the
+//     per-SM copy engine, which also executes the tcgen05 scale copies, as free as it can be.
+//   * the down accumulators form two buffers of group_chunks chunks; down groups alternate
+//     between them, so one group's MMAs overlap the epilogue's reading of the previous one.
 //
 // Warp roles (352 threads, one CTA per SM): warp 0 lane 0 issues the copies; warps 1 and 2
 // (lane 0) issue tcgen05 copies and MMAs for alternate ring stages (an issued tcgen05
