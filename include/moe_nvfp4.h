@@ -218,8 +218,8 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
  * memory round trips would cost more than the work (Basalt pages: "What Basalt changes in a
  * Blackwell local inference stack", section "Experts can move without becoming free").
  *   x_bf16 [T][d]; ts_in float32[1] static activation scale or NULL (dynamic amax);
- *   Wr float32 [E][d]; br float32 [E] or NULL; W: both groups packed by moe_pack_experts,
- *   slices included.
+ *   Wr float32 [E][d]; br float32 [E] or NULL; W: both groups with the decode pack
+ *   (dec_pack) of moe_pack_experts.
  *   Outputs: xq_codes [T][d/2], xq_scales [T][d/16], xq_ts [1]; topk_idx [T][k],
  *   topk_w [T][k]; counts [E], offsets [E+1], sorted_assign [T*k], assign_pos [T*k];
  *   y_acc float32 [T][d] (the unrounded output); y_bf16 [T][d]; rms_renorm as moe_combine.
@@ -227,7 +227,9 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
  *   call (it holds the arrival counter of the kernel's grid-wide barrier, which every call
  *   leaves at a multiple of the grid size; after a MOE_ERR_TIMEOUT from
  *   moe_get_device_status, zero it again).
- * Limits: 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024.
+ * Limits: 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024,
+ * and at most 32 units per CTA in the worst case ((min(T*k, E) + shared) * I/64 units over
+ * all SMs but one); otherwise MOE_ERR_UNSUPPORTED_SHAPE.
  * The kernel uses all SMs but one and waits at grid-wide barriers, so it must not share the
  * GPU with a kernel that occupies more than one SM until this one ends.
  */

@@ -342,7 +342,8 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
   if ((s = device_info(&sms, &dstatus)) != MOE_OK) return s;
   if (!layer_dec_supported(T, d, I, E, k, W->has_shared ? 1 : 0, sms))
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
-                "moe_layer_decode needs 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024");
+                "moe_layer_decode needs 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, "
+                "k <= E <= 1024 and at most 32 units per CTA");
   if ((s = check_ws(ws, ws_bytes, layer_dec_ws_bytes(T, E))) != MOE_OK) return s;
   LayerDecArgs a;
   a.x = x;
