@@ -97,3 +97,30 @@ def test_workspace_sizes_monotone():
     assert B.moe_workspace_size(B.MOE_OP_LAYER, 8, 2048, 512, 10, 512) >= \
         B.moe_workspace_size(B.MOE_OP_FFN, 8, 2048, 512, 10, 512)
     assert B.moe_workspace_size(B.MOE_OP_ROUTE, -1, 2048, 512, 10, 512) == 0
+
+
+def test_pack_and_layer_decode_validation():
+    """Host-side checks of moe_pack_experts (the decode pack's shape rule) and of
+    moe_layer_decode (alignment, the decode pack), which run before any device call."""
+    L = B.lib()
+    INV, SHAPE = 1, 2
+    p = ctypes.c_void_p(0x10000)
+    # d = 256 is packable for the tensor-core scales but not for the decode pack
+    w = B._WeightsC(4, 256, 64, p.value, p.value, p.value, p.value, p.value, p.value)
+    assert L.moe_pack_experts(ctypes.byref(w), p, p, p, None) == SHAPE
+    assert L.moe_pack_experts(ctypes.byref(w), p, p, ctypes.c_void_p(0x10008), None) == INV
+    assert L.moe_pack_experts(ctypes.byref(w), None, p, None, None) == INV
+    # moe_layer_decode: weights without the decode pack, and a misaligned scale buffer
+    w5 = B._WeightsC(16, 512, 64, p.value, p.value, p.value, p.value, p.value, p.value)
+    ex = B._ExpertsC(w5, B._WeightsC(), 0)
+    args = [p, 4, None, p, None, ctypes.byref(ex), 2, p, p, p, p, p, p, p, p, p, p, p, 0, p, 1 << 20, None]
+    assert L.moe_layer_decode(*args) == SHAPE
+    assert b"decode pack" in L.moe_last_error()
+    args[8] = ctypes.c_void_p(0x10004)  # xq_scales
+    assert L.moe_layer_decode(*args) == INV
+
+
+def test_dec_pack_bytes_formula():
+    """The binding's decode-pack size is the header's E*I*d*27/16 bytes (18 KB blocks)."""
+    for E, d, I in [(1, 512, 64), (512, 2048, 512), (256, 4096, 2048), (8, 1024, 192)]:
+        assert B.dec_pack_bytes(E, d, I) == E * I * d * 27 // 16
