@@ -207,15 +207,15 @@ def moe_permute(topk_idx, E, counts, offsets, sorted_assign, assign_pos, ws, str
         _stream(stream)))
 
 
-def moe_pack_experts(w: ExpertWeights, stream=None, slices: bool = True):
+def moe_pack_experts(w: ExpertWeights, stream=None, decode_pack: bool = True):
     """Allocate and fill the derived layouts used by the tensor-core paths: re-tiled scales,
-    and (slices=True, d % 512 == 0) the decode pack: all weights again as the 18 KB blocks
+    and (decode_pack=True, d % 512 == 0) the decode pack: all weights again as the 18 KB blocks
     the decode kernel copies into shared memory."""
     if w.gu_sf_tiled is None:
         w.gu_sf_tiled = torch.empty_like(w.gu_scales)
     if w.dn_sf_tiled is None:
         w.dn_sf_tiled = torch.empty_like(w.dn_scales)
-    if slices and w.dec_pack is None and w.d % 512 == 0:
+    if decode_pack and w.dec_pack is None and w.d % 512 == 0:
         w.dec_pack = torch.empty(dec_pack_bytes(w.E, w.d, w.I), dtype=torch.uint8,
                                  device=w.gu_codes.device)
     s = w.struct()

@@ -41,7 +41,6 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
-#include "tmap.h"
 #include "trace.cuh"
 
 namespace moe {
