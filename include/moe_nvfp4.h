@@ -258,8 +258,9 @@ moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32
  *   Same arguments, outputs and results as moe_route, minus ws/ws_bytes. The scratch is one
  *   256 KiB array compiled into the library and held by every GPU that loads it until the
  *   process exits; calls whose scratch need (moe_workspace_size(MOE_OP_ROUTE, ...)) exceeds
- *   256 KiB return MOE_ERR_UNSUPPORTED_SHAPE. With T*k <= 4096 that allows T*E <= 65536
- *   (e.g. 64 tokens with 1024 experts, or 128 tokens with 512 experts).
+ *   256 KiB return MOE_ERR_UNSUPPORTED_SHAPE. With T*k <= 4096 the scratch is the T*E float32
+ *   router logits alone, so T*E <= 65536 fits (e.g. 64 tokens with 1024 experts, or 128
+ *   tokens with 512 experts); above 4096 assignments per-chunk histograms are added.
  *   It allocates nothing. The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress); make that first call before capturing any stream.
  *   All calls share the one array, which keeps the last call's contents (nothing in it needs

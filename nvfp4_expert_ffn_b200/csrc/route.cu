@@ -384,8 +384,11 @@ cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* cou
                     (const int32_t*)chunk_hist, sorted_assign, assign_pos);
 }
 
+// Per-chunk histograms of the three-kernel permutation; the single-CTA permutation of at
+// most kPermChunk assignments keeps its histogram in shared memory and needs none.
 size_t permute_ws_bytes(int64_t T, int k, int E) {
   const int64_t n = T * k;
+  if (n <= kPermChunk) return 0;
   const int64_t nchunk = (n + kPermChunk - 1) / kPermChunk;
   return (size_t)(nchunk * E * sizeof(int32_t));
 }

@@ -19,8 +19,9 @@
 
 namespace moe {
 
-// Largest scratch a call may need: the router logits (T*E float32, padded to 256 bytes)
-// plus, above 4096 assignments, the permutation's per-chunk histograms.
+// Scratch of one call: the router logits (T*E float32, padded to 256 bytes), plus the
+// permutation's per-chunk histograms when there are more than 4096 assignments (T*k).
+// With at most 4096 assignments the array holds up to 65536 logits: T*E <= 65536.
 constexpr size_t kNoAllocScratchBytes = 256 * 1024;
 
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];

@@ -124,3 +124,13 @@ def test_dec_pack_bytes_formula():
     """The binding's decode-pack size is the header's E*I*d*27/16 bytes (18 KB blocks)."""
     for E, d, I in [(1, 512, 64), (512, 2048, 512), (256, 4096, 2048), (8, 1024, 192)]:
         assert B.dec_pack_bytes(E, d, I) == E * I * d * 27 // 16
+
+
+def test_route_workspace_has_no_permutation_scratch_up_to_4096_assignments():
+    """The routing scratch is the T*E float32 logits (padded to 256 bytes); the per-chunk
+    histograms of the multi-kernel permutation are added only above 4096 assignments."""
+    E, d, k = 512, 2048, 10
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 128, d, E, k, 512) == 128 * E * 4
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 409, d, E, k, 512) == 409 * E * 4
+    # 410 tokens x 10 = 4100 assignments: two chunks of histograms
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 410, d, E, k, 512) == 410 * E * 4 + 2 * E * 4

@@ -74,3 +74,27 @@ def test_noalloc_rejects_sizes_above_its_array():
     with pytest.raises(B.MoeError) as err:
         B.moe_route_noalloc(x, Wr.cuda(), br.cuda(), cfg.k, *(o[n] for n in NAMES))
     assert err.value.status == 2 and "scratch" in str(err.value)
+
+
+def test_noalloc_boundary_of_its_array():
+    """128 tokens x 512 experts of float32 logits fill the 256 KiB array exactly (1280
+    assignments need no permutation scratch): accepted and equal to moe_route. One more
+    token needs more than the array holds and is rejected before anything is launched."""
+    cfg = synth.CONFIGS["decode"]
+    Wr, br = synth.make_router(0, cfg)
+    Wr, br = Wr.cuda(), br.cuda()
+    x = synth.make_x(0, cfg, 128, step=4).cuda()
+    want = _with_workspace(x, Wr, br, cfg.k)
+    got = _no_alloc(x, Wr, br, cfg.k)
+    torch.cuda.synchronize()
+    for n in NAMES:
+        a, b = got[n].cpu().numpy(), want[n].cpu().numpy()
+        if n == "topk_w":
+            np.testing.assert_allclose(a, b, rtol=2e-6, atol=1e-7)
+        else:
+            assert np.array_equal(a, b), n
+    x = synth.make_x(0, cfg, 129, step=5).cuda()
+    o = _outputs(129, cfg.k, cfg.E)
+    with pytest.raises(B.MoeError) as err:
+        B.moe_route_noalloc(x, Wr, br, cfg.k, *(o[n] for n in NAMES))
+    assert err.value.status == 2 and "scratch" in str(err.value)
