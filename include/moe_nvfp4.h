@@ -224,14 +224,17 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
  *   topk_w [T][k]; counts [E], offsets [E+1], sorted_assign [T*k], assign_pos [T*k];
  *   y_acc float32 [T][d] (the unrounded output); y_bf16 [T][d]; rms_renorm as moe_combine.
  *   ws: moe_workspace_size(MOE_OP_LAYER_DECODE, ...) bytes, zero-filled before the first
- *   call (it holds the arrival counter of the kernel's grid-wide barrier, which every call
- *   leaves at a multiple of the grid size; after a MOE_ERR_TIMEOUT from
- *   moe_get_device_status, zero it again).
+ *   call. It holds the arrival counter of the kernel's grid-wide barrier, which every call
+ *   leaves at a multiple of the grid size, and a mark that a CTA sets when it gives up at a
+ *   bounded wait (moe_get_device_status then reports MOE_ERR_TIMEOUT). A call that finds the
+ *   mark set computes nothing, writes no output and sets the device status to
+ *   MOE_ERR_WORKSPACE; zero the workspace again to recover.
  * Limits: 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024,
  * and at most 32 units per CTA in the worst case ((min(T*k, E) + shared) * I/64 units over
  * all SMs but one); otherwise MOE_ERR_UNSUPPORTED_SHAPE.
- * The kernel uses all SMs but one and waits at grid-wide barriers, so it must not share the
- * GPU with a kernel that occupies more than one SM until this one ends.
+ * The kernel uses all SMs but one and waits at grid-wide barriers. It is launched as a
+ * cooperative grid, so the launch fails (MOE_ERR_CUDA) rather than start when its CTAs cannot
+ * all be resident; while it runs, other kernels on the GPU get one SM.
  */
 moe_status moe_layer_decode(const uint16_t* x_bf16, int32_t T, const float* ts_in, const float* Wr,
                             const float* br, const moe_experts_t* W, int32_t k, uint8_t* xq_codes,
@@ -262,7 +265,8 @@ moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32
  *   router logits alone, so T*E <= 65536 fits (e.g. 64 tokens with 1024 experts, or 128
  *   tokens with 512 experts); above 4096 assignments per-chunk histograms are added.
  *   It allocates nothing. The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before capturing any stream.
+ *   (cudaGetSymbolAddress); make that first call before capturing any stream. The address is
+ *   kept for the life of the process, so no call may follow a cudaDeviceReset.
  *   All calls share the one array, which keeps the last call's contents (nothing in it needs
  *   to start at zero). Calls that overlap on the GPU - on different streams or from
  *   different host threads - race on it and give undefined results.
@@ -275,9 +279,18 @@ moe_status moe_route_noalloc(const uint16_t* x_bf16, int32_t T, int32_t d, const
 /* Bytes of workspace needed by one op (MOE_OP_*) for these sizes (MOE_OP_LAYER: max). */
 size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k, int32_t I);
 
-/* Synchronise `stream` and return the device status word (MOE_OK or MOE_ERR_TIMEOUT);
- * `clear` != 0 resets it afterwards. */
+/* Synchronise `stream` and return the device status word of the current device: MOE_OK,
+ * MOE_ERR_TIMEOUT (a bounded device-side wait ran out; the kernel stopped early and its
+ * outputs are not valid) or MOE_ERR_WORKSPACE (moe_layer_decode found its workspace marked
+ * by an earlier call that gave up). `clear` != 0 resets it afterwards. */
 moe_status moe_get_device_status(void* stream, int32_t clear, int32_t* status_out);
+
+/* How long a device-side wait (for a copy, a tensor-core result, another CTA) may last before
+ * the kernel gives up and reports MOE_ERR_TIMEOUT, for kernels launched on the current device
+ * from now on, including replays of captured graphs. Default 2 s; allowed 1 ms .. 60 s. A
+ * short limit can end a long call early: the waits of the PREFILL path last up to the length
+ * of the call. */
+moe_status moe_set_wait_limit_ns(uint64_t ns);
 
 /* Static description of a status code, and a per-thread detail of the last failure. */
 const char* moe_status_string(moe_status s);

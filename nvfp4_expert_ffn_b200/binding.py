@@ -22,6 +22,8 @@ MOE_OK = 0
 MOE_FFN_ACCUMULATE, MOE_FFN_PER_ASSIGN = 0, 1
 MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_CUDA_CORE = 0, 1, 2, 3
 MOE_OP_LAYER, MOE_OP_ROUTE, MOE_OP_QUANT, MOE_OP_FFN, MOE_OP_LAYER_DECODE = 0, 1, 2, 3, 4
+MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE = 4, 5
+DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
 
 # (name, restype, argtypes) of every C export; tests check the header declares the same set
 _P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
@@ -39,6 +41,7 @@ EXPORTS = {
                                 _P, _P, _I32, _P, _SZ, _P]),
     "moe_workspace_size": (_SZ, [_I32, _I64, _I32, _I32, _I32, _I32]),
     "moe_get_device_status": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
+    "moe_set_wait_limit_ns": (_I32, [ctypes.c_uint64]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_version": (_I32, []),
@@ -263,3 +266,7 @@ def moe_get_device_status(clear=True, stream=None) -> int:
                                                                  1 if clear else 0,
                                                                  ctypes.byref(out)))
     return out.value
+
+
+def moe_set_wait_limit_ns(ns: int) -> None:
+    _check("moe_set_wait_limit_ns", lib().moe_set_wait_limit_ns(int(ns)))

@@ -124,7 +124,7 @@ const char* moe_status_string(moe_status s) {
     case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
     case MOE_ERR_CUDA: return "CUDA error";
     case MOE_ERR_TIMEOUT: return "device wait timed out";
-    case MOE_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MOE_ERR_WORKSPACE: return "workspace too small, misaligned, or marked by a call that gave up";
   }
   return "unknown status";
 }
@@ -396,6 +396,16 @@ moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32
   if (s != MOE_OK) return s;
   cudaError_t e = launch_hist(counts, E, cum, rank_out, reset ? 1 : 0, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_hist launch");
+}
+
+moe_status moe_set_wait_limit_ns(uint64_t ns) {
+  if (ns < 1000000ull || ns > 60000000000ull)
+    return fail(MOE_ERR_INVALID_ARG, "wait limit must be between 1 ms and 60 s");
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = set_wait_limits((unsigned long long)ns);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_set_wait_limit_ns");
 }
 
 moe_status moe_get_device_status(void* stream, int32_t clear, int32_t* status_out) {

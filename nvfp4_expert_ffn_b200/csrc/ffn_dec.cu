@@ -221,6 +221,8 @@ bool ffn_dec_supported(int64_t T, int d, int I, int mode, int E, int k, int has_
 
 size_t ffn_dec_ws_bytes(int E) { return 256 + a256d((size_t)(E + 1) * 4) + a256d((size_t)(E + 1) * kDecMaxT * 4); }
 
+cudaError_t set_wait_limit_ffn_dec(unsigned long long ns) { return set_wait_limit_here(ns); }
+
 cudaError_t init_ffn_dec_attributes() {
   // the largest configuration; launches use at most this much
   return cudaFuncSetAttribute(ffn_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmemBudget);

@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) ffn_decode_fused_kernel(FfnA
               ok = 0;
               break;
             }
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > wait_limit_ns()) {
               s_abort = 1;
               atomicExch(c.status, kStatusTimeout);
               ok = 0;
@@ -505,6 +505,8 @@ cudaError_t launch_ffn_decode(const FfnArgs& a, int num_sms, int32_t* status, cu
   ffn_decode_fused_kernel<<<grid, kFusedThreads, smem, st>>>(a, c);
   return cudaGetLastError();
 }
+
+cudaError_t set_wait_limit_ffn_decode(unsigned long long ns) { return set_wait_limit_here(ns); }
 
 cudaError_t init_ffn_decode_attributes() {
   return cudaFuncSetAttribute(ffn_decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

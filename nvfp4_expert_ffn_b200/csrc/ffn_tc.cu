@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
               ok = 0;
               break;
             }
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > wait_limit_ns()) {
               s_abort = 1;
               atomicExch(p.status, kStatusTimeout);
               ok = 0;
@@ -672,6 +672,8 @@ size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I) {
 bool ffn_tc_supported(int d, int I) { return d % kStageK == 0 && I % kStageK == 0 && d <= 16384 && I <= 16384; }
 
 size_t ffn_tc_smem_bytes() { return (size_t)kTcStages * kStageBytes + (size_t)kEpiWarps * 2 * kEpiStageBytes + 1024; }
+
+cudaError_t set_wait_limit_ffn_tc(unsigned long long ns) { return set_wait_limit_here(ns); }
 
 cudaError_t init_ffn_tc_attributes() {
   return cudaFuncSetAttribute(tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ffn_tc_smem_bytes());

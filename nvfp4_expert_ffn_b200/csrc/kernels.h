@@ -33,6 +33,27 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// As launch_pdl, and cooperative: the launch fails instead of starting unless every CTA of
+// the grid can be resident at once (kernels that wait at grid-wide barriers).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  g_launch_count.fetch_add(1, std::memory_order_relaxed);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // per-thread detail string returned by moe_last_error()
 void set_last_error(const std::string& msg);
 
@@ -131,6 +152,19 @@ cudaError_t launch_pack_dec(const ExpertGroup& g, int E, int d, int I, const uin
 size_t dec_pack_bytes(int E, int d, int I);
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
                            int num_sms, cudaStream_t st);
+
+// the bounded-wait limit of each translation unit with device-side waits, on the current device
+cudaError_t set_wait_limit_ffn_decode(unsigned long long ns);
+cudaError_t set_wait_limit_ffn_tc(unsigned long long ns);
+cudaError_t set_wait_limit_ffn_dec(unsigned long long ns);
+cudaError_t set_wait_limit_layer_dec(unsigned long long ns);
+inline cudaError_t set_wait_limits(unsigned long long ns) {
+  cudaError_t e = set_wait_limit_ffn_decode(ns);
+  if (e == cudaSuccess) e = set_wait_limit_ffn_tc(ns);
+  if (e == cudaSuccess) e = set_wait_limit_ffn_dec(ns);
+  if (e == cudaSuccess) e = set_wait_limit_layer_dec(ns);
+  return e;
+}
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t init_route_attributes();

@@ -22,7 +22,12 @@
 //   barrier
 //   phase 4  CTA t < T converts row t of y_acc to bf16 (optionally RMS-renormalised).
 // The grid barrier counts arrivals in a workspace word that must be zero before the first
-// call; every call leaves it at a multiple of the grid size.
+// call; every call leaves it at a multiple of the grid size. A CTA that gives up at a
+// bounded wait marks the workspace (a second word), since the counter may then be left
+// between multiples; later calls on a marked workspace do nothing but report
+// MOE_ERR_WORKSPACE until the caller zeroes it. The launch is cooperative: it fails rather
+// than start a grid whose CTAs cannot all be resident, so the barrier cannot wait on a CTA
+// that has not started.
 #include <cuda_bf16.h>
 
 #include "dec_core.cuh"
@@ -60,6 +65,7 @@ struct LayerArgs {
   // workspace
   float* logits;       // [T][E]
   unsigned long long* sync;  // arrival counter of the grid barrier (zero before the first call)
+  unsigned int* poison;      // nonzero once a call on this workspace gave up at a bounded wait
   int32_t* status;
 };
 
@@ -96,7 +102,7 @@ MOE_DEV bool grid_wait(unsigned long long* count, unsigned long long target, vol
       if (c >= target) break;
       if (*abort) {
         ok = 0;
-      } else if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      } else if (globaltimer_ns() - t0 > wait_limit_ns()) {
         *abort = 1;
         atomicExch(status, kStatusTimeout);
         ok = 0;
@@ -183,8 +189,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   }
   MOE_PDL_PROLOGUE();
   RT_TRACE(g_layer_trace, 0, 1);
+  // a workspace marked by an earlier call that gave up: report it and do nothing (the mark is
+  // written by the predecessor kernels this one has just waited for)
+  __shared__ int s_live;
+  if (threadIdx.x == 0) {
+    s_live = 1;
+    if (*reinterpret_cast<volatile unsigned int*>(p.poison) != 0u) {
+      s_live = 0;
+      *abort = 1;
+      atomicExch(p.status, kStatusWorkspace);
+    }
+  }
+  __syncthreads();
+  const bool live = s_live != 0;
+  float ts = 1.0f;
 
   // ---------------------------------------------------------------- phase 1
+  if (live) {
   // x -> shared memory (every load of a round in flight before the stores)
   {
     const int nx = T * d / 8;
@@ -208,7 +229,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   RT_TRACE(g_layer_trace, 0, 2);
   // NVFP4 tensor scale: amax / (6 * 448) over all T tokens (every CTA computes the same), or
   // the static scale
-  float ts;
   if (p.ts_in) {
     ts = *p.ts_in;
   } else {
@@ -266,7 +286,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   // reduce-scatter leaves lane l with the warp's sum of (row l / 8, token l % 8), and warp 0
   // adds the warps' sums
   if (nrows > 0) {
-    mbar_wait(&s_wbar, 0, abort, p.status);
+    {
+      volatile int no_abort = 0;  // the rows' copies land before anything else happens
+      if (!mbar_wait(&s_wbar, 0, &no_abort, p.status)) *abort = 1;
+    }
     RT_TRACE(g_layer_trace, 2, 3);
     for (int r0 = 0; r0 < nrows; r0 += 4) {
       float v[32];
@@ -325,6 +348,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   if (b == 0) {
     float4* y4 = reinterpret_cast<float4*>(p.y_acc);
     for (int i = threadIdx.x; i < T * d / 4; i += blockDim.x) y4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  } else if (nrows > 0) {
+    // marked workspace: only wait for the router rows' copies, which must land before exit
+    volatile int no_abort = 0;
+    mbar_wait(&s_wbar, 0, &no_abort, p.status);
   }
   RT_TRACE(g_layer_trace, 0, 3);
   bool ok = grid_sync(p.sync, abort, p.status);
@@ -540,6 +568,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
       reinterpret_cast<uint32_t*>(p.y + (size_t)t * d)[n2] = lo | (hi << 16);
     }
   }
+  // a CTA that gave up (or found the workspace marked) marks it for the calls that follow
+  if (threadIdx.x == 0 && *abort) atomicExch(p.poison, 1u);
   RT_TRACE(g_layer_trace, 1, 1);
 }
 
@@ -561,6 +591,8 @@ bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, 
   const int64_t slots = (T * k < E ? T * k : E) + has_shared;
   return (slots * (I / 64) + G - 1) / G <= kDecMaxUnits;
 }
+
+cudaError_t set_wait_limit_layer_dec(unsigned long long ns) { return set_wait_limit_here(ns); }
 
 cudaError_t init_layer_dec_attributes() {
   return cudaFuncSetAttribute(layer_dec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmemBudget);
@@ -592,9 +624,11 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
   p.y_acc = a.y_acc;
   p.y = a.y;
   p.sync = reinterpret_cast<unsigned long long*>(w);
+  p.poison = reinterpret_cast<unsigned int*>(w + 8);
   p.logits = reinterpret_cast<float*>(w + 256);
   p.status = status;
-  return launch_pdl(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st, p);
+  return launch_pdl_coop(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st,
+                         p);
 }
 
 }  // namespace moe

@@ -13,9 +13,10 @@
 
 namespace moe {
 
-// float -> unsigned key with the same order
+// float -> unsigned key with the same order; -0.0 and +0.0 get the same key (they are equal
+// logits, so the lower expert id goes first)
 MOE_DEV uint32_t ordered_key(float v) {
-  const uint32_t u = __float_as_uint(v);
+  const uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -12,7 +12,17 @@ namespace moe {
 
 constexpr int32_t kStatusTimeout = 4;                   // MOE_ERR_TIMEOUT
 constexpr int32_t kStatusUnsupported = 2;               // MOE_ERR_UNSUPPORTED_SHAPE
-constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;  // 2 s
+constexpr int32_t kStatusWorkspace = 5;                 // MOE_ERR_WORKSPACE
+constexpr unsigned long long kDefaultWaitLimitNs = 2000ull * 1000ull * 1000ull;  // 2 s
+
+// How long a device-side wait may last before the kernel gives up (moe_set_wait_limit_ns).
+// Each translation unit that includes this header has its own copy of the word on each
+// device; set_wait_limit_here() writes this unit's copy on the current device.
+static __device__ unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
+static inline cudaError_t set_wait_limit_here(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
 
 MOE_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -21,6 +31,8 @@ MOE_DEV uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
+
+MOE_DEV uint64_t wait_limit_ns() { return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns); }
 
 MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
@@ -63,15 +75,15 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete. Gives up after kWaitLimitNs (or as
+// Wait for the phase with the given parity to complete. Gives up after wait_limit_ns() (or as
 // soon as *abort is set by another thread): records MOE_ERR_TIMEOUT in *status, sets
 // *abort, and returns false.
 MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  const uint64_t t0 = globaltimer_ns(), limit = wait_limit_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit) {
       *abort = 1;
       if (status) atomicExch(status, kStatusTimeout);
       return false;

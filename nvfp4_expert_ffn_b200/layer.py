@@ -77,6 +77,7 @@ class MoeLayer:
         self.path = B.MOE_PATH_AUTO
         self._side = torch.cuda.Stream(device=dev)
         self._ev = [torch.cuda.Event() for _ in range(4)]
+        self._hist_pending = False  # the last call's histogram may still read self.counts
         # calls of at most 8 tokens go through the one-kernel decode layer when the shapes allow;
         # its workspace holds a barrier counter and must start zeroed
         can_fuse = (d % 512 == 0 and d <= 4096 and I % 64 == 0 and k <= 32 and E <= 1024
@@ -98,6 +99,9 @@ class MoeLayer:
         assert T <= self.T_max
         main = torch.cuda.current_stream() if stream is None else stream
         side, ev = self._side, self._ev
+        if self._hist_pending:
+            main.wait_event(ev[3])  # this call rewrites the counts the last histogram reads
+        self._hist_pending = not join
         if self.fused and T <= 8:
             B.moe_layer_decode(x, self.static_ts, self.Wr, self.br, self.experts, k,
                                self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
@@ -135,34 +139,53 @@ class MoeLayer:
         return self.y[:T]
 
     def join(self, stream=None) -> None:
-        """Make `stream` (default: current) wait for this layer's side-stream work."""
+        """Make `stream` (default: current) wait for this layer's side-stream work; later
+        calls on that stream need not wait for it again."""
         (torch.cuda.current_stream() if stream is None else stream).wait_event(self._ev[3])
+        self._hist_pending = False
 
-    def graphed(self, T: int) -> "GraphedMoeLayer":
-        """A replayable CUDA graph of forward() for a fixed token count (decode loops)."""
-        return GraphedMoeLayer(self, T)
+    def graphed(self, T: int, n_slots: int = 1, stream=None) -> "GraphedMoeLayer":
+        """A replayable CUDA graph of forward() with its host copies, for a fixed token count."""
+        return GraphedMoeLayer(self, T, n_slots=n_slots, stream=stream)
 
 
 class GraphedMoeLayer:
-    """forward() of one layer captured once as a CUDA graph; step() copies a pinned host
-    batch in, replays the graph and copies the result back (all on one stream)."""
+    """forward() of one layer for a fixed token count, captured once as a CUDA graph together
+    with its host copies: each replay copies one pinned host input slot to the device, runs
+    the layer and copies y back to a pinned host buffer - one launch per step.
 
-    def __init__(self, layer: MoeLayer, T: int, rms_renorm: bool = False):
+    Write a step's input (bf16 bits [T][d]) into ``x_host[slot]`` before ``run(slot)``, and
+    read ``y_host`` after synchronising ``stream``. All replays go to ``stream``."""
+
+    def __init__(self, layer: MoeLayer, T: int, rms_renorm: bool = False, n_slots: int = 1,
+                 stream: Optional[torch.cuda.Stream] = None):
         self.layer, self.T = layer, T
         dev = layer.xq_codes.device
         self.x = torch.zeros(T, layer.d, dtype=torch.int16, device=dev)
-        self.stream = torch.cuda.Stream(device=dev)
+        self.x_host = [torch.zeros(T, layer.d, dtype=torch.int16).pin_memory() for _ in range(n_slots)]
+        self.y_host = torch.zeros(T, layer.d, dtype=torch.int16).pin_memory()
+        self.stream = stream if stream is not None else torch.cuda.Stream(device=dev)
         with torch.cuda.stream(self.stream):
             layer.forward(self.x, rms_renorm)  # first calls do per-device set-up
         self.stream.synchronize()
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph, stream=self.stream):
-            self.y = layer.forward(self.x, rms_renorm)
+        self.graphs = []
+        for slot in range(n_slots):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self.x.copy_(self.x_host[slot], non_blocking=True)
+                y = layer.forward(self.x, rms_renorm)
+                self.y_host.copy_(y, non_blocking=True)
+            self.graphs.append(g)
+
+    def run(self, slot: int = 0) -> None:
+        """Asynchronous on self.stream: x_host[slot] -> device, the layer, y -> y_host."""
+        self.graphs[slot].replay()
 
     def step(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
-        """x_host, y_host: pinned host tensors [T][d] of bf16 bits. Asynchronous on
-        self.stream; synchronise (or read y_host after self.stream.synchronize())."""
-        with torch.cuda.stream(self.stream):
-            self.x.copy_(x_host, non_blocking=True)
-            self.graph.replay()
-            y_host.copy_(self.y, non_blocking=True)
+        """Copy a host batch into slot 0 (synchronising the stream first, since the last
+        replay may still be reading it), run, and copy y_host out after the replay ends."""
+        self.stream.synchronize()
+        self.x_host[0].copy_(x_host)
+        self.run(0)
+        self.stream.synchronize()
+        y_host.copy_(self.y_host)

@@ -11,6 +11,7 @@ import torch
 
 from oracle import moe as omoe
 from oracle import nvfp4 as onv
+from oracle.weights import OracleWeights, expert_from_bf16  # noqa: F401
 from nvfp4_expert_ffn_b200 import binding as B
 from nvfp4_expert_ffn_b200 import synth
 
@@ -45,9 +46,7 @@ def assert_close_layer(y_gpu, y_ref, what=""):
     return rel, mabs / rms
 
 
-def oracle_expert_from_bf16(g, u, dn) -> omoe.Expert:
-    return omoe.Expert.from_f32(bits_to_f32(g.cpu().numpy()), bits_to_f32(u.cpu().numpy()),
-                                bits_to_f32(dn.cpu().numpy()))
+oracle_expert_from_bf16 = expert_from_bf16
 
 
 def weights_to_gpu(experts, device="cuda", pack=False) -> B.ExpertWeights:
@@ -64,31 +63,6 @@ def weights_to_gpu(experts, device="cuda", pack=False) -> B.ExpertWeights:
     if pack:
         B.moe_pack_experts(w)
     return w
-
-
-class OracleWeights:
-    """Lazily quantised oracle experts of a synth layer (only the experts a test touches)."""
-
-    def __init__(self, seed, cfg, layer=0):
-        self.seed, self.cfg, self.layer = seed, cfg, layer
-        self._cache = {}
-        self._shared = None
-
-    def __getitem__(self, e) -> omoe.Expert:
-        if e not in self._cache:
-            self._cache[e] = oracle_expert_from_bf16(
-                *synth.make_expert_weights_bf16(self.seed, self.cfg, e, self.layer))
-        return self._cache[e]
-
-    @property
-    def shared(self) -> omoe.Expert:
-        if self._shared is None:
-            self._shared = oracle_expert_from_bf16(
-                *synth.make_expert_weights_bf16(self.seed, self.cfg, 0, self.layer, shared=True))
-        return self._shared
-
-    def __len__(self):
-        return self.cfg.E
 
 
 def topk_margins(logits, k) -> np.ndarray:

@@ -69,7 +69,7 @@ def test_host_validation_without_gpu():
     # hist: E out of range
     assert L.moe_expert_hist(p, 0, p, None, 0, None) == SHAPE
     assert b"E must be" in L.moe_last_error()
-    assert L.moe_status_string(5) == b"workspace too small or misaligned"
+    assert L.moe_status_string(5) == b"workspace too small, misaligned, or marked by a call that gave up"
 
 
 def test_ffn_weight_validation():
@@ -134,3 +134,11 @@ def test_route_workspace_has_no_permutation_scratch_up_to_4096_assignments():
     assert B.moe_workspace_size(B.MOE_OP_ROUTE, 409, d, E, k, 512) == 409 * E * 4
     # 410 tokens x 10 = 4100 assignments: two chunks of histograms
     assert B.moe_workspace_size(B.MOE_OP_ROUTE, 410, d, E, k, 512) == 410 * E * 4 + 2 * E * 4
+
+
+def test_wait_limit_rejects_out_of_range_without_gpu():
+    """moe_set_wait_limit_ns checks its range on the host before any device call."""
+    L = B.lib()
+    assert L.moe_set_wait_limit_ns(999_999) == 1
+    assert L.moe_set_wait_limit_ns(60_000_000_001) == 1
+    assert b"wait limit" in L.moe_last_error()

@@ -9,8 +9,8 @@ from nvfp4_expert_ffn_b200 import binding as B
 from nvfp4_expert_ffn_b200 import layer as L
 from nvfp4_expert_ffn_b200 import synth
 
-from helpers import (OracleWeights, assert_close_layer, bits_to_f32, compare_topk,
-                     oracle_expert_from_bf16, weights_to_gpu)
+from helpers import (OracleWeights, assert_close_layer, bits_to_f32, check_permutation_valid,
+                     compare_topk, oracle_expert_from_bf16, weights_to_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +40,10 @@ def test_layer_matches_oracle(cfg_name, T, fused):
     assert_close_layer(bits_to_f32(y.cpu().numpy())[keep], ref["y"][keep], cfg_name)
     assert np.array_equal(lay.xq_codes[:T].cpu().numpy(), ref["x_codes"])
     assert np.array_equal(lay.xq_scales[:T].cpu().numpy(), ref["x_scales"])
+    # whatever the tie excuses, the permutation is a stable counting sort of the GPU's own top-k
+    check_permutation_valid(lay.topk_idx[:T].cpu().numpy(), lay.counts.cpu().numpy(),
+                            lay.offsets.cpu().numpy(), lay.sorted_assign[:T * cfg.k].cpu().numpy(),
+                            lay.assign_pos[:T * cfg.k].cpu().numpy(), cfg.E)
     if not excused:
         assert np.array_equal(lay.counts.cpu().numpy(), ref["counts"])
         assert np.array_equal(lay.offsets.cpu().numpy(), ref["offsets"])
@@ -106,6 +110,23 @@ def test_graphed_layer_step_matches_forward():
         torch.cuda.synchronize()
         assert torch.equal(got, want) or np.allclose(
             bits_to_f32(got.numpy()), bits_to_f32(want.numpy()), rtol=1e-2, atol=1e-3)
+
+
+def test_graphed_layer_slots_copy_in_and_out_inside_the_graph():
+    """run(slot) replays one graph that copies pinned x_host[slot] in, runs the layer and
+    copies y out: each slot's result equals an eager forward of the same input."""
+    cfg, lay, Wr, br = _layer("decode", T_max=8)
+    runner = lay.graphed(4, n_slots=3)
+    xs = [synth.make_x(6, cfg, 4, step=s) for s in range(3)]
+    for s in range(3):
+        runner.x_host[s].copy_(xs[s])
+    for s in (2, 0, 1):
+        runner.run(s)
+        runner.stream.synchronize()
+        got = runner.y_host.clone()
+        want = lay.forward(xs[s].cuda()).cpu()
+        torch.cuda.synchronize()
+        assert np.allclose(bits_to_f32(got.numpy()), bits_to_f32(want.numpy()), rtol=1e-2, atol=1e-3)
 
 
 def test_fused_decode_layer_repeated_calls():

@@ -9,7 +9,7 @@ candidates are gathered one per lane and each is ranked against the others (equa
 lower id); with more candidates the kernel falls back to k rounds of a warp arg-max, which is
 the sorted order by definition. This model follows those steps on the same float32 bit keys,
 so a wrong threshold, a candidate lost or a wrong tie rule shows up as a difference from the
-oracle. (Keys order -0.0 below +0.0; the inputs here hold no signed zeros.)
+oracle. Both zeros map to the key of +0.0, so logits of -0.0 and +0.0 tie like equal values.
 """
 import numpy as np
 import pytest
@@ -20,7 +20,9 @@ pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
 
 
 def _keys(row_f32):
-    u = row_f32.astype(np.float32).view(np.uint32).astype(np.uint64)
+    r = row_f32.astype(np.float32)
+    r = np.where(r == 0.0, np.float32(0.0), r)  # -0.0 -> +0.0
+    u = r.view(np.uint32).astype(np.uint64)
     neg = (u >> 31) == 1
     return np.where(neg, (~u) & 0xFFFFFFFF, u | 0x80000000).astype(np.uint64)
 
@@ -110,3 +112,16 @@ def test_threshold_selection_small_E():
         for k in range(1, E + 1, max(1, E // 4)):
             rows = rng.standard_normal((4, E)).astype(np.float32)
             assert _check_rows(rows, k) == 0
+
+
+def test_threshold_selection_signed_zeros():
+    """Logits of exactly -0.0 and +0.0 around the k-th place are equal values: the oracle
+    takes the lower expert ids first, and so do the kernels' keys (both zeros share one key)."""
+    E, k = 64, 8
+    rng = np.random.default_rng(21)
+    rows = -np.abs(rng.standard_normal((16, E))).astype(np.float32) - 1.0
+    for t in range(rows.shape[0]):
+        zeros = rng.choice(E, 12, replace=False)
+        rows[t, zeros] = np.where(rng.random(12) < 0.5, np.float32(-0.0), np.float32(0.0))
+        rows[t, rng.choice(np.setdiff1d(np.arange(E), zeros), 3, replace=False)] = 1.0
+    assert _check_rows(rows, k) == 0
