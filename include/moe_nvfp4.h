@@ -106,7 +106,10 @@ typedef struct moe_experts {
 
 /*
  * nvfp4_quantize_act - NVFP4 quantisation of a bf16 matrix (activations, or weights at
- * load time). Steps: amax over the whole matrix (unless ts_in is given), then per 16-block
+ * load time): step A4 of the layer. Source: "Basalt" project page, "All the numbers", list
+ * "Engines: commit, and what is not NVIDIA's weights" (routed experts are NVIDIA's NVFP4;
+ * the llama.cpp row keeps NVIDIA's activation input_scale, the static scale ts_in here).
+ * Steps: amax over the whole matrix (unless ts_in is given), then per 16-block
  *   sb = (amax_b / 6) / ts; s = E4M3(sb); q_i = E2M1(x_i / (E4M3value(s) * ts)).
  *   x_bf16  [rows][cols] device; cols % 16 == 0
  *   ts_in   device float32[1] static tensor scale, or NULL for the dynamic amax/2688
@@ -120,11 +123,18 @@ moe_status nvfp4_quantize_act(const uint16_t* x_bf16, int64_t rows, int32_t cols
 
 /*
  * moe_route - router (A1), softmax/top-k/renormalisation (A2) and permutation (A3).
+ * Source: "What Basalt changes in a Blackwell local inference stack", section "Experts can
+ * move without becoming free" (each token selects a subset of the experts) and the "Basalt"
+ * project page, section "Expert tiers" (each token uses only a few experts).
  *   x_bf16 [T][d]; Wr float32 [E][d]; br float32 [E] or NULL.
  *   topk_idx int32 [T][k] (descending logit), topk_w float32 [T][k],
  *   counts int32 [E], offsets int32 [E+1], sorted_assign int32 [T*k] (assignment ids
  *   a = t*k + j grouped by expert, increasing a within an expert), assign_pos int32 [T*k]
  *   (inverse of sorted_assign). 1 <= k <= 32, k <= E <= 1024, d % 16 == 0.
+ * From 256 tokens on, with E % 128 == 0 and d % 64 == 0, the logits come from a bf16-split
+ * tensor-core product and every expert near each token's k-th logit is recomputed exactly,
+ * so the top-k is that of the float32 logits; the workspace then also holds the split
+ * router matrix (moe_workspace_size accounts for it).
  */
 moe_status moe_route(const uint16_t* x_bf16, int32_t T, int32_t d, const float* Wr,
                      const float* br, int32_t E, int32_t k, int32_t* topk_idx,
@@ -134,7 +144,8 @@ moe_status moe_route(const uint16_t* x_bf16, int32_t T, int32_t d, const float* 
 
 /*
  * moe_permute - the permutation step (A3) alone, from given top-k indices: a stable
- * counting sort of the T*k assignments by expert, with the per-expert histogram.
+ * counting sort of the T*k assignments by expert, with the per-expert histogram (the
+ * routing counts of "Basalt" project page, section "Expert tiers").
  * Same outputs and limits as moe_route.
  */
 moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
@@ -143,7 +154,9 @@ moe_status moe_permute(const int32_t* topk_idx, int32_t T, int32_t k, int32_t E,
 
 /*
  * moe_pack_experts - derived layouts of an expert group for the tensor-core paths, written
- * once per weight load into caller-owned buffers (set them in W afterwards):
+ * once per weight load into caller-owned buffers (set them in W afterwards). The pages have
+ * no counterpart (they keep NVIDIA's NVFP4 bytes unchanged, "Basalt" project page,
+ * "Engines" list); these are the same bytes rearranged for the tensor core:
  *   gu_sf_tiled (E*2I*d/16 bytes), dn_sf_tiled (E*d*I/16 bytes): the E4M3 scale bytes in
  *     512-byte atoms of 128 weight rows x 4 scale blocks, the layout the tensor core reads
  *     its scales in (gate/up atoms [E][I/64][d/64], atom rows 0-63 gate, 64-127 up; down
@@ -166,7 +179,10 @@ moe_status moe_pack_experts(const moe_expert_weights_t* W, uint8_t* gu_sf_tiled,
 
 /*
  * moe_expert_ffn - expert SwiGLU FFN for all routed assignments (A5-A7) and the shared
- * expert (A8).
+ * expert (A8). Source: "What Basalt changes in a Blackwell local inference stack", section
+ * "Experts can move without becoming free" (only the selected experts run for a token) and
+ * the "Basalt" project page, "Engines" list (the experts' weights are NVFP4) and section
+ * "Expert tiers" (every kernel, FP4 included, written for Blackwell).
  *   xq_codes [T][d/2], xq_scales [T][d/16], xq_ts float32[1]: the NVFP4 activation.
  *   offsets [E+1], sorted_assign [T*k], topk_w [T][k]: from moe_route / moe_permute.
  *   mode MOE_FFN_ACCUMULATE: out = float32 [T][d], set by the call to
@@ -195,7 +211,9 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales,
                           float* shared_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * moe_combine - weighted combine (A9) and cast to bf16.
+ * moe_combine - weighted combine (A9) and cast to bf16: a token's output is the sum of its
+ * selected experts' outputs, weighted by the routing weights ("What Basalt changes in a
+ * Blackwell local inference stack", section "Experts can move without becoming free").
  *   mode MOE_FFN_ACCUMULATE: expert_out = y_acc float32 [T][d]; y = bf16(y_acc).
  *   mode MOE_FFN_PER_ASSIGN: y[t] = sum_j topk_w[t,j] * expert_out[assign_pos[t*k+j]]
  *        + shared_out[t] (shared_out may be NULL).
@@ -244,7 +262,10 @@ moe_status moe_layer_decode(const uint16_t* x_bf16, int32_t T, const float* ts_i
                             void* ws, size_t ws_bytes, void* stream);
 
 /*
- * moe_expert_hist - cumulative routing counts and hot-to-cold ranking (A10).
+ * moe_expert_hist - cumulative routing counts and hot-to-cold ranking (A10). Source:
+ * "Basalt" project page, section "Expert tiers" (the busiest experts are kept in VRAM, and
+ * the tiers follow the conversation as it shifts) and its FAQ "Can it use a second GPU or
+ * system RAM?".
  *   counts int32 [E] (this call's histogram), cum int64 [E] in/out (cum += counts, or
  *   cum = counts when reset != 0), rank_out int32 [E] or NULL: expert ids from most to
  *   least routed, equal counts by lower id. E <= 4096.

@@ -217,10 +217,11 @@ moe_status moe_route(const uint16_t* x, int32_t T, int32_t d, const float* Wr, c
     if (s != MOE_OK) return s;
   }
   int sms = 0;
-  s = device_info(&sms);
+  int32_t* dstatus = nullptr;
+  s = device_info(&sms, &dstatus);
   if (s != MOE_OK) return s;
   cudaError_t e = launch_route(x, T, d, Wr, br, E, k, topk_idx, topk_w, counts, offsets,
-                               sorted_assign, assign_pos, ws, sms, (cudaStream_t)stream);
+                               sorted_assign, assign_pos, ws, sms, dstatus, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_route launch");
 }
 

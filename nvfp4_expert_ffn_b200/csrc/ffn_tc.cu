@@ -160,9 +160,11 @@ __global__ void __launch_bounds__(256) tc_row_gather_kernel(TcParams p) {
       wgt = p.topk_w[a];
       slot = q;
     }
-    const uint4* csrc = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
-    uint4* cdst = reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
-    for (int c = lane; c < d / 32; c += 32) cdst[c] = __ldg(csrc + c);
+    if (p.a1) {
+      const uint4* csrc = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
+      uint4* cdst = reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
+      for (int c = lane; c < d / 32; c += 32) cdst[c] = __ldg(csrc + c);
+    }
     const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
     for (int kc = lane; kc < d / 64; kc += 32)
       *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (r % 32) * 16 + (r / 32) * 4) =
@@ -627,6 +629,354 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
   if (threadIdx.x == 0) TC_TRACE_AT(g_tc_trace, kEvExit, 0);
 }
 
+// ---------------------------------------------------------------- 4. m-tile kernel
+// One job = the whole FFN of one m-tile (up to 128 rows of one expert), run by one CTA:
+//   gate/up: I/128 tiles of N = 256 weight rows (gate and up rows of two 64-row slices of I,
+//            in the order the scale atoms hold them), K = d; SwiGLU and the NVFP4
+//            quantisation of h in the epilogue, h written into this CTA's shared memory in
+//            the layout the down GEMM reads as its A operand;
+//   down:    d/256 tiles of N = 256 output rows, K = I, A = that h tile; the epilogue adds
+//            w * o into y with bulk reductions (or stores o).
+// The activation scale atoms of the m-tile (K = d) and then those of h (K = I) stay in TMEM
+// for all of the job's tiles, so a K = 64 step needs only the two weight scale copies next to
+// its N = 256 MMA (each tcgen05.cp takes the tensor pipe about as long as a 128-column MMA).
+// One N = 256 accumulator (TMEM has no room for a second one beside the scales): the
+// epilogue takes its columns into registers first and releases it before its own math.
+constexpr int kMtN = 256;
+constexpr int kMtStages = 2;
+constexpr int kMtABytes = kTileM * kStageK / 2;      // 16 KB: gathered activation rows
+constexpr int kMtBBytes = kMtN * kStageK / 2;        // 32 KB: weight rows
+constexpr int kMtSfbBytes = 8 * kAtom;               // 4 KB: two atoms per K = 64 step
+constexpr int kMtStageBytes = kMtABytes + kMtBBytes + kMtSfbBytes;
+constexpr int kMtColSfa = 256, kMtColSfb = 384;      // TMEM columns (accumulator at 0)
+constexpr int kMtMaxD = 2048, kMtMaxI = 768;
+constexpr uint32_t kMtIdesc = idesc_mxf4nvf4(kTileM, kMtN);
+
+__host__ __device__ inline size_t mt_h_bytes(int I) { return (size_t)(I / kStageK) * kMtABytes; }
+__host__ __device__ inline size_t mt_smem_bytes(int d, int I) {
+  return (size_t)kMtStages * kMtStageBytes + mt_h_bytes(I) + (size_t)(I / 64) * kAtom + (size_t)(d / 64) * kAtom +
+         (size_t)kEpiWarps * kEpiStageBytes + 1024;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
+  MOE_PDL_PROLOGUE();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t full[kMtStages], empty[kMtStages], acc_full, acc_empty, sfa_full, sfa_empty, h_ready,
+      final_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+  __shared__ int s_epi_go[2];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = p.d, I = p.I;
+  const int nt1 = I / 128, nt2 = d / kMtN;      // tiles per job
+  const int nks1 = d / kStageK, nks2 = I / kStageK;
+  uint8_t* const ring = smem;
+  uint8_t* const htile = smem + (size_t)kMtStages * kMtStageBytes;   // [I/256][128 rows][128 B]
+  uint8_t* const hsf = htile + mt_h_bytes(I);                         // [I/64][512]
+  uint8_t* const xsf = hsf + (size_t)(I / 64) * kAtom;                // [d/64][512]
+  float* const ystage = reinterpret_cast<float*>(xsf + (size_t)(d / 64) * kAtom);
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kMtStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    mbar_init(&acc_full, 1);
+    mbar_init(&acc_empty, kEpiWarps);
+    mbar_init(&sfa_full, 1);
+    mbar_init(&sfa_empty, 1);
+    mbar_init(&h_ready, 1);
+    mbar_init(&final_bar, 1);
+    fence_barrier_init();
+    s_abort = 0;
+    prefetch_tensormap(&maps.xg);
+    prefetch_tensormap(&maps.b1);
+    prefetch_tensormap(&maps.b2);
+  }
+  if (warp == 1) tmem_alloc(&s_tmem, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int n_m = *p.n_mtiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    uint32_t it = 0, jc = 0;
+    bool alive = true;
+    auto wait_empty = [&](uint32_t itx) -> bool {
+      int ok = 1;
+      if (lane == 0)
+        ok = mbar_wait(&empty[itx % kMtStages], ((itx / kMtStages) & 1) ^ 1, &s_abort, p.status) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+    for (int m = blockIdx.x; m < n_m && alive; m += gridDim.x, ++jc) {
+      const int e = p.mt_expert[m];
+      const bool sh = (e == p.E);
+      const int eloc = sh ? 0 : e;
+      const ExpertGroup& G = sh ? p.shared : p.routed;
+      const int valid = p.mt_valid[m];
+      const int ngather = (valid + 3) / 4;
+      // the 4 rows this lane gathers (padding rows of a group repeat the m-tile's first row)
+      int rowtok[4];
+      const int tok0 = p.row_token[(size_t)m * kTileM];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        rowtok[i] = r < valid ? p.row_token[(size_t)m * kTileM + r] : tok0;
+      }
+      // the m-tile's activation scale atoms (pre-gathered) for the whole of K = d
+      if (lane == 0) {
+        if (!mbar_wait(&sfa_empty, (jc & 1) ^ 1, &s_abort, p.status)) alive = false;
+        else {
+          mbar_arrive_expect_tx(&sfa_full, (uint32_t)(d / 64) * kAtom);
+          bulk_g2s(xsf, p.sfa1 + (size_t)m * (d / 64) * kAtom, (uint32_t)(d / 64) * kAtom, &sfa_full);
+        }
+      }
+      alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
+      // gate/up stages: activation rows by gather4, two 64-row gate+up boxes, their scales
+      for (int j = 0; j < nt1 && alive; ++j) {
+        for (int ks = 0; ks < nks1; ++ks, ++it) {
+          const uint32_t st = it % kMtStages;
+          if (!wait_empty(it)) {
+            alive = false;
+            break;
+          }
+          uint8_t* sb = ring + (size_t)st * kMtStageBytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[st], (uint32_t)(ngather * 512 + kMtBBytes + kMtSfbBytes));
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              tma_load_4d(sb + kMtABytes + hh * (kMtBBytes / 2), sh ? &maps.b1s : &maps.b1, &full[st], ks * 128,
+                          64 * (2 * j + hh), 0, eloc);
+              bulk_g2s(sb + kMtABytes + kMtBBytes + hh * (kMtSfbBytes / 2),
+                       G.gu_sf_tiled + (((size_t)eloc * (I / 64) + 2 * j + hh) * (d / 64) + 4 * ks) * kAtom,
+                       kMtSfbBytes / 2, &full[st]);
+            }
+          }
+          __syncwarp();
+          if (lane < ngather)
+            tma_gather4(sb + 4 * lane * 128, &maps.xg, &full[st], ks * 128, rowtok[0], rowtok[1], rowtok[2],
+                        rowtok[3]);
+        }
+      }
+      // down stages: two 128-row boxes of output rows and their scales
+      for (int n = 0; n < nt2 && alive; ++n) {
+        for (int ks = 0; ks < nks2; ++ks, ++it) {
+          const uint32_t st = it % kMtStages;
+          if (!wait_empty(it)) {
+            alive = false;
+            break;
+          }
+          uint8_t* sb = ring + (size_t)st * kMtStageBytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[st], (uint32_t)(kMtBBytes + kMtSfbBytes));
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              tma_load_3d(sb + kMtABytes + hh * (kMtBBytes / 2), sh ? &maps.b2s : &maps.b2, &full[st], ks * 128,
+                          kMtN * n + 128 * hh, eloc);
+              bulk_g2s(sb + kMtABytes + kMtBBytes + hh * (kMtSfbBytes / 2),
+                       G.dn_sf_tiled + (((size_t)eloc * (d / 128) + 2 * n + hh) * (I / 64) + 4 * ks) * kAtom,
+                       kMtSfbBytes / 2, &full[st]);
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+    // no copy may still be landing when the CTA exits
+    if (lane == 0) {
+      for (uint32_t jj = (it > (uint32_t)kMtStages ? it - kMtStages : 0); jj < it; ++jj) {
+        volatile int no_abort = 0;
+        mbar_wait(&full[jj % kMtStages], (jj / kMtStages) & 1, &no_abort, p.status);
+      }
+      if (jc > 0) {
+        volatile int no_abort = 0;
+        mbar_wait(&sfa_full, (jc - 1) & 1, &no_abort, p.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tc = 0, jc = 0;
+      bool ok = true;
+      auto tile = [&](int nks, bool phase1) -> bool {
+        if (!mbar_wait(&acc_empty, (tc & 1) ^ 1, &s_abort, p.status)) return false;
+        tc_fence_after();
+        for (int ks = 0; ks < nks; ++ks, ++it) {
+          const uint32_t st = it % kMtStages;
+          if (!mbar_wait(&full[st], (it / kMtStages) & 1, &s_abort, p.status)) return false;
+          tc_fence_after();
+          const uint8_t* sb = ring + (size_t)st * kMtStageBytes;
+          const uint32_t aB = smem_u32(sb + kMtABytes);
+          const uint32_t aA = phase1 ? smem_u32(sb) : smem_u32(htile + (size_t)ks * kMtABytes);
+          const uint32_t aS = smem_u32(sb + kMtABytes + kMtBBytes);
+          const uint32_t sfb = tmem + kMtColSfb + 32 * st;
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc) {
+            tmem_cp_sf(sfb + 8 * kc, sdesc_sf(aS + kAtom * kc));                     // rows 0-127
+            tmem_cp_sf(sfb + 8 * kc + 4, sdesc_sf(aS + kMtSfbBytes / 2 + kAtom * kc));  // rows 128-255
+          }
+#pragma unroll
+          for (int kc = 0; kc < 4; ++kc)
+            mma_mxf4nvf4(tmem, sdesc_sw128(aA + 32 * kc), sdesc_sw128(aB + 32 * kc), kMtIdesc,
+                         tmem + kMtColSfa + 4 * (4 * ks + kc), sfb + 8 * kc, (ks | kc) ? 1u : 0u);
+          mma_commit(&empty[st]);
+        }
+        mma_commit(&acc_full);
+        ++tc;
+        return true;
+      };
+      for (int m = blockIdx.x; m < n_m && ok; m += gridDim.x, ++jc) {
+        // activation scale atoms of the m-tile -> TMEM for the job's gate/up tiles
+        if (!mbar_wait(&sfa_full, jc & 1, &s_abort, p.status)) break;
+        tc_fence_after();
+        for (int a = 0; a < d / 64; ++a) tmem_cp_sf(tmem + kMtColSfa + 4 * a, sdesc_sf(smem_u32(xsf + (size_t)a * kAtom)));
+        mma_commit(&sfa_empty);
+        for (int j = 0; j < nt1 && ok; ++j) ok = tile(nks1, true);
+        if (!ok) break;
+        // h (written by the epilogue into shared memory) and its scale atoms -> TMEM
+        if (!mbar_wait(&h_ready, jc & 1, &s_abort, p.status)) break;
+        tc_fence_after();
+        for (int a = 0; a < I / 64; ++a) tmem_cp_sf(tmem + kMtColSfa + 4 * a, sdesc_sf(smem_u32(hsf + (size_t)a * kAtom)));
+        for (int n = 0; n < nt2 && ok; ++n) ok = tile(nks2, false);
+      }
+      // all issued tensor-core work has completed before TMEM is released
+      mma_commit(&final_bar);
+      volatile int no_abort = 0;
+      mbar_wait(&final_bar, 0, &no_abort, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    // warp w takes TMEM lane quarter q = w % 4 (m-tile rows 32q..32q+31) and half `half` of the
+    // accumulator's 256 columns. One thread waits; a named barrier publishes its decision.
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int half = ew >> 2;
+    const int row = 32 * q + lane;
+    const float ts_x = *p.xq_ts;
+    float* stage_f = ystage + (size_t)ew * (kEpiStageBytes / 4);
+    uint32_t tc = 0, jc = 0;
+    bool go = true;
+    auto wait_acc = [&]() -> bool {
+      if (ew == 0 && lane == 0) s_epi_go[tc & 1] = mbar_wait(&acc_full, tc & 1, &s_abort, p.status) ? 1 : 0;
+      named_bar_sync(2, 32 * kEpiWarps);
+      const bool g = s_epi_go[tc & 1] != 0;
+      tc_fence_after();
+      return g;
+    };
+    // 128 accumulator columns of this thread's row: [128*half, 128*half + 128)
+    auto drain = [&](uint32_t (&v)[4][32]) {
+      const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + 128 * half;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(base + 32 * c, v[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty);
+      ++tc;
+    };
+    for (int m = blockIdx.x; m < n_m && go; m += gridDim.x, ++jc) {
+      const int e = p.mt_expert[m];
+      const bool sh = (e == p.E);
+      const int eloc = sh ? 0 : e;
+      const ExpertGroup& G = sh ? p.shared : p.routed;
+      const bool valid = row < p.mt_valid[m];
+      const size_t prow = (size_t)m * kTileM + row;
+      // ---- gate/up tiles: SwiGLU and NVFP4 h into the shared-memory h tile
+      const float sg = G.gu_ts[2 * eloc] * ts_x, su = G.gu_ts[2 * eloc + 1] * ts_x;
+      for (int j = 0; j < nt1 && go; ++j) {
+        if (!(go = wait_acc())) break;
+        uint32_t v[4][32];
+        drain(v);
+        // columns [0,64) gate and [64,128) up of h columns 128j + 64*half .. +63
+        uint32_t packed[16];
+        uint32_t sbytes = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          float h[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int c = 16 * b + i;
+            const float gv = __uint_as_float(v[c >> 5][c & 31]) * sg;
+            const float uv = __uint_as_float(v[2 + (c >> 5)][c & 31]) * su;
+            h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
+          }
+          uint2 cw;
+          const uint32_t sb = quantize_block16(h, 1.0f, &cw);
+          packed[4 * b] = cw.x;
+          packed[4 * b + 1] = cw.y;
+          sbytes |= sb << (8 * b);
+        }
+        if (!valid) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) packed[i] = packed[i + 1] = 0u;
+          sbytes = 0u;
+        }
+        // 32 code bytes at h column 128j + 64*half: K stage kt, 16-byte pieces c0, c0 + 1 of
+        // the row (128-byte swizzle: piece c of row r at r*128 + (c ^ (r % 8))*16)
+        const int hc = 128 * j + 64 * half;
+        uint8_t* hrow = htile + (size_t)(hc / kStageK) * kMtABytes + (size_t)row * 128;
+        const int c0 = (hc % kStageK) / 32;
+        *reinterpret_cast<uint4*>(hrow + ((c0 ^ (row & 7)) * 16)) = make_uint4(packed[0], packed[1], packed[4], packed[5]);
+        *reinterpret_cast<uint4*>(hrow + (((c0 + 1) ^ (row & 7)) * 16)) =
+            make_uint4(packed[8], packed[9], packed[12], packed[13]);
+        *reinterpret_cast<uint32_t*>(hsf + (size_t)(hc / 64) * kAtom + (row % 32) * 16 + (row / 32) * 4) = sbytes;
+      }
+      if (!go) break;
+      // h complete: visible to the tensor core (async proxy), then released to the MMA issuer
+      fence_proxy_async_smem();
+      named_bar_sync(2, 32 * kEpiWarps);
+      if (ew == 0 && lane == 0) mbar_arrive(&h_ready);
+      // ---- down tiles: w * o added into y (or o stored), 32 columns per bulk operation
+      const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
+      int tok = 0, slot = 0;
+      float wgt = 0.0f;
+      if (valid) {
+        tok = p.row_token[prow];
+        wgt = p.row_weight[prow];
+        slot = p.row_slot[prow];
+      }
+      const float f = p.mode == 0 ? wgt * ts_o : ts_o;
+      for (int n = 0; n < nt2 && go; ++n) {
+        if (!(go = wait_acc())) break;
+        uint32_t v[4][32];
+        drain(v);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          bulk_wait_read<0>();  // the staging row of the previous chunk has been read
+          __syncwarp();
+          float4* rowp = reinterpret_cast<float4*>(stage_f + kEpiRowFloats * lane);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            rowp[i] = make_float4(__uint_as_float(v[c][4 * i]) * f, __uint_as_float(v[c][4 * i + 1]) * f,
+                                  __uint_as_float(v[c][4 * i + 2]) * f, __uint_as_float(v[c][4 * i + 3]) * f);
+          fence_proxy_async_smem();
+          if (valid) {
+            const int n0 = kMtN * n + 128 * half + 32 * c;
+            if (p.mode == 0)
+              bulk_reduce_add_f32(p.out + (size_t)tok * d + n0, rowp, 128);
+            else
+              bulk_s2g((sh ? p.shared_out + (size_t)tok * d : p.out + (size_t)slot * d) + n0, rowp, 128);
+          }
+          bulk_commit();
+        }
+      }
+    }
+    bulk_wait_all();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 namespace {
 
@@ -638,6 +988,8 @@ struct TcLayout {
   size_t off_hdr, off_expert, off_valid, off_first, off_done, off_tok, off_w, off_slot, off_a1, off_sfa1, off_h,
       off_sfa2, total;
 };
+
+bool mt_supported(int d, int I) { return d <= kMtMaxD && I <= kMtMaxI && d % kStageK == 0 && I % kStageK == 0; }
 
 TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   TcLayout L;
@@ -653,9 +1005,12 @@ TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   L.off_tok = o; o += a256(L.rows_cap * 4);
   L.off_w = o; o += a256(L.rows_cap * 4);
   L.off_slot = o; o += a256(L.rows_cap * 4);
-  const bool big = T > kSmallT;  // large T: activation rows gathered before the FFN kernel
-  L.off_a1 = o; o += big ? a256(L.rows_cap * (d / 2)) : 0;
-  L.off_sfa1 = o; o += big ? a256(L.rows_cap * (d / kBlock)) : 0;
+  // the previous kernel gathers activation rows for large T; the m-tile kernel needs only the
+  // rows' scale atoms (every T)
+  const bool mt = mt_supported(d, I);
+  const bool big = T > kSmallT;
+  L.off_a1 = o; o += (big && !mt) ? a256(L.rows_cap * (d / 2)) : 0;
+  L.off_sfa1 = o; o += (big || mt) ? a256(L.rows_cap * (d / kBlock)) : 0;
   L.off_h = o; o += a256(L.rows_cap * (I / 2));
   L.off_sfa2 = o; o += a256(L.rows_cap * (I / kBlock));
   L.total = o;
@@ -676,7 +1031,10 @@ size_t ffn_tc_smem_bytes() { return (size_t)kTcStages * kStageBytes + (size_t)kE
 cudaError_t set_wait_limit_ffn_tc(unsigned long long ns) { return set_wait_limit_here(ns); }
 
 cudaError_t init_ffn_tc_attributes() {
-  return cudaFuncSetAttribute(tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ffn_tc_smem_bytes());
+  cudaError_t e = cudaFuncSetAttribute(tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ffn_tc_smem_bytes());
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(tc_ffn_mt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)mt_smem_bytes(kMtMaxD, kMtMaxI));
 }
 
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t, int num_sms,
@@ -701,8 +1059,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.row_token = reinterpret_cast<int32_t*>(w + L.off_tok);
   p.row_weight = reinterpret_cast<float*>(w + L.off_w);
   p.row_slot = reinterpret_cast<int32_t*>(w + L.off_slot);
-  p.a1 = a.T > kSmallT ? w + L.off_a1 : nullptr;
-  p.sfa1 = a.T > kSmallT ? w + L.off_sfa1 : nullptr;
+  const bool mt = mt_supported(a.d, a.I);
+  p.a1 = (a.T > kSmallT && !mt) ? w + L.off_a1 : nullptr;
+  p.sfa1 = (a.T > kSmallT || mt) ? w + L.off_sfa1 : nullptr;
   p.h_codes = w + L.off_h;
   p.sfa2 = w + L.off_sfa2;
   p.max_m = L.max_m;
@@ -768,6 +1127,11 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     if (zc > num_sms) zc = num_sms;
   }
   if ((e = launch_pdl(tc_schedule_kernel, dim3(1 + zc), dim3(1024), 0, st, p)) != cudaSuccess) return e;
+  if (mt) {
+    // the rows' tokens, weights, output slots and scale atoms, then one job per m-tile
+    if ((e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess) return e;
+    return launch_pdl(tc_ffn_mt_kernel, dim3(num_sms), dim3(kTcThreads), mt_smem_bytes(a.d, a.I), st, maps, p);
+  }
   if (p.a1 && (e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess)
     return e;
   return launch_pdl(tc_ffn_kernel, dim3(num_sms), dim3(kTcThreads), ffn_tc_smem_bytes(), st, maps, p);

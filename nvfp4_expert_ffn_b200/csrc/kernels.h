@@ -96,7 +96,13 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t rows, int cols, const flo
 cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const float* br, int E,
                          int k, int32_t* topk_idx, float* topk_w, int32_t* counts, int32_t* offsets,
                          int32_t* sorted_assign, int32_t* assign_pos, void* ws, int num_sms,
-                         cudaStream_t st);
+                         int32_t* status, cudaStream_t st);
+// tensor-core router (many tokens): approximate bf16-split logits, then an exact top-k
+bool router_tc_supported(int64_t T, int d, int E);
+size_t router_tc_ws_bytes(int d, int E);
+cudaError_t launch_router_tc(const uint16_t* x, int T, int d, const float* Wr, const float* br, int E, int k,
+                             int32_t* topk_idx, float* topk_w, float* logits, uint16_t* w2, int num_sms,
+                             int32_t* status, cudaStream_t st);
 size_t route_ws_bytes(int64_t T, int d, int E, int k);
 
 cudaError_t launch_permute(const int32_t* idx, int T, int k, int E, int32_t* counts,
@@ -158,8 +164,10 @@ cudaError_t set_wait_limit_ffn_decode(unsigned long long ns);
 cudaError_t set_wait_limit_ffn_tc(unsigned long long ns);
 cudaError_t set_wait_limit_ffn_dec(unsigned long long ns);
 cudaError_t set_wait_limit_layer_dec(unsigned long long ns);
+cudaError_t set_wait_limit_router_tc(unsigned long long ns);
 inline cudaError_t set_wait_limits(unsigned long long ns) {
   cudaError_t e = set_wait_limit_ffn_decode(ns);
+  if (e == cudaSuccess) e = set_wait_limit_router_tc(ns);
   if (e == cudaSuccess) e = set_wait_limit_ffn_tc(ns);
   if (e == cudaSuccess) e = set_wait_limit_ffn_dec(ns);
   if (e == cudaSuccess) e = set_wait_limit_layer_dec(ns);
@@ -168,12 +176,15 @@ inline cudaError_t set_wait_limits(unsigned long long ns) {
 
 // one-time per-device kernel attribute setup (dynamic shared memory limits)
 cudaError_t init_route_attributes();
+cudaError_t init_router_tc_attributes();
 cudaError_t init_ffn_decode_attributes();
 cudaError_t init_ffn_tc_attributes();
 cudaError_t init_ffn_dec_attributes();
 cudaError_t init_layer_dec_attributes();
 inline cudaError_t init_kernel_attributes() {
   cudaError_t e = init_route_attributes();
+  if (e != cudaSuccess) return e;
+  e = init_router_tc_attributes();
   if (e != cudaSuccess) return e;
   e = init_ffn_decode_attributes();
   if (e != cudaSuccess) return e;

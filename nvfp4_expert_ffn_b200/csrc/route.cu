@@ -393,19 +393,29 @@ size_t permute_ws_bytes(int64_t T, int k, int E) {
   return (size_t)(nchunk * E * sizeof(int32_t));
 }
 
+// Workspace: the router logits [T][E] float32; with the tensor-core router the bf16 split
+// of Wr [E][2d]; then the permutation's chunk histograms.
 size_t route_ws_bytes(int64_t T, int d, int E, int k) {
   const size_t logits = ((size_t)T * E * sizeof(float) + 255) & ~(size_t)255;
-  return logits + permute_ws_bytes(T, k, E);
+  const size_t w2 = router_tc_supported(T, d, E) ? router_tc_ws_bytes(d, E) : 0;
+  return logits + w2 + permute_ws_bytes(T, k, E);
 }
 
 cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const float* br,
                          int E, int k, int32_t* topk_idx, float* topk_w, int32_t* counts,
                          int32_t* offsets, int32_t* sorted_assign, int32_t* assign_pos, void* ws,
-                         int num_sms, cudaStream_t st) {
+                         int num_sms, int32_t* status, cudaStream_t st) {
   if (T == 0) return launch_permute(nullptr, 0, k, E, counts, offsets, sorted_assign, assign_pos,
                                     nullptr, st);
   float* logits = reinterpret_cast<float*>(ws);
   const size_t logits_bytes = ((size_t)T * E * sizeof(float) + 255) & ~(size_t)255;
+  if (router_tc_supported(T, d, E)) {
+    uint16_t* w2 = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(ws) + logits_bytes);
+    void* perm_ws = reinterpret_cast<char*>(ws) + logits_bytes + router_tc_ws_bytes(d, E);
+    cudaError_t e0 = launch_router_tc(x, T, d, Wr, br, E, k, topk_idx, topk_w, logits, w2, num_sms, status, st);
+    if (e0 != cudaSuccess) return e0;
+    return launch_permute(topk_idx, T, k, E, counts, offsets, sorted_assign, assign_pos, perm_ws, st);
+  }
   void* perm_ws = reinterpret_cast<char*>(ws) + logits_bytes;
   if (T <= kGemvMaxT) {
     // 4 warps (one expert row each) per CTA: E = 512 spreads the router matrix over 128 SMs

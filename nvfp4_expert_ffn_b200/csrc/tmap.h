@@ -35,4 +35,14 @@ inline cudaError_t encode_u8(CUtensorMap* map, const void* base, int rank, const
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 16-bit element tensor (bf16 bits), same conventions as encode_u8 (strides in bytes).
+inline cudaError_t encode_u16(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swizzle) {
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  CUresult r = tmap_encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, (cuuint32_t)rank, const_cast<void*>(base),
+                                dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace moe

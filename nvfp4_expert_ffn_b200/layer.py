@@ -139,10 +139,11 @@ class MoeLayer:
         return self.y[:T]
 
     def join(self, stream=None) -> None:
-        """Make `stream` (default: current) wait for this layer's side-stream work; later
-        calls on that stream need not wait for it again."""
-        (torch.cuda.current_stream() if stream is None else stream).wait_event(self._ev[3])
-        self._hist_pending = False
+        """Make `stream` (default: current) wait for the side-stream work of the last
+        forward(join=False) of this layer, if one is outstanding (otherwise nothing to do)."""
+        if self._hist_pending:
+            (torch.cuda.current_stream() if stream is None else stream).wait_event(self._ev[3])
+            self._hist_pending = False
 
     def graphed(self, T: int, n_slots: int = 1, stream=None) -> "GraphedMoeLayer":
         """A replayable CUDA graph of forward() with its host copies, for a fixed token count."""
@@ -179,7 +180,8 @@ class GraphedMoeLayer:
 
     def run(self, slot: int = 0) -> None:
         """Asynchronous on self.stream: x_host[slot] -> device, the layer, y -> y_host."""
-        self.graphs[slot].replay()
+        with torch.cuda.stream(self.stream):  # a graph replays on the current stream
+            self.graphs[slot].replay()
 
     def step(self, x_host: torch.Tensor, y_host: torch.Tensor) -> None:
         """Copy a host batch into slot 0 (synchronising the stream first, since the last

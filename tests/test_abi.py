@@ -127,13 +127,18 @@ def test_dec_pack_bytes_formula():
 
 
 def test_route_workspace_has_no_permutation_scratch_up_to_4096_assignments():
-    """The routing scratch is the T*E float32 logits (padded to 256 bytes); the per-chunk
-    histograms of the multi-kernel permutation are added only above 4096 assignments."""
+    """The routing scratch is the T*E float32 logits (padded to 256 bytes); from 256 tokens
+    on (tensor-core router) the bf16 split of the router matrix, E*2d*2 bytes; the per-chunk
+    histograms of the multi-kernel permutation only above 4096 assignments."""
     E, d, k = 512, 2048, 10
+    w2 = E * 2 * d * 2
     assert B.moe_workspace_size(B.MOE_OP_ROUTE, 128, d, E, k, 512) == 128 * E * 4
-    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 409, d, E, k, 512) == 409 * E * 4
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 255, d, E, k, 512) == 255 * E * 4
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 409, d, E, k, 512) == 409 * E * 4 + w2
     # 410 tokens x 10 = 4100 assignments: two chunks of histograms
-    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 410, d, E, k, 512) == 410 * E * 4 + 2 * E * 4
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 410, d, E, k, 512) == 410 * E * 4 + w2 + 2 * E * 4
+    # E not a multiple of 128: the CUDA-core router, no split matrix
+    assert B.moe_workspace_size(B.MOE_OP_ROUTE, 409, d, 500, k, 512) == (409 * 500 * 4 + 255) // 256 * 256
 
 
 def test_wait_limit_rejects_out_of_range_without_gpu():

@@ -55,8 +55,30 @@ def _check_route(x, Wr, br, k):
     return len(excused)
 
 
+@pytest.mark.parametrize("cfg_name", ["prefill", "wide"])
+def test_tensor_core_router_error_is_far_below_its_margin(cfg_name):
+    """From 256 tokens on, moe_route takes approximate logits from a bf16-split tensor-core
+    GEMM (left in the first T*E*4 bytes of the workspace) and recomputes exactly every expert
+    within 2*delta (delta = 2e-3) of the k-th. That is exact as long as each approximate logit
+    is within delta of the true one: check it is within delta/20 of the oracle's."""
+    c = synth.CONFIGS[cfg_name]
+    T = c.T_list[0]
+    x = synth.make_x(0, c, T)
+    Wr, br = synth.make_router(0, c)
+    brg = br if c.zipf_s > 0 else None
+    b = route_buffers(T, c.k, c.E, c.d)
+    B.moe_route(x.cuda(), Wr.cuda(), None if brg is None else brg.cuda(), c.k, b["topk_idx"], b["topk_w"],
+                b["counts"], b["offsets"], b["sorted_assign"], b["assign_pos"], b["ws"])
+    torch.cuda.synchronize()
+    approx = b["ws"][:T * c.E * 4].view(torch.float32).view(T, c.E).cpu().numpy().astype(np.float64)
+    logits = omoe.router_logits(bits_to_f32(x.numpy()), Wr.numpy(), None if brg is None else brg.numpy())
+    err = np.abs(approx - logits).max()
+    print(f"{cfg_name}: max |approximate - oracle logit| = {err:.3e}")
+    assert err < 2e-3 / 20
+
+
 @pytest.mark.parametrize("cfg,T", [("tiny", 16), ("decode", 1), ("decode", 4), ("decode", 8),
-                                   ("decode", 9), ("decode", 100), ("prefill", 16384),
+                                   ("decode", 9), ("decode", 100), ("decode", 300), ("prefill", 16384),
                                    ("wide", 27140)])
 def test_route_matches_oracle(cfg, T):
     c = synth.CONFIGS[cfg]
