@@ -407,6 +407,97 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
     return out
 
 
+def build_stack(device, n_layers: int = 48, epochs: int = 4, n_x: int = 64):
+    """The decode stack: n_layers distinct decode layers (own weights, router and Zipf(1.0)
+    popularity each; decode pack only, every weight byte held once), the router bias of every
+    64-step epoch, and n_x input draws of 8 tokens."""
+    from nvfp4_expert_ffn_b200 import binding as B
+    from nvfp4_expert_ffn_b200 import layer as L
+    from nvfp4_expert_ffn_b200 import synth
+    cfg = synth.CONFIGS["stack48"]
+    ws_q = torch.empty(B.moe_workspace_size(B.MOE_OP_QUANT, 1, cfg.d, 1, 1, cfg.I), dtype=torch.uint8, device=device)
+    layers, biases = [], []
+    for li in range(n_layers):
+        routed = L.quantize_weights_gpu(SEED, cfg, layer=li, device=device, ws=ws_q, decode_only=True)
+        shared = L.quantize_weights_gpu(SEED, cfg, layer=li, shared=True, device=device, ws=ws_q, decode_only=True)
+        Wr, _ = synth.make_router(SEED, cfg, layer=li)
+        biases.append([synth.make_router(SEED, cfg, layer=li, epoch=ep)[1].to(device) for ep in range(epochs)])
+        layers.append(L.MoeLayer(B.Experts(routed, shared), Wr.to(device), biases[-1][0], cfg.k, 8, device=device,
+                                 fused=True))
+    xs = torch.stack([synth.make_x(SEED, cfg, 8, step=s) for s in range(n_x)]).to(device)
+    return cfg, layers, biases, xs
+
+
+def measure_stack(timer, cfg, layers, biases, xs, K, W, stream, world, peaks):
+    """Step = 8 tokens through every layer (RMS renormalisation between layers); step s uses
+    input draw s % len(xs) and the router biases of epoch (s // 64) % epochs."""
+    n_ep = len(biases[0])
+    x_in = torch.empty_like(xs[0])
+    graphs = []
+    for ep in range(n_ep):
+        for lay, b in zip(layers, biases):
+            lay.br = b[ep]
+
+        def step(i):
+            h = x_in
+            for lay in layers:
+                h = lay.forward(h, rms_renorm=True, join=False)
+
+        def finish():
+            for lay in layers:
+                lay.join(stream)
+
+        with torch.cuda.stream(stream):
+            step(0)
+            finish()
+        torch.cuda.synchronize()
+        graphs.append(timer.capture(step, 1, finish))
+    lps = graphs[0][1]
+
+    def run(n, s0=0):
+        for s in range(s0, s0 + n):
+            x_in.copy_(xs[s % len(xs)], non_blocking=True)
+            graphs[(s // 64) % n_ep][0].replay()
+
+    # touched experts per layer and step (for the bytes), on a sample of steps
+    U = []
+    with torch.cuda.stream(stream):
+        for s in (0, 64, 128, 192):
+            run(1, s)
+            stream.synchronize()
+            U.extend(int((lay.counts > 0).sum().item()) for lay in layers)
+    with torch.cuda.stream(stream):
+        run(W)
+    torch.cuda.synchronize()
+    if timer.dist is not None:
+        timer.dist.barrier()
+    t0h = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        run(K)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    timer.windows.append((t0h, time.time()))
+    ms = max_over_ranks(timer.dist, e0.elapsed_time(e1), timer.device)
+    per_layer_bytes = float(np.mean([algorithmic_bytes(cfg, u, 8) for u in U]))
+    step_bytes = per_layer_bytes * len(layers)
+    ach = step_bytes / (ms / K * 1e-3) / 1e9
+    return {"value": round(whole_job_rate(world, 8, K, ms), 1), "unit": "tokens/s", "ms_per_step": round(ms / K, 6),
+            "steps": K, "T": 8, "layers": len(layers), "touched_experts_avg": round(float(np.mean(U)), 2),
+            "gpu_launches": int(round(lps * K)), "gpu_launches_per_step": lps,
+            "roofline": {"kernel": "whole step: 48 x (layer_dec_kernel + hist_kernel)", "bound": "hbm",
+                         "achieved": round(ach, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": round(ach / peaks["hbm"], 4), "peak_kind": peaks["kind"] + " (HBM copy, burst)",
+                         "frac_vs_nominal_8tbs": round(ach / NOMINAL_HBM_GBS, 4),
+                         "bytes_per_step": int(step_bytes), "traffic": None},
+            "workload": (f"48-layer decode stack: d={cfg.d}, {cfg.E} experts/layer, top-{cfg.k} + 1 shared, "
+                         f"I={cfg.I}, 8 tokens per step, per-layer RMS renormalisation, Zipf(1.0) routing "
+                         f"re-drawn every 64 steps, {len(layers)} x {cfg.E} experts resident "
+                         f"({len(layers) * (cfg.E + 1) * 3 * cfg.d * cfg.I * 0.5625 / 1e9:.1f} GB, decode pack only)")}
+
+
 def near_tie_record():
     """Tokens excused from the bit-exact top-k comparison in the parity tests (k-th/(k+1)-th
     oracle logit margin under 1e-6), per test input, from tests/golden/near_ties.json."""
@@ -453,6 +544,20 @@ def run_gpu(args):
             extra["prefill_T16384"]["workload"] = ("prefill MoE layer: the decode layer's weights, Zipf(0.8) "
                                                    "routing, T=16384 tokens per step, 2 layer copies")
             del players
+            if not args.no_stack:
+                del copies, xs
+                torch.cuda.empty_cache()
+                copies = []
+                scfg, slayers, sbiases, sxs = build_stack(device)
+                extra["stack48"] = measure_stack(timer, scfg, slayers, sbiases, sxs, 256, max(W, 8), stream, world,
+                                                 peaks)
+                del slayers
+    elif args.workload == "stack48":
+        T = 8
+        cfg, slayers, sbiases, sxs = build_stack(device)
+        main = measure_stack(timer, cfg, slayers, sbiases, sxs, K, W, stream, world, peaks)
+        workload = main["workload"]
+        l2 = "48 layers x 513 experts resident (43.6 GB), far above L2"
     else:
         cfg, layers, xs = build_prefill_layers(device, args.workload, None, args.layers)
         T = xs[0].shape[0]
@@ -585,11 +690,12 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--T", type=int, default=0, help="decode tokens per step (default 8)")
-    ap.add_argument("--workload", choices=["decode", "prefill", "wide"], default="decode")
+    ap.add_argument("--workload", choices=["decode", "prefill", "wide", "stack48"], default="decode")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-stack", action="store_true", help="leave out the 48-layer decode stack")
     ap.add_argument("--layers", type=int, default=8, help="distinct layer copies rotated")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

@@ -84,6 +84,10 @@ typedef enum moe_status {
  *   dec_pack  the decode pack written by moe_pack_experts for the DECODE path and
  *            moe_layer_decode (NULL if absent): every weight byte and scale of the group
  *            again, as the 18432-byte blocks the decode kernel copies into shared memory.
+ * A group that has its decode pack may leave gu_codes, gu_scales, dn_codes, dn_scales and the
+ * re-tiled scales NULL (all four natural arrays, or none): moe_layer_decode and the DECODE
+ * path of moe_expert_ffn read only the pack and the tensor scales, so a decode-only model
+ * holds each weight byte once. The other paths then return an error.
  */
 typedef struct moe_expert_weights {
   int32_t E, d, I;

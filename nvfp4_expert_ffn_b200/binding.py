@@ -113,27 +113,42 @@ class _ExpertsC(ctypes.Structure):
 @dataclass
 class ExpertWeights:
     """NVFP4 weights of an expert group on the GPU (natural layout, see moe_nvfp4.h)."""
-    gu_codes: torch.Tensor   # uint8 [E][2I][d/2]
-    gu_scales: torch.Tensor  # uint8 [E][2I][d/16]
-    gu_ts: torch.Tensor      # float32 [E][2]
-    dn_codes: torch.Tensor   # uint8 [E][d][I/2]
-    dn_scales: torch.Tensor  # uint8 [E][d][I/16]
-    dn_ts: torch.Tensor      # float32 [E]
+    gu_codes: Optional[torch.Tensor]   # uint8 [E][2I][d/2]
+    gu_scales: Optional[torch.Tensor]  # uint8 [E][2I][d/16]
+    gu_ts: torch.Tensor                # float32 [E][2]
+    dn_codes: Optional[torch.Tensor]   # uint8 [E][d][I/2]
+    dn_scales: Optional[torch.Tensor]  # uint8 [E][d][I/16]
+    dn_ts: torch.Tensor                # float32 [E]
     gu_sf_tiled: Optional[torch.Tensor] = None
     dn_sf_tiled: Optional[torch.Tensor] = None
     dec_pack: Optional[torch.Tensor] = None
+    dims: tuple = ()                   # (E, d, I), taken from gu_codes when not given
+
+    def __post_init__(self):
+        if not self.dims:
+            E, twoI, dh = self.gu_codes.shape
+            self.dims = (E, 2 * dh, twoI // 2)
 
     @property
     def E(self):
-        return self.gu_codes.shape[0]
-
-    @property
-    def I(self):
-        return self.gu_codes.shape[1] // 2
+        return self.dims[0]
 
     @property
     def d(self):
-        return self.gu_codes.shape[2] * 2
+        return self.dims[1]
+
+    @property
+    def I(self):
+        return self.dims[2]
+
+    def release_natural(self) -> None:
+        """Drop the natural-layout arrays and the re-tiled scales, keeping the decode pack and
+        the tensor scales: enough for moe_layer_decode and the DECODE path, with every
+        weight byte held once."""
+        if self.dec_pack is None:
+            raise ValueError("release_natural needs the decode pack (moe_pack_experts)")
+        self.gu_codes = self.gu_scales = self.dn_codes = self.dn_scales = None
+        self.gu_sf_tiled = self.dn_sf_tiled = None
 
     def struct(self) -> _WeightsC:
         p = lambda t: None if t is None else _ptr(t).value  # noqa: E731

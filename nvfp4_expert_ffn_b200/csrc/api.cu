@@ -85,14 +85,29 @@ moe_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return MOE_OK;
 }
 
-moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E, int d, int I) {
+// The tensor scales are always needed. The natural-layout codes and scales may all be NULL
+// when the group carries its decode pack (which holds the same bytes), for the calls that read
+// only the pack; `natural` reports whether they are present.
+moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E, int d, int I, bool* natural) {
   const std::string n(name);
   if (w.E != E || w.d != d || w.I != I) return fail(MOE_ERR_INVALID_ARG, n + ": inconsistent E/d/I");
-  const void* ps[6] = {w.gu_codes, w.gu_scales, w.gu_ts, w.dn_codes, w.dn_scales, w.dn_ts};
-  for (const void* p : ps) {
-    if (!p) return fail(MOE_ERR_INVALID_ARG, n + ": null weight pointer");
+  const void* ts[2] = {w.gu_ts, w.dn_ts};
+  for (const void* p : ts) {
+    if (!p) return fail(MOE_ERR_INVALID_ARG, n + ": null tensor-scale pointer");
     if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, n + ": weight pointer not 16-byte aligned");
   }
+  const void* nat[4] = {w.gu_codes, w.gu_scales, w.dn_codes, w.dn_scales};
+  int present = 0;
+  for (const void* p : nat) {
+    if (p && !aligned16(p)) return fail(MOE_ERR_INVALID_ARG, n + ": weight pointer not 16-byte aligned");
+    present += p ? 1 : 0;
+  }
+  if (present != 0 && present != 4)
+    return fail(MOE_ERR_INVALID_ARG, n + ": the natural-layout codes and scales must all be given or all NULL");
+  if (present == 0 && !w.dec_pack)
+    return fail(MOE_ERR_INVALID_ARG, n + ": null weight pointer (neither the natural layout nor the decode pack)");
+  if (w.dec_pack && !aligned16(w.dec_pack)) return fail(MOE_ERR_INVALID_ARG, n + ": dec_pack not 16-byte aligned");
+  *natural = present == 4;
   return MOE_OK;
 }
 
@@ -262,12 +277,14 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   if (mode != MOE_FFN_ACCUMULATE && mode != MOE_FFN_PER_ASSIGN) return fail(MOE_ERR_INVALID_ARG, "bad mode");
   if (path != MOE_PATH_AUTO && path != MOE_PATH_DECODE && path != MOE_PATH_PREFILL && path != MOE_PATH_CUDA_CORE)
     return fail(MOE_ERR_INVALID_ARG, "bad path");
-  moe_status s = check_weights(W->routed, "routed", E, d, I);
+  bool nat_r = false, nat_s = true;
+  moe_status s = check_weights(W->routed, "routed", E, d, I, &nat_r);
   if (s != MOE_OK) return s;
   if (W->has_shared) {
-    s = check_weights(W->shared, "shared", 1, d, I);
+    s = check_weights(W->shared, "shared", 1, d, I, &nat_s);
     if (s != MOE_OK) return s;
   }
+  const bool natural = nat_r && nat_s;
   if (T == 0) return MOE_OK;
   if (!xq_codes || !xq_scales || !xq_ts || !offsets || !sorted_assign || !topk_w || !out)
     return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
@@ -281,17 +298,23 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales, con
   if (s != MOE_OK) return s;
   const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
                       (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
-  const bool tc_ok = ffn_tc_supported(d, I) && packed;
+  const bool tc_ok = ffn_tc_supported(d, I) && packed && natural;
   const bool dec_packed = W->routed.dec_pack && (!W->has_shared || W->shared.dec_pack);
   const bool dec_ok = ffn_dec_supported(T, d, I, mode, E, k, W->has_shared ? 1 : 0, sms) && dec_packed;
   if (path == MOE_PATH_PREFILL && !tc_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
-                "tensor-core path needs d % 256 == 0, I % 256 == 0 and scales packed by moe_pack_experts");
+                "tensor-core path needs d % 256 == 0, I % 256 == 0, the natural-layout weights and scales "
+                "packed by moe_pack_experts");
   if (path == MOE_PATH_DECODE && !dec_ok)
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "decode path needs T <= 8, ACCUMULATE mode, d % 512 == 0, I % 64 == 0 and the decode pack");
+  if (path == MOE_PATH_CUDA_CORE && !natural)
+    return fail(MOE_ERR_INVALID_ARG, "the CUDA-core path reads the natural-layout weights, which are NULL");
   const int kind = path == MOE_PATH_AUTO ? (dec_ok ? MOE_PATH_DECODE : tc_ok ? MOE_PATH_PREFILL : MOE_PATH_CUDA_CORE)
                                          : path;
+  if (kind == MOE_PATH_CUDA_CORE && !natural)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE,
+                "without the natural-layout weights only the DECODE path (T <= 8) can run this call");
   const size_t need = kind == MOE_PATH_DECODE    ? ffn_dec_ws_bytes(E)
                       : kind == MOE_PATH_PREFILL ? ffn_tc_ws_bytes(T, d, E, k, I)
                                                  : ffn_decode_ws_bytes(T, d, E, k, I);
@@ -327,9 +350,10 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
                             int32_t rms_renorm, void* ws, size_t ws_bytes, void* stream) {
   if (!W) return fail(MOE_ERR_INVALID_ARG, "null weights");
   const int E = W->routed.E, d = W->routed.d, I = W->routed.I;
-  moe_status s = check_weights(W->routed, "routed", E, d, I);
+  bool nat = false;
+  moe_status s = check_weights(W->routed, "routed", E, d, I, &nat);
   if (s != MOE_OK) return s;
-  if (W->has_shared && (s = check_weights(W->shared, "shared", 1, d, I)) != MOE_OK) return s;
+  if (W->has_shared && (s = check_weights(W->shared, "shared", 1, d, I, &nat)) != MOE_OK) return s;
   if (!x || !Wr || !xq_codes || !xq_scales || !xq_ts || !topk_idx || !topk_w || !counts || !offsets ||
       !sorted_assign || !assign_pos || !y_acc || !y)
     return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");

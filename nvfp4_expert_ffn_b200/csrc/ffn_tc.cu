@@ -521,31 +521,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
-        float h[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float gv = __uint_as_float(g[i]) * sg, uv = __uint_as_float(u[i]) * su;
-          h[i] = gv * __frcp_rn(1.0f + __expf(-gv)) * uv;
-        }
+        // SwiGLU and the NVFP4 quantisation of h (tensor scale 1), IEEE float32 steps as in the
+        // activation quantiser
         uint32_t packed[8];
         uint32_t sbytes = 0;
 #pragma unroll
         for (int b = 0; b < 2; ++b) {
-          float amax = 0.0f;
+          float h[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(h[16 * b + i]));
-          const uint32_t sb = f32_to_e4m3_sat(__fdiv_rn(amax, kE2M1Max));  // tensor scale of h is 1
-          const float sval = e4m3_to_f32(sb);
-          const float rs = sval != 0.0f ? __frcp_rn(sval) : 0.0f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = f32x2_to_e2m1x2(h[16 * b + 2 * i] * rs, h[16 * b + 2 * i + 1] * rs);
-            const uint32_t hi = f32x2_to_e2m1x2(h[16 * b + 8 + 2 * i] * rs, h[16 * b + 9 + 2 * i] * rs);
-            if (i == 0) packed[4 * b] = lo, packed[4 * b + 2] = hi;
-            else packed[4 * b] |= lo << (8 * i), packed[4 * b + 2] |= hi << (8 * i);
+          for (int i = 0; i < 16; ++i) {
+            const float gv = __uint_as_float(g[16 * b + i]) * sg, uv = __uint_as_float(u[16 * b + i]) * su;
+            h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
           }
-          if (sval == 0.0f) packed[4 * b] = packed[4 * b + 2] = 0;
-          sbytes |= sb << (8 * b);
+          uint2 cw;
+          sbytes |= quantize_block16(h, 1.0f, &cw) << (8 * b);
+          packed[4 * b] = cw.x;      // elements 0-7 of the block
+          packed[4 * b + 2] = cw.y;  // elements 8-15
         }
         if (valid) {
           // 32 codes = 16 bytes at h columns 64j + 32*half
@@ -658,8 +649,16 @@ __host__ __device__ inline size_t mt_smem_bytes(int d, int I) {
          (size_t)kEpiWarps * kEpiStageBytes + 1024;
 }
 
+// trace id of tile `t` (0..nt1-1 gate/up, then down) of this CTA's job `jc` (first 4 jobs only)
+#define MT_TRACE(ev, jc, t)                                        \
+  do {                                                             \
+    if ((jc) < 4) TC_TRACE_AT(g_tc_trace, ev, (jc) * 64 + (t));    \
+  } while (0)
+
 __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
+  TC_TRACE_DECL
   MOE_PDL_PROLOGUE();
+  TC_TRACE_BEGIN(g_tc_trace);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ uint64_t full[kMtStages], empty[kMtStages], acc_full, acc_empty, sfa_full, sfa_empty, h_ready,
@@ -701,6 +700,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
   tc_fence_after();
   const uint32_t tmem = s_tmem;
   const int n_m = *p.n_mtiles;
+  if (threadIdx.x == 0) TC_TRACE_AT(g_tc_trace, kEvSetupDone, n_m);
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -744,6 +744,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
             alive = false;
             break;
           }
+          if (ks == 0 && lane == 0) MT_TRACE(kEvProdTile, jc, j);
           uint8_t* sb = ring + (size_t)st * kMtStageBytes;
           if (lane == 0) {
             mbar_arrive_expect_tx(&full[st], (uint32_t)(ngather * 512 + kMtBBytes + kMtSfbBytes));
@@ -770,6 +771,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
             alive = false;
             break;
           }
+          if (ks == 0 && lane == 0) MT_TRACE(kEvProdTile, jc, nt1 + n);
           uint8_t* sb = ring + (size_t)st * kMtStageBytes;
           if (lane == 0) {
             mbar_arrive_expect_tx(&full[st], (uint32_t)(kMtBBytes + kMtSfbBytes));
@@ -803,13 +805,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
     if (lane == 0) {
       uint32_t it = 0, tc = 0, jc = 0;
       bool ok = true;
+      int tix = 0;  // tile index within the job, for the trace
       auto tile = [&](int nks, bool phase1) -> bool {
         if (!mbar_wait(&acc_empty, (tc & 1) ^ 1, &s_abort, p.status)) return false;
         tc_fence_after();
+        MT_TRACE(kEvMmaSlot, jc, tix);
         for (int ks = 0; ks < nks; ++ks, ++it) {
           const uint32_t st = it % kMtStages;
           if (!mbar_wait(&full[st], (it / kMtStages) & 1, &s_abort, p.status)) return false;
           tc_fence_after();
+          if (ks == 0) MT_TRACE(kEvMmaFirst, jc, tix);
           const uint8_t* sb = ring + (size_t)st * kMtStageBytes;
           const uint32_t aB = smem_u32(sb + kMtABytes);
           const uint32_t aA = phase1 ? smem_u32(sb) : smem_u32(htile + (size_t)ks * kMtABytes);
@@ -827,10 +832,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
           mma_commit(&empty[st]);
         }
         mma_commit(&acc_full);
+        MT_TRACE(kEvMmaLast, jc, tix);
         ++tc;
+        ++tix;
         return true;
       };
       for (int m = blockIdx.x; m < n_m && ok; m += gridDim.x, ++jc) {
+        tix = 0;
         // activation scale atoms of the m-tile -> TMEM for the job's gate/up tiles
         if (!mbar_wait(&sfa_full, jc & 1, &s_abort, p.status)) break;
         tc_fence_after();
@@ -841,6 +849,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
         // h (written by the epilogue into shared memory) and its scale atoms -> TMEM
         if (!mbar_wait(&h_ready, jc & 1, &s_abort, p.status)) break;
         tc_fence_after();
+        MT_TRACE(kEvProdDone1, jc, 0);
         for (int a = 0; a < I / 64; ++a) tmem_cp_sf(tmem + kMtColSfa + 4 * a, sdesc_sf(smem_u32(hsf + (size_t)a * kAtom)));
         for (int n = 0; n < nt2 && ok; ++n) ok = tile(nks2, false);
       }
@@ -862,8 +871,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
     float* stage_f = ystage + (size_t)ew * (kEpiStageBytes / 4);
     uint32_t tc = 0, jc = 0;
     bool go = true;
+    int tix = 0;
     auto wait_acc = [&]() -> bool {
-      if (ew == 0 && lane == 0) s_epi_go[tc & 1] = mbar_wait(&acc_full, tc & 1, &s_abort, p.status) ? 1 : 0;
+      if (ew == 0 && lane == 0) {
+        s_epi_go[tc & 1] = mbar_wait(&acc_full, tc & 1, &s_abort, p.status) ? 1 : 0;
+        MT_TRACE(kEvEpiStart, jc, tix);
+      }
       named_bar_sync(2, 32 * kEpiWarps);
       const bool g = s_epi_go[tc & 1] != 0;
       tc_fence_after();
@@ -878,9 +891,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty);
+      if (ew == 0 && lane == 0) MT_TRACE(kEvDrainEnd, jc, tix);
       ++tc;
     };
     for (int m = blockIdx.x; m < n_m && go; m += gridDim.x, ++jc) {
+      tix = 0;
       const int e = p.mt_expert[m];
       const bool sh = (e == p.E);
       const int eloc = sh ? 0 : e;
@@ -926,6 +941,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
         *reinterpret_cast<uint4*>(hrow + (((c0 + 1) ^ (row & 7)) * 16)) =
             make_uint4(packed[8], packed[9], packed[12], packed[13]);
         *reinterpret_cast<uint32_t*>(hsf + (size_t)(hc / 64) * kAtom + (row % 32) * 16 + (row / 32) * 4) = sbytes;
+        if (ew == 0 && lane == 0) MT_TRACE(kEvEpiEnd, jc, tix);
+        ++tix;
       }
       if (!go) break;
       // h complete: visible to the tensor core (async proxy), then released to the MMA issuer
@@ -965,6 +982,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
           }
           bulk_commit();
         }
+        if (ew == 0 && lane == 0) MT_TRACE(kEvEpiEnd, jc, tix);
+        ++tix;
       }
     }
     bulk_wait_all();
@@ -975,6 +994,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (threadIdx.x == 0) TC_TRACE_AT(g_tc_trace, kEvExit, 0);
 }
 
 // ---------------------------------------------------------------- host side

@@ -17,10 +17,12 @@ from . import synth
 
 def quantize_weights_gpu(seed: int, cfg: synth.LayerShape, layer: int = 0, device="cuda",
                          experts: Optional[range] = None, shared: bool = False,
-                         ws: Optional[torch.Tensor] = None, pack: bool = True) -> B.ExpertWeights:
-    """Generate an expert group's bf16 weights on the GPU and quantise each matrix
-    (gate, up, down of every expert, one tensor scale each) with nvfp4_quantize_act; then
-    re-tile the scales for the tensor-core path (moe_pack_experts) when the shape allows."""
+                         ws: Optional[torch.Tensor] = None, pack: bool = True,
+                         decode_only: bool = False, chunk: int = 32) -> B.ExpertWeights:
+    """Generate an expert group's bf16 weights on the GPU (a chunk of experts at a time) and
+    quantise each matrix (gate, up, down of every expert, one tensor scale each) with
+    nvfp4_quantize_act; then re-tile the scales for the tensor-core path (moe_pack_experts)
+    when the shape allows. decode_only: keep only the decode pack and the tensor scales."""
     E = 1 if shared else cfg.E
     d, I = cfg.d, cfg.I
     w = B.ExpertWeights(
@@ -33,13 +35,18 @@ def quantize_weights_gpu(seed: int, cfg: synth.LayerShape, layer: int = 0, devic
     if ws is None:
         ws = torch.empty(B.moe_workspace_size(B.MOE_OP_QUANT, 1, d, 1, 1, I),
                          dtype=torch.uint8, device=device)
-    for e in range(E):
-        g, u, dn = synth.make_expert_weights_bf16(seed, cfg, e, layer, shared, device)
-        B.nvfp4_quantize_act(g, w.gu_codes[e, :I], w.gu_scales[e, :I], w.gu_ts[e, 0:1], ws=ws)
-        B.nvfp4_quantize_act(u, w.gu_codes[e, I:], w.gu_scales[e, I:], w.gu_ts[e, 1:2], ws=ws)
-        B.nvfp4_quantize_act(dn, w.dn_codes[e], w.dn_scales[e], w.dn_ts[e:e + 1], ws=ws)
+    for e0 in range(0, E, chunk):
+        ids = range(e0, min(E, e0 + chunk))
+        g, u, dn = synth.make_experts_weights_bf16(seed, cfg, ids, layer, shared, device)
+        for r, e in enumerate(ids):
+            B.nvfp4_quantize_act(g[r], w.gu_codes[e, :I], w.gu_scales[e, :I], w.gu_ts[e, 0:1], ws=ws)
+            B.nvfp4_quantize_act(u[r], w.gu_codes[e, I:], w.gu_scales[e, I:], w.gu_ts[e, 1:2], ws=ws)
+            B.nvfp4_quantize_act(dn[r], w.dn_codes[e], w.dn_scales[e], w.dn_ts[e:e + 1], ws=ws)
+        del g, u, dn
     if pack and d % 128 == 0 and I % 64 == 0:
         B.moe_pack_experts(w)
+        if decode_only:
+            w.release_natural()
     return w
 
 

@@ -173,6 +173,35 @@ def make_expert_weights_bf16(seed: int, cfg: LayerShape, expert: int, layer: int
     return mk(tg).view(cfg.I, cfg.d), mk(tu).view(cfg.I, cfg.d), mk(td).view(cfg.d, cfg.I)
 
 
+def normal_f32_rows(keys, n: int, std: float, device="cpu") -> torch.Tensor:
+    """normal_f32(keys[r], n, std) for every key at once: a [len(keys)][n] float32 tensor,
+    bit-identical row by row (the same integer steps, with the key broadcast per row)."""
+    key = torch.tensor([_s64(k) for k in keys], dtype=torch.int64, device=device)[:, None]
+    z = torch.arange(n, dtype=torch.int64, device=device)[None, :] + 1
+    z = z * _s64(_GOLDEN) + key
+    z = (z ^ _lsr(z, 30)) * _s64(_M1)
+    z = (z ^ _lsr(z, 27)) * _s64(_M2)
+    h = z ^ _lsr(z, 31)
+    s = (h & 0xFFFF) + (_lsr(h, 16) & 0xFFFF) + (_lsr(h, 32) & 0xFFFF) + _lsr(h, 48)
+    zi = (2 * s - 4 * 65535).to(torch.float32)
+    c = torch.tensor(np.float32(std * _IH4_SCALE), dtype=torch.float32, device=device)
+    return zi * c
+
+
+def make_experts_weights_bf16(seed: int, cfg: LayerShape, experts, layer: int = 0,
+                              shared: bool = False, device="cpu"):
+    """make_expert_weights_bf16 for several experts at once: gate [n][I][d], up [n][I][d],
+    down [n][d][I] as bf16 bit patterns, row e equal to expert experts[e]'s draws."""
+    tg, tu, td = (TID_SGATE, TID_SUP, TID_SDOWN) if shared else (TID_GATE, TID_UP, TID_DOWN)
+    base = (seed, cfg.cid, layer)
+    n = cfg.I * cfg.d
+    ex = list(experts)
+    mk = lambda tid: f32_to_bf16_bits(  # noqa: E731
+        normal_f32_rows([stream_key(*base, tid, e) for e in ex], n, cfg.weight_std, device))
+    return (mk(tg).view(len(ex), cfg.I, cfg.d), mk(tu).view(len(ex), cfg.I, cfg.d),
+            mk(td).view(len(ex), cfg.d, cfg.I))
+
+
 def make_expert_weights_f32(seed: int, cfg: LayerShape, expert: int, layer: int = 0,
                             shared: bool = False, device="cpu"):
     """The same weights widened (exactly) to float32."""

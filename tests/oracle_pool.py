@@ -34,16 +34,34 @@ def _expert_rows(cfg_name, seed, layer, e, shared, x_hat_rows):
     return e, shared, omoe.expert_ffn(x_hat_rows, ex)
 
 
-def expert_outputs(cfg_name, seed, layer, tasks, workers=None):
-    """tasks: list of (expert id, shared flag, x_hat rows float64 [n][d]). Returns a dict
-    (expert id, shared) -> o rows float64 [n][d], in the order of the given rows."""
-    workers = workers or min(32, os.cpu_count() or 1)
-    out = {}
-    with cf.ProcessPoolExecutor(max_workers=workers, mp_context=mp.get_context("spawn"),
-                                initializer=_init_worker) as ex:
-        futs = [ex.submit(_expert_rows, cfg_name, seed, layer, e, sh, np.ascontiguousarray(rows))
+class OraclePool:
+    """A pool of host processes kept across many expert_outputs calls (use as a context
+    manager)."""
+
+    def __init__(self, workers=None):
+        self.workers = workers or min(32, os.cpu_count() or 1)
+        self.ex = cf.ProcessPoolExecutor(max_workers=self.workers, mp_context=mp.get_context("spawn"),
+                                         initializer=_init_worker)
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.ex.shutdown()
+
+    def expert_outputs(self, cfg_name, seed, layer, tasks):
+        """tasks: list of (expert id, shared flag, x_hat rows float64 [n][d]). Returns a dict
+        (expert id, shared) -> o rows float64 [n][d], in the order of the given rows."""
+        futs = [self.ex.submit(_expert_rows, cfg_name, seed, layer, e, sh, np.ascontiguousarray(rows))
                 for e, sh, rows in tasks]
+        out = {}
         for f in cf.as_completed(futs):
             e, sh, o = f.result()
             out[(e, sh)] = o
-    return out
+        return out
+
+
+def expert_outputs(cfg_name, seed, layer, tasks, workers=None):
+    """One-off OraclePool.expert_outputs."""
+    with OraclePool(workers) as pool:
+        return pool.expert_outputs(cfg_name, seed, layer, tasks)

@@ -147,3 +147,25 @@ def test_wait_limit_rejects_out_of_range_without_gpu():
     assert L.moe_set_wait_limit_ns(999_999) == 1
     assert L.moe_set_wait_limit_ns(60_000_000_001) == 1
     assert b"wait limit" in L.moe_last_error()
+
+
+def test_natural_weights_all_or_none():
+    """A group may leave its natural-layout arrays NULL only all together and only when it has
+    the decode pack; the checks run on the host before any device call."""
+    L = B.lib()
+    INV = 1
+    p = ctypes.c_void_p(0x10000)
+    # natural arrays NULL, no decode pack: nothing to read
+    w = B._WeightsC(8, 512, 64, None, None, p.value, None, None, p.value, None, None, None)
+    ex = B._ExpertsC(w, B._WeightsC(), 0)
+    assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == INV
+    assert b"neither" in L.moe_last_error()
+    # some natural arrays given, others NULL
+    w = B._WeightsC(8, 512, 64, p.value, None, p.value, p.value, p.value, p.value, None, None, p.value)
+    ex = B._ExpertsC(w, B._WeightsC(), 0)
+    assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == INV
+    assert b"all be given or all NULL" in L.moe_last_error()
+    # tensor scales are always needed
+    w = B._WeightsC(8, 512, 64, None, None, None, None, None, p.value, None, None, p.value)
+    ex = B._ExpertsC(w, B._WeightsC(), 0)
+    assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == INV

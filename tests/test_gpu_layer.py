@@ -153,3 +153,24 @@ def test_fused_decode_layer_repeated_calls():
     y = lay.forward(x).clone()
     torch.cuda.synchronize()
     assert np.allclose(bits_to_f32(y.cpu().numpy()), bits_to_f32(outs[0].numpy()), rtol=1e-2, atol=1e-3)
+
+
+def test_decode_layer_with_weights_held_once():
+    """After release_natural() a group keeps only its decode pack and tensor scales (each
+    weight byte once): the one-kernel decode layer gives the same result as before, and the
+    paths that read the natural layout refuse instead of reading freed memory."""
+    cfg, lay, Wr, br = _layer("decode", T_max=8, fused=True)
+    x = synth.make_x(8, cfg, 8).cuda()
+    y1 = lay.forward(x).clone()
+    for g in (lay.experts.routed, lay.experts.shared):
+        g.release_natural()
+    torch.cuda.empty_cache()
+    y2 = lay.forward(x).clone()
+    torch.cuda.synchronize()
+    assert B.moe_get_device_status() == 0
+    a, b = bits_to_f32(y2.cpu().numpy()), bits_to_f32(y1.cpu().numpy())
+    assert np.abs(a - b).max() <= 1e-2 * np.sqrt((b ** 2).mean())
+    with pytest.raises(B.MoeError):
+        B.moe_expert_ffn(lay.xq_codes[:8], lay.xq_scales[:8], lay.xq_ts[:1], lay.experts, cfg.k, lay.offsets,
+                         lay.sorted_assign[:8 * cfg.k], lay.topk_w[:8], B.MOE_FFN_ACCUMULATE, B.MOE_PATH_PREFILL,
+                         lay.y_acc[:8], None, lay.ws)

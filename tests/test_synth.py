@@ -40,3 +40,15 @@ def test_zipf_bias_is_log_rank_permutation():
     assert not torch.equal(br, br2)
     _, b0 = synth.make_router(0, synth.CONFIGS["wide"])
     assert not b0.any()
+
+
+def test_batched_expert_draws_equal_single_draws():
+    """The batched generator gives, row by row, the bits of the one-expert generator."""
+    cfg = synth.CONFIGS["tiny"]
+    g, u, dn = synth.make_experts_weights_bf16(3, cfg, [0, 5, 7], layer=2)
+    for r, e in enumerate([0, 5, 7]):
+        g1, u1, d1 = synth.make_expert_weights_bf16(3, cfg, e, layer=2)
+        assert torch.equal(g[r], g1) and torch.equal(u[r], u1) and torch.equal(dn[r], d1)
+    gs, us, ds = synth.make_experts_weights_bf16(3, cfg, [0], layer=2, shared=True)
+    g1, u1, d1 = synth.make_expert_weights_bf16(3, cfg, 0, layer=2, shared=True)
+    assert torch.equal(gs[0], g1) and torch.equal(ds[0], d1)
