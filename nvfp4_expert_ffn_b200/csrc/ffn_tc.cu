@@ -85,6 +85,8 @@ struct TcParams {
   ExpertGroup routed, shared;
   int has_shared;
   int E, d, I, T, k, mode;
+  int t0, t1;   // tokens of this call's chunk: [t0, t1)
+  int zero_y;   // accumulate mode: zero out (all T rows) before the chunk
   float* out;
   float* shared_out;
   int32_t* status;
@@ -99,9 +101,28 @@ MOE_DEV void schedule_body(const TcParams& p) {
   const int nslots = p.E + (p.has_shared ? 1 : 0);
   for (int e0 = 0; e0 < nslots; e0 += blockDim.x) {
     const int e = e0 + threadIdx.x;
-    int cnt = 0;
-    if (e < p.E) cnt = p.offsets[e + 1] - p.offsets[e];
-    else if (e < nslots) cnt = p.T;
+    // the expert's rows with tokens in [t0, t1): its assignments are sorted by id a = t*k + j,
+    // so they form one run of its segment, found by two binary searches
+    int cnt = 0, lo = 0;
+    if (e < p.E) {
+      const int s0 = p.offsets[e], s1 = p.offsets[e + 1];
+      auto lower = [&](int key) {
+        int a = s0, b = s1;
+        while (a < b) {
+          const int mid = (a + b) >> 1;
+          if (p.sorted_assign[mid] < key) a = mid + 1;
+          else b = mid;
+        }
+        return a;
+      };
+      lo = p.t0 == 0 ? s0 : lower(p.t0 * p.k);
+      const int hi = p.t1 >= p.T ? s1 : lower(p.t1 * p.k);
+      cnt = hi - lo;
+      lo -= s0;
+    } else if (e < nslots) {
+      cnt = p.t1 - p.t0;
+      lo = p.t0;  // the shared expert's row i is token i
+    }
     const int nm = (cnt + kTileM - 1) / kTileM;
     int total;
     const int base = block_exclusive_scan(nm, tmp, &total) + carry;
@@ -110,7 +131,7 @@ MOE_DEV void schedule_body(const TcParams& p) {
       if (m < p.max_m) {
         p.mt_expert[m] = e;
         p.mt_valid[m] = min(kTileM, cnt - i * kTileM);
-        p.mt_first[m] = i * kTileM;
+        p.mt_first[m] = lo + i * kTileM;
         p.done1[m] = 0;
       }
     }
@@ -127,6 +148,7 @@ __global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
     schedule_body(p);
     return;
   }
+  if (!p.zero_y) return;
   // accumulate mode: y is summed into by the FFN kernel, so it starts at zero
   const size_t n4 = (size_t)p.T * p.d / 4;
   float4* o4 = reinterpret_cast<float4*>(p.out);
@@ -627,35 +649,42 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
 //            quantisation of h in the epilogue, h written into this CTA's shared memory in
 //            the layout the down GEMM reads as its A operand;
 //   down:    d/256 tiles of N = 256 output rows, K = I, A = that h tile; the epilogue adds
-//            w * o into y with bulk reductions (or stores o).
+//            w * o into y with vector reductions from registers (or stores o).
 // The activation scale atoms of the m-tile (K = d) and then those of h (K = I) stay in TMEM
 // for all of the job's tiles, so a K = 64 step needs only the two weight scale copies next to
 // its N = 256 MMA (each tcgen05.cp takes the tensor pipe about as long as a 128-column MMA).
 // One N = 256 accumulator (TMEM has no room for a second one beside the scales): the
-// epilogue takes its columns into registers first and releases it before its own math.
+// epilogue takes its columns into registers first and releases it before its own math; 16
+// epilogue warps (four per TMEM lane quarter, 64 columns each) keep that math short.
+// y of every token the call covers receives about k + 1 reductions; the caller splits the
+// tokens into chunks whose y fits in L2 (launch_ffn_tc).
 constexpr int kMtN = 256;
-constexpr int kMtStages = 2;
+constexpr int kMtStages = 3;
+constexpr int kMtEpiWarps = 16;
+constexpr int kMtThreads = 64 + 32 * kMtEpiWarps;
 constexpr int kMtABytes = kTileM * kStageK / 2;      // 16 KB: gathered activation rows
 constexpr int kMtBBytes = kMtN * kStageK / 2;        // 32 KB: weight rows
 constexpr int kMtSfbBytes = 8 * kAtom;               // 4 KB: two atoms per K = 64 step
 constexpr int kMtStageBytes = kMtABytes + kMtBBytes + kMtSfbBytes;
 constexpr int kMtColSfa = 256, kMtColSfb = 384;      // TMEM columns (accumulator at 0)
 constexpr int kMtMaxD = 2048, kMtMaxI = 768;
+constexpr size_t kMtSmemMax = 226 * 1024;
 constexpr uint32_t kMtIdesc = idesc_mxf4nvf4(kTileM, kMtN);
+constexpr size_t kMtChunkYBytes = 64ull << 20;       // y bytes of one token chunk (L2 is 126 MB)
+constexpr bool kMtPregather = true;  // above 64 tokens: one TMA box of pre-gathered rows per stage
 
 __host__ __device__ inline size_t mt_h_bytes(int I) { return (size_t)(I / kStageK) * kMtABytes; }
 __host__ __device__ inline size_t mt_smem_bytes(int d, int I) {
-  return (size_t)kMtStages * kMtStageBytes + mt_h_bytes(I) + (size_t)(I / 64) * kAtom + (size_t)(d / 64) * kAtom +
-         (size_t)kEpiWarps * kEpiStageBytes + 1024;
+  return (size_t)kMtStages * kMtStageBytes + mt_h_bytes(I) + (size_t)(I / 64) * kAtom + (size_t)(d / 64) * kAtom + 1024;
 }
 
-// trace id of tile `t` (0..nt1-1 gate/up, then down) of this CTA's job `jc` (first 4 jobs only)
+// trace id of tile `t` (0..nt1-1 gate/up, then down) of this CTA's job `jc` (first 2 jobs only)
 #define MT_TRACE(ev, jc, t)                                        \
   do {                                                             \
-    if ((jc) < 4) TC_TRACE_AT(g_tc_trace, ev, (jc) * 64 + (t));    \
+    if ((jc) < 2) TC_TRACE_AT(g_tc_trace, ev, (jc) * 64 + (t));    \
   } while (0)
 
-__global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
+__global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_constant__ TcMaps maps, TcParams p) {
   TC_TRACE_DECL
   MOE_PDL_PROLOGUE();
   TC_TRACE_BEGIN(g_tc_trace);
@@ -671,11 +700,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
   const int d = p.d, I = p.I;
   const int nt1 = I / 128, nt2 = d / kMtN;      // tiles per job
   const int nks1 = d / kStageK, nks2 = I / kStageK;
+  // CTAs that work on the same expert at the same time visit its weight tiles and K stages in
+  // orders rotated by their index, so that they do not all request the same lines from L2 at
+  // once (the sums do not depend on the order)
+  const int rj = blockIdx.x % nt1, rn = blockIdx.x % nt2;
+  const int rk1 = (blockIdx.x / nt1) % nks1, rk2 = (blockIdx.x / nt2) % nks2;
   uint8_t* const ring = smem;
   uint8_t* const htile = smem + (size_t)kMtStages * kMtStageBytes;   // [I/256][128 rows][128 B]
   uint8_t* const hsf = htile + mt_h_bytes(I);                         // [I/64][512]
   uint8_t* const xsf = hsf + (size_t)(I / 64) * kAtom;                // [d/64][512]
-  float* const ystage = reinterpret_cast<float*>(xsf + (size_t)(d / 64) * kAtom);
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < kMtStages; ++st) {
@@ -683,14 +716,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
       mbar_init(&empty[st], 1);
     }
     mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, kEpiWarps);
+    mbar_init(&acc_empty, kMtEpiWarps);
     mbar_init(&sfa_full, 1);
     mbar_init(&sfa_empty, 1);
     mbar_init(&h_ready, 1);
     mbar_init(&final_bar, 1);
     fence_barrier_init();
     s_abort = 0;
-    prefetch_tensormap(&maps.xg);
+    prefetch_tensormap(p.a1 ? &maps.a1 : &maps.xg);
     prefetch_tensormap(&maps.b1);
     prefetch_tensormap(&maps.b2);
   }
@@ -737,17 +770,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
       }
       alive = __shfl_sync(0xffffffffu, alive ? 1 : 0, 0) != 0;
       // gate/up stages: activation rows by gather4, two 64-row gate+up boxes, their scales
-      for (int j = 0; j < nt1 && alive; ++j) {
-        for (int ks = 0; ks < nks1; ++ks, ++it) {
+      for (int jq = 0; jq < nt1 && alive; ++jq) {
+        const int j = (jq + rj) % nt1;
+        for (int kq = 0; kq < nks1; ++kq, ++it) {
+          const int ks = (kq + rk1) % nks1;
           const uint32_t st = it % kMtStages;
           if (!wait_empty(it)) {
             alive = false;
             break;
           }
-          if (ks == 0 && lane == 0) MT_TRACE(kEvProdTile, jc, j);
+          if (kq == 0 && lane == 0) MT_TRACE(kEvProdTile, jc, jq);
           uint8_t* sb = ring + (size_t)st * kMtStageBytes;
           if (lane == 0) {
-            mbar_arrive_expect_tx(&full[st], (uint32_t)(ngather * 512 + kMtBBytes + kMtSfbBytes));
+            mbar_arrive_expect_tx(&full[st], (uint32_t)((p.a1 ? kMtABytes : ngather * 512) + kMtBBytes + kMtSfbBytes));
+            if (p.a1) tma_load_2d(sb, &maps.a1, &full[st], ks * 128, m * kTileM);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
               tma_load_4d(sb + kMtABytes + hh * (kMtBBytes / 2), sh ? &maps.b1s : &maps.b1, &full[st], ks * 128,
@@ -758,20 +794,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
             }
           }
           __syncwarp();
-          if (lane < ngather)
+          if (!p.a1 && lane < ngather)
             tma_gather4(sb + 4 * lane * 128, &maps.xg, &full[st], ks * 128, rowtok[0], rowtok[1], rowtok[2],
                         rowtok[3]);
         }
       }
       // down stages: two 128-row boxes of output rows and their scales
-      for (int n = 0; n < nt2 && alive; ++n) {
-        for (int ks = 0; ks < nks2; ++ks, ++it) {
+      for (int nq = 0; nq < nt2 && alive; ++nq) {
+        const int n = (nq + rn) % nt2;
+        for (int kq = 0; kq < nks2; ++kq, ++it) {
+          const int ks = (kq + rk2) % nks2;
           const uint32_t st = it % kMtStages;
           if (!wait_empty(it)) {
             alive = false;
             break;
           }
-          if (ks == 0 && lane == 0) MT_TRACE(kEvProdTile, jc, nt1 + n);
+          if (kq == 0 && lane == 0) MT_TRACE(kEvProdTile, jc, nt1 + nq);
           uint8_t* sb = ring + (size_t)st * kMtStageBytes;
           if (lane == 0) {
             mbar_arrive_expect_tx(&full[st], (uint32_t)(kMtBBytes + kMtSfbBytes));
@@ -810,11 +848,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
         if (!mbar_wait(&acc_empty, (tc & 1) ^ 1, &s_abort, p.status)) return false;
         tc_fence_after();
         MT_TRACE(kEvMmaSlot, jc, tix);
-        for (int ks = 0; ks < nks; ++ks, ++it) {
+        const int rk = phase1 ? rk1 : rk2;
+        for (int kq = 0; kq < nks; ++kq, ++it) {
+          const int ks = (kq + rk) % nks;  // the producer's order
           const uint32_t st = it % kMtStages;
           if (!mbar_wait(&full[st], (it / kMtStages) & 1, &s_abort, p.status)) return false;
           tc_fence_after();
-          if (ks == 0) MT_TRACE(kEvMmaFirst, jc, tix);
+          if (kq == 0) MT_TRACE(kEvMmaFirst, jc, tix);
           const uint8_t* sb = ring + (size_t)st * kMtStageBytes;
           const uint32_t aB = smem_u32(sb + kMtABytes);
           const uint32_t aA = phase1 ? smem_u32(sb) : smem_u32(htile + (size_t)ks * kMtABytes);
@@ -822,13 +862,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
           const uint32_t sfb = tmem + kMtColSfb + 32 * st;
 #pragma unroll
           for (int kc = 0; kc < 4; ++kc) {
-            tmem_cp_sf(sfb + 8 * kc, sdesc_sf(aS + kAtom * kc));                     // rows 0-127
+            tmem_cp_sf(sfb + 8 * kc, sdesc_sf(aS + kAtom * kc));                        // rows 0-127
             tmem_cp_sf(sfb + 8 * kc + 4, sdesc_sf(aS + kMtSfbBytes / 2 + kAtom * kc));  // rows 128-255
           }
 #pragma unroll
           for (int kc = 0; kc < 4; ++kc)
             mma_mxf4nvf4(tmem, sdesc_sw128(aA + 32 * kc), sdesc_sw128(aB + 32 * kc), kMtIdesc,
-                         tmem + kMtColSfa + 4 * (4 * ks + kc), sfb + 8 * kc, (ks | kc) ? 1u : 0u);
+                         tmem + kMtColSfa + 4 * (4 * ks + kc), sfb + 8 * kc, (kq | kc) ? 1u : 0u);
           mma_commit(&empty[st]);
         }
         mma_commit(&acc_full);
@@ -861,14 +901,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
-    // warp w takes TMEM lane quarter q = w % 4 (m-tile rows 32q..32q+31) and half `half` of the
-    // accumulator's 256 columns. One thread waits; a named barrier publishes its decision.
+    // warp w takes TMEM lane quarter q = w % 4 (m-tile rows 32q..32q+31) and column quarter
+    // cq = (w - 2) / 4: accumulator columns [64cq, 64cq + 64) in the down tiles; in the
+    // gate/up tiles the gate and up columns of 32 h columns (see below). One thread waits; a
+    // named barrier publishes its decision.
     const int ew = warp - 2;
     const int q = warp & 3;
-    const int half = ew >> 2;
+    const int cq = ew >> 2;
     const int row = 32 * q + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
     const float ts_x = *p.xq_ts;
-    float* stage_f = ystage + (size_t)ew * (kEpiStageBytes / 4);
     uint32_t tc = 0, jc = 0;
     bool go = true;
     int tix = 0;
@@ -877,16 +919,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
         s_epi_go[tc & 1] = mbar_wait(&acc_full, tc & 1, &s_abort, p.status) ? 1 : 0;
         MT_TRACE(kEvEpiStart, jc, tix);
       }
-      named_bar_sync(2, 32 * kEpiWarps);
+      named_bar_sync(2, 32 * kMtEpiWarps);
       const bool g = s_epi_go[tc & 1] != 0;
       tc_fence_after();
       return g;
     };
-    // 128 accumulator columns of this thread's row: [128*half, 128*half + 128)
-    auto drain = [&](uint32_t (&v)[4][32]) {
-      const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + 128 * half;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(base + 32 * c, v[c]);
+    // two 32-column groups of this thread's row, at columns c0 and c1
+    auto drain = [&](uint32_t c0, uint32_t c1, uint32_t (&v)[2][32]) {
+      tmem_ld32(lane_base + c0, v[0]);
+      tmem_ld32(lane_base + c1, v[1]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -902,54 +943,51 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
       const ExpertGroup& G = sh ? p.shared : p.routed;
       const bool valid = row < p.mt_valid[m];
       const size_t prow = (size_t)m * kTileM + row;
-      // ---- gate/up tiles: SwiGLU and NVFP4 h into the shared-memory h tile
+      // ---- gate/up tiles: SwiGLU and NVFP4 h into the shared-memory h tile. Tile j holds gate
+      // rows of slice s = 2j + (cq >> 1) at columns 128(cq >> 1) .. +63 and its up rows 64
+      // columns later; this thread takes h columns 32(cq & 1) .. +31 of that slice.
       const float sg = G.gu_ts[2 * eloc] * ts_x, su = G.gu_ts[2 * eloc + 1] * ts_x;
-      for (int j = 0; j < nt1 && go; ++j) {
+      const uint32_t cg = 128 * (cq >> 1) + 32 * (cq & 1);
+      for (int jq = 0; jq < nt1 && go; ++jq) {
+        const int j = (jq + rj) % nt1;
         if (!(go = wait_acc())) break;
-        uint32_t v[4][32];
-        drain(v);
-        // columns [0,64) gate and [64,128) up of h columns 128j + 64*half .. +63
-        uint32_t packed[16];
+        uint32_t v[2][32];
+        drain(cg, cg + 64, v);
+        uint32_t packed[4];
         uint32_t sbytes = 0;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < 2; ++b) {
           float h[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int c = 16 * b + i;
-            const float gv = __uint_as_float(v[c >> 5][c & 31]) * sg;
-            const float uv = __uint_as_float(v[2 + (c >> 5)][c & 31]) * su;
+            const float gv = __uint_as_float(v[0][16 * b + i]) * sg;
+            const float uv = __uint_as_float(v[1][16 * b + i]) * su;
             h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
           }
           uint2 cw;
-          const uint32_t sb = quantize_block16(h, 1.0f, &cw);
-          packed[4 * b] = cw.x;
-          packed[4 * b + 1] = cw.y;
-          sbytes |= sb << (8 * b);
+          sbytes |= quantize_block16(h, 1.0f, &cw) << (8 * b);
+          packed[2 * b] = cw.x;
+          packed[2 * b + 1] = cw.y;
         }
-        if (!valid) {
-#pragma unroll
-          for (int i = 0; i < 16; i += 4) packed[i] = packed[i + 1] = 0u;
-          sbytes = 0u;
-        }
-        // 32 code bytes at h column 128j + 64*half: K stage kt, 16-byte pieces c0, c0 + 1 of
-        // the row (128-byte swizzle: piece c of row r at r*128 + (c ^ (r % 8))*16)
-        const int hc = 128 * j + 64 * half;
+        if (!valid) packed[0] = packed[1] = packed[2] = packed[3] = sbytes = 0u;
+        // 16 code bytes at h column hc: K stage hc / 256, 16-byte piece (hc % 256) / 32 of the
+        // row (128-byte swizzle: piece c of row r at r*128 + (c ^ (r % 8))*16)
+        const int hc = 128 * j + 64 * (cq >> 1) + 32 * (cq & 1);
         uint8_t* hrow = htile + (size_t)(hc / kStageK) * kMtABytes + (size_t)row * 128;
-        const int c0 = (hc % kStageK) / 32;
-        *reinterpret_cast<uint4*>(hrow + ((c0 ^ (row & 7)) * 16)) = make_uint4(packed[0], packed[1], packed[4], packed[5]);
-        *reinterpret_cast<uint4*>(hrow + (((c0 + 1) ^ (row & 7)) * 16)) =
-            make_uint4(packed[8], packed[9], packed[12], packed[13]);
-        *reinterpret_cast<uint32_t*>(hsf + (size_t)(hc / 64) * kAtom + (row % 32) * 16 + (row / 32) * 4) = sbytes;
+        const int pc = (hc % kStageK) / 32;
+        *reinterpret_cast<uint4*>(hrow + ((pc ^ (row & 7)) * 16)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        // the two scale bytes: blocks (hc % 64) / 16 and the next of atom hc / 64
+        *reinterpret_cast<uint16_t*>(hsf + (size_t)(hc / 64) * kAtom + (row % 32) * 16 + (row / 32) * 4 +
+                                     (hc % 64) / 16) = (uint16_t)sbytes;
         if (ew == 0 && lane == 0) MT_TRACE(kEvEpiEnd, jc, tix);
         ++tix;
       }
       if (!go) break;
       // h complete: visible to the tensor core (async proxy), then released to the MMA issuer
       fence_proxy_async_smem();
-      named_bar_sync(2, 32 * kEpiWarps);
+      named_bar_sync(2, 32 * kMtEpiWarps);
       if (ew == 0 && lane == 0) mbar_arrive(&h_ready);
-      // ---- down tiles: w * o added into y (or o stored), 32 columns per bulk operation
+      // ---- down tiles: w * o added into y (or o stored), 64 columns per thread
       const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
       int tok = 0, slot = 0;
       float wgt = 0.0f;
@@ -959,34 +997,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_mt_kernel(const __grid_c
         slot = p.row_slot[prow];
       }
       const float f = p.mode == 0 ? wgt * ts_o : ts_o;
-      for (int n = 0; n < nt2 && go; ++n) {
+      float* dst = p.mode == 0 ? p.out + (size_t)tok * d
+                               : (sh ? p.shared_out + (size_t)tok * d : p.out + (size_t)slot * d);
+      for (int nq = 0; nq < nt2 && go; ++nq) {
+        const int n = (nq + rn) % nt2;
         if (!(go = wait_acc())) break;
-        uint32_t v[4][32];
-        drain(v);
+        uint32_t v[2][32];
+        drain(64 * cq, 64 * cq + 32, v);
+        if (valid) {
+          float* o = dst + kMtN * n + 64 * cq;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          bulk_wait_read<0>();  // the staging row of the previous chunk has been read
-          __syncwarp();
-          float4* rowp = reinterpret_cast<float4*>(stage_f + kEpiRowFloats * lane);
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            rowp[i] = make_float4(__uint_as_float(v[c][4 * i]) * f, __uint_as_float(v[c][4 * i + 1]) * f,
-                                  __uint_as_float(v[c][4 * i + 2]) * f, __uint_as_float(v[c][4 * i + 3]) * f);
-          fence_proxy_async_smem();
-          if (valid) {
-            const int n0 = kMtN * n + 128 * half + 32 * c;
-            if (p.mode == 0)
-              bulk_reduce_add_f32(p.out + (size_t)tok * d + n0, rowp, 128);
-            else
-              bulk_s2g((sh ? p.shared_out + (size_t)tok * d : p.out + (size_t)slot * d) + n0, rowp, 128);
-          }
-          bulk_commit();
+            for (int i = 0; i < 8; ++i) {
+              const float a0 = __uint_as_float(v[c][4 * i]) * f, a1 = __uint_as_float(v[c][4 * i + 1]) * f;
+              const float a2 = __uint_as_float(v[c][4 * i + 2]) * f, a3 = __uint_as_float(v[c][4 * i + 3]) * f;
+              if (p.mode == 0)
+                red_add_v4(o + 32 * c + 4 * i, a0, a1, a2, a3);
+              else
+                *reinterpret_cast<float4*>(o + 32 * c + 4 * i) = make_float4(a0, a1, a2, a3);
+            }
         }
         if (ew == 0 && lane == 0) MT_TRACE(kEvEpiEnd, jc, tix);
         ++tix;
       }
     }
-    bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -1009,7 +1044,9 @@ struct TcLayout {
       off_sfa2, total;
 };
 
-bool mt_supported(int d, int I) { return d <= kMtMaxD && I <= kMtMaxI && d % kStageK == 0 && I % kStageK == 0; }
+bool mt_supported(int d, int I) {
+  return d <= kMtMaxD && I <= kMtMaxI && d % kStageK == 0 && I % kStageK == 0 && mt_smem_bytes(d, I) <= kMtSmemMax;
+}
 
 TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   TcLayout L;
@@ -1029,7 +1066,7 @@ TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   // rows' scale atoms (every T)
   const bool mt = mt_supported(d, I);
   const bool big = T > kSmallT;
-  L.off_a1 = o; o += (big && !mt) ? a256(L.rows_cap * (d / 2)) : 0;
+  L.off_a1 = o; o += (big && (!mt || kMtPregather)) ? a256(L.rows_cap * (d / 2)) : 0;
   L.off_sfa1 = o; o += (big || mt) ? a256(L.rows_cap * (d / kBlock)) : 0;
   L.off_h = o; o += a256(L.rows_cap * (I / 2));
   L.off_sfa2 = o; o += a256(L.rows_cap * (I / kBlock));
@@ -1053,8 +1090,7 @@ cudaError_t set_wait_limit_ffn_tc(unsigned long long ns) { return set_wait_limit
 cudaError_t init_ffn_tc_attributes() {
   cudaError_t e = cudaFuncSetAttribute(tc_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ffn_tc_smem_bytes());
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(tc_ffn_mt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)mt_smem_bytes(kMtMaxD, kMtMaxI));
+  return cudaFuncSetAttribute(tc_ffn_mt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMtSmemMax);
 }
 
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t, int num_sms,
@@ -1080,7 +1116,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.row_weight = reinterpret_cast<float*>(w + L.off_w);
   p.row_slot = reinterpret_cast<int32_t*>(w + L.off_slot);
   const bool mt = mt_supported(a.d, a.I);
-  p.a1 = (a.T > kSmallT && !mt) ? w + L.off_a1 : nullptr;
+  p.a1 = (a.T > kSmallT && (!mt || kMtPregather)) ? w + L.off_a1 : nullptr;
   p.sfa1 = (a.T > kSmallT || mt) ? w + L.off_sfa1 : nullptr;
   p.h_codes = w + L.off_h;
   p.sfa2 = w + L.off_sfa2;
@@ -1095,6 +1131,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.shared = a.shared;
   p.has_shared = a.has_shared;
   p.E = a.E; p.d = a.d; p.I = a.I; p.T = a.T; p.k = a.k; p.mode = a.mode;
+  p.t0 = 0;
+  p.t1 = a.T;
+  p.zero_y = a.mode == 0 ? 1 : 0;
   p.out = a.out;
   p.shared_out = a.shared_out;
   p.status = status;
@@ -1146,13 +1185,24 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     zc = (int)((n4 + 4095) / 4096);
     if (zc > num_sms) zc = num_sms;
   }
-  if ((e = launch_pdl(tc_schedule_kernel, dim3(1 + zc), dim3(1024), 0, st, p)) != cudaSuccess) return e;
-  if (mt) {
-    // the rows' tokens, weights, output slots and scale atoms, then one job per m-tile
-    if ((e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess) return e;
-    return launch_pdl(tc_ffn_mt_kernel, dim3(num_sms), dim3(kTcThreads), mt_smem_bytes(a.d, a.I), st, maps, p);
+  // m-tile kernel: token chunks whose accumulate-mode y fits in L2 next to the streamed
+  // weights. Each chunk: m-tiles over the chunk's rows (the first launch also zeroes y), the
+  // rows' tokens, weights, output slots and scale atoms, then one job per m-tile.
+  const size_t ybytes = (size_t)a.T * a.d * sizeof(float);
+  const int nchunk = (mt && a.mode == 0) ? (int)((ybytes + kMtChunkYBytes - 1) / kMtChunkYBytes) : 1;
+  for (int c = 0; c < nchunk; ++c) {
+    p.t0 = (int)((int64_t)a.T * c / nchunk);
+    p.t1 = (int)((int64_t)a.T * (c + 1) / nchunk);
+    p.zero_y = (c == 0 && a.mode == 0) ? 1 : 0;
+    if ((e = launch_pdl(tc_schedule_kernel, dim3(c == 0 ? 1 + zc : 1), dim3(1024), 0, st, p)) != cudaSuccess) return e;
+    if (!mt) break;
+    if ((e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess) return e;
+    if ((e = launch_pdl(tc_ffn_mt_kernel, dim3(num_sms), dim3(kMtThreads), mt_smem_bytes(a.d, a.I), st, maps, p)) !=
+        cudaSuccess)
+      return e;
   }
-  if (p.a1 && (e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 4), dim3(256), 0, st, p)) != cudaSuccess)
+  if (mt) return cudaSuccess;
+  if (p.a1 && (e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess)
     return e;
   return launch_pdl(tc_ffn_kernel, dim3(num_sms), dim3(kTcThreads), ffn_tc_smem_bytes(), st, maps, p);
 }

@@ -21,10 +21,11 @@
 //   phase 3  the units (expert, 64-column slice of I), adding into y_acc.
 //   barrier
 //   phase 4  CTA t < T converts row t of y_acc to bf16 (optionally RMS-renormalised).
-// The grid barrier counts arrivals in a workspace word that must be zero before the first
-// call; every call leaves it at a multiple of the grid size. A CTA that gives up at a
-// bounded wait marks the workspace (a second word), since the counter may then be left
-// between multiples; later calls on a marked workspace do nothing but report
+// The grid barrier counts arrivals in eight workspace words (CTA b arrives on word b % 8, so
+// that 147 arrivals do not queue on one address) that must be zero before the first call;
+// every call leaves each word at a multiple of the number of CTAs that arrive on it. A CTA
+// that gives up at a bounded wait marks the workspace (another word), since the counters may
+// then be left between multiples; later calls on a marked workspace do nothing but report
 // MOE_ERR_WORKSPACE until the caller zeroes it. The launch is cooperative: it fails rather
 // than start a grid whose CTAs cannot all be resident, so the barrier cannot wait on a CTA
 // that has not started.
@@ -64,42 +65,56 @@ struct LayerArgs {
   uint16_t* y;         // [T][d] bf16
   // workspace
   float* logits;       // [T][E]
-  unsigned long long* sync;  // arrival counter of the grid barrier (zero before the first call)
+  unsigned long long* sync;  // arrival counters of the grid barrier (zero before the first call)
   unsigned int* poison;      // nonzero once a call on this workspace gave up at a bounded wait
   int32_t* status;
 };
 
-// Grid-wide barrier on a 64-bit arrival counter that only grows: thread 0 of each CTA adds
-// one and waits (bounded) until the count reaches the next multiple of the grid size. The
-// counter starts at zero and every call adds two multiples, so it stays aligned. Writes
+// Grid-wide barrier on eight 64-bit arrival counters that only grow (kBarStripes words,
+// kBarStride words apart): thread 0 of CTA b adds one to counter b % 8, which gives the
+// barrier's generation g (its old value over the number of CTAs of that counter), then
+// waits (bounded) until every counter s holds (g + 1) times the number of its CTAs. The
+// counters start at zero and every call adds two generations, so they stay aligned. Writes
 // before the arrival are visible to every CTA after the wait; the CTA may work between the
 // two halves.
-//
-// Arrival (every thread calls it): returns, in thread 0, the count to wait for (0 if the
+constexpr int kBarStripes = 8, kBarStride = 16;  // 16 words = one 128-byte line per counter
+
+MOE_DEV unsigned long long stripe_ctas(int s) { return (gridDim.x - s + kBarStripes - 1) / kBarStripes; }
+
+// Arrival (every thread calls it): returns, in thread 0, the generation to wait for (0 if the
 // kernel is aborting and did not arrive).
 MOE_DEV unsigned long long grid_arrive(unsigned long long* count, volatile int* abort) {
   __syncthreads();
   unsigned long long target = 0;
   if (threadIdx.x == 0 && !*abort) {
-    const unsigned long long G = gridDim.x;
+    const int s = blockIdx.x % kBarStripes;
     __threadfence();
-    const unsigned long long old = atomicAdd(count, 1ull);
-    target = (old / G + 1) * G;
+    const unsigned long long old = atomicAdd(count + kBarStride * s, 1ull);
+    target = old / stripe_ctas(s) + 1;
   }
   return target;
 }
 
-// Wait (every thread calls it, thread 0 with the arrival's target): false after an abort or
-// a timeout.
+// Wait (every thread calls it, thread 0 with the arrival's generation): false after an abort
+// or a timeout.
 MOE_DEV bool grid_wait(unsigned long long* count, unsigned long long target, volatile int* abort, int32_t* status) {
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
     int ok = target != 0 && !*abort ? 1 : 0;
     const uint64_t t0 = globaltimer_ns();
-    while (ok) {
+    int s = 0;  // the first counter not yet seen at its target
+    while (ok && s < kBarStripes) {
+      const unsigned long long need = stripe_ctas(s);
+      if (need == 0) {
+        ++s;
+        continue;
+      }
       unsigned long long c;
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count) : "memory");
-      if (c >= target) break;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count + kBarStride * s) : "memory");
+      if (c >= target * need) {
+        ++s;
+        continue;
+      }
       if (*abort) {
         ok = 0;
       } else if (globaltimer_ns() - t0 > wait_limit_ns()) {
@@ -579,7 +594,9 @@ size_t a256l(size_t v) { return (v + 255) & ~(size_t)255; }
 int layer_grid(int num_sms) { return num_sms > 1 ? num_sms - 1 : 1; }
 }  // namespace
 
-size_t layer_dec_ws_bytes(int64_t T, int E) { return 256 + a256l((size_t)T * E * 4); }
+// workspace: the barrier counters (one 128-byte line each) and the mark, then the logits
+constexpr size_t kLayerWsHeader = 2048, kLayerWsPoison = 1024;
+size_t layer_dec_ws_bytes(int64_t T, int E) { return kLayerWsHeader + a256l((size_t)T * E * 4); }
 
 bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms) {
   const int G = layer_grid(num_sms);
@@ -624,8 +641,8 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
   p.y_acc = a.y_acc;
   p.y = a.y;
   p.sync = reinterpret_cast<unsigned long long*>(w);
-  p.poison = reinterpret_cast<unsigned int*>(w + 8);
-  p.logits = reinterpret_cast<float*>(w + 256);
+  p.poison = reinterpret_cast<unsigned int*>(w + kLayerWsPoison);
+  p.logits = reinterpret_cast<float*>(w + kLayerWsHeader);
   p.status = status;
   return launch_pdl_coop(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st,
                          p);

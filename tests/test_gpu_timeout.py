@@ -1,10 +1,10 @@
 """A bounded device-side wait that runs out, and recovery afterwards (the one-kernel decode
 layer's grid barrier).
 
-The wait limit is shortened to 5 ms and the barrier's arrival counter in the workspace is
-moved one past a multiple of the grid size, so the last CTA to arrive at the first barrier
-waits for arrivals that never come: its wait gives up, sets the device status to
-MOE_ERR_TIMEOUT and marks the workspace. Every access stays inside its buffers and every
+The wait limit is shortened to 5 ms and the first of the barrier's arrival counters in the
+workspace is moved one past a whole generation, so the last CTA to arrive on it at the first
+barrier counts itself into the next generation and waits for arrivals that never come: its
+wait gives up, sets the device status to MOE_ERR_TIMEOUT and marks the workspace. Every access stays inside its buffers and every
 wait is bounded, so the GPU context stays usable. The next call on the marked workspace does
 nothing and reports MOE_ERR_WORKSPACE; after the caller zeroes the workspace the layer gives
 its normal result again.
@@ -18,6 +18,7 @@ from nvfp4_expert_ffn_b200 import layer as L
 from nvfp4_expert_ffn_b200 import synth
 
 from helpers import bits_to_f32
+from test_gpu_layer import barrier_generations
 
 pytestmark = pytest.mark.gpu
 
@@ -33,11 +34,10 @@ def test_decode_layer_wait_runs_out_then_recovers():
     y0 = lay.forward(x).clone()
     assert B.moe_get_device_status(clear=True) == 0
     counter = lay.ws_dec[:8].view(torch.int64)
-    grid = torch.cuda.get_device_properties(0).multi_processor_count - 1
-    assert int(counter[0]) % grid == 0
+    assert None not in barrier_generations(lay.ws_dec)
     B.moe_set_wait_limit_ns(5_000_000)
     try:
-        counter += 1  # one arrival too many: a multiple of the grid size is never reached again
+        counter += 1  # one arrival too many on the first counter: its next generation never completes
         lay.forward(x)
         assert B.moe_get_device_status(clear=True) == B.MOE_ERR_TIMEOUT
         # the workspace is marked: the next call computes nothing and says so
@@ -53,7 +53,8 @@ def test_decode_layer_wait_runs_out_then_recovers():
         assert B.moe_get_device_status(clear=True) == 0
         a, b = bits_to_f32(y.cpu().numpy()), bits_to_f32(y0.cpu().numpy())
         assert np.abs(a - b).max() <= 1e-2 * np.sqrt((b ** 2).mean())
-        assert int(counter[0]) % grid == 0
+        gens = barrier_generations(lay.ws_dec)
+        assert gens[0] is not None and all(g == gens[0] for g in gens)
     finally:
         B.moe_set_wait_limit_ns(B.DEFAULT_WAIT_LIMIT_NS)
 
