@@ -85,8 +85,6 @@ struct TcParams {
   ExpertGroup routed, shared;
   int has_shared;
   int E, d, I, T, k, mode;
-  int t0, t1;   // tokens of this call's chunk: [t0, t1)
-  int zero_y;   // accumulate mode: zero out (all T rows) before the chunk
   float* out;
   float* shared_out;
   int32_t* status;
@@ -101,28 +99,9 @@ MOE_DEV void schedule_body(const TcParams& p) {
   const int nslots = p.E + (p.has_shared ? 1 : 0);
   for (int e0 = 0; e0 < nslots; e0 += blockDim.x) {
     const int e = e0 + threadIdx.x;
-    // the expert's rows with tokens in [t0, t1): its assignments are sorted by id a = t*k + j,
-    // so they form one run of its segment, found by two binary searches
-    int cnt = 0, lo = 0;
-    if (e < p.E) {
-      const int s0 = p.offsets[e], s1 = p.offsets[e + 1];
-      auto lower = [&](int key) {
-        int a = s0, b = s1;
-        while (a < b) {
-          const int mid = (a + b) >> 1;
-          if (p.sorted_assign[mid] < key) a = mid + 1;
-          else b = mid;
-        }
-        return a;
-      };
-      lo = p.t0 == 0 ? s0 : lower(p.t0 * p.k);
-      const int hi = p.t1 >= p.T ? s1 : lower(p.t1 * p.k);
-      cnt = hi - lo;
-      lo -= s0;
-    } else if (e < nslots) {
-      cnt = p.t1 - p.t0;
-      lo = p.t0;  // the shared expert's row i is token i
-    }
+    int cnt = 0;
+    if (e < p.E) cnt = p.offsets[e + 1] - p.offsets[e];
+    else if (e < nslots) cnt = p.T;
     const int nm = (cnt + kTileM - 1) / kTileM;
     int total;
     const int base = block_exclusive_scan(nm, tmp, &total) + carry;
@@ -131,7 +110,7 @@ MOE_DEV void schedule_body(const TcParams& p) {
       if (m < p.max_m) {
         p.mt_expert[m] = e;
         p.mt_valid[m] = min(kTileM, cnt - i * kTileM);
-        p.mt_first[m] = lo + i * kTileM;
+        p.mt_first[m] = i * kTileM;
         p.done1[m] = 0;
       }
     }
@@ -148,7 +127,6 @@ __global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
     schedule_body(p);
     return;
   }
-  if (!p.zero_y) return;
   // accumulate mode: y is summed into by the FFN kernel, so it starts at zero
   const size_t n4 = (size_t)p.T * p.d / 4;
   float4* o4 = reinterpret_cast<float4*>(p.out);
@@ -670,7 +648,6 @@ constexpr int kMtColSfa = 256, kMtColSfb = 384;      // TMEM columns (accumulato
 constexpr int kMtMaxD = 2048, kMtMaxI = 768;
 constexpr size_t kMtSmemMax = 226 * 1024;
 constexpr uint32_t kMtIdesc = idesc_mxf4nvf4(kTileM, kMtN);
-constexpr size_t kMtChunkYBytes = 64ull << 20;       // y bytes of one token chunk (L2 is 126 MB)
 constexpr bool kMtPregather = true;  // above 64 tokens: one TMA box of pre-gathered rows per stage
 
 __host__ __device__ inline size_t mt_h_bytes(int I) { return (size_t)(I / kStageK) * kMtABytes; }
@@ -1131,9 +1108,6 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.shared = a.shared;
   p.has_shared = a.has_shared;
   p.E = a.E; p.d = a.d; p.I = a.I; p.T = a.T; p.k = a.k; p.mode = a.mode;
-  p.t0 = 0;
-  p.t1 = a.T;
-  p.zero_y = a.mode == 0 ? 1 : 0;
   p.out = a.out;
   p.shared_out = a.shared_out;
   p.status = status;
@@ -1185,23 +1159,12 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     zc = (int)((n4 + 4095) / 4096);
     if (zc > num_sms) zc = num_sms;
   }
-  // m-tile kernel: token chunks whose accumulate-mode y fits in L2 next to the streamed
-  // weights. Each chunk: m-tiles over the chunk's rows (the first launch also zeroes y), the
-  // rows' tokens, weights, output slots and scale atoms, then one job per m-tile.
-  const size_t ybytes = (size_t)a.T * a.d * sizeof(float);
-  const int nchunk = (mt && a.mode == 0) ? (int)((ybytes + kMtChunkYBytes - 1) / kMtChunkYBytes) : 1;
-  for (int c = 0; c < nchunk; ++c) {
-    p.t0 = (int)((int64_t)a.T * c / nchunk);
-    p.t1 = (int)((int64_t)a.T * (c + 1) / nchunk);
-    p.zero_y = (c == 0 && a.mode == 0) ? 1 : 0;
-    if ((e = launch_pdl(tc_schedule_kernel, dim3(c == 0 ? 1 + zc : 1), dim3(1024), 0, st, p)) != cudaSuccess) return e;
-    if (!mt) break;
+  if ((e = launch_pdl(tc_schedule_kernel, dim3(1 + zc), dim3(1024), 0, st, p)) != cudaSuccess) return e;
+  if (mt) {
+    // m-tile kernel: rows gathered once per m-tile, then one job per m-tile
     if ((e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess) return e;
-    if ((e = launch_pdl(tc_ffn_mt_kernel, dim3(num_sms), dim3(kMtThreads), mt_smem_bytes(a.d, a.I), st, maps, p)) !=
-        cudaSuccess)
-      return e;
+    return launch_pdl(tc_ffn_mt_kernel, dim3(num_sms), dim3(kMtThreads), mt_smem_bytes(a.d, a.I), st, maps, p);
   }
-  if (mt) return cudaSuccess;
   if (p.a1 && (e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess)
     return e;
   return launch_pdl(tc_ffn_kernel, dim3(num_sms), dim3(kTcThreads), ffn_tc_smem_bytes(), st, maps, p);

@@ -65,56 +65,42 @@ struct LayerArgs {
   uint16_t* y;         // [T][d] bf16
   // workspace
   float* logits;       // [T][E]
-  unsigned long long* sync;  // arrival counters of the grid barrier (zero before the first call)
+  unsigned long long* sync;  // arrival counter of the grid barrier (zero before the first call)
   unsigned int* poison;      // nonzero once a call on this workspace gave up at a bounded wait
   int32_t* status;
 };
 
-// Grid-wide barrier on eight 64-bit arrival counters that only grow (kBarStripes words,
-// kBarStride words apart): thread 0 of CTA b adds one to counter b % 8, which gives the
-// barrier's generation g (its old value over the number of CTAs of that counter), then
-// waits (bounded) until every counter s holds (g + 1) times the number of its CTAs. The
-// counters start at zero and every call adds two generations, so they stay aligned. Writes
+// Grid-wide barrier on a 64-bit arrival counter that only grows: thread 0 of each CTA adds
+// one and waits (bounded) until the count reaches the next multiple of the grid size. The
+// counter starts at zero and every call adds two multiples, so it stays aligned. Writes
 // before the arrival are visible to every CTA after the wait; the CTA may work between the
 // two halves.
-constexpr int kBarStripes = 8, kBarStride = 16;  // 16 words = one 128-byte line per counter
-
-MOE_DEV unsigned long long stripe_ctas(int s) { return (gridDim.x - s + kBarStripes - 1) / kBarStripes; }
-
-// Arrival (every thread calls it): returns, in thread 0, the generation to wait for (0 if the
+//
+// Arrival (every thread calls it): returns, in thread 0, the count to wait for (0 if the
 // kernel is aborting and did not arrive).
 MOE_DEV unsigned long long grid_arrive(unsigned long long* count, volatile int* abort) {
   __syncthreads();
   unsigned long long target = 0;
   if (threadIdx.x == 0 && !*abort) {
-    const int s = blockIdx.x % kBarStripes;
+    const unsigned long long G = gridDim.x;
     __threadfence();
-    const unsigned long long old = atomicAdd(count + kBarStride * s, 1ull);
-    target = old / stripe_ctas(s) + 1;
+    const unsigned long long old = atomicAdd(count, 1ull);
+    target = (old / G + 1) * G;
   }
   return target;
 }
 
-// Wait (every thread calls it, thread 0 with the arrival's generation): false after an abort
-// or a timeout.
+// Wait (every thread calls it, thread 0 with the arrival's target): false after an abort or
+// a timeout.
 MOE_DEV bool grid_wait(unsigned long long* count, unsigned long long target, volatile int* abort, int32_t* status) {
   __shared__ int s_ok;
   if (threadIdx.x == 0) {
     int ok = target != 0 && !*abort ? 1 : 0;
     const uint64_t t0 = globaltimer_ns();
-    int s = 0;  // the first counter not yet seen at its target
-    while (ok && s < kBarStripes) {
-      const unsigned long long need = stripe_ctas(s);
-      if (need == 0) {
-        ++s;
-        continue;
-      }
+    while (ok) {
       unsigned long long c;
-      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count + kBarStride * s) : "memory");
-      if (c >= target * need) {
-        ++s;
-        continue;
-      }
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(c) : "l"(count) : "memory");
+      if (c >= target) break;
       if (*abort) {
         ok = 0;
       } else if (globaltimer_ns() - t0 > wait_limit_ns()) {
