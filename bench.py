@@ -229,7 +229,33 @@ def algorithmic_bytes(cfg, U: int, T: int) -> float:
             + T * cfg.d * (2 + 0.5625 + 4 + 2))
 
 
-def measure_decode(timer, cfg, copies, xs, T, K, W, e2e_steps, stream, world, peaks):
+def hot_tier_on(layers, n_layers_sharing: int, stream):
+    """Give every layer a hot tier of as many experts as this process's L2 set-aside holds
+    for n_layers_sharing layers, ranked by each layer's routing so far. Returns the tier's
+    description (n_hot 0 when the set-aside holds less than one expert per layer)."""
+    from nvfp4_expert_ffn_b200 import binding as B
+    lay0 = layers[0]
+    setaside = B.moe_set_l2_persisting(1 << 40)
+    per_expert = B.dec_pack_bytes(1, lay0.d, lay0.I)
+    n_hot = int(setaside // (n_layers_sharing * per_expert))
+    with torch.cuda.stream(stream):
+        for lay in layers:
+            lay.update_hot_tier(n_hot, stream=stream)
+    torch.cuda.synchronize()
+    return {"n_hot_per_layer": n_hot, "l2_setaside_bytes": setaside, "expert_bytes": per_expert,
+            "ranking": "each layer's cumulative routing counts (moe_expert_hist)"}
+
+
+def hot_tier_off(layers, stream):
+    from nvfp4_expert_ffn_b200 import binding as B
+    with torch.cuda.stream(stream):
+        for lay in layers:
+            lay.update_hot_tier(0, stream=stream)
+    torch.cuda.synchronize()
+    B.moe_set_l2_persisting(0)
+
+
+def measure_decode(timer, cfg, copies, xs, T, K, W, e2e_steps, stream, world, peaks, hot=False):
     from nvfp4_expert_ffn_b200 import binding as B
     n = len(copies)
     cycle = n * X_DRAWS
@@ -262,6 +288,7 @@ def measure_decode(timer, cfg, copies, xs, T, K, W, e2e_steps, stream, world, pe
             U.append(int((copies[i % n].counts > 0).sum().item()))
     Ui = [U[i % cycle] for i in range(K)]
     bytes_k = [algorithmic_bytes(cfg, u, T) for u in Ui]
+    tier = hot_tier_on(copies, n, stream) if hot else None
     warm, _ = timer.plan(step, W, cycle, finish)
     main, lps = timer.plan(step, K, cycle, finish)
     kplan, _ = timer.plan(kernel, K, cycle) if fused else (None, 0)
@@ -312,6 +339,9 @@ def measure_decode(timer, cfg, copies, xs, T, K, W, e2e_steps, stream, world, pe
                       "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2,
                       "steps": e2e_steps, "api": "GraphedMoeLayer.run: pinned x -> device, layer, y -> pinned"}
         del runners
+    if tier is not None:
+        out["hot_tier"] = tier
+        hot_tier_off(copies, stream)
     return out
 
 
@@ -404,6 +434,9 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
                       "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2,
                       "steps": e2e_steps, "api": "GraphedMoeLayer.run: pinned x -> device, layer, y -> pinned"}
         del runners
+    if tier is not None:
+        out["hot_tier"] = tier
+        hot_tier_off(copies, stream)
     return out
 
 
@@ -428,11 +461,16 @@ def build_stack(device, n_layers: int = 48, epochs: int = 4, n_x: int = 64):
     return cfg, layers, biases, xs
 
 
-def measure_stack(timer, cfg, layers, biases, xs, K, W, stream, world, peaks):
+def measure_stack(timer, cfg, layers, biases, xs, K, W, stream, world, peaks, hot=False):
     """Step = 8 tokens through every layer (RMS renormalisation between layers); step s uses
-    input draw s % len(xs) and the router biases of epoch (s // 64) % epochs."""
+    input draw s % len(xs) and the router biases of epoch (s // 64) % epochs. With hot=True
+    every layer keeps a hot tier in L2 that follows the drift: at the start of each epoch the
+    layers' routing counts restart, and after its first 8 steps each layer's tier is refilled
+    with its most-routed experts of those steps (inside the timed region)."""
     n_ep = len(biases[0])
     x_in = torch.empty_like(xs[0])
+    tier = hot_tier_on(layers, len(layers), stream) if hot else None
+    n_hot = tier["n_hot_per_layer"] if tier else 0
     graphs = []
     for ep in range(n_ep):
         for lay, b in zip(layers, biases):
@@ -456,6 +494,12 @@ def measure_stack(timer, cfg, layers, biases, xs, K, W, stream, world, peaks):
 
     def run(n, s0=0):
         for s in range(s0, s0 + n):
+            if n_hot > 0 and s % 64 == 0:
+                for lay in layers:
+                    lay.cum.zero_()
+            elif n_hot > 0 and s % 64 == 8:
+                for lay in layers:
+                    lay.update_hot_tier(n_hot, stream=stream)
             x_in.copy_(xs[s % len(xs)], non_blocking=True)
             graphs[(s // 64) % n_ep][0].replay()
 
@@ -484,7 +528,10 @@ def measure_stack(timer, cfg, layers, biases, xs, K, W, stream, world, peaks):
     per_layer_bytes = float(np.mean([algorithmic_bytes(cfg, u, 8) for u in U]))
     step_bytes = per_layer_bytes * len(layers)
     ach = step_bytes / (ms / K * 1e-3) / 1e9
+    if tier is not None:
+        hot_tier_off(layers, stream)
     return {"value": round(whole_job_rate(world, 8, K, ms), 1), "unit": "tokens/s", "ms_per_step": round(ms / K, 6),
+            "hot_tier": tier,
             "steps": K, "T": 8, "layers": len(layers), "touched_experts_avg": round(float(np.mean(U)), 2),
             "gpu_launches": int(round(lps * K)), "gpu_launches_per_step": lps,
             "roofline": {"kernel": "whole step: 48 x (layer_dec_kernel + hist_kernel)", "bound": "hbm",
@@ -538,6 +585,9 @@ def run_gpu(args):
                 if Tx != T:
                     extra[f"decode_T{Tx}"] = measure_decode(timer, cfg, copies, xs, Tx, K, W, e2e_steps, stream,
                                                             world, peaks)
+            if not args.no_hot:
+                extra[f"decode_T{T}_hot_tier"] = measure_decode(timer, cfg, copies, xs, T, K, W, 0, stream, world,
+                                                                peaks, hot=True)
             pcfg, players, pxs = build_prefill_layers(device, "prefill", copies, 2)
             extra["prefill_T16384"] = measure_prefill(timer, pcfg, players, pxs, K, W, e2e_steps, stream, world,
                                                       peaks)
@@ -551,6 +601,9 @@ def run_gpu(args):
                 scfg, slayers, sbiases, sxs = build_stack(device)
                 extra["stack48"] = measure_stack(timer, scfg, slayers, sbiases, sxs, 256, max(W, 8), stream, world,
                                                  peaks)
+                if not args.no_hot:
+                    extra["stack48_hot_tier"] = measure_stack(timer, scfg, slayers, sbiases, sxs, 256, max(W, 8),
+                                                              stream, world, peaks, hot=True)
                 del slayers
     elif args.workload == "stack48":
         T = 8
@@ -691,6 +744,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--T", type=int, default=0, help="decode tokens per step (default 8)")
     ap.add_argument("--workload", choices=["decode", "prefill", "wide", "stack48"], default="decode")
+    ap.add_argument("--no-hot", action="store_true", help="skip the hot-tier (L2 persisting) measurements")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-steps", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -100,6 +100,14 @@ typedef struct moe_expert_weights {
   const uint8_t* gu_sf_tiled;
   const uint8_t* dn_sf_tiled;
   const uint8_t* dec_pack;
+  /* Optional hot tier of the group (NULL, NULL, 0 for none), read by moe_layer_decode:
+   * hot_pack holds copies of n_hot experts' decode-pack units, [n_hot][I/64][d/256 +
+   * d/512][18432] (slot s: the same bytes as expert hot_slot^-1(s)'s dec_pack rows), and
+   * hot_slot int32 [E] (device) the slot of each expert, or -1. moe_hot_tier_update fills
+   * both. */
+  const uint8_t* hot_pack;
+  const int32_t* hot_slot;
+  int32_t n_hot;
 } moe_expert_weights_t;
 
 typedef struct moe_experts {
@@ -246,15 +254,18 @@ moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const floa
  *   topk_w [T][k]; counts [E], offsets [E+1], sorted_assign [T*k], assign_pos [T*k];
  *   y_acc float32 [T][d] (the unrounded output); y_bf16 [T][d]; rms_renorm as moe_combine.
  *   ws: moe_workspace_size(MOE_OP_LAYER_DECODE, ...) bytes, zero-filled before the first
- *   call. It holds the arrival counter of the kernel's grid-wide barrier, which every call
- *   leaves at a multiple of the grid size, and a mark that a CTA sets when it gives up at a
- *   bounded wait (moe_get_device_status then reports MOE_ERR_TIMEOUT). A call that finds the
- *   mark set computes nothing, writes no output and sets the device status to
+ *   call. Its first 2048 bytes are a header: at byte 0 the 64-bit arrival count of the
+ *   kernel's grid-wide barrier and of its final done count, which every call leaves at a
+ *   multiple of the grid size; at byte 1024 a mark that a CTA sets when it gives up at a
+ *   bounded wait (moe_get_device_status then reports MOE_ERR_TIMEOUT); at byte 1536 a word
+ *   the library never writes: while it is nonzero, CTA 0 holds back its barrier arrival, so
+ *   the other CTAs' bounded waits run out (tests use it to exercise that path). A call that
+ *   finds the mark set computes nothing, writes no output and sets the device status to
  *   MOE_ERR_WORKSPACE; zero the workspace again to recover.
  * Limits: 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, k <= E <= 1024,
  * and at most 32 units per CTA in the worst case ((min(T*k, E) + shared) * I/64 units over
  * all SMs but one); otherwise MOE_ERR_UNSUPPORTED_SHAPE.
- * The kernel uses all SMs but one and waits at grid-wide barriers. It is launched as a
+ * The kernel uses all SMs but one and waits at a grid-wide barrier. It is launched as a
  * cooperative grid, so the launch fails (MOE_ERR_CUDA) rather than start when its CTAs cannot
  * all be resident; while it runs, other kernels on the GPU get one SM.
  */
@@ -276,6 +287,35 @@ moe_status moe_layer_decode(const uint16_t* x_bf16, int32_t T, const float* ts_i
  */
 moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32_t* rank_out,
                            int32_t reset, void* stream);
+
+/*
+ * moe_hot_tier_update - puts the top-ranked experts of a group into its hot tier. Source:
+ * "Basalt" project page, section "Expert tiers" (the busiest experts are kept in the
+ * fastest memory and the tiers follow the conversation as it shifts) and its FAQ "Can it
+ * use a second GPU or system RAM?". On one B200 every expert is in HBM; the fastest tier
+ * is the L2 cache, so the hot tier is a compact copy of the hot experts' decode-pack units
+ * that moe_layer_decode reads instead of dec_pack and marks as persisting in L2 for its
+ * launch (an access-policy window; see moe_set_l2_persisting for the set-aside it uses).
+ *   W: the group, with its decode pack; rank int32 [E] device: expert ids from most to
+ *   least routed (moe_expert_hist's rank_out); n_hot in [0, E];
+ *   hot_pack: n_hot * (I/64) * (d/256 + d/512) * 18432 bytes, 16-byte aligned, out;
+ *   hot_slot int32 [E] device out: slot i < n_hot for expert rank[i], -1 for the others.
+ * Stream-ordered: calls on the same stream after it read the new tier, calls before it
+ * the old one. Put the two pointers and n_hot into the group's hot_pack, hot_slot and
+ * n_hot (once; later updates rewrite the same buffers). Needs E % 4 == 0 and d % 512 == 0.
+ */
+moe_status moe_hot_tier_update(const moe_expert_weights_t* W, const int32_t* rank, int32_t n_hot,
+                               uint8_t* hot_pack, int32_t* hot_slot, void* stream);
+
+/*
+ * moe_set_l2_persisting - size of the L2 set-aside for lines accessed as persisting (the
+ * hot tier's window) in this process's CUDA context on the current device, clamped to the
+ * device's maximum; 0 gives the set-aside back and returns persisting lines to normal. It
+ * is part of the context's state, not a setting of the GPU: it ends with the context
+ * (process exit or cudaDeviceReset) and other processes do not see it. Writes the size in
+ * effect to *bytes_out when not NULL.
+ */
+moe_status moe_set_l2_persisting(size_t bytes, size_t* bytes_out);
 
 /*
  * moe_route_noalloc - moe_route for callers that cannot give the library any scratch

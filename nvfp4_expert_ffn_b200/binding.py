@@ -42,6 +42,8 @@ EXPORTS = {
     "moe_workspace_size": (_SZ, [_I32, _I64, _I32, _I32, _I32, _I32]),
     "moe_get_device_status": (_I32, [_P, _I32, ctypes.POINTER(_I32)]),
     "moe_set_wait_limit_ns": (_I32, [ctypes.c_uint64]),
+    "moe_hot_tier_update": (_I32, [_P, _P, _I32, _P, _P, _P]),
+    "moe_set_l2_persisting": (_I32, [_SZ, ctypes.POINTER(_SZ)]),
     "moe_status_string": (ctypes.c_char_p, [_I32]),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_version": (_I32, []),
@@ -103,7 +105,7 @@ class _WeightsC(ctypes.Structure):
                 ("gu_codes", _P), ("gu_scales", _P), ("gu_ts", _P),
                 ("dn_codes", _P), ("dn_scales", _P), ("dn_ts", _P),
                 ("gu_sf_tiled", _P), ("dn_sf_tiled", _P),
-                ("dec_pack", _P)]
+                ("dec_pack", _P), ("hot_pack", _P), ("hot_slot", _P), ("n_hot", _I32)]
 
 
 class _ExpertsC(ctypes.Structure):
@@ -123,6 +125,9 @@ class ExpertWeights:
     dn_sf_tiled: Optional[torch.Tensor] = None
     dec_pack: Optional[torch.Tensor] = None
     dims: tuple = ()                   # (E, d, I), taken from gu_codes when not given
+    hot_pack: Optional[torch.Tensor] = None   # uint8: n_hot experts' decode-pack units
+    hot_slot: Optional[torch.Tensor] = None   # int32 [E]: slot in hot_pack or -1
+    n_hot: int = 0
 
     def __post_init__(self):
         if not self.dims:
@@ -154,7 +159,8 @@ class ExpertWeights:
         p = lambda t: None if t is None else _ptr(t).value  # noqa: E731
         return _WeightsC(self.E, self.d, self.I, p(self.gu_codes), p(self.gu_scales),
                          p(self.gu_ts), p(self.dn_codes), p(self.dn_scales), p(self.dn_ts),
-                         p(self.gu_sf_tiled), p(self.dn_sf_tiled), p(self.dec_pack))
+                         p(self.gu_sf_tiled), p(self.dn_sf_tiled), p(self.dec_pack),
+                         p(self.hot_pack), p(self.hot_slot), self.n_hot)
 
 
 @dataclass
@@ -281,6 +287,28 @@ def moe_get_device_status(clear=True, stream=None) -> int:
                                                                  1 if clear else 0,
                                                                  ctypes.byref(out)))
     return out.value
+
+
+def moe_hot_tier_update(w: ExpertWeights, rank, n_hot: int, stream=None) -> None:
+    """Copy the units of experts rank[:n_hot] into w's hot tier (allocated here on first
+    use, sized for n_hot) and point w at it; n_hot = 0 turns the tier off."""
+    if n_hot > 0 and (w.hot_pack is None or w.hot_pack.numel() < dec_pack_bytes(n_hot, w.d, w.I)):
+        w.hot_pack = torch.empty(dec_pack_bytes(n_hot, w.d, w.I), dtype=torch.uint8,
+                                 device=w.dec_pack.device)
+    if w.hot_slot is None:
+        w.hot_slot = torch.empty(w.E, dtype=torch.int32, device=w.dec_pack.device)
+    s = w.struct()
+    _check("moe_hot_tier_update", lib().moe_hot_tier_update(
+        ctypes.byref(s), _ptr(rank), n_hot, _ptr(w.hot_pack), _ptr(w.hot_slot), _stream(stream)))
+    w.n_hot = n_hot
+
+
+def moe_set_l2_persisting(nbytes: int) -> int:
+    """Set this process's L2 set-aside for persisting lines (clamped to the device's
+    maximum; 0 releases it); returns the size in effect."""
+    out = _SZ(0)
+    _check("moe_set_l2_persisting", lib().moe_set_l2_persisting(int(nbytes), ctypes.byref(out)))
+    return int(out.value)
 
 
 def moe_set_wait_limit_ns(ns: int) -> None:

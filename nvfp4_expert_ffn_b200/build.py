@@ -27,7 +27,7 @@ LIB = os.path.join(LIBDIR, "libmoe_nvfp4.so")
 BUILD = os.path.join(ROOT, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-Xcompiler", "-fPIC",
                      "-Xptxas", "-v", "-I", os.path.join(ROOT, "include"), "-I", CSRC]
 
 
@@ -52,7 +52,7 @@ def _compile(src: str, outdir: str = BUILD, extra: tuple = ()) -> tuple[str, str
 def build(jobs: int = 8, verbose: bool = False, trace: bool = False) -> str:
     outdir = os.path.join(BUILD, "trace") if trace else BUILD
     lib = os.path.join(outdir, "libmoe_nvfp4_trace.so") if trace else LIB
-    extra = ("-DMOE_TRACE",) if trace else ()
+    extra = ("-DMOE_TRACE", "-lineinfo") if trace else ()
     os.makedirs(outdir, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))

@@ -112,8 +112,8 @@ moe_status check_weights(const moe_expert_weights_t& w, const char* name, int E,
 }
 
 ExpertGroup to_group(const moe_expert_weights_t& w) {
-  return ExpertGroup{w.gu_codes,    w.gu_scales,   w.gu_ts,          w.dn_codes,      w.dn_scales,
-                     w.dn_ts,       w.gu_sf_tiled, w.dn_sf_tiled, w.dec_pack};
+  return ExpertGroup{w.gu_codes, w.gu_scales,   w.gu_ts,       w.dn_codes, w.dn_scales, w.dn_ts,
+                     w.gu_sf_tiled, w.dn_sf_tiled, w.dec_pack, w.hot_pack, w.hot_slot, w.n_hot};
 }
 
 }  // namespace
@@ -362,6 +362,13 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
     return fail(MOE_ERR_INVALID_ARG, "x, Wr, xq_codes, xq_scales, y_acc and y must be 16-byte aligned");
   const bool packed = W->routed.dec_pack && (!W->has_shared || W->shared.dec_pack);
   if (!packed) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "weights need the decode pack of moe_pack_experts");
+  const moe_expert_weights_t& R = W->routed;
+  if (R.n_hot < 0 || R.n_hot > E) return fail(MOE_ERR_INVALID_ARG, "routed.n_hot must be in [0, E]");
+  if (R.n_hot > 0) {
+    if (!R.hot_pack || !R.hot_slot || !aligned16(R.hot_pack) || !aligned16(R.hot_slot))
+      return fail(MOE_ERR_INVALID_ARG, "a hot tier needs 16-byte aligned hot_pack and hot_slot");
+    if (E % 4 != 0) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "a hot tier needs E % 4 == 0");
+  }
   int sms = 0;
   int32_t* dstatus = nullptr;
   if ((s = device_info(&sms, &dstatus)) != MOE_OK) return s;
@@ -421,6 +428,41 @@ moe_status moe_expert_hist(const int32_t* counts, int32_t E, int64_t* cum, int32
   if (s != MOE_OK) return s;
   cudaError_t e = launch_hist(counts, E, cum, rank_out, reset ? 1 : 0, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_hist launch");
+}
+
+moe_status moe_hot_tier_update(const moe_expert_weights_t* W, const int32_t* rank, int32_t n_hot,
+                               uint8_t* hot_pack, int32_t* hot_slot, void* stream) {
+  if (!W) return fail(MOE_ERR_INVALID_ARG, "null weights");
+  if (!W->dec_pack) return fail(MOE_ERR_INVALID_ARG, "the group needs its decode pack (moe_pack_experts)");
+  if (!rank || !hot_slot || (n_hot > 0 && !hot_pack)) return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+  if (n_hot < 0 || n_hot > W->E) return fail(MOE_ERR_INVALID_ARG, "n_hot must be in [0, E]");
+  if (W->E % 4 != 0 || W->d % 512 != 0 || W->I % 64 != 0)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "a hot tier needs E % 4 == 0, d % 512 == 0 and I % 64 == 0");
+  if ((hot_pack && !aligned16(hot_pack)) || !aligned16(hot_slot) || !aligned16(W->dec_pack))
+    return fail(MOE_ERR_INVALID_ARG, "hot_pack, hot_slot and dec_pack must be 16-byte aligned");
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  cudaError_t e = launch_hot_tier(W->dec_pack, rank, W->E, W->d, W->I, n_hot, hot_pack, hot_slot, sms,
+                                  (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_hot_tier_update launch");
+}
+
+moe_status moe_set_l2_persisting(size_t bytes, size_t* bytes_out) {
+  int sms = 0;
+  moe_status s = device_info(&sms);
+  if (s != MOE_OK) return s;
+  int dev = 0, max_bytes = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&max_bytes, cudaDevAttrMaxPersistingL2CacheSize, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "persisting L2 maximum");
+  const size_t b = bytes < (size_t)max_bytes ? bytes : (size_t)max_bytes;
+  if (b == 0 && (e = cudaCtxResetPersistingL2Cache()) != cudaSuccess) return cuda_fail(e, "cudaCtxResetPersistingL2Cache");
+  if ((e = cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, b)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize)");
+  if (bytes_out && (e = cudaDeviceGetLimit(bytes_out, cudaLimitPersistingL2CacheSize)) != cudaSuccess)
+    return cuda_fail(e, "cudaDeviceGetLimit(cudaLimitPersistingL2CacheSize)");
+  return MOE_OK;
 }
 
 moe_status moe_set_wait_limit_ns(uint64_t ns) {

@@ -59,6 +59,9 @@ constexpr int kDecDnN = 16;                                    // 16 token colum
 constexpr uint32_t kDecIdescT = idesc_mxf4nvf4(128, kDecDnN);  // 128 weight rows x 16 token columns
 constexpr int kDecHBytes = 1024;                       // h codes (8 rows x 32 B) + its atom at +512
 constexpr size_t kDecSmemBudget = 224 * 1024;          // dynamic shared memory; the rest is static
+// The weight stream is read once per call: its L2 lines go first, so that the activations,
+// logits, router rows and the kernel's own code stay in L2 while it passes.
+constexpr bool kDecStreamEvictFirst = true;
 
 // TMEM columns (512 allocated): gate/up accumulators of the two MMA issuers, h scale slots
 // (per issuer, per unit parity), the weight-scale ring, the resident activation scales
@@ -81,12 +84,14 @@ struct DecArgs {
 };
 
 // This CTA's units, in shared memory: expert id (E = the shared expert), slice j, and the
-// routing weight of each of the 8 tokens (0: token not routed to the expert).
+// routing weight of each of the 8 tokens (0: token not routed to the expert); optionally
+// where each unit's stages start (else the unit's place in the group's decode pack).
 struct DecUnits {
   int n;
   const int* e;
   const int* j;
   const float* w;  // [n][8]
+  const uint8_t* const* base = nullptr;
 };
 
 struct DecBars {
@@ -218,6 +223,7 @@ MOE_DEV void dec_run(const DecArgs& p, const DecSmem& sm, DecBars& bar, const De
     if (lane == 0) {
       uint32_t it = 0;
       bool alive = true;
+      const uint64_t pol = l2_policy_evict_first();
       for (int jb = 0; jb < 2 * nu && alive; ++jb) {
         const bool gu = job_is_gu(jb);
         const int u = job_unit(jb);
@@ -240,8 +246,11 @@ MOE_DEV void dec_run(const DecArgs& p, const DecSmem& sm, DecBars& bar, const De
           // four scale atoms (gate/up K block (q + rot) % nks1, or down chunks 4(q - nks1)..+3)
           const int qp = q < nks1 ? (q + rot) % nks1 : q;
           mbar_arrive_expect_tx(&full[st], kDecStageBytes);
-          bulk_g2s(sb, G.dec_pack + (((size_t)el * nt1 + j) * (nks1 + nks2) + qp) * kDecStageBytes, kDecStageBytes,
-                   &full[st]);
+          const uint8_t* ub =
+              U.base ? U.base[u] : G.dec_pack + ((size_t)el * nt1 + j) * (nks1 + nks2) * kDecStageBytes;
+          const uint8_t* src = ub + (size_t)qp * kDecStageBytes;
+          if (kDecStreamEvictFirst) bulk_g2s_hint(sb, src, kDecStageBytes, &full[st], pol);
+          else bulk_g2s(sb, src, kDecStageBytes, &full[st]);
         }
       }
       // no copy may still be landing when the CTA exits
@@ -379,7 +388,7 @@ MOE_DEV void dec_run(const DecArgs& p, const DecSmem& sm, DecBars& bar, const De
     uint32_t gc = 0;
     for (int jb = 0; jb < 2 * nu; ++jb) {
       const int u = job_unit(jb);
-      const int e = U.e[u], j = U.j[u];
+      const int e = U.e[u];
       const bool sh = e == p.E;
       const int el = sh ? 0 : e;
       const ExpertGroup& G = sh ? p.shared : p.routed;

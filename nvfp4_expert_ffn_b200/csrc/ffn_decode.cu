@@ -21,7 +21,6 @@
 namespace moe {
 
 constexpr int kTokChunk = 8;      // tokens processed together per unit pass
-constexpr int kFfnThreads = 256;  // 8 warps
 
 __host__ __device__ __forceinline__ size_t align16(size_t v) { return (v + 15) & ~(size_t)15; }
 

@@ -34,22 +34,28 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 // As launch_pdl, and cooperative: the launch fails instead of starting unless every CTA of
-// the grid can be resident at once (kernels that wait at grid-wide barriers).
+// the grid can be resident at once (kernels that wait at grid-wide barriers). With `win`,
+// the launch also carries that L2 access-policy window.
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl_coop(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                   cudaStream_t st, Args&&... args) {
+                                   cudaStream_t st, const cudaAccessPolicyWindow* win, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeCooperative;
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  if (win) {
+    attr[2].id = cudaLaunchAttributeAccessPolicyWindow;
+    attr[2].val.accessPolicyWindow = *win;
+    cfg.numAttrs = 3;
+  }
   g_launch_count.fetch_add(1, std::memory_order_relaxed);
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
@@ -68,6 +74,9 @@ struct ExpertGroup {
   const uint8_t* gu_sf_tiled;
   const uint8_t* dn_sf_tiled;
   const uint8_t* dec_pack;  // [E][I/64][d/256 + d/512][18432]: decode stages (moe_pack_experts)
+  const uint8_t* hot_pack;  // [n_hot][I/64][d/256 + d/512][18432]: copies of the hot experts' units
+  const int32_t* hot_slot;  // [E]: slot in hot_pack, or -1
+  int n_hot;
 };
 
 struct FfnArgs {
@@ -156,6 +165,8 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
 cudaError_t launch_pack_dec(const ExpertGroup& g, int E, int d, int I, const uint8_t* gu_sf_tiled,
                             const uint8_t* dn_sf_tiled, uint8_t* dec_pack, int num_sms, cudaStream_t st);
 size_t dec_pack_bytes(int E, int d, int I);
+cudaError_t launch_hot_tier(const uint8_t* dec_pack, const int32_t* rank, int E, int d, int I, int n_hot,
+                            uint8_t* hot_pack, int32_t* hot_slot, int num_sms, cudaStream_t st);
 cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* gu_t, uint8_t* dn_t,
                            int num_sms, cudaStream_t st);
 

@@ -7,28 +7,29 @@
 // and as separate kernels each costs a launch and a chain of dependent memory round trips.
 // Here one CTA per SM (all but one SM, left to a side-stream kernel such as the cumulative
 // histogram) runs:
+//   prologue (before the kernel waits on its predecessor) the CTA's router rows are copied
+//            into shared memory and, with a shared expert, CTA j < I/64 starts bringing its
+//            shared-expert unit (slice j) into L2: neither depends on the previous kernel.
 //   phase 1  every CTA loads x, takes the global amax itself (the NVFP4 tensor scale),
 //            quantises its share of the 64-element groups into the xq output buffers, and
-//            computes the router logits of its expert rows (E / grid rows, the router
-//            weights copied in before the kernel waits on its predecessor); CTA 0 zeroes
-//            y_acc.
+//            computes the router logits of its expert rows; CTA 0 zeroes y_acc.
 //   barrier
-//   phase 2  every CTA reads all tokens' codes into its MMA operand tiles (their scales go
-//            on to TMEM while the rest of the phase runs) and all logits, runs the top-k of
-//            all tokens itself and derives its own units from the bitmap of chosen experts;
-//            the last CTA also writes the routing outputs (top-k, counts, offsets,
-//            permutation).
+//   phase 2  warp t < T reads token t's logits from L2 and runs its top-k while the other
+//            warps read all tokens' codes and scales into the MMA operand tiles (one round
+//            of loads); then warp 0 derives this CTA's units from the bitmap of chosen
+//            experts, and the last CTA also writes the routing outputs (top-k, counts,
+//            offsets, permutation).
 //   phase 3  the units (expert, 64-column slice of I), adding into y_acc.
-//   barrier
-//   phase 4  CTA t < T converts row t of y_acc to bf16 (optionally RMS-renormalised).
-// The grid barrier counts arrivals in eight workspace words (CTA b arrives on word b % 8, so
-// that 147 arrivals do not queue on one address) that must be zero before the first call;
-// every call leaves each word at a multiple of the number of CTAs that arrive on it. A CTA
-// that gives up at a bounded wait marks the workspace (another word), since the counters may
-// then be left between multiples; later calls on a marked workspace do nothing but report
-// MOE_ERR_WORKSPACE until the caller zeroes it. The launch is cooperative: it fails rather
-// than start a grid whose CTAs cannot all be resident, so the barrier cannot wait on a CTA
-// that has not started.
+//   phase 4  each CTA counts itself done; the one that comes last converts y_acc to bf16
+//            (optionally RMS-renormalised). The others exit without waiting.
+// The barrier and the done count share one 64-bit workspace word that must be zero before
+// the first call; every call adds 2G to it (G CTAs). A CTA that gives up at a bounded wait
+// marks the workspace (a second word), since the count may then be left between multiples
+// of G; later calls on a marked workspace do nothing but report MOE_ERR_WORKSPACE until the
+// caller zeroes it. A third word, which the library never writes, makes CTA 0 hold back its
+// barrier arrival while it is nonzero: a test sets it to make the other CTAs' bounded waits
+// run out. The launch is cooperative: it fails rather than start a grid whose CTAs cannot
+// all be resident, so the barrier cannot wait on a CTA that has not started.
 #include <cuda_bf16.h>
 
 #include "dec_core.cuh"
@@ -67,12 +68,14 @@ struct LayerArgs {
   float* logits;       // [T][E]
   unsigned long long* sync;  // arrival counter of the grid barrier (zero before the first call)
   unsigned int* poison;      // nonzero once a call on this workspace gave up at a bounded wait
+  const unsigned int* hold;  // nonzero: CTA 0 does not arrive at the barrier (set only by tests)
   int32_t* status;
 };
 
 // Grid-wide barrier on a 64-bit arrival counter that only grows: thread 0 of each CTA adds
 // one and waits (bounded) until the count reaches the next multiple of the grid size. The
-// counter starts at zero and every call adds two multiples, so it stays aligned. Writes
+// counter starts at zero and every call adds two multiples (the barrier's arrivals, then
+// phase 4's done count), so it stays aligned. Writes
 // before the arrival are visible to every CTA after the wait; the CTA may work between the
 // two halves.
 //
@@ -121,40 +124,38 @@ MOE_DEV bool grid_sync(unsigned long long* count, volatile int* abort, int32_t* 
 }
 
 // Shared-memory scratch of phases 1 and 2, on the weight ring (not in use before phase 3):
-// the bf16 activations (phase 1), then at the same place the logits (phase 2); the top-k of
-// each token, the permutation's counters, the router's partial sums and rows.
+// the bf16 activations (phase 1), the top-k of each token, the permutation's counters, the
+// router's partial sums and rows.
 struct LayerScratch {
   uint16_t* xb;   // [8][d] (phase 1)
-  float* logits;  // [8][E] (phase 2, over xb)
   int* tidx;      // [8][32] expert ids of each token's top-k
   float* tw;      // [8][32] their weights
   int* perm;      // [1024] counters of the permutation
   int* sidx;      // [256] top-k expert ids, assignment order
   float* part;    // [kDecThreads] router partial sums (phase 1)
   uint32_t* tks;  // [8][64] top-k scratch of each token's warp
+  int* hslot;     // [1024] the routed group's hot-tier slots (with a hot tier)
   float* wr;      // [rows][d] this CTA's router rows (phase 1)
 };
 
-__host__ __device__ inline size_t layer_scratch_head(int d) {
-  const size_t xb = 16 * (size_t)d, lg = (size_t)kDecMaxT * 1024 * 4;
-  return xb > lg ? xb : lg;
-}
+__host__ __device__ inline size_t layer_scratch_head(int d) { return 16 * (size_t)d; }
 
 MOE_DEV LayerScratch layer_scratch(uint8_t* ring, int d) {
   LayerScratch s;
   s.xb = reinterpret_cast<uint16_t*>(ring);
-  s.logits = reinterpret_cast<float*>(ring);
   s.tidx = reinterpret_cast<int*>(ring + layer_scratch_head(d));
   s.tw = reinterpret_cast<float*>(s.tidx + kDecMaxT * kLayerMaxK);
   s.perm = reinterpret_cast<int*>(s.tw + kDecMaxT * kLayerMaxK);
   s.sidx = s.perm + 1024;
   s.part = reinterpret_cast<float*>(s.sidx + 256);
   s.tks = reinterpret_cast<uint32_t*>(s.part + kDecThreads);
-  s.wr = reinterpret_cast<float*>(s.tks + kDecMaxT * 64);
+  s.hslot = reinterpret_cast<int*>(s.tks + kDecMaxT * 64);
+  s.wr = reinterpret_cast<float*>(s.hslot + 1024);
   return s;
 }
 // bytes of scratch past the head
-constexpr size_t kLayerScratchTail = 2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 256 + kDecThreads + kDecMaxT * 64) * 4;
+constexpr size_t kLayerScratchTail =
+    2 * kDecMaxT * kLayerMaxK * 4 + (1024 + 256 + kDecThreads + kDecMaxT * 64 + 1024) * 4;
 static_assert(kLayerScratchTail % 16 == 0, "router rows must start 16-byte aligned");
 
 __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) {
@@ -177,9 +178,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   // this CTA's router rows b, b + G, ... are copied into shared memory before the kernel
   // waits on its predecessor (the router weights are not written by anything)
   const int nrows = b < E ? (E - 1 - b) / G + 1 : 0;
-  __shared__ uint64_t s_wbar;
+  __shared__ uint64_t s_wbar, s_hbar;
   __shared__ float s_bias[kLayerMaxRows];
-  if (threadIdx.x == 0) mbar_init(&s_wbar, 1);
+  __shared__ const uint8_t* s_ub[kDecMaxUnits];  // where each unit's stages start
+  __shared__ int s_hot;                           // the hot-tier slots are on their way
+  if (threadIdx.x == 0) {
+    mbar_init(&s_wbar, 1);
+    mbar_init(&s_hbar, 1);
+  }
   if (threadIdx.x < 32) s_bits[threadIdx.x] = 0u;
   if (threadIdx.x < nrows) s_bias[threadIdx.x] = p.br ? __ldg(p.br + b + threadIdx.x * G) : 0.0f;
   dec_init(bar, p.nstages);  // includes the barrier-init fence
@@ -188,6 +194,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
     for (int r = 0; r < nrows; ++r)
       bulk_g2s(sc.wr + (size_t)r * d, p.Wr + (size_t)(b + r * G) * d, (uint32_t)(d * 4), &s_wbar);
   }
+  // units 0 .. I/64 - 1 are the shared expert's slices and go to CTAs 0 .. I/64 - 1 (the unit
+  // table of phase 2): such a CTA starts its unit's stages on their way into L2 now
+  if (threadIdx.x == 32 && p.has_shared && b < p.I / 64) {
+    const uint32_t unit_bytes = (uint32_t)((d / 256 + d / 512) * kDecStageBytes);
+    prefetch_l2_bulk(p.shared.dec_pack + (size_t)b * unit_bytes, unit_bytes);
+  }
   MOE_PDL_PROLOGUE();
   RT_TRACE(g_layer_trace, 0, 1);
   // a workspace marked by an earlier call that gave up: report it and do nothing (the mark is
@@ -195,10 +207,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   __shared__ int s_live;
   if (threadIdx.x == 0) {
     s_live = 1;
+    s_hot = 0;
     if (*reinterpret_cast<volatile unsigned int*>(p.poison) != 0u) {
       s_live = 0;
       *abort = 1;
       atomicExch(p.status, kStatusWorkspace);
+    } else {
+      if (b == 0 && *reinterpret_cast<const volatile unsigned int*>(p.hold) != 0u)
+        *abort = 1;  // held back: no arrival, so every other CTA's barrier wait runs out
+      if (p.routed.n_hot > 0) {
+        // the routed group's hot-tier slots (written by the update that came before this
+        // call, so only now), needed when the unit table is built
+        s_hot = 1;
+        mbar_arrive_expect_tx(&s_hbar, (uint32_t)(E * 4));
+        bulk_g2s(sc.hslot, p.routed.hot_slot, (uint32_t)(E * 4), &s_hbar);
+      }
     }
   }
   __syncthreads();
@@ -207,7 +230,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
 
   // ---------------------------------------------------------------- phase 1
   if (live) {
-  // x -> shared memory (every load of a round in flight before the stores)
+  // x -> shared memory (every load of a round in flight before the stores), with each
+  // thread's running maximum of |x| (bf16 magnitudes order like their bit patterns)
+  uint32_t mx2 = 0;
   {
     const int nx = T * d / 8;
     const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
@@ -217,37 +242,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * blockDim.x;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
         if (i < nx) v[u] = __ldg(x4 + i);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * blockDim.x;
         if (i < nx) xb4[i] = v[u];
+        mx2 = __vmaxu2(mx2, v[u].x & 0x7FFF7FFFu);
+        mx2 = __vmaxu2(mx2, v[u].y & 0x7FFF7FFFu);
+        mx2 = __vmaxu2(mx2, v[u].z & 0x7FFF7FFFu);
+        mx2 = __vmaxu2(mx2, v[u].w & 0x7FFF7FFFu);
       }
     }
   }
-  __syncthreads();
-  RT_TRACE(g_layer_trace, 0, 2);
   // NVFP4 tensor scale: amax / (6 * 448) over all T tokens (every CTA computes the same), or
   // the static scale
-  if (p.ts_in) {
-    ts = *p.ts_in;
-  } else {
-    uint32_t m = 0;
-    const uint4* xb4 = reinterpret_cast<const uint4*>(sc.xb);
-    for (int i = threadIdx.x; i < T * d / 8; i += blockDim.x) {
-      const uint4 v = xb4[i];
-      m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
-      m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
-      m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
-      m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
-    }
-    float f = warp_max(fmaxf(bf16_to_f32(m & 0xFFFFu), bf16_to_f32(m >> 16)));
+  {
+    float f = warp_max(fmaxf(bf16_to_f32(mx2 & 0xFFFFu), bf16_to_f32(mx2 >> 16)));
     if (lane == 0) s_red[warp] = f;
-    __syncthreads();
-    f = lane < (int)(blockDim.x >> 5) ? s_red[lane] : 0.0f;
-    f = warp_max(f);
-    ts = f > 0.0f ? __fdiv_rn(f, kE2M1Max * kE4M3Max) : 1.0f;
+    __syncthreads();  // also: x is in shared memory
+    RT_TRACE(g_layer_trace, 0, 2);
+    if (p.ts_in) {
+      ts = *p.ts_in;
+    } else {
+      f = lane < (int)(blockDim.x >> 5) ? s_red[lane] : 0.0f;
+      f = warp_max(f);
+      ts = f > 0.0f ? __fdiv_rn(f, kE2M1Max * kE4M3Max) : 1.0f;
+    }
   }
   RT_TRACE(g_layer_trace, 2, 0);
   // this CTA's share of the 64-element groups (b, b + G, ...), one warp per group of four
@@ -358,6 +380,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   RT_TRACE(g_layer_trace, 0, 3);
   bool ok = grid_sync(p.sync, abort, p.status);
   RT_TRACE(g_layer_trace, 0, 4);
+  if (threadIdx.x == 0 && s_hot) {
+    // long landed by now; waited for on every path, as it must land before the CTA exits
+    volatile int no_abort = 0;
+    if (!mbar_wait(&s_hbar, 0, &no_abort, p.status)) {
+      *abort = 1;
+      ok = false;
+    }
+  }
 
   // ---------------------------------------------------------------- phase 2
   // Data written by other CTAs before the barrier is read through L2 (ld.global.cg).
@@ -365,89 +395,65 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   const bool writer = b == G - 1;  // the CTA with the fewest units writes the routing outputs
   int nu = 0;
   if (ok) {
-    // all tokens' codes -> the 8-row tiles (rows >= T zero), scales -> atoms, logits -> shared
-    // memory; each thread's loads of a round go out together
-    {
-      const int q4 = d / 256;  // 16-byte pieces of a token's scale row
-      uint4 sv = make_uint4(0u, 0u, 0u, 0u);
-      if (threadIdx.x < kDecMaxT * q4 && (int)threadIdx.x / q4 < T)
-        sv = __ldcg(reinterpret_cast<const uint4*>(p.xq_scales + (size_t)(threadIdx.x / q4) * (d / kBlock)) +
-                    threadIdx.x % q4);
-      const int nc = kDecMaxT * (d / 32);
-      // every CTA reads the same few lines right after the barrier: each starts at a different
-      // place so that the requests to one L2 line do not all arrive at once
-      const int rot_c = (b * 37) % nc;
-      for (int i0 = threadIdx.x; i0 < nc; i0 += 4 * blockDim.x) {
-        uint4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int iu = i0 + u * blockDim.x;
-          const int i = iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc;
-          const int t = i / (d / 32), c = i % (d / 32);
-          v[u] = make_uint4(0u, 0u, 0u, 0u);
-          if (iu < nc && t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + c);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int iu = i0 + u * blockDim.x;
-          const int i = iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc;
-          if (iu < nc) *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(i / (d / 32), i % (d / 32))) = v[u];
-        }
-      }
-      RT_TRACE(g_layer_trace, 3, 3);
-      // the scale words of token t arrive as d/256 16-byte pieces (loaded above); word kc of
-      // token t goes to the four rows t, t + 8, t + 16, t + 24 of atom kc
-      if (threadIdx.x < kDecMaxT * q4) {
-        const int t = threadIdx.x / q4, c4 = threadIdx.x % q4;
-        const uint32_t wv[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-#pragma unroll
-          for (int r1 = 0; r1 < 4; ++r1) dec_xsf_store(sm.xsf, 4 * c4 + w, t + 8 * r1, wv[w]);
-      }
-      RT_TRACE(g_layer_trace, 3, 4);
-      // the logits -> shared memory, the same way
-      const int nl = T * E;
-      const int rot_l = (b * 131) % nl;
-      for (int i0 = threadIdx.x; i0 < nl; i0 += 8 * blockDim.x) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int iu = i0 + u * blockDim.x;
-          const int i = iu + rot_l < nl ? iu + rot_l : iu + rot_l - nl;
-          v[u] = iu < nl ? __ldcg(p.logits + i) : 0.0f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int iu = i0 + u * blockDim.x;
-          const int i = iu + rot_l < nl ? iu + rot_l : iu + rot_l - nl;
-          if (iu < nl) sc.logits[i] = v[u];
-        }
-      }
-    }
-    fence_proxy_async_smem();  // the tiles and atoms are read by tcgen05 (async proxy)
-    __syncthreads();
-    RT_TRACE(g_layer_trace, 3, 0);
-    // the activation scale atoms -> TMEM for the whole of phase 3, issued by a warp the top-k
-    // leaves idle (both issuers' arrivals on xsf_ready come from here)
-    if (warp == kDecThreads / 32 - 1 && lane == 0) {
-      tc_fence_after();
-      for (int a = 0; a < d / 64; ++a)
-        tmem_cp_sf(bar.tmem + kColX + 4 * a, sdesc_sf(smem_u32(sm.xsf + (size_t)a * kDecAtom)));
-      mma_commit(&bar.xsf_ready);
-      mma_commit(&bar.xsf_ready);
-    }
-    // top-k of every token (one warp each); the chosen experts are marked in s_bits
     if (warp < T) {
-      topk_dispatch(sc.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
-                    writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
-                    sc.tw + warp * kLayerMaxK, sc.tks + warp * 64);
+      // token `warp`: its logits straight from L2 into the top-k; the chosen experts are
+      // marked in s_bits
+      unsigned long long* stamps = nullptr;
+#ifdef MOE_TRACE
+      if (warp == 0 && b < kTraceCtas) stamps = &g_layer_trace[4][b][0];
+#endif
+      topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
+                          writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
+                          sc.tw + warp * kLayerMaxK, sc.tks + warp * 64, stamps);
+      RT_TRACE(g_layer_trace, 3, 0);
       __syncwarp();
       if (lane < k) {
         const int e = sc.tidx[warp * kLayerMaxK + lane];
         atomicOr(&s_bits[e >> 5], 1u << (e & 31));
       }
+    } else {
+      // the other warps: all tokens' codes -> the 8-row tiles (rows >= T zero) and their
+      // scale words -> the atoms (word kc of token t goes to rows t, t + 8, t + 16, t + 24 of
+      // atom kc), each thread's loads of a round in flight together. Every CTA reads the same
+      // few lines right after the barrier, so each starts the codes at its own place.
+      const int tid = (int)threadIdx.x - 32 * T, nth = (int)blockDim.x - 32 * T;
+      const int cpr = d / 32, q4 = d / 256;       // 16-byte code / scale pieces of a token row
+      const int nc = kDecMaxT * cpr, ns = kDecMaxT * q4;
+      const int rot_c = (b * 37) % nc;
+      auto code_piece = [&](int iu) { return iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc; };
+      for (int i0 = tid; i0 < nc + ns; i0 += 8 * nth) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int iu = i0 + u * nth;
+          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          if (iu < nc) {
+            const int i = code_piece(iu), t = i / cpr;
+            if (t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + i % cpr);
+          } else if (iu < nc + ns) {
+            const int t = (iu - nc) / q4;
+            if (t < T)
+              v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_scales + (size_t)t * (d / kBlock)) + (iu - nc) % q4);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int iu = i0 + u * nth;
+          if (iu < nc) {
+            const int i = code_piece(iu);
+            *reinterpret_cast<uint4*>(sm.xs + dec_xs_offset(i / cpr, i % cpr)) = v[u];
+          } else if (iu < nc + ns) {
+            const int t = (iu - nc) / q4, c4 = (iu - nc) % q4;
+            const uint32_t wv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+#pragma unroll
+              for (int r1 = 0; r1 < 4; ++r1) dec_xsf_store(sm.xsf, 4 * c4 + w, t + 8 * r1, wv[w]);
+          }
+        }
+      }
     }
+    fence_proxy_async_smem();  // the tiles and atoms are read by tcgen05 (async proxy)
     __syncthreads();
     RT_TRACE(g_layer_trace, 3, 1);
     if (warp == 0) {
@@ -488,6 +494,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
         }
         s_ue[lane] = e;
         s_uj[lane] = ug % nt1;
+        // the unit's stages: the shared expert's, a hot expert's copy, or its decode pack
+        const size_t unit_bytes = (size_t)(d / 256 + d / 512) * kDecStageBytes;
+        int hs = (e < E && s_hot) ? sc.hslot[e] : -1;
+        if (hs >= p.routed.n_hot) hs = -1;  // not a slot of this tier: read the decode pack
+        s_ub[lane] = e == E ? p.shared.dec_pack + (size_t)(ug % nt1) * unit_bytes
+                     : hs >= 0 ? p.routed.hot_pack + ((size_t)hs * nt1 + ug % nt1) * unit_bytes
+                               : p.routed.dec_pack + ((size_t)e * nt1 + ug % nt1) * unit_bytes;
       }
       if (lane == 0) s_nu = n;
       __syncwarp();
@@ -505,6 +518,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
         }
         s_uw[u * kDecMaxT + t] = wt;
       }
+      RT_TRACE(g_layer_trace, 3, 3);
     } else if (warp == 1 && writer) {
       // the routing outputs: assignment a = t*k + j in expert order
       for (int a = lane; a < T * k; a += 32) sc.sidx[a] = sc.tidx[(a / k) * kLayerMaxK + a % k];
@@ -530,10 +544,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   a.nstages = p.nstages;
   a.group_chunks = p.group_chunks;
   a.ts_x = ts;
-  a.xsf_loaded = 1;
+  a.xsf_loaded = 0;  // the MMA issuers copy the activation scale atoms to TMEM
   a.out = p.y_acc;
   a.status = p.status;
-  dec_run(a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw});
+  dec_run(a, sm, bar, DecUnits{nu, s_ue, s_uj, s_uw, s_ub});
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(bar.tmem, 512);
@@ -541,32 +555,56 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
 
   RT_TRACE(g_layer_trace, 0, 6);
   // ---------------------------------------------------------------- phase 4
-  ok = grid_sync(p.sync, abort, p.status) && ok;
+  // Each CTA that finished its units counts itself on the barrier word (the call's second G
+  // arrivals); the one whose arrival completes the multiple of G has seen every other CTA's
+  // additions into y_acc and converts it: row t by warp t, to bf16, optionally scaled to
+  // unit root-mean-square. The others exit at once.
+  __shared__ int s_last;
+  __syncthreads();  // every unit's additions are issued and complete
+  if (threadIdx.x == 0) {
+    s_last = 0;
+    if (ok && !*abort) {
+      __threadfence();
+      const unsigned long long old = atomicAdd(p.sync, 1ull);
+      s_last = old % (unsigned long long)G == (unsigned long long)(G - 1) ? 1 : 0;
+      __threadfence();
+    }
+  }
+  __syncthreads();
   RT_TRACE(g_layer_trace, 1, 0);
-  if (ok && b < T) {
-    // row t = b of y_acc -> bf16, optionally scaled to unit root-mean-square
-    const int t = b;
-    const float* row = p.y_acc + (size_t)t * d;
+  if (s_last && warp < T) {
+    const int t = warp, n4 = d / 4;
+    const float4* row = reinterpret_cast<const float4*>(p.y_acc + (size_t)t * d);
+    uint2* out = reinterpret_cast<uint2*>(p.y + (size_t)t * d);
     float scale = 1.0f;
     if (p.rms) {
       float ss = 0.0f;
-      for (int n = threadIdx.x; n < d; n += blockDim.x) {
-        const float v = __ldcg(row + n);
-        ss = fmaf(v, v, ss);
+      for (int c0 = lane; c0 < n4; c0 += 32 * 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = c0 + 32 * u < n4 ? __ldcg(row + c0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          ss = fmaf(v[u].x, v[u].x, ss);
+          ss = fmaf(v[u].y, v[u].y, ss);
+          ss = fmaf(v[u].z, v[u].z, ss);
+          ss = fmaf(v[u].w, v[u].w, ss);
+        }
       }
-      ss = warp_sum(ss);
-      if (lane == 0) s_red[warp] = ss;
-      __syncthreads();
-      float tot = lane < (int)(blockDim.x >> 5) ? s_red[lane] : 0.0f;
-      tot = warp_sum(tot);
-      const float ms = tot / (float)d;
+      const float ms = warp_sum(ss) / (float)d;
       scale = ms > 0.0f ? rsqrtf(ms) : 0.0f;
     }
-    for (int n2 = threadIdx.x; n2 < d / 2; n2 += blockDim.x) {
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(row) + n2);
-      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v.x * scale));
-      const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(v.y * scale));
-      reinterpret_cast<uint32_t*>(p.y + (size_t)t * d)[n2] = lo | (hi << 16);
+    auto bf2 = [&](float lo, float hi) {
+      return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo * scale)) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi * scale)) << 16);
+    };
+    for (int c0 = lane; c0 < n4; c0 += 32 * 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = c0 + 32 * u < n4 ? __ldcg(row + c0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (c0 + 32 * u < n4) out[c0 + 32 * u] = make_uint2(bf2(v[u].x, v[u].y), bf2(v[u].z, v[u].w));
     }
   }
   // a CTA that gave up (or found the workspace marked) marks it for the calls that follow
@@ -580,8 +618,9 @@ size_t a256l(size_t v) { return (v + 255) & ~(size_t)255; }
 int layer_grid(int num_sms) { return num_sms > 1 ? num_sms - 1 : 1; }
 }  // namespace
 
-// workspace: the barrier counters (one 128-byte line each) and the mark, then the logits
-constexpr size_t kLayerWsHeader = 2048, kLayerWsPoison = 1024;
+// workspace: the barrier word, the mark and the hold word (each on its own line), then the
+// logits
+constexpr size_t kLayerWsHeader = 2048, kLayerWsPoison = 1024, kLayerWsHold = 1536;
 size_t layer_dec_ws_bytes(int64_t T, int E) { return kLayerWsHeader + a256l((size_t)T * E * 4); }
 
 bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms) {
@@ -628,10 +667,27 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
   p.y = a.y;
   p.sync = reinterpret_cast<unsigned long long*>(w);
   p.poison = reinterpret_cast<unsigned int*>(w + kLayerWsPoison);
+  p.hold = reinterpret_cast<const unsigned int*>(w + kLayerWsHold);
   p.logits = reinterpret_cast<float*>(w + kLayerWsHeader);
   p.status = status;
+  // a hot tier: its copies are read as persisting in L2, everything else as streaming
+  cudaAccessPolicyWindow win = {};
+  const cudaAccessPolicyWindow* wp = nullptr;
+  if (a.routed.n_hot > 0) {
+    int dev = 0, max_win = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&max_win, cudaDevAttrMaxAccessPolicyWindowSize, dev);
+    if (e != cudaSuccess) return e;
+    const size_t bytes = (size_t)a.routed.n_hot * (a.I / 64) * (a.d / 256 + a.d / 512) * kDecStageBytes;
+    win.base_ptr = const_cast<uint8_t*>(a.routed.hot_pack);
+    win.num_bytes = bytes < (size_t)max_win ? bytes : (size_t)max_win;
+    win.hitRatio = 1.0f;
+    win.hitProp = cudaAccessPropertyPersisting;
+    win.missProp = cudaAccessPropertyStreaming;
+    if (win.num_bytes > 0) wp = &win;
+  }
   return launch_pdl_coop(layer_dec_kernel, dim3(layer_grid(num_sms)), dim3(kDecThreads), dec_smem_bytes(a.d), st,
-                         p);
+                         wp, p);
 }
 
 }  // namespace moe

@@ -442,8 +442,8 @@ cudaError_t launch_route(const uint16_t* x, int T, int d, const float* Wr, const
 
 // ---------------------------------------------------------------- cumulative histogram
 // One CTA: cum[e] += counts[e] (or = on reset); then a bitonic sort in shared memory of
-// keys (cum descending, id ascending) packed into 64 bits: key = (2^51-1-cum) << 12 | e.
-constexpr int kHistMaxE = 4096;
+// keys (cum descending, id ascending) packed into 64 bits: key = (2^51-1-cum) << 12 | e
+// (E <= 4096, checked by the caller).
 
 __global__ void __launch_bounds__(1024) hist_kernel(const int32_t* __restrict__ counts, int E,
                                                     int64_t* __restrict__ cum,

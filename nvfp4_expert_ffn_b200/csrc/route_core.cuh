@@ -33,9 +33,25 @@ MOE_DEV uint32_t ordered_key(float v) {
 // each candidate's rank is counted against the other 31. Otherwise k rounds of a warp
 // arg-max pick the winners one at a time, and only the winning lane rescans its entries.
 // Both give the same picks in the same order.
+// stamps (trace builds only): lane 0 records globaltimer after the loads, the threshold, the
+// selection and the weights into stamps[0..3]
+#ifdef MOE_TRACE
+#define TOPK_STAMP(i)                                                    \
+  do {                                                                   \
+    if (stamps != nullptr && lane == 0) stamps[i] = globaltimer_ns_rc(); \
+  } while (0)
+MOE_DEV unsigned long long globaltimer_ns_rc() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#else
+#define TOPK_STAMP(i) do { } while (0)
+#endif
 template <int NPER, bool kL2 = false>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* idx_out, float* w_out,
-                        int* idx_smem = nullptr, float* w_smem = nullptr, uint32_t* scratch = nullptr) {
+                        int* idx_smem = nullptr, float* w_smem = nullptr, uint32_t* scratch = nullptr,
+                        unsigned long long* stamps = nullptr) {
   const int lane = threadIdx.x & 31;
   uint32_t key[NPER];
 #pragma unroll
@@ -71,12 +87,14 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
 #pragma unroll
       for (int j = 0; j < w; ++j) m[j] = max(m[j], m[j + w]);
     const uint32_t lmax = m[0];
+    TOPK_STAMP(0);
     // threshold: the k-th largest lane maximum = the smallest maximum with fewer than k
     // maxima strictly above it (lanes without entries hold 0, below every key)
     int above = 0;
 #pragma unroll 8
     for (int o = 1; o < 32; ++o) above += __shfl_sync(0xffffffffu, lmax, (lane + o) & 31) > lmax ? 1 : 0;
     const uint32_t th = __reduce_min_sync(0xffffffffu, above < k ? lmax : 0xffffffffu);
+    TOPK_STAMP(1);
     int c = 0;
 #pragma unroll
     for (int j = 0; j < NPER; ++j) c += (lane + 32 * j < E && key[j] >= th) ? 1 : 0;
@@ -145,6 +163,7 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
       }
     }
   }
+  TOPK_STAMP(2);
   auto key_to_float = [](uint32_t kk) {
     return __uint_as_float((kk & 0x80000000u) ? (kk & 0x7fffffffu) : ~kk);
   };
@@ -157,15 +176,17 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
     if (idx_smem) idx_smem[lane] = my_e;
     if (w_smem) w_smem[lane] = w;
   }
+  TOPK_STAMP(3);
 }
 
 // scratch: NULL, or 64 words of shared memory for this warp
 template <bool kL2 = false>
 MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w, int* idx_smem = nullptr,
-                           float* w_smem = nullptr, uint32_t* scratch = nullptr) {
-  if (E <= 256) topk_token<8, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch);
-  else if (E <= 512) topk_token<16, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch);
-  else topk_token<32, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch);
+                           float* w_smem = nullptr, uint32_t* scratch = nullptr,
+                           unsigned long long* stamps = nullptr) {
+  if (E <= 256) topk_token<8, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
+  else if (E <= 512) topk_token<16, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
+  else topk_token<32, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
 }
 
 // The permutation of n <= 32*k assignments by one warp, without block-wide barriers:

@@ -145,6 +145,16 @@ class MoeLayer:
             main.wait_event(ev[3])
         return self.y[:T]
 
+    def update_hot_tier(self, n_hot: int, stream=None) -> None:
+        """Refill the routed group's hot tier with the n_hot experts this layer has routed most
+        so far (the ranking of its cumulative histogram); 0 turns the tier off. Enqueued on
+        `stream` (default: current) after this layer's outstanding histogram. The one-kernel
+        decode layer then reads those experts' units from the tier, as persisting in L2 (the
+        process's set-aside: binding.moe_set_l2_persisting)."""
+        main = torch.cuda.current_stream() if stream is None else stream
+        self.join(main)
+        B.moe_hot_tier_update(self.experts.routed, self.rank, n_hot, stream=main)
+
     def join(self, stream=None) -> None:
         """Make `stream` (default: current) wait for the side-stream work of the last
         forward(join=False) of this layer, if one is outstanding (otherwise nothing to do)."""

@@ -169,3 +169,34 @@ def test_natural_weights_all_or_none():
     w = B._WeightsC(8, 512, 64, None, None, None, None, None, p.value, None, None, p.value)
     ex = B._ExpertsC(w, B._WeightsC(), 0)
     assert L.moe_expert_ffn(p, p, p, 4, ctypes.byref(ex), 2, p, p, p, 0, 0, p, None, p, 1 << 20, None) == INV
+
+
+def test_hot_tier_validation_without_gpu():
+    """moe_hot_tier_update and moe_layer_decode check the hot tier's arguments on the host
+    before any device call."""
+    L = B.lib()
+    INV, UNSUP = 1, 2
+    p = ctypes.c_void_p(0x10000)
+    w = B._WeightsC(8, 512, 64, p.value, p.value, p.value, p.value, p.value, p.value, None, None, p.value)
+    # no decode pack
+    w_nopack = B._WeightsC(8, 512, 64, p.value, p.value, p.value, p.value, p.value, p.value, None, None, None)
+    assert L.moe_hot_tier_update(ctypes.byref(w_nopack), p, 2, p, p, None) == INV
+    # n_hot out of range, missing buffers
+    assert L.moe_hot_tier_update(ctypes.byref(w), p, -1, p, p, None) == INV
+    assert L.moe_hot_tier_update(ctypes.byref(w), p, 9, p, p, None) == INV
+    assert L.moe_hot_tier_update(ctypes.byref(w), p, 2, None, p, None) == INV
+    assert L.moe_hot_tier_update(ctypes.byref(w), None, 2, p, p, None) == INV
+    # shapes the tier does not take: E % 4 != 0, d % 512 != 0
+    w6 = B._WeightsC(6, 512, 64, p.value, p.value, p.value, p.value, p.value, p.value, None, None, p.value)
+    assert L.moe_hot_tier_update(ctypes.byref(w6), p, 2, p, p, None) == UNSUP
+    w256 = B._WeightsC(8, 256, 64, p.value, p.value, p.value, p.value, p.value, p.value, None, None, p.value)
+    assert L.moe_hot_tier_update(ctypes.byref(w256), p, 2, p, p, None) == UNSUP
+    # misaligned hot_pack
+    assert L.moe_hot_tier_update(ctypes.byref(w), p, 2, ctypes.c_void_p(0x10008), p, None) == INV
+    # the layer call refuses a tier with n_hot > 0 but no buffers, or n_hot < 0
+    for hot_pack, hot_slot, n_hot in ((None, p.value, 2), (p.value, None, 2), (p.value, p.value, -1)):
+        wr = B._WeightsC(8, 512, 64, p.value, p.value, p.value, p.value, p.value, p.value, None, None, p.value,
+                         hot_pack, hot_slot, n_hot)
+        ex = B._ExpertsC(wr, B._WeightsC(), 0)
+        args = [p, 4, None, p, None, ctypes.byref(ex), 2] + [p] * 11 + [0, p, 1 << 20, None]
+        assert L.moe_layer_decode(*args) == INV, (hot_pack, hot_slot, n_hot)

@@ -1,11 +1,11 @@
 """A bounded device-side wait that runs out, and recovery afterwards (the one-kernel decode
 layer's grid barrier).
 
-The wait limit is shortened to 5 ms and the first of the barrier's arrival counters in the
-workspace is moved one past a whole generation, so the last CTA to arrive on it at the first
-barrier counts itself into the next generation and waits for arrivals that never come: its
-wait gives up, sets the device status to MOE_ERR_TIMEOUT and marks the workspace. Every access stays inside its buffers and every
-wait is bounded, so the GPU context stays usable. The next call on the marked workspace does
+The wait limit is shortened to 5 ms and the workspace's hold word (byte 1536, which the
+library never writes) is set, so CTA 0 holds back its barrier arrival and every other CTA
+waits for an arrival that never comes: their waits give up, set the device status to
+MOE_ERR_TIMEOUT and mark the workspace. Every access stays inside its buffers and every wait
+is bounded, so the GPU context stays usable. The next call on the marked workspace does
 nothing and reports MOE_ERR_WORKSPACE; after the caller zeroes the workspace the layer gives
 its normal result again.
 """
@@ -33,11 +33,11 @@ def test_decode_layer_wait_runs_out_then_recovers():
     x = synth.make_x(0, cfg, 8, step=9).cuda()
     y0 = lay.forward(x).clone()
     assert B.moe_get_device_status(clear=True) == 0
-    counter = lay.ws_dec[:8].view(torch.int64)
+    hold = lay.ws_dec[1536:1540].view(torch.int32)
     assert None not in barrier_generations(lay.ws_dec)
     B.moe_set_wait_limit_ns(5_000_000)
     try:
-        counter += 1  # one arrival too many: the next generation never completes
+        hold.fill_(1)  # CTA 0 does not arrive: the barrier never completes
         lay.forward(x)
         assert B.moe_get_device_status(clear=True) == B.MOE_ERR_TIMEOUT
         # the workspace is marked: the next call computes nothing and says so
