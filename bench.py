@@ -345,9 +345,11 @@ def measure_decode(timer, cfg, copies, xs, T, K, W, e2e_steps, stream, world, pe
     return out
 
 
-def build_prefill_layers(device, workload, decode_copies, n_copies: int):
+def build_prefill_layers(device, workload, decode_copies, n_copies: int, static_scales: bool = False):
     """Layers of the prefill workload. prefill: the decode copies' weights (the same layer)
-    with the prefill router (Zipf(0.8) popularity); wide: its own seeded weights."""
+    with the prefill router (Zipf(0.8) popularity); wide: its own seeded weights. With
+    static_scales each layer quantises every expert's rows with the expert's own static
+    input scales (synth.make_input_scales) instead of one per-call activation scale."""
     from nvfp4_expert_ffn_b200 import binding as B
     from nvfp4_expert_ffn_b200 import layer as L
     from nvfp4_expert_ffn_b200 import synth
@@ -361,8 +363,9 @@ def build_prefill_layers(device, workload, decode_copies, n_copies: int):
             experts = B.Experts(L.quantize_weights_gpu(SEED, cfg, layer=li, device=device),
                                 L.quantize_weights_gpu(SEED, cfg, layer=li, shared=True, device=device))
         Wr, br = synth.make_router(SEED, cfg, layer=li)
+        scales = tuple(t.to(device) for t in synth.make_input_scales(cfg)) if static_scales else None
         layers.append(L.MoeLayer(experts, Wr.to(device), br.to(device) if cfg.zipf_s > 0 else None, cfg.k, T,
-                                 device=device, fused=False))
+                                 device=device, fused=False, input_scales=scales))
         xs.append(synth.make_x(SEED, cfg, T, layer=li).to(device))
     return cfg, layers, xs
 
@@ -381,9 +384,14 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
 
     def ffn(i):  # the dominant call alone: the expert FFN (schedule, row gather, tcgen05 GEMMs)
         lay = layers[i % n]
-        B.moe_expert_ffn(lay.xq_codes[:T], lay.xq_scales[:T], lay.xq_ts[:1], lay.experts, k, lay.offsets,
-                         lay.sorted_assign[:T * k], lay.topk_w[:T], B.MOE_FFN_ACCUMULATE, lay.path, lay.y_acc[:T],
-                         None, lay.ws)
+        if lay.input_scales is not None:
+            B.moe_expert_ffn_static(xs[i % n], lay.experts, lay.input_scales[0], lay.input_scales[1], k, lay.offsets,
+                                    lay.sorted_assign[:T * k], lay.topk_w[:T], B.MOE_FFN_ACCUMULATE, lay.y_acc[:T],
+                                    None, lay.ws)
+        else:
+            B.moe_expert_ffn(lay.xq_codes[:T], lay.xq_scales[:T], lay.xq_ts[:1], lay.experts, k, lay.offsets,
+                             lay.sorted_assign[:T * k], lay.topk_w[:T], B.MOE_FFN_ACCUMULATE, lay.path,
+                             lay.y_acc[:T], None, lay.ws)
 
     with torch.cuda.stream(stream):
         for i in range(n):
@@ -406,7 +414,8 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
     out = {"value": round(whole_job_rate(world, T, K, ms), 1), "unit": "tokens/s", "ms_per_step": round(ms / K, 6),
            "T": T, "touched_experts_avg": round(float(np.mean(U)), 2),
            "gpu_launches": int(round(lps * K)), "gpu_launches_per_step": lps,
-           "roofline": {"kernel": "moe_expert_ffn (schedule, row gather, tcgen05 block-scaled grouped GEMMs)",
+           "roofline": {"kernel": ("moe_expert_ffn_static" if layers[0].input_scales is not None else "moe_expert_ffn")
+                        + " (schedule, row gather, tcgen05 block-scaled grouped GEMMs)",
                         "bound": "tensor", "achieved": round(tf, 1), "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                         "frac": round(tf / fp4_peak, 4),
                         "peak_kind": f"{peaks['kind']} bf16 (burst) x 4, the nominal dense FP4 : bf16 ratio",
@@ -434,9 +443,6 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
                       "h2d_bytes_per_step": T * cfg.d * 2, "d2h_bytes_per_step": T * cfg.d * 2,
                       "steps": e2e_steps, "api": "GraphedMoeLayer.run: pinned x -> device, layer, y -> pinned"}
         del runners
-    if tier is not None:
-        out["hot_tier"] = tier
-        hot_tier_off(copies, stream)
     return out
 
 
@@ -593,6 +599,13 @@ def run_gpu(args):
                                                       peaks)
             extra["prefill_T16384"]["workload"] = ("prefill MoE layer: the decode layer's weights, Zipf(0.8) "
                                                    "routing, T=16384 tokens per step, 2 layer copies")
+            del players
+            pcfg, players, pxs = build_prefill_layers(device, "prefill", copies, 2, static_scales=True)
+            extra["prefill_T16384_static_scales"] = measure_prefill(timer, pcfg, players, pxs, K, W, 0, stream,
+                                                                    world, peaks)
+            extra["prefill_T16384_static_scales"]["workload"] = (
+                "prefill_T16384 with static per-expert input scales: every expert quantises its own rows "
+                "(moe_expert_ffn_static), no per-call activation quantisation")
             del players
             if not args.no_stack:
                 del copies, xs

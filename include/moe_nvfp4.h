@@ -69,6 +69,7 @@ typedef enum moe_status {
 #define MOE_OP_QUANT 2
 #define MOE_OP_FFN 3
 #define MOE_OP_LAYER_DECODE 4 /* moe_layer_decode (zero-filled before its first use) */
+#define MOE_OP_FFN_STATIC 5   /* moe_expert_ffn_static */
 
 /*
  * Expert weights of one expert group (E routed experts, or E = 1 for the shared expert),
@@ -223,6 +224,29 @@ moe_status moe_expert_ffn(const uint8_t* xq_codes, const uint8_t* xq_scales,
                           float* shared_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_expert_ffn_static - moe_expert_ffn with static per-expert input scales: each expert
+ * quantises its own token rows from the bf16 activations with its own static tensor scale,
+ * and its h with its own static scale, instead of one per-call quantisation of the
+ * activations and h scale 1.0. Source: "Basalt" project page, "All the numbers", list
+ * "Engines: commit, and what is not NVIDIA's weights" (the llama.cpp row keeps NVIDIA's
+ * experts bit-exact including their input_scale).
+ *   x_bf16 [T][d] (16-byte aligned); in_scale_gu, in_scale_dn: float32 [E + has_shared]
+ *   (device; the shared expert's at index E): per expert, the tensor scale of its
+ *   activations and of its h (dequantisation multipliers, e.g. a calibrated amax / 2688).
+ *   Block scales and codes follow nvfp4_quantize_act with ts_in = the expert's scale.
+ *   Other arguments, modes and outputs as moe_expert_ffn. Always the tcgen05 PREFILL kernel
+ *   (any T; needs d % 256 == 0, I % 256 == 0, d <= 2048, I <= 768, the natural-layout
+ *   weights and the scales packed by moe_pack_experts), with every routed row quantised
+ *   once per (token, expert) by the row-gather step. The workspace is
+ *   moe_workspace_size(MOE_OP_FFN_STATIC, ...).
+ */
+moe_status moe_expert_ffn_static(const uint16_t* x_bf16, int32_t T, const moe_experts_t* W,
+                                 const float* in_scale_gu, const float* in_scale_dn, int32_t k,
+                                 const int32_t* offsets, const int32_t* sorted_assign,
+                                 const float* topk_w, int32_t mode, float* out, float* shared_out,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_combine - weighted combine (A9) and cast to bf16: a token's output is the sum of its
  * selected experts' outputs, weighted by the routing weights ("What Basalt changes in a
  * Blackwell local inference stack", section "Experts can move without becoming free").
@@ -310,7 +334,8 @@ moe_status moe_hot_tier_update(const moe_expert_weights_t* W, const int32_t* ran
 /*
  * moe_set_l2_persisting - size of the L2 set-aside for lines accessed as persisting (the
  * hot tier's window) in this process's CUDA context on the current device, clamped to the
- * device's maximum; 0 gives the set-aside back and returns persisting lines to normal. It
+ * device's maximum (the driver may round it up to its granularity); 0 gives the set-aside
+ * back and returns persisting lines to normal. It
  * is part of the context's state, not a setting of the GPU: it ends with the context
  * (process exit or cudaDeviceReset) and other processes do not see it. Writes the size in
  * effect to *bytes_out when not NULL.

@@ -22,6 +22,7 @@ MOE_OK = 0
 MOE_FFN_ACCUMULATE, MOE_FFN_PER_ASSIGN = 0, 1
 MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL, MOE_PATH_CUDA_CORE = 0, 1, 2, 3
 MOE_OP_LAYER, MOE_OP_ROUTE, MOE_OP_QUANT, MOE_OP_FFN, MOE_OP_LAYER_DECODE = 0, 1, 2, 3, 4
+MOE_OP_FFN_STATIC = 5
 MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE = 4, 5
 DEFAULT_WAIT_LIMIT_NS = 2_000_000_000
 
@@ -35,6 +36,7 @@ EXPORTS = {
     "moe_pack_experts": (_I32, [_P, _P, _P, _P, _P]),
     "moe_expert_ffn": (_I32, [_P, _P, _P, _I32, _P, _I32, _P, _P, _P, _I32, _I32, _P, _P, _P,
                               _SZ, _P]),
+    "moe_expert_ffn_static": (_I32, [_P, _I32, _P, _P, _P, _I32, _P, _P, _P, _I32, _P, _P, _P, _SZ, _P]),
     "moe_combine": (_I32, [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _I32, _P, _P]),
     "moe_expert_hist": (_I32, [_P, _I32, _P, _P, _I32, _P]),
     "moe_layer_decode": (_I32, [_P, _I32, _P, _P, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -260,6 +262,16 @@ def moe_expert_ffn(xq_codes, xq_scales, xq_ts, experts: Experts, k, offsets, sor
     _check("moe_expert_ffn", lib().moe_expert_ffn(
         _ptr(xq_codes), _ptr(xq_scales), _ptr(xq_ts), T, ctypes.byref(s), k, _ptr(offsets),
         _ptr(sorted_assign), _ptr(topk_w), mode, path, _ptr(out), _ptr(shared_out), _ptr(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def moe_expert_ffn_static(x, experts: Experts, in_scale_gu, in_scale_dn, k, offsets, sorted_assign,
+                          topk_w, mode, out, shared_out, ws, stream=None):
+    T = x.shape[0]
+    s = experts.struct()
+    _check("moe_expert_ffn_static", lib().moe_expert_ffn_static(
+        _ptr(x), T, ctypes.byref(s), _ptr(in_scale_gu), _ptr(in_scale_dn), k, _ptr(offsets),
+        _ptr(sorted_assign), _ptr(topk_w), mode, _ptr(out), _ptr(shared_out), _ptr(ws),
         0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
 
 

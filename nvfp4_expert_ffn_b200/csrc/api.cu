@@ -159,7 +159,8 @@ size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k
       size_t m = q > r ? q : r;
       return m > f ? m : f;
     }
-    case MOE_OP_LAYER_DECODE: return layer_dec_ws_bytes(T, E);
+    case MOE_OP_LAYER_DECODE: return layer_dec_ws_bytes(T, d, E);
+    case MOE_OP_FFN_STATIC: return align256(ffn_tc_static_ws_bytes(T, d, E, k, I));
   }
   return 0;
 }
@@ -376,7 +377,7 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "moe_layer_decode needs 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, "
                 "k <= E <= 1024 and at most 32 units per CTA");
-  if ((s = check_ws(ws, ws_bytes, layer_dec_ws_bytes(T, E))) != MOE_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, layer_dec_ws_bytes(T, d, E))) != MOE_OK) return s;
   LayerDecArgs a;
   a.x = x;
   a.ts_in = ts_in;
@@ -400,6 +401,58 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
   a.y = y;
   cudaError_t e = launch_layer_dec(a, ws, sms, dstatus, (cudaStream_t)stream);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_layer_decode launch");
+}
+
+moe_status moe_expert_ffn_static(const uint16_t* x, int32_t T, const moe_experts_t* W, const float* in_gu,
+                                 const float* in_dn, int32_t k, const int32_t* offsets,
+                                 const int32_t* sorted_assign, const float* topk_w, int32_t mode, float* out,
+                                 float* shared_out, void* ws, size_t ws_bytes, void* stream) {
+  if (!W) return fail(MOE_ERR_INVALID_ARG, "null weights");
+  const int E = W->routed.E, d = W->routed.d, I = W->routed.I;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (k < 1 || k > 32 || E < k || E > 1024) return fail(MOE_ERR_UNSUPPORTED_SHAPE, "need 1 <= k <= 32, k <= E <= 1024");
+  if (mode != MOE_FFN_ACCUMULATE && mode != MOE_FFN_PER_ASSIGN) return fail(MOE_ERR_INVALID_ARG, "bad mode");
+  if (d <= 0 || I <= 0 || ffn_tc_static_ws_bytes(1, d, E, k, I) == 0)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "static input scales need d % 256 == 0, I % 256 == 0, d <= 2048, I <= 768");
+  bool nat_r = false, nat_s = true;
+  moe_status s = check_weights(W->routed, "routed", E, d, I, &nat_r);
+  if (s != MOE_OK) return s;
+  if (W->has_shared && (s = check_weights(W->shared, "shared", 1, d, I, &nat_s)) != MOE_OK) return s;
+  const bool packed = W->routed.gu_sf_tiled && W->routed.dn_sf_tiled &&
+                      (!W->has_shared || (W->shared.gu_sf_tiled && W->shared.dn_sf_tiled));
+  if (!(nat_r && nat_s) || !packed)
+    return fail(MOE_ERR_UNSUPPORTED_SHAPE, "static input scales need the natural-layout weights and packed scales");
+  if (T == 0) return MOE_OK;
+  if (!x || !in_gu || !in_dn || !offsets || !sorted_assign || !topk_w || !out)
+    return fail(MOE_ERR_INVALID_ARG, "null tensor pointer");
+  if (!aligned16(x) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "x_bf16 and out must be 16-byte aligned");
+  if (mode == MOE_FFN_PER_ASSIGN && W->has_shared && !shared_out)
+    return fail(MOE_ERR_INVALID_ARG, "shared_out needed in PER_ASSIGN mode with a shared expert");
+  int sms = 0;
+  int32_t* dstatus = nullptr;
+  if ((s = device_info(&sms, &dstatus)) != MOE_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, ffn_tc_static_ws_bytes(T, d, E, k, I))) != MOE_OK) return s;
+  FfnArgs a;
+  a.xq_codes = nullptr;
+  a.xq_scales = nullptr;
+  a.xq_ts = nullptr;
+  a.x_bf16 = x;
+  a.in_gu = in_gu;
+  a.in_dn = in_dn;
+  a.T = T; a.d = d; a.I = I; a.E = E; a.k = k;
+  a.routed = to_group(W->routed);
+  a.shared = W->has_shared ? to_group(W->shared) : ExpertGroup{};
+  a.has_shared = W->has_shared ? 1 : 0;
+  a.offsets = offsets;
+  a.sorted_assign = sorted_assign;
+  a.topk_w = topk_w;
+  a.mode = mode;
+  a.out = out;
+  a.shared_out = shared_out;
+  a.h_codes = nullptr;
+  a.h_scales = nullptr;
+  cudaError_t e = launch_ffn_tc(a, ws, sms, dstatus, (cudaStream_t)stream);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "moe_expert_ffn_static launch");
 }
 
 moe_status moe_combine(int32_t T, int32_t d, int32_t k, int32_t mode, const float* expert_out,

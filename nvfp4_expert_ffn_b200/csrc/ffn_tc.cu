@@ -79,6 +79,9 @@ struct TcParams {
   const uint8_t* xq_codes;
   const uint8_t* xq_scales;
   const float* xq_ts;
+  const uint16_t* x_bf16;  // static input scales: rows are quantised from here (else NULL)
+  const float* in_gu;      // [E + 1] static activation scale of each expert (shared at E)
+  const float* in_dn;      // [E + 1] static h scale of each expert, or NULL (1.0)
   const int32_t* offsets;
   const int32_t* sorted_assign;
   const float* topk_w;
@@ -160,15 +163,38 @@ __global__ void __launch_bounds__(256) tc_row_gather_kernel(TcParams p) {
       wgt = p.topk_w[a];
       slot = q;
     }
-    if (p.a1) {
-      const uint4* csrc = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
-      uint4* cdst = reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
-      for (int c = lane; c < d / 32; c += 32) cdst[c] = __ldg(csrc + c);
+    if (p.x_bf16) {
+      // static input scales: the token's bf16 row quantised with its expert's own tensor
+      // scale. Lane l takes 16-element blocks l, l + 32, ...: its 8 code bytes go to the
+      // gathered row, its scale byte into the m-tile's scale atom.
+      const float ts = p.in_gu[e];
+      const uint4* xsrc = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)t * d);
+      uint2* cdst = reinterpret_cast<uint2*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
+      for (int blk = lane; blk < d / kBlock; blk += 32) {
+        const uint4 lo = __ldg(xsrc + 2 * blk), hi = __ldg(xsrc + 2 * blk + 1);
+        const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[2 * i] = __uint_as_float(wv[i] << 16);
+          v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        }
+        uint2 cw;
+        const uint32_t sb = quantize_block16(v, ts, &cw);
+        cdst[blk] = cw;
+        p.sfa1[((size_t)m * (d / 64) + blk / 4) * kAtom + (r % 32) * 16 + (r / 32) * 4 + blk % 4] = (uint8_t)sb;
+      }
+    } else {
+      if (p.a1) {
+        const uint4* csrc = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
+        uint4* cdst = reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
+        for (int c = lane; c < d / 32; c += 32) cdst[c] = __ldg(csrc + c);
+      }
+      const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
+      for (int kc = lane; kc < d / 64; kc += 32)
+        *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (r % 32) * 16 + (r / 32) * 4) =
+            __ldg(ssrc + kc);
     }
-    const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
-    for (int kc = lane; kc < d / 64; kc += 32)
-      *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (r % 32) * 16 + (r / 32) * 4) =
-          __ldg(ssrc + kc);
     if (lane == 0) {
       const size_t prow = (size_t)m * kTileM + r;
       p.row_token[prow] = t;
@@ -887,7 +913,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
     const int cq = ew >> 2;
     const int row = 32 * q + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16);
-    const float ts_x = *p.xq_ts;
+    const float ts_call = p.x_bf16 ? 1.0f : *p.xq_ts;  // per-call activation scale
     uint32_t tc = 0, jc = 0;
     bool go = true;
     int tix = 0;
@@ -923,6 +949,10 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
       // ---- gate/up tiles: SwiGLU and NVFP4 h into the shared-memory h tile. Tile j holds gate
       // rows of slice s = 2j + (cq >> 1) at columns 128(cq >> 1) .. +63 and its up rows 64
       // columns later; this thread takes h columns 32(cq & 1) .. +31 of that slice.
+      // tensor scales of this expert's activations and h: static per expert, or the call's
+      // activation scale and 1.0
+      const float ts_x = p.x_bf16 ? p.in_gu[e] : ts_call;
+      const float ts_h = p.in_dn ? p.in_dn[e] : 1.0f;
       const float sg = G.gu_ts[2 * eloc] * ts_x, su = G.gu_ts[2 * eloc + 1] * ts_x;
       const uint32_t cg = 128 * (cq >> 1) + 32 * (cq & 1);
       for (int jq = 0; jq < nt1 && go; ++jq) {
@@ -942,7 +972,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
             h[i] = __fdiv_rn(gv, 1.0f + expf(-gv)) * uv;
           }
           uint2 cw;
-          sbytes |= quantize_block16(h, 1.0f, &cw) << (8 * b);
+          sbytes |= quantize_block16(h, ts_h, &cw) << (8 * b);
           packed[2 * b] = cw.x;
           packed[2 * b + 1] = cw.y;
         }
@@ -970,7 +1000,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
       // each holds 4 consecutive columns of one row: row t/4 + 8(t%2) of the half, columns
       // 8i + 4((t/2)%2) .. +3. A warp's vector reduction covers 16 rows x 32 contiguous bytes
       // (two lanes per row) instead of 32 rows x 16 bytes, which L2 absorbs about twice as fast.
-      const float ts_o = G.dn_ts[eloc];  // h tensor scale is 1
+      const float ts_o = G.dn_ts[eloc] * ts_h;
       int orow = -1;  // output row of this thread's m-tile row (lane = row), -1 if padding
       float f = 0.0f;
       if (valid) {
@@ -1051,7 +1081,7 @@ bool mt_supported(int d, int I) {
   return d <= kMtMaxD && I <= kMtMaxI && d % kStageK == 0 && I % kStageK == 0 && mt_smem_bytes(d, I) <= kMtSmemMax;
 }
 
-TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
+TcLayout tc_layout(int64_t T, int d, int E, int k, int I, bool per_expert_rows = false) {
   TcLayout L;
   const int64_t n = T * k;
   L.max_m = (int)((n + kTileM - 1) / kTileM + (n < E ? n : E) + (T + kTileM - 1) / kTileM + 2);
@@ -1069,7 +1099,7 @@ TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
   // rows' scale atoms (every T)
   const bool mt = mt_supported(d, I);
   const bool big = T > kSmallT;
-  L.off_a1 = o; o += (big && (!mt || kMtPregather)) ? a256(L.rows_cap * (d / 2)) : 0;
+  L.off_a1 = o; o += ((big && (!mt || kMtPregather)) || per_expert_rows) ? a256(L.rows_cap * (d / 2)) : 0;
   L.off_sfa1 = o; o += (big || mt) ? a256(L.rows_cap * (d / kBlock)) : 0;
   L.off_h = o; o += a256(L.rows_cap * (I / 2));
   L.off_sfa2 = o; o += a256(L.rows_cap * (I / kBlock));
@@ -1082,6 +1112,11 @@ TcLayout tc_layout(int64_t T, int d, int E, int k, int I) {
 size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I) {
   if (d % kStageK || I % kStageK) return 0;
   return tc_layout(T, d, E, k, I).total;
+}
+
+size_t ffn_tc_static_ws_bytes(int64_t T, int d, int E, int k, int I) {
+  if (!mt_supported(d, I)) return 0;
+  return tc_layout(T, d, E, k, I, true).total;
 }
 
 bool ffn_tc_supported(int d, int I) { return d % kStageK == 0 && I % kStageK == 0 && d <= 16384 && I <= 16384; }
@@ -1107,7 +1142,8 @@ cudaError_t launch_pack_sf(const ExpertGroup& g, int E, int d, int I, uint8_t* g
 cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st) {
   cudaError_t e = get_encode();
   if (e != cudaSuccess) return e;
-  const TcLayout L = tc_layout(a.T, a.d, a.E, a.k, a.I);
+  const bool per_expert = a.x_bf16 != nullptr;  // static input scales: rows quantised per expert
+  const TcLayout L = tc_layout(a.T, a.d, a.E, a.k, a.I, per_expert);
   uint8_t* w = reinterpret_cast<uint8_t*>(ws);
   TcParams p;
   p.n_mtiles = reinterpret_cast<int32_t*>(w + L.off_hdr);
@@ -1119,7 +1155,8 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.row_weight = reinterpret_cast<float*>(w + L.off_w);
   p.row_slot = reinterpret_cast<int32_t*>(w + L.off_slot);
   const bool mt = mt_supported(a.d, a.I);
-  p.a1 = (a.T > kSmallT && (!mt || kMtPregather)) ? w + L.off_a1 : nullptr;
+  if (per_expert && !mt) return cudaErrorInvalidValue;  // the caller checks the shapes
+  p.a1 = ((a.T > kSmallT && (!mt || kMtPregather)) || per_expert) ? w + L.off_a1 : nullptr;
   p.sfa1 = (a.T > kSmallT || mt) ? w + L.off_sfa1 : nullptr;
   p.h_codes = w + L.off_h;
   p.sfa2 = w + L.off_sfa2;
@@ -1127,6 +1164,9 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   p.xq_codes = a.xq_codes;
   p.xq_scales = a.xq_scales;
   p.xq_ts = a.xq_ts;
+  p.x_bf16 = a.x_bf16;
+  p.in_gu = a.in_gu;
+  p.in_dn = a.in_dn;
   p.offsets = a.offsets;
   p.sorted_assign = a.sorted_assign;
   p.topk_w = a.topk_w;
@@ -1140,7 +1180,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
 
   TcMaps maps;
   const int d = a.d, I = a.I;
-  {
+  if (a.xq_codes) {
     cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)a.T};
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
     cuuint32_t box[2] = {128, 1};
@@ -1151,6 +1191,7 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
     cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
     cuuint32_t box[2] = {128, 128};
     if ((e = encode_u8(&maps.a1, p.a1, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess) return e;
+    if (!a.xq_codes) maps.xg = maps.a1;  // not read: the rows come from a1
   } else {
     maps.a1 = maps.xg;
   }

@@ -83,6 +83,12 @@ struct FfnArgs {
   const uint8_t* xq_codes;
   const uint8_t* xq_scales;
   const float* xq_ts;
+  // static per-expert input scales (tcgen05 m-tile path only): the bf16 activations, which
+  // each expert's rows are quantised from with in_gu[e], and h's scale in_dn[e]; NULL for the
+  // per-call quantised activations above and h scale 1
+  const uint16_t* x_bf16 = nullptr;
+  const float* in_gu = nullptr;
+  const float* in_dn = nullptr;
   int T, d, I, E, k;
   ExpertGroup routed, shared;
   int has_shared;
@@ -132,6 +138,9 @@ cudaError_t launch_combine(int T, int d, int k, int mode, const float* expert_ou
 // tensor-core (tcgen05) FFN path
 bool ffn_tc_supported(int d, int I);
 size_t ffn_tc_ws_bytes(int64_t T, int d, int E, int k, int I);
+// the m-tile kernel's workspace when rows are quantised per expert (static input scales);
+// 0 when the m-tile kernel does not take these shapes
+size_t ffn_tc_static_ws_bytes(int64_t T, int d, int E, int k, int I);
 cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
 // tcgen05 decode FFN (at most 8 tokens)
 bool ffn_dec_supported(int64_t T, int d, int I, int mode, int E, int k, int has_shared, int grid);
@@ -160,7 +169,7 @@ struct LayerDecArgs {
   uint16_t* y;
 };
 bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms);
-size_t layer_dec_ws_bytes(int64_t T, int E);
+size_t layer_dec_ws_bytes(int64_t T, int d, int E);
 cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
 cudaError_t launch_pack_dec(const ExpertGroup& g, int E, int d, int I, const uint8_t* gu_sf_tiled,
                             const uint8_t* dn_sf_tiled, uint8_t* dec_pack, int num_sms, cudaStream_t st);

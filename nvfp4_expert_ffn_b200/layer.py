@@ -55,8 +55,12 @@ class MoeLayer:
 
     def __init__(self, experts: B.Experts, Wr: torch.Tensor, br: Optional[torch.Tensor], k: int,
                  T_max: int, static_ts: Optional[torch.Tensor] = None, device="cuda",
-                 fused: Optional[bool] = None):
+                 fused: Optional[bool] = None, input_scales: Optional[tuple] = None):
+        """input_scales: optional (in_gu, in_dn) float32 [E + 1] device tensors, static
+        per-expert input scales (moe_expert_ffn_static); the layer then skips the per-call
+        activation quantisation and always runs the five-call path."""
         self.experts, self.Wr, self.br, self.k = experts, Wr, br, k
+        self.input_scales = input_scales
         r = experts.routed
         self.E, self.d, self.I = r.E, r.d, r.I
         self.T_max = T_max
@@ -77,6 +81,8 @@ class MoeLayer:
         self.cum = torch.zeros(E, dtype=torch.int64, device=dev)
         self.rank = torch.empty(E, dtype=torch.int32, device=dev)
         ws = B.moe_workspace_size(B.MOE_OP_LAYER, T_max, d, E, k, I)
+        if input_scales is not None:
+            ws = max(ws, B.moe_workspace_size(B.MOE_OP_FFN_STATIC, T_max, d, E, k, I))
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
         # the quantiser runs concurrently with the router, so it gets its own workspace
         self.ws_q = torch.empty(B.moe_workspace_size(B.MOE_OP_QUANT, T_max, d, E, k, I),
@@ -90,6 +96,7 @@ class MoeLayer:
         can_fuse = (d % 512 == 0 and d <= 4096 and I % 64 == 0 and k <= 32 and E <= 1024
                     and experts.routed.dec_pack is not None
                     and (experts.shared is None or experts.shared.dec_pack is not None))
+        can_fuse = can_fuse and input_scales is None
         self.fused = can_fuse if fused is None else (fused and can_fuse)
         self.ws_dec = torch.zeros(
             max(256, B.moe_workspace_size(B.MOE_OP_LAYER_DECODE, min(T_max, 8), d, E, k, I)),
@@ -122,20 +129,27 @@ class MoeLayer:
             if join:
                 main.wait_event(ev[3])
             return self.y[:T]
-        ev[0].record(main)
-        side.wait_event(ev[0])
-        B.nvfp4_quantize_act(x, self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
-                             ts_in=self.static_ts, ws=self.ws_q, stream=side)
-        ev[1].record(side)
+        static = self.input_scales is not None
+        if not static:
+            ev[0].record(main)
+            side.wait_event(ev[0])
+            B.nvfp4_quantize_act(x, self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1],
+                                 ts_in=self.static_ts, ws=self.ws_q, stream=side)
+            ev[1].record(side)
         B.moe_route(x, self.Wr, self.br, k, self.topk_idx[:T], self.topk_w[:T], self.counts,
                     self.offsets, self.sorted_assign[:T * k], self.assign_pos[:T * k], self.ws,
                     stream=main)
         ev[2].record(main)
-        main.wait_event(ev[1])
-        B.moe_expert_ffn(self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1], self.experts, k,
-                         self.offsets, self.sorted_assign[:T * k], self.topk_w[:T],
-                         B.MOE_FFN_ACCUMULATE, self.path, self.y_acc[:T], None, self.ws,
-                         stream=main)
+        if static:
+            B.moe_expert_ffn_static(x, self.experts, self.input_scales[0], self.input_scales[1], k,
+                                    self.offsets, self.sorted_assign[:T * k], self.topk_w[:T],
+                                    B.MOE_FFN_ACCUMULATE, self.y_acc[:T], None, self.ws, stream=main)
+        else:
+            main.wait_event(ev[1])
+            B.moe_expert_ffn(self.xq_codes[:T], self.xq_scales[:T], self.xq_ts[:1], self.experts, k,
+                             self.offsets, self.sorted_assign[:T * k], self.topk_w[:T],
+                             B.MOE_FFN_ACCUMULATE, self.path, self.y_acc[:T], None, self.ws,
+                             stream=main)
         side.wait_event(ev[2])
         B.moe_expert_hist(self.counts, self.cum, self.rank, stream=side)
         ev[3].record(side)

@@ -160,6 +160,19 @@ def make_router(seed: int, cfg: LayerShape, layer: int = 0, epoch: int = 0, devi
     return Wr, br
 
 
+def make_input_scales(cfg: LayerShape):
+    """Static per-expert input scales (float32 [E + 1], the shared expert's last), standing
+    in for calibrated ones: in_gu[e] = (1 + (e % 7) / 7) * 2*sqrt(3) / 2688 for the
+    activations (2*sqrt(3) bounds |x| of the synthetic activations, so no block scale
+    saturates) and in_dn[e] = (1 + (e % 5) / 5) / 64 for h. The factors vary by expert so that
+    experts quantise the same token differently."""
+    e = np.arange(cfg.E + 1)
+    x_bound = np.float32(2.0 * np.sqrt(3.0))
+    in_gu = ((1.0 + (e % 7) / 7.0) * (x_bound / np.float32(2688.0))).astype(np.float32)
+    in_dn = ((1.0 + (e % 5) / 5.0) / 64.0).astype(np.float32)
+    return torch.from_numpy(in_gu), torch.from_numpy(in_dn)
+
+
 def make_expert_weights_bf16(seed: int, cfg: LayerShape, expert: int, layer: int = 0,
                              shared: bool = False, device="cpu"):
     """Unquantised weights of one expert as bf16 bit patterns (int16), the precision a

@@ -27,6 +27,9 @@ oracle takes the plainest reading, listed in each function's docstring:
      before the down projection; a shared expert, if present, is added with weight 1.
   R6 token permutation is a stable counting sort of the (token, slot) assignments by expert.
   R7 cumulative per-expert counts rank experts hot to cold (ties to the lower index).
+  R13 static per-expert input scales (the input_scale of NVIDIA's experts): when given, an
+     expert's token rows are quantised with its own static tensor scale in_gu[e] and its h
+     with in_dn[e], instead of the per-call dynamic scale and 1.0.
 
 Precision: float32 where the reading fixes float32 (quantiser steps, logits, routing
 weights, h), float64 elsewhere (dot products, combine).

@@ -128,11 +128,12 @@ class Expert:
         return g, u, dn
 
 
-def expert_ffn(x_hat, expert: Expert, dense=None):
+def expert_ffn(x_hat, expert: Expert, dense=None, h_ts=1.0):
     """Reading R5 for a batch of dequantised token rows x_hat float64 [n][d]:
         g = x_hat Wg^T, u = x_hat Wu^T         (float64)
         h = silu(g) * u                        (float64, rounded once to float32)
-        h_hat = NVFP4(h) with tensor scale 1.0 (blocks of 16 along I)
+        h_hat = NVFP4(h) with tensor scale h_ts (blocks of 16 along I); h_ts is 1.0 unless
+                the expert has a static input scale for its down projection (R13)
         o = h_hat Wd^T                         (float64)
     Returns o float64 [n][d]."""
     Wg, Wu, Wd = dense if dense is not None else expert.dense()
@@ -142,9 +143,52 @@ def expert_ffn(x_hat, expert: Expert, dense=None):
     g = x_hat @ Wg.T
     u = x_hat @ Wu.T
     h = (silu(g) * u).astype(F32)
-    hc, hs, hts = nvfp4.quantize(h, ts=F32(1.0))
+    hc, hs, hts = nvfp4.quantize(h, ts=F32(h_ts))
     h_hat = nvfp4.dequantize(hc, hs, hts)
     return h_hat @ Wd.T
+
+
+def expert_ffn_static(x_f32, expert: Expert, in_gu, in_dn, dense=None):
+    """Reading R13, static per-expert input scales ("Basalt" project page, "All the numbers",
+    list "Engines: commit, and what is not NVIDIA's weights": NVIDIA's NVFP4 experts come
+    with their input_scale): the expert's token rows x (float32 [n][d], the bf16
+    activations) are quantised to NVFP4 with the expert's own static tensor scale in_gu
+    instead of the per-call dynamic one, and h with the expert's static scale in_dn; the
+    rest is expert_ffn. Returns o float64 [n][d]."""
+    xc, xs, xts = nvfp4.quantize(np.asarray(x_f32, dtype=F32), ts=F32(in_gu))
+    return expert_ffn(nvfp4.dequantize(xc, xs, xts), expert, dense, h_ts=in_dn)
+
+
+def ffn_static_forward(x_bits, idx, w, experts, shared, in_gu, in_dn, tokens=None):
+    """The expert FFN and the combine (A5-A9) with static per-expert input scales (R13) for a
+    given routing: y[t] = sum_j w[t, j] * o_{idx[t, j]}(x_t) + o_shared(x_t), every o from
+    expert_ffn_static with that expert's scales (the shared expert's at index E of in_gu and
+    in_dn). x_bits: bf16 bit patterns [T][d]; idx, w: [T][k]. Rows outside `tokens` (default
+    all) are NaN. Returns y float64 [T][d]."""
+    x_bits = np.asarray(x_bits)
+    T, d = x_bits.shape
+    E = len(experts)
+    k = np.asarray(idx).shape[1]
+    x_f32 = (x_bits.astype(np.uint16).astype(np.uint32) << 16).view(F32).reshape(T, d)
+    tokens = np.arange(T) if tokens is None else np.asarray(sorted(set(tokens)))
+    idx, w = np.asarray(idx), np.asarray(w)
+    o = {}
+    for e in range(E):
+        rows = [(t, j) for t in tokens for j in range(k) if idx[t, j] == e]
+        if rows:
+            oe = expert_ffn_static(x_f32[[t for t, _ in rows]], experts[e], in_gu[e], in_dn[e])
+            for (t, j), r in zip(rows, oe):
+                o[(t, j)] = r
+    o_shared = None
+    if shared is not None:
+        o_shared = np.zeros((T, d))
+        o_shared[tokens] = expert_ffn_static(x_f32[tokens], shared, in_gu[E], in_dn[E])
+    y = np.full((T, d), np.nan)
+    if tokens.size:
+        o_assign = np.concatenate([np.stack([o[(t, j)] for j in range(k)]) for t in tokens])
+        y[tokens] = combine(len(tokens), d, idx[tokens], w[tokens], o_assign,
+                            None if o_shared is None else o_shared[tokens])
+    return y
 
 
 # --------------------------------------------------------------------------- combine (A9)

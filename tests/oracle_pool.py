@@ -34,6 +34,14 @@ def _expert_rows(cfg_name, seed, layer, e, shared, x_hat_rows):
     return e, shared, omoe.expert_ffn(x_hat_rows, ex)
 
 
+def _expert_rows_static(cfg_name, seed, layer, e, shared, x_rows, in_gu, in_dn):
+    from nvfp4_expert_ffn_b200 import synth
+    from oracle import moe as omoe
+    from oracle.weights import synth_expert
+    ex = synth_expert(seed, synth.CONFIGS[cfg_name], e, layer, shared=shared)
+    return e, shared, omoe.expert_ffn_static(x_rows, ex, in_gu, in_dn)
+
+
 class OraclePool:
     """A pool of host processes kept across many expert_outputs calls (use as a context
     manager)."""
@@ -54,6 +62,19 @@ class OraclePool:
         (expert id, shared) -> o rows float64 [n][d], in the order of the given rows."""
         futs = [self.ex.submit(_expert_rows, cfg_name, seed, layer, e, sh, np.ascontiguousarray(rows))
                 for e, sh, rows in tasks]
+        out = {}
+        for f in cf.as_completed(futs):
+            e, sh, o = f.result()
+            out[(e, sh)] = o
+        return out
+
+
+    def expert_outputs_static(self, cfg_name, seed, layer, tasks):
+        """As expert_outputs with static input scales: tasks are (expert id, shared flag,
+        x rows float32 [n][d], in_gu, in_dn) and the rows are the unquantised activations."""
+        futs = [self.ex.submit(_expert_rows_static, cfg_name, seed, layer, e, sh, np.ascontiguousarray(rows),
+                               gu, dn)
+                for e, sh, rows, gu, dn in tasks]
         out = {}
         for f in cf.as_completed(futs):
             e, sh, o = f.result()

@@ -111,6 +111,9 @@ def test_layer_output_unchanged_and_tier_is_read():
 
 
 def test_l2_persisting_setaside_set_and_released():
+    # the driver rounds the set-aside up to its own granularity
     got = B.moe_set_l2_persisting(8 << 20)
-    assert 0 < got <= 8 << 20
+    assert got >= 8 << 20
+    most = B.moe_set_l2_persisting(1 << 40)
+    assert got <= most < (1 << 40)
     assert B.moe_set_l2_persisting(0) == 0
