@@ -36,10 +36,17 @@ METRIC = "MoE-layer tokens/s (decode T=1–8, prefill T=16K); % of HBM BW / FP4 
 SEED = 0
 X_DRAWS = 4             # input draws per decode layer copy
 NOMINAL_HBM_GBS = 8000.0  # B200 spec-sheet HBM3e bandwidth, for context beside the measured peak
-# DRAM bytes / algorithmic bytes of layer_dec_kernel from an ncu capture without cache control
-# inside the rotating decode loop; None until the current kernel has been captured
-DECODE_TRAFFIC_RATIO = None
-DECODE_TRAFFIC_SOURCE = None
+# DRAM bytes (read + write) per launch of the dominant kernels from ncu captures of the
+# current kernels (profiles/); None when the kernel has changed since its capture
+DECODE_TRAFFIC_RATIO = 0.874  # layer_dec_kernel: traffic / algorithmic bytes in the rotating loop
+DECODE_TRAFFIC_SOURCE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                         "--cache-control none (1 pass) on 10 launches inside the 8-copy rotating decode loop "
+                         "(T=8): 49.88 MB per launch against 57.09 MB of algorithmic bytes; the ratio is "
+                         "applied to this run's algorithmic bytes")
+PREFILL_TRAFFIC_BYTES = 3_271_831_000  # tc_ffn_mt_kernel, T = 16384, one launch
+PREFILL_TRAFFIC_SOURCE = ("ncu --set full capture of tc_ffn_mt_kernel at T=16384 (caches flushed): "
+                          "dram__bytes_read.sum 2.168 GB + dram__bytes_write.sum 1.104 GB; the m-tile "
+                          "kernel only, not the schedule and row-gather launches of the call")
 
 
 def _peaks():
@@ -237,7 +244,7 @@ def hot_tier_on(layers, n_layers_sharing: int, stream):
     lay0 = layers[0]
     setaside = B.moe_set_l2_persisting(1 << 40)
     per_expert = B.dec_pack_bytes(1, lay0.d, lay0.I)
-    n_hot = int(setaside // (n_layers_sharing * per_expert))
+    n_hot = int(round(setaside / (n_layers_sharing * per_expert)))
     with torch.cuda.stream(stream):
         for lay in layers:
             lay.update_hot_tier(n_hot, stream=stream)
@@ -420,7 +427,11 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
                         "frac": round(tf / fp4_peak, 4),
                         "peak_kind": f"{peaks['kind']} bf16 (burst) x 4, the nominal dense FP4 : bf16 ratio",
                         "flops_per_launch": flops, "weight_bytes_per_launch": int(wbytes),
-                        "avg_launch_us": round(ms_f / K * 1e3, 3), "traffic": None}}
+                        "avg_launch_us": round(ms_f / K * 1e3, 3),
+                        "traffic": (PREFILL_TRAFFIC_BYTES if cfg.name == "prefill" and layers[0].input_scales is None
+                                    else None),
+                        "traffic_source": (PREFILL_TRAFFIC_SOURCE if cfg.name == "prefill"
+                                           and layers[0].input_scales is None else None)}}
     if e2e_steps:
         runners = [lay.graphed(T, n_slots=1, stream=stream) for lay in layers]
         for r, x in zip(runners, xs):

@@ -159,7 +159,7 @@ size_t moe_workspace_size(int32_t op, int64_t T, int32_t d, int32_t E, int32_t k
       size_t m = q > r ? q : r;
       return m > f ? m : f;
     }
-    case MOE_OP_LAYER_DECODE: return layer_dec_ws_bytes(T, d, E);
+    case MOE_OP_LAYER_DECODE: return layer_dec_ws_bytes(T, E);
     case MOE_OP_FFN_STATIC: return align256(ffn_tc_static_ws_bytes(T, d, E, k, I));
   }
   return 0;
@@ -377,7 +377,7 @@ moe_status moe_layer_decode(const uint16_t* x, int32_t T, const float* ts_in, co
     return fail(MOE_ERR_UNSUPPORTED_SHAPE,
                 "moe_layer_decode needs 1 <= T <= 8, d % 512 == 0, d <= 4096, I % 64 == 0, 1 <= k <= 32, "
                 "k <= E <= 1024 and at most 32 units per CTA");
-  if ((s = check_ws(ws, ws_bytes, layer_dec_ws_bytes(T, d, E))) != MOE_OK) return s;
+  if ((s = check_ws(ws, ws_bytes, layer_dec_ws_bytes(T, E))) != MOE_OK) return s;
   LayerDecArgs a;
   a.x = x;
   a.ts_in = ts_in;

@@ -169,7 +169,7 @@ struct LayerDecArgs {
   uint16_t* y;
 };
 bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms);
-size_t layer_dec_ws_bytes(int64_t T, int d, int E);
+size_t layer_dec_ws_bytes(int64_t T, int E);
 cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32_t* status, cudaStream_t st);
 cudaError_t launch_pack_dec(const ExpertGroup& g, int E, int d, int I, const uint8_t* gu_sf_tiled,
                             const uint8_t* dn_sf_tiled, uint8_t* dec_pack, int num_sms, cudaStream_t st);

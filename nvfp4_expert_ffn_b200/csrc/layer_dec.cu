@@ -38,8 +38,6 @@
 namespace moe {
 
 constexpr int kLayerMaxK = 32;
-constexpr int kLayerReplicas = 8;  // copies of the data that every CTA reads after the barrier
-constexpr bool kWarmTopk = true;
 constexpr int kLayerMaxRows = kDecThreads / 32;  // router rows per CTA (the host checks E <= grid * this)
 
 RT_TRACE_ARRAY(g_layer_trace)
@@ -66,11 +64,8 @@ struct LayerArgs {
   int32_t* assign_pos;     // [T*k]
   float* y_acc;        // [T][d]
   uint16_t* y;         // [T][d] bf16
-  // workspace: kLayerReplicas copies of the logits and of the quantised activations, so that
-  // each line read by every CTA after the barrier has G / kLayerReplicas readers
-  float* logits;       // [R][T][E], copy r at r * rep_logits floats
-  uint8_t* xq_rep;     // [R][T][d/2 + d/16]: codes then scales of each copy, rep_xq bytes apart
-  size_t rep_logits, rep_xq;
+  // workspace
+  float* logits;       // [T][E]
   unsigned long long* sync;  // arrival counter of the grid barrier (zero before the first call)
   unsigned int* poison;      // nonzero once a call on this workspace gave up at a bounded wait
   const unsigned int* hold;  // nonzero: CTA 0 does not arrive at the barrier (set only by tests)
@@ -303,18 +298,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
       const uint32_t swd = sbyte | (__shfl_down_sync(0xffffffffu, sbyte, 8) << 8) |
                            (__shfl_down_sync(0xffffffffu, sbyte, 16) << 16) |
                            (__shfl_down_sync(0xffffffffu, sbyte, 24) << 24);
-      if ((lane & 3) == 0) {
-        reinterpret_cast<uint32_t*>(p.xq_codes)[8 * g + (lane >> 2)] = word;
-#pragma unroll
-        for (int r = 0; r < kLayerReplicas; ++r)
-          reinterpret_cast<uint32_t*>(p.xq_rep + r * p.rep_xq)[8 * g + (lane >> 2)] = word;
-      }
-      if (lane == 0) {
-        reinterpret_cast<uint32_t*>(p.xq_scales)[g] = swd;
-#pragma unroll
-        for (int r = 0; r < kLayerReplicas; ++r)
-          reinterpret_cast<uint32_t*>(p.xq_rep + r * p.rep_xq + (size_t)T * (d / 2))[g] = swd;
-      }
+      if ((lane & 3) == 0) reinterpret_cast<uint32_t*>(p.xq_codes)[8 * g + (lane >> 2)] = word;
+      if (lane == 0) reinterpret_cast<uint32_t*>(p.xq_scales)[g] = swd;
     }
     if (b == G - 1 && threadIdx.x == 0) *p.xq_ts = ts;
   }
@@ -376,11 +361,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
         float sum = 0.0f;
         for (int w = 0; w < (int)(blockDim.x >> 5); ++w) sum += sc.part[32 * w + lane];
         const int r = r0 + (lane >> 3), t = lane & 7;
-        if (r < nrows && t < T) {
-          const float v = sum + s_bias[r];
-#pragma unroll
-          for (int c = 0; c < kLayerReplicas; ++c) p.logits[c * p.rep_logits + (size_t)t * E + b + r * G] = v;
-        }
+        if (r < nrows && t < T) p.logits[(size_t)t * E + b + r * G] = sum + s_bias[r];
       }
       __syncthreads();
     }
@@ -397,19 +378,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
     mbar_wait(&s_wbar, 0, &no_abort, p.status);
   }
   RT_TRACE(g_layer_trace, 0, 3);
-  const unsigned long long bar_target = grid_arrive(p.sync, abort);
-  // While the other CTAs arrive, the top-k warps run the top-k once on a dummy row, so that
-  // its instructions (run once per launch, after a weight stream that has flushed the
-  // caches) are fetched before the real logits can be read.
-  if (kWarmTopk && live && warp < T && 16 * d >= 4 * E * kDecMaxT) {
-    float* dummy = reinterpret_cast<float*>(sc.xb) + (size_t)warp * E;
-    for (int e = lane; e < E; e += 32) dummy[e] = (float)((e * 37) % 101);
-    __syncwarp();
-    topk_dispatch(dummy, E, k, nullptr, nullptr, sc.tidx + warp * kLayerMaxK, sc.tw + warp * kLayerMaxK,
-                  sc.tks + warp * 64);
-    __syncwarp();
-  }
-  bool ok = grid_wait(p.sync, bar_target, abort, p.status);
+  bool ok = grid_sync(p.sync, abort, p.status);
   RT_TRACE(g_layer_trace, 0, 4);
   if (threadIdx.x == 0 && s_hot) {
     // long landed by now; waited for on every path, as it must land before the CTA exits
@@ -425,6 +394,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   const int nt1 = p.I / 64;
   const bool writer = b == G - 1;  // the CTA with the fewest units writes the routing outputs
   int nu = 0;
+#ifdef MOE_TRACE
+  // trace builds: the latency of one L2 load of data older than this launch (the router bias)
+  // and of one logit written by another CTA before the barrier, in SM cycles
+  if (ok && threadIdx.x == 0 && b < kTraceCtas && p.br) {
+    unsigned long long c0, c1, c2;
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c0));
+    const float a = __ldcg(p.br + (b * 7) % E);
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c1) : "f"(a));
+    const float l = __ldcg(p.logits + (size_t)((b * 131 + 17) % (T * E)));
+    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c2) : "f"(l));
+    g_layer_trace[5][b][0] = c1 - c0;
+    g_layer_trace[5][b][1] = c2 - c1;
+    g_layer_trace[5][b][2] = __float_as_uint(a + l);
+  }
+#endif
   if (ok) {
     if (warp < T) {
       // token `warp`: its logits straight from L2 into the top-k; the chosen experts are
@@ -433,8 +417,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
 #ifdef MOE_TRACE
       if (warp == 0 && b < kTraceCtas) stamps = &g_layer_trace[4][b][0];
 #endif
-      topk_dispatch<true>(p.logits + (b % kLayerReplicas) * p.rep_logits + (size_t)warp * E, E, k,
-                          writer ? p.topk_idx + (size_t)warp * k : nullptr,
+      topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
                           writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
                           sc.tw + warp * kLayerMaxK, sc.tks + warp * 64, stamps);
       RT_TRACE(g_layer_trace, 3, 0);
@@ -452,8 +435,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
       const int cpr = d / 32, q4 = d / 256;       // 16-byte code / scale pieces of a token row
       const int nc = kDecMaxT * cpr, ns = kDecMaxT * q4;
       const int rot_c = (b * 37) % nc;
-      const uint8_t* rep_codes = p.xq_rep + (b % kLayerReplicas) * p.rep_xq;  // this CTA's copy
-      const uint8_t* rep_scales = rep_codes + (size_t)T * (d / 2);
       auto code_piece = [&](int iu) { return iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc; };
       for (int i0 = tid; i0 < nc + ns; i0 += 8 * nth) {
         uint4 v[8];
@@ -463,11 +444,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
           v[u] = make_uint4(0u, 0u, 0u, 0u);
           if (iu < nc) {
             const int i = code_piece(iu), t = i / cpr;
-            if (t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(rep_codes + (size_t)t * (d / 2)) + i % cpr);
+            if (t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + i % cpr);
           } else if (iu < nc + ns) {
             const int t = (iu - nc) / q4;
             if (t < T)
-              v[u] = __ldcg(reinterpret_cast<const uint4*>(rep_scales + (size_t)t * (d / kBlock)) + (iu - nc) % q4);
+              v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_scales + (size_t)t * (d / kBlock)) + (iu - nc) % q4);
           }
         }
 #pragma unroll
@@ -653,14 +634,10 @@ size_t a256l(size_t v) { return (v + 255) & ~(size_t)255; }
 int layer_grid(int num_sms) { return num_sms > 1 ? num_sms - 1 : 1; }
 }  // namespace
 
-// workspace: the barrier word, the mark and the hold word (each on its own line), then
-// kLayerReplicas copies of the logits, then as many copies of the quantised activations
+// workspace: the barrier word, the mark and the hold word (each on its own line), then the
+// logits
 constexpr size_t kLayerWsHeader = 2048, kLayerWsPoison = 1024, kLayerWsHold = 1536;
-size_t rep_logits_bytes(int64_t T, int E) { return a256l((size_t)T * E * 4); }
-size_t rep_xq_bytes(int64_t T, int d) { return a256l((size_t)T * (d / 2 + d / 16)); }
-size_t layer_dec_ws_bytes(int64_t T, int d, int E) {
-  return kLayerWsHeader + kLayerReplicas * (rep_logits_bytes(T, E) + rep_xq_bytes(T, d));
-}
+size_t layer_dec_ws_bytes(int64_t T, int E) { return kLayerWsHeader + a256l((size_t)T * E * 4); }
 
 bool layer_dec_supported(int64_t T, int d, int I, int E, int k, int has_shared, int num_sms) {
   const int G = layer_grid(num_sms);
@@ -708,9 +685,6 @@ cudaError_t launch_layer_dec(const LayerDecArgs& a, void* ws, int num_sms, int32
   p.poison = reinterpret_cast<unsigned int*>(w + kLayerWsPoison);
   p.hold = reinterpret_cast<const unsigned int*>(w + kLayerWsHold);
   p.logits = reinterpret_cast<float*>(w + kLayerWsHeader);
-  p.rep_logits = rep_logits_bytes(a.T, a.E) / 4;
-  p.xq_rep = w + kLayerWsHeader + kLayerReplicas * rep_logits_bytes(a.T, a.E);
-  p.rep_xq = rep_xq_bytes(a.T, a.d);
   p.status = status;
   // a hot tier: its copies are read as persisting in L2, everything else as streaming
   cudaAccessPolicyWindow win = {};

@@ -200,3 +200,26 @@ def test_hot_tier_validation_without_gpu():
         ex = B._ExpertsC(wr, B._WeightsC(), 0)
         args = [p, 4, None, p, None, ctypes.byref(ex), 2] + [p] * 11 + [0, p, 1 << 20, None]
         assert L.moe_layer_decode(*args) == INV, (hot_pack, hot_slot, n_hot)
+
+
+def test_static_scales_validation_without_gpu():
+    """moe_expert_ffn_static refuses shapes the m-tile kernel does not take, weights without
+    their packed scales, and missing scale arrays, on the host."""
+    L = B.lib()
+    INV, UNSUP = 1, 2
+    p = ctypes.c_void_p(0x10000)
+
+    def call(E, d, I, packed=True, gu=p, dn=p, T=16):
+        sf = p.value if packed else None
+        w = B._WeightsC(E, d, I, p.value, p.value, p.value, p.value, p.value, p.value, sf, sf, None)
+        ex = B._ExpertsC(w, B._WeightsC(), 0)
+        return L.moe_expert_ffn_static(p, T, ctypes.byref(ex), gu, dn, 2, p, p, p, 0, p, None, p, 1 << 30, None)
+
+    assert call(8, 4096, 512) == UNSUP      # d above the m-tile kernel's 2048
+    assert call(8, 2048, 1024) == UNSUP     # I above 768
+    assert call(8, 2048, 320) == UNSUP      # I % 256 != 0
+    assert call(8, 2048, 512, packed=False) == UNSUP
+    assert call(8, 2048, 512, gu=None) == INV
+    assert call(8, 2048, 512, dn=None) == INV
+    assert call(8, 2048, 512, T=-1) == INV
+    assert call(8, 2048, 512, T=0) == 0     # nothing to do
