@@ -238,21 +238,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
     const uint4* x4 = reinterpret_cast<const uint4*>(p.x);
     uint4* xb4 = reinterpret_cast<uint4*>(sc.xb);
     for (int i0 = threadIdx.x; i0 < nx; i0 += 8 * blockDim.x) {
+      // all of a round's loads in flight together (past the end: piece 0, not used)
       uint4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * blockDim.x;
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-        if (i < nx) v[u] = __ldg(x4 + i);
+        v[u] = __ldg(x4 + (i < nx ? i : 0));
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = i0 + u * blockDim.x;
-        if (i < nx) xb4[i] = v[u];
-        mx2 = __vmaxu2(mx2, v[u].x & 0x7FFF7FFFu);
-        mx2 = __vmaxu2(mx2, v[u].y & 0x7FFF7FFFu);
-        mx2 = __vmaxu2(mx2, v[u].z & 0x7FFF7FFFu);
-        mx2 = __vmaxu2(mx2, v[u].w & 0x7FFF7FFFu);
+        if (i < nx) {
+          xb4[i] = v[u];
+          mx2 = __vmaxu2(mx2, v[u].x & 0x7FFF7FFFu);
+          mx2 = __vmaxu2(mx2, v[u].y & 0x7FFF7FFFu);
+          mx2 = __vmaxu2(mx2, v[u].z & 0x7FFF7FFFu);
+          mx2 = __vmaxu2(mx2, v[u].w & 0x7FFF7FFFu);
+        }
       }
     }
   }
@@ -415,7 +417,34 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
       // marked in s_bits
       unsigned long long* stamps = nullptr;
 #ifdef MOE_TRACE
-      if (warp == 0 && b < kTraceCtas) stamps = &g_layer_trace[4][b][0];
+      if (warp == 0 && b < kTraceCtas) {
+        stamps = &g_layer_trace[4][b][0];
+        // trace builds: the 16 logit loads of the top-k alone, through L2 and plain, timed
+        {
+          const float* row = p.logits + (size_t)warp * E;
+          float acc = 0.0f, acc2 = 0.0f;
+          const unsigned long long c0 = clock64();
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __ldcg(row + ((lane + 32 * j) % E));
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc += v[j];
+          const unsigned long long c1 = clock64() + (acc == 12345.0f ? 1u : 0u);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = row[(lane + 32 * j) % E];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc2 += v[j];
+          const unsigned long long c2 = clock64() + (acc2 == 12345.0f ? 1u : 0u);
+          if (lane == 0) {
+            g_layer_trace[7][b][0] = c1 - c0;
+            g_layer_trace[7][b][1] = c2 - c1;
+          }
+        }
+        // trace builds: the same top-k once before, into the scratch only, with its own stamps
+        topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, nullptr, nullptr, sc.tidx + warp * kLayerMaxK,
+                            sc.tw + warp * kLayerMaxK, sc.tks + warp * 64, &g_layer_trace[6][b][0]);
+        __syncwarp();
+      }
 #endif
       topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
                           writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
@@ -437,19 +466,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
       const int rot_c = (b * 37) % nc;
       auto code_piece = [&](int iu) { return iu + rot_c < nc ? iu + rot_c : iu + rot_c - nc; };
       for (int i0 = tid; i0 < nc + ns; i0 += 8 * nth) {
+        // every load of the round in flight together: pieces of rows >= T and past the end
+        // read piece 0 of the codes and are replaced by zeros
         uint4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int iu = i0 + u * nth;
-          v[u] = make_uint4(0u, 0u, 0u, 0u);
+          const uint4* src = reinterpret_cast<const uint4*>(p.xq_codes);
           if (iu < nc) {
             const int i = code_piece(iu), t = i / cpr;
-            if (t < T) v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + i % cpr);
+            if (t < T) src = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2)) + i % cpr;
           } else if (iu < nc + ns) {
             const int t = (iu - nc) / q4;
-            if (t < T)
-              v[u] = __ldcg(reinterpret_cast<const uint4*>(p.xq_scales + (size_t)t * (d / kBlock)) + (iu - nc) % q4);
+            if (t < T) src = reinterpret_cast<const uint4*>(p.xq_scales + (size_t)t * (d / kBlock)) + (iu - nc) % q4;
           }
+          v[u] = __ldcg(src);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int iu = i0 + u * nth;
+          const bool real = iu < nc ? code_piece(iu) / cpr < T : (iu < nc + ns && (iu - nc) / q4 < T);
+          if (!real) v[u] = make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {

@@ -34,11 +34,17 @@ MOE_DEV uint32_t ordered_key(float v) {
 // arg-max pick the winners one at a time, and only the winning lane rescans its entries.
 // Both give the same picks in the same order.
 // stamps (trace builds only): lane 0 records globaltimer after the loads, the threshold, the
-// selection and the weights into stamps[0..3]
+// selection and the weights into stamps[0..3], and the SM cycles since the previous point
+// (the first since entry) into stamps[4..7]
 #ifdef MOE_TRACE
 #define TOPK_STAMP(i)                                                    \
   do {                                                                   \
-    if (stamps != nullptr && lane == 0) stamps[i] = globaltimer_ns_rc(); \
+    if (stamps != nullptr && lane == 0) {                                \
+      stamps[i] = globaltimer_ns_rc();                                   \
+      const unsigned long long c_ = clock64();                           \
+      stamps[4 + (i)] = c_ - clk_prev;                                   \
+      clk_prev = c_;                                                     \
+    }                                                                    \
   } while (0)
 MOE_DEV unsigned long long globaltimer_ns_rc() {
   unsigned long long t;
@@ -53,14 +59,21 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
                         int* idx_smem = nullptr, float* w_smem = nullptr, uint32_t* scratch = nullptr,
                         unsigned long long* stamps = nullptr) {
   const int lane = threadIdx.x & 31;
-  uint32_t key[NPER];
+#ifdef MOE_TRACE
+  unsigned long long clk_prev = clock64();
+#endif
+  // every load first (entries past E read entry 0 and are masked below), so that they are
+  // all in flight together, then the keys
+  float val[NPER];
 #pragma unroll
   for (int j = 0; j < NPER; ++j) {
     const int e = lane + 32 * j;
-    float v = 0.0f;
-    if (e < E) v = kL2 ? __ldcg(row + e) : row[e];
-    key[j] = e < E ? ordered_key(v) : 0u;  // 0 is below every float's key
+    const float* src = row + (e < E ? e : 0);
+    val[j] = kL2 ? __ldcg(src) : *src;
   }
+  uint32_t key[NPER];
+#pragma unroll
+  for (int j = 0; j < NPER; ++j) key[j] = lane + 32 * j < E ? ordered_key(val[j]) : 0u;  // 0: below every key
   // does (ka, ea) come before (kb, eb): larger key, or equal key and lower index
   auto before = [](uint32_t ka, int ea, uint32_t kb, int eb) { return ka > kb || (ka == kb && ea < eb); };
   uint32_t taken = 0;
