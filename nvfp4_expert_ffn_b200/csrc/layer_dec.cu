@@ -392,63 +392,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
   }
 
   // ---------------------------------------------------------------- phase 2
-  // Data written by other CTAs before the barrier is read through L2 (ld.global.cg).
+  // Data written by other CTAs before the barrier is read with plain loads: the barrier's
+  // acquire, fence and block barrier make it visible, and plain loads are all in flight
+  // together (ld.global.cg loads were measured to complete one after another).
   const int nt1 = p.I / 64;
   const bool writer = b == G - 1;  // the CTA with the fewest units writes the routing outputs
   int nu = 0;
-#ifdef MOE_TRACE
-  // trace builds: the latency of one L2 load of data older than this launch (the router bias)
-  // and of one logit written by another CTA before the barrier, in SM cycles
-  if (ok && threadIdx.x == 0 && b < kTraceCtas && p.br) {
-    unsigned long long c0, c1, c2;
-    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c0));
-    const float a = __ldcg(p.br + (b * 7) % E);
-    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c1) : "f"(a));
-    const float l = __ldcg(p.logits + (size_t)((b * 131 + 17) % (T * E)));
-    asm volatile("mov.u64 %0, %%clock64;" : "=l"(c2) : "f"(l));
-    g_layer_trace[5][b][0] = c1 - c0;
-    g_layer_trace[5][b][1] = c2 - c1;
-    g_layer_trace[5][b][2] = __float_as_uint(a + l);
-  }
-#endif
   if (ok) {
     if (warp < T) {
       // token `warp`: its logits straight from L2 into the top-k; the chosen experts are
       // marked in s_bits
       unsigned long long* stamps = nullptr;
 #ifdef MOE_TRACE
-      if (warp == 0 && b < kTraceCtas) {
-        stamps = &g_layer_trace[4][b][0];
-        // trace builds: the 16 logit loads of the top-k alone, through L2 and plain, timed
-        {
-          const float* row = p.logits + (size_t)warp * E;
-          float acc = 0.0f, acc2 = 0.0f;
-          const unsigned long long c0 = clock64();
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __ldcg(row + ((lane + 32 * j) % E));
-#pragma unroll
-          for (int j = 0; j < 16; ++j) acc += v[j];
-          const unsigned long long c1 = clock64() + (acc == 12345.0f ? 1u : 0u);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = row[(lane + 32 * j) % E];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) acc2 += v[j];
-          const unsigned long long c2 = clock64() + (acc2 == 12345.0f ? 1u : 0u);
-          if (lane == 0) {
-            g_layer_trace[7][b][0] = c1 - c0;
-            g_layer_trace[7][b][1] = c2 - c1;
-          }
-        }
-        // trace builds: the same top-k once before, into the scratch only, with its own stamps
-        topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, nullptr, nullptr, sc.tidx + warp * kLayerMaxK,
-                            sc.tw + warp * kLayerMaxK, sc.tks + warp * 64, &g_layer_trace[6][b][0]);
-        __syncwarp();
-      }
+      if (warp == 0 && b < kTraceCtas) stamps = &g_layer_trace[4][b][0];
 #endif
-      topk_dispatch<true>(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
-                          writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
-                          sc.tw + warp * kLayerMaxK, sc.tks + warp * 64, stamps);
+      topk_dispatch(p.logits + (size_t)warp * E, E, k, writer ? p.topk_idx + (size_t)warp * k : nullptr,
+                    writer ? p.topk_w + (size_t)warp * k : nullptr, sc.tidx + warp * kLayerMaxK,
+                    sc.tw + warp * kLayerMaxK, sc.tks + warp * 64, stamps);
       RT_TRACE(g_layer_trace, 3, 0);
       __syncwarp();
       if (lane < k) {
@@ -480,7 +440,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
             const int t = (iu - nc) / q4;
             if (t < T) src = reinterpret_cast<const uint4*>(p.xq_scales + (size_t)t * (d / kBlock)) + (iu - nc) % q4;
           }
-          v[u] = __ldcg(src);
+          v[u] = *src;
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -635,13 +595,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
       for (int c0 = lane; c0 < n4; c0 += 32 * 8) {
         float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = c0 + 32 * u < n4 ? __ldcg(row + c0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 8; ++u) v[u] = row[c0 + 32 * u < n4 ? c0 + 32 * u : 0];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          ss = fmaf(v[u].x, v[u].x, ss);
-          ss = fmaf(v[u].y, v[u].y, ss);
-          ss = fmaf(v[u].z, v[u].z, ss);
-          ss = fmaf(v[u].w, v[u].w, ss);
+          if (c0 + 32 * u < n4) {
+            ss = fmaf(v[u].x, v[u].x, ss);
+            ss = fmaf(v[u].y, v[u].y, ss);
+            ss = fmaf(v[u].z, v[u].z, ss);
+            ss = fmaf(v[u].w, v[u].w, ss);
+          }
         }
       }
       const float ms = warp_sum(ss) / (float)d;
@@ -654,7 +616,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) layer_dec_kernel(LayerArgs p) 
     for (int c0 = lane; c0 < n4; c0 += 32 * 8) {
       float4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = c0 + 32 * u < n4 ? __ldcg(row + c0 + 32 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 8; ++u) v[u] = row[c0 + 32 * u < n4 ? c0 + 32 * u : 0];
 #pragma unroll
       for (int u = 0; u < 8; ++u)
         if (c0 + 32 * u < n4) out[c0 + 32 * u] = make_uint2(bf2(v[u].x, v[u].y), bf2(v[u].z, v[u].w));

@@ -22,9 +22,10 @@ MOE_DEV uint32_t ordered_key(float v) {
 
 // One warp per token. Lane L holds logits L, L+32, ... (keys that order like the floats).
 // Outputs (each may be NULL): idx_out / w_out in global memory, idx_smem / w_smem in shared
-// memory, k entries each, in descending logit order, ties to the lower expert id. With
-// kL2 = true the logits are read through L2 (ld.global.cg: written by other CTAs of the same
-// kernel).
+// memory, k entries each, in descending logit order, ties to the lower expert id. The logits
+// are read with plain loads: a row written by other CTAs of the same kernel is visible once
+// the grid barrier (acquire, fence, block barrier) has passed, and plain loads pipeline where
+// ld.global.cg loads were measured to complete one after another.
 //
 // With a 64-word shared scratch and k <= 32 the selection first takes a threshold: the k-th
 // largest of the 32 lane maxima. At least k logits reach it (those k maxima), so every logit
@@ -54,7 +55,7 @@ MOE_DEV unsigned long long globaltimer_ns_rc() {
 #else
 #define TOPK_STAMP(i) do { } while (0)
 #endif
-template <int NPER, bool kL2 = false>
+template <int NPER>
 MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* idx_out, float* w_out,
                         int* idx_smem = nullptr, float* w_smem = nullptr, uint32_t* scratch = nullptr,
                         unsigned long long* stamps = nullptr) {
@@ -69,7 +70,7 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
   for (int j = 0; j < NPER; ++j) {
     const int e = lane + 32 * j;
     const float* src = row + (e < E ? e : 0);
-    val[j] = kL2 ? __ldcg(src) : *src;
+    val[j] = *src;
   }
   uint32_t key[NPER];
 #pragma unroll
@@ -193,13 +194,12 @@ MOE_DEV void topk_token(const float* __restrict__ row, int E, int k, int32_t* id
 }
 
 // scratch: NULL, or 64 words of shared memory for this warp
-template <bool kL2 = false>
 MOE_DEV void topk_dispatch(const float* row, int E, int k, int32_t* idx, float* w, int* idx_smem = nullptr,
                            float* w_smem = nullptr, uint32_t* scratch = nullptr,
                            unsigned long long* stamps = nullptr) {
-  if (E <= 256) topk_token<8, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
-  else if (E <= 512) topk_token<16, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
-  else topk_token<32, kL2>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
+  if (E <= 256) topk_token<8>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
+  else if (E <= 512) topk_token<16>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
+  else topk_token<32>(row, E, k, idx, w, idx_smem, w_smem, scratch, stamps);
 }
 
 // The permutation of n <= 32*k assignments by one warp, without block-wide barriers:
