@@ -205,8 +205,9 @@ class GraphedMoeLayer:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=self.stream):
                 self.x.copy_(self.x_host[slot], non_blocking=True)
-                y = layer.forward(self.x, rms_renorm)
-                self.y_host.copy_(y, non_blocking=True)
+                y = layer.forward(self.x, rms_renorm, join=False)
+                self.y_host.copy_(y, non_blocking=True)  # y does not wait for the histogram
+                layer.join(self.stream)
             self.graphs.append(g)
 
     def run(self, slot: int = 0) -> None:
