@@ -43,10 +43,8 @@ DECODE_TRAFFIC_SOURCE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.s
                          "--cache-control none (1 pass) on 10 launches inside the 8-copy rotating decode loop "
                          "(T=8): 49.88 MB per launch against 57.09 MB of algorithmic bytes; the ratio is "
                          "applied to this run's algorithmic bytes")
-PREFILL_TRAFFIC_BYTES = 3_271_831_000  # tc_ffn_mt_kernel, T = 16384, one launch
-PREFILL_TRAFFIC_SOURCE = ("ncu --set full capture of tc_ffn_mt_kernel at T=16384 (caches flushed): "
-                          "dram__bytes_read.sum 2.168 GB + dram__bytes_write.sum 1.104 GB; the m-tile "
-                          "kernel only, not the schedule and row-gather launches of the call")
+PREFILL_TRAFFIC_BYTES = None  # tc_ffn_mt_kernel, T = 16384, one launch
+PREFILL_TRAFFIC_SOURCE = None
 
 
 def _peaks():
@@ -343,8 +341,10 @@ def measure_decode(timer, cfg, copies, xs, T, K, W, e2e_steps, stream, world, pe
             "frac": round(ach / peaks["hbm"], 4), "peak_kind": peaks["kind"] + " (HBM copy, burst)",
             "frac_vs_nominal_8tbs": round(ach / NOMINAL_HBM_GBS, 4),
             "bytes_per_launch": int(avg_b), "avg_launch_us": round(ms_k / K * 1e3, 3),
-            "traffic": None if DECODE_TRAFFIC_RATIO is None else int(avg_b * DECODE_TRAFFIC_RATIO),
-            "traffic_source": DECODE_TRAFFIC_SOURCE}
+            # the ratio was captured at T = 8 without a hot tier; other token counts are not measured
+            "traffic": (int(avg_b * DECODE_TRAFFIC_RATIO) if DECODE_TRAFFIC_RATIO is not None and T == 8 and not hot
+                        else None),
+            "traffic_source": DECODE_TRAFFIC_SOURCE if T == 8 and not hot else None}
     # end to end through the public API: each step is one replay of a graphed layer step that
     # copies the step's input from pinned host memory, runs the layer and copies y back
     if e2e_steps:
@@ -444,8 +444,8 @@ def measure_prefill(timer, cfg, layers, xs, K, W, e2e_steps, stream, world, peak
                         "peak_kind": f"{peaks['kind']} bf16 (burst) x 4, the nominal dense FP4 : bf16 ratio",
                         "flops_per_launch": flops, "weight_bytes_per_launch": int(wbytes),
                         "avg_launch_us": round(ms_f / K * 1e3, 3),
-                        "traffic": (PREFILL_TRAFFIC_BYTES if cfg.name == "prefill" and layers[0].input_scales is None
-                                    else None),
+                        "traffic": (PREFILL_TRAFFIC_BYTES if PREFILL_TRAFFIC_BYTES is not None and cfg.name == "prefill"
+                                    and layers[0].input_scales is None else None),
                         "traffic_source": (PREFILL_TRAFFIC_SOURCE if cfg.name == "prefill"
                                            and layers[0].input_scales is None else None)}}
     if e2e_steps:

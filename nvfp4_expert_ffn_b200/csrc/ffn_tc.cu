@@ -672,8 +672,14 @@ constexpr int kMtSfbBytes = 8 * kAtom;               // 4 KB: two atoms per K = 
 constexpr int kMtStageBytes = kMtABytes + kMtBBytes + kMtSfbBytes;
 constexpr int kMtColSfa = 256, kMtColSfb = 384;      // TMEM columns (accumulator at 0)
 constexpr int kMtMaxD = 2048, kMtMaxI = 768;
-constexpr size_t kMtSmemMax = 226 * 1024;
+constexpr size_t kMtSmemMax = 225 * 1024;  // + 2 KB of static shared memory = the 227 KB limit
 constexpr uint32_t kMtIdesc = idesc_mxf4nvf4(kTileM, kMtN);
+// Down tiles computed transposed, D[output column][token] (weights the A operand, two M = 128
+// halves of a 256-column tile; h the N = 128 B operand): each thread of the epilogue then
+// holds one output column for 32 tokens, and a warp's reduction covers 32 consecutive floats
+// (128 bytes) of one token's row of y.
+constexpr bool kMtDownTransposed = true;
+constexpr uint32_t kMtIdescDownT = idesc_mxf4nvf4(128, kTileM);
 constexpr bool kMtPregather = true;  // above 64 tokens: one TMA box of pre-gathered rows per stage
 
 __host__ __device__ inline size_t mt_h_bytes(int I) { return (size_t)(I / kStageK) * kMtABytes; }
@@ -698,6 +704,8 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
   __shared__ int s_epi_go[2];
+  __shared__ int s_orow[kTileM];  // this job's rows: output row (-1: padding) and factor, for the
+  __shared__ float s_f[kTileM];   // transposed down read-out
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = p.d, I = p.I;
@@ -868,10 +876,22 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
             tmem_cp_sf(sfb + 8 * kc, sdesc_sf(aS + kAtom * kc));                        // rows 0-127
             tmem_cp_sf(sfb + 8 * kc + 4, sdesc_sf(aS + kMtSfbBytes / 2 + kAtom * kc));  // rows 128-255
           }
+          if (phase1 || !kMtDownTransposed) {
 #pragma unroll
-          for (int kc = 0; kc < 4; ++kc)
-            mma_mxf4nvf4(tmem, sdesc_sw128(aA + 32 * kc), sdesc_sw128(aB + 32 * kc), kMtIdesc,
-                         tmem + kMtColSfa + 4 * (4 * ks + kc), sfb + 8 * kc, (kq | kc) ? 1u : 0u);
+            for (int kc = 0; kc < 4; ++kc)
+              mma_mxf4nvf4(tmem, sdesc_sw128(aA + 32 * kc), sdesc_sw128(aB + 32 * kc), kMtIdesc,
+                           tmem + kMtColSfa + 4 * (4 * ks + kc), sfb + 8 * kc, (kq | kc) ? 1u : 0u);
+          } else {
+            // output rows 0-127 and 128-255 of the tile (the two boxes) as A, h as B, into
+            // accumulator columns 0-127 and 128-255; the weight scales are the A scales
+#pragma unroll
+            for (int kc = 0; kc < 4; ++kc)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh)
+                mma_mxf4nvf4(tmem + 128 * hh, sdesc_sw128(aB + hh * (kMtBBytes / 2) + 32 * kc),
+                             sdesc_sw128(aA + 32 * kc), kMtIdescDownT, sfb + 8 * kc + 4 * hh,
+                             tmem + kMtColSfa + 4 * (4 * ks + kc), (kq | kc) ? 1u : 0u);
+          }
           mma_commit(&empty[st]);
         }
         mma_commit(&acc_full);
@@ -1009,6 +1029,48 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
         f = p.mode == 0 ? p.row_weight[prow] * ts_o : ts_o;
       }
       float* const obase = (p.mode != 0 && sh) ? p.shared_out : p.out;
+      if (kMtDownTransposed) {
+        // D[output column][token]: thread = output column 32q + lane of each 128-column half,
+        // its 32 registers = tokens 32cq .. 32cq + 31 (their output rows and factors from
+        // shared memory, published by the first tile's barrier)
+        if (cq == 0) {
+          s_orow[row] = orow;
+          s_f[row] = f;
+        }
+        for (int nq = 0; nq < nt2 && go; ++nq) {
+          const int n = (nq + rn) % nt2;
+          if (!(go = wait_acc())) break;
+          uint32_t v[2][32];
+          tmem_ld32(lane_base + 32 * cq, v[0]);
+          tmem_ld32(lane_base + 128 + 32 * cq, v[1]);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty);
+          if (ew == 0 && lane == 0) MT_TRACE(kEvDrainEnd, jc, tix);
+          ++tc;
+          const int ocol = kMtN * n + 32 * q + lane;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int orr = s_orow[32 * cq + j];
+            const float fr = s_f[32 * cq + j];
+            if (orr >= 0) {
+              float* o = obase + (size_t)orr * d + ocol;
+              const float a0 = __uint_as_float(v[0][j]) * fr, a1 = __uint_as_float(v[1][j]) * fr;
+              if (p.mode == 0) {
+                red_add_f32(o, a0);
+                red_add_f32(o + 128, a1);
+              } else {
+                o[0] = a0;
+                o[128] = a1;
+              }
+            }
+          }
+          if (ew == 0 && lane == 0) MT_TRACE(kEvEpiEnd, jc, tix);
+          ++tix;
+        }
+        continue;
+      }
       const bool odd = (lane & 1) != 0;
       const int src0 = (lane >> 2) + 8 * (lane & 1);  // quarter row of half 0 after the swap
       int orh[2];
