@@ -38,13 +38,15 @@ X_DRAWS = 4             # input draws per decode layer copy
 NOMINAL_HBM_GBS = 8000.0  # B200 spec-sheet HBM3e bandwidth, for context beside the measured peak
 # DRAM bytes (read + write) per launch of the dominant kernels from ncu captures of the
 # current kernels (profiles/); None when the kernel has changed since its capture
-DECODE_TRAFFIC_RATIO = 0.874  # layer_dec_kernel: traffic / algorithmic bytes in the rotating loop
+DECODE_TRAFFIC_RATIO = 0.899  # layer_dec_kernel: traffic / algorithmic bytes in the rotating loop
 DECODE_TRAFFIC_SOURCE = ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
-                         "--cache-control none (1 pass) on 10 launches inside the 8-copy rotating decode loop "
-                         "(T=8): 49.88 MB per launch against 57.09 MB of algorithmic bytes; the ratio is "
+                         "--cache-control none (1 pass) on 16 launches inside the 8-copy rotating decode loop "
+                         "(T=8): 51.27 MB per launch against 57.05 MB of algorithmic bytes; the ratio is "
                          "applied to this run's algorithmic bytes")
-PREFILL_TRAFFIC_BYTES = None  # tc_ffn_mt_kernel, T = 16384, one launch
-PREFILL_TRAFFIC_SOURCE = None
+PREFILL_TRAFFIC_BYTES = 3_275_270_000  # tc_ffn_mt_kernel, T = 16384, one launch
+PREFILL_TRAFFIC_SOURCE = ("ncu --set full (caches flushed before the passes) on one launch of tc_ffn_mt_kernel "
+                          "at T=16384: 2.173 GB read + 1.103 GB written; about 2.1 GB of it is the float32 "
+                          "output y (128 MB) leaving L2 between its 11 reductions per token")
 
 
 def _peaks():
