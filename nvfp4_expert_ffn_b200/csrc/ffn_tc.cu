@@ -140,66 +140,100 @@ __global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
 
 // ---------------------------------------------------------------- 1b. row gather (large T)
 // With many rows per m-tile, every phase-1 tile of an m-tile would gather the same rows
-// again, 4 rows per TMA request; instead one warp per row copies the row's d/2 code bytes
-// into a contiguous [m-tile row][d/2] buffer (one TMA box per stage then), its d/16 scale
-// bytes into the m-tile's scale atoms, and writes the row's (token, weight, output slot).
+// again, 4 rows per TMA request; instead the rows' d/2 code bytes are copied into a
+// contiguous [m-tile row][d/2] buffer (one TMA box per stage then), their d/16 scale bytes
+// into the m-tile's scale atoms, and each row's (token, weight, output slot) is written.
+// A warp takes 32 rows of one m-tile: lane r resolves row r's token through the expert's
+// offset and the sorted assignment, so the 32 rows' chains of dependent index loads overlap;
+// the warp then copies the rows kGatherRows at a time, all their loads issued before the
+// stores.
+constexpr int kGatherRows = 8;
+
 __global__ void __launch_bounds__(256) tc_row_gather_kernel(TcParams p) {
   MOE_PDL_PROLOGUE();
   const int n_m = *p.n_mtiles;
   const int lane = threadIdx.x & 31;
   const int nw = (gridDim.x * blockDim.x) >> 5;
   const int d = p.d;
-  for (int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < n_m * kTileM; w += nw) {
-    const int m = w / kTileM, r = w % kTileM;
-    if (r >= p.mt_valid[m]) continue;
+  for (int g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < n_m * (kTileM / 32); g += nw) {
+    const int m = g / (kTileM / 32), r0 = 32 * (g % (kTileM / 32));
+    const int valid = p.mt_valid[m];
+    if (r0 >= valid) continue;
     const int e = p.mt_expert[m];
-    const int i = p.mt_first[m] + r;
-    int t = i, slot = -1;
-    float wgt = 1.0f;
-    if (e < p.E) {
-      const int q = p.offsets[e] + i;
-      const int a = p.sorted_assign[q];
-      t = a / p.k;
-      wgt = p.topk_w[a];
-      slot = q;
-    }
-    if (p.x_bf16) {
-      // static input scales: the token's bf16 row quantised with its expert's own tensor
-      // scale. Lane l takes 16-element blocks l, l + 32, ...: its 8 code bytes go to the
-      // gathered row, its scale byte into the m-tile's scale atom.
-      const float ts = p.in_gu[e];
-      const uint4* xsrc = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)t * d);
-      uint2* cdst = reinterpret_cast<uint2*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
-      for (int blk = lane; blk < d / kBlock; blk += 32) {
-        const uint4 lo = __ldg(xsrc + 2 * blk), hi = __ldg(xsrc + 2 * blk + 1);
-        const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        float v[16];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v[2 * i] = __uint_as_float(wv[i] << 16);
-          v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-        }
-        uint2 cw;
-        const uint32_t sb = quantize_block16(v, ts, &cw);
-        cdst[blk] = cw;
-        p.sfa1[((size_t)m * (d / 64) + blk / 4) * kAtom + (r % 32) * 16 + (r / 32) * 4 + blk % 4] = (uint8_t)sb;
+    const int nr = min(32, valid - r0);
+    const int r = r0 + lane;
+    int t = 0;
+    if (lane < nr) {
+      const int i = p.mt_first[m] + r;
+      int slot = -1;
+      float wgt = 1.0f;
+      t = i;
+      if (e < p.E) {
+        const int q = p.offsets[e] + i;
+        const int a = p.sorted_assign[q];
+        t = a / p.k;
+        wgt = p.topk_w[a];
+        slot = q;
       }
-    } else {
-      if (p.a1) {
-        const uint4* csrc = reinterpret_cast<const uint4*>(p.xq_codes + (size_t)t * (d / 2));
-        uint4* cdst = reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r) * (d / 2));
-        for (int c = lane; c < d / 32; c += 32) cdst[c] = __ldg(csrc + c);
-      }
-      const uint32_t* ssrc = reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)t * (d / kBlock));
-      for (int kc = lane; kc < d / 64; kc += 32)
-        *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (r % 32) * 16 + (r / 32) * 4) =
-            __ldg(ssrc + kc);
-    }
-    if (lane == 0) {
       const size_t prow = (size_t)m * kTileM + r;
       p.row_token[prow] = t;
       p.row_weight[prow] = wgt;
       p.row_slot[prow] = slot;
+    }
+    if (p.x_bf16) {
+      // static input scales: each token's bf16 row quantised with its expert's own tensor
+      // scale. Lane l takes 16-element blocks l, l + 32, ...: its 8 code bytes go to the
+      // gathered row, its scale byte into the m-tile's scale atom.
+      const float ts = p.in_gu[e];
+      for (int j = 0; j < nr; ++j) {
+        const int tj = __shfl_sync(0xffffffffu, t, j);
+        const int rj = r0 + j;
+        const uint4* xsrc = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)tj * d);
+        uint2* cdst = reinterpret_cast<uint2*>(p.a1 + ((size_t)m * kTileM + rj) * (d / 2));
+        for (int blk = lane; blk < d / kBlock; blk += 32) {
+          const uint4 lo = __ldg(xsrc + 2 * blk), hi = __ldg(xsrc + 2 * blk + 1);
+          const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[2 * i] = __uint_as_float(wv[i] << 16);
+            v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+          }
+          uint2 cw;
+          const uint32_t sb = quantize_block16(v, ts, &cw);
+          cdst[blk] = cw;
+          p.sfa1[((size_t)m * (d / 64) + blk / 4) * kAtom + (rj % 32) * 16 + (rj / 32) * 4 + blk % 4] = (uint8_t)sb;
+        }
+      }
+      continue;
+    }
+    for (int j0 = 0; j0 < nr; j0 += kGatherRows) {
+      int tj[kGatherRows];
+#pragma unroll
+      for (int u = 0; u < kGatherRows; ++u) tj[u] = __shfl_sync(0xffffffffu, t, (j0 + u) & 31);
+      if (p.a1) {
+        for (int c = lane; c < d / 32; c += 32) {
+          uint4 v[kGatherRows];
+#pragma unroll
+          for (int u = 0; u < kGatherRows; ++u)
+            if (j0 + u < nr) v[u] = __ldg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)tj[u] * (d / 2)) + c);
+#pragma unroll
+          for (int u = 0; u < kGatherRows; ++u)
+            if (j0 + u < nr) reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r0 + j0 + u) * (d / 2))[c] = v[u];
+        }
+      }
+      for (int kc = lane; kc < d / 64; kc += 32) {
+        uint32_t v[kGatherRows];
+#pragma unroll
+        for (int u = 0; u < kGatherRows; ++u)
+          if (j0 + u < nr) v[u] = __ldg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)tj[u] * (d / kBlock)) + kc);
+#pragma unroll
+        for (int u = 0; u < kGatherRows; ++u) {
+          const int rj = r0 + j0 + u;
+          if (j0 + u < nr)
+            *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (rj % 32) * 16 + (rj / 32) * 4) = v[u];
+        }
+      }
     }
   }
 }
@@ -651,17 +685,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) tc_ffn_kernel(const __grid_cons
 //   gate/up: I/128 tiles of N = 256 weight rows (gate and up rows of two 64-row slices of I,
 //            in the order the scale atoms hold them), K = d; SwiGLU and the NVFP4
 //            quantisation of h in the epilogue, h written into this CTA's shared memory in
-//            the layout the down GEMM reads as its A operand;
-//   down:    d/256 tiles of N = 256 output rows, K = I, A = that h tile; the epilogue adds
-//            w * o into y with vector reductions from registers (or stores o).
+//            the layout the down GEMM reads as its token operand;
+//   down:    d/256 tiles of 256 output rows, K = I, computed transposed (the two 128-row
+//            weight boxes as A, that h tile as the N = 128 B operand); the epilogue adds
+//            w * o into y with reductions from registers (or stores o).
 // The activation scale atoms of the m-tile (K = d) and then those of h (K = I) stay in TMEM
 // for all of the job's tiles, so a K = 64 step needs only the two weight scale copies next to
 // its N = 256 MMA (each tcgen05.cp takes the tensor pipe about as long as a 128-column MMA).
 // One N = 256 accumulator (TMEM has no room for a second one beside the scales): the
 // epilogue takes its columns into registers first and releases it before its own math; 16
 // epilogue warps (four per TMEM lane quarter, 64 columns each) keep that math short.
-// y of every token the call covers receives about k + 1 reductions; the caller splits the
-// tokens into chunks whose y fits in L2 (launch_ffn_tc).
+// y of every token the call covers receives about k + 1 float32 reductions, 128 contiguous
+// bytes of one row per warp instruction (the down tiles are computed transposed).
 constexpr int kMtN = 256;
 constexpr int kMtStages = 3;
 constexpr int kMtEpiWarps = 16;
