@@ -35,6 +35,9 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s (decode T=1–8, prefill T=16K); % of HBM BW / FP4 MMA peak"
 SEED = 0
 X_DRAWS = 4             # input draws per decode layer copy
+# prefill layer copies: each has its own buffers and, end to end, its own stream, so one step's
+# 64 MB host copies in and out overlap the neighbouring steps' compute
+PREFILL_COPIES = 3
 NOMINAL_HBM_GBS = 8000.0  # B200 spec-sheet HBM3e bandwidth, for context beside the measured peak
 # DRAM bytes (read + write) per launch of the dominant kernels from ncu captures of the
 # current kernels (profiles/); None when the kernel has changed since its capture
@@ -615,11 +618,11 @@ def run_gpu(args):
             if not args.no_hot:
                 extra[f"decode_T{T}_hot_tier"] = measure_decode(timer, cfg, copies, xs, T, K, W, 0, stream, world,
                                                                 peaks, hot=True)
-            pcfg, players, pxs = build_prefill_layers(device, "prefill", copies, 2)
+            pcfg, players, pxs = build_prefill_layers(device, "prefill", copies, PREFILL_COPIES)
             extra["prefill_T16384"] = measure_prefill(timer, pcfg, players, pxs, K, W, e2e_steps, stream, world,
                                                       peaks)
             extra["prefill_T16384"]["workload"] = ("prefill MoE layer: the decode layer's weights, Zipf(0.8) "
-                                                   "routing, T=16384 tokens per step, 2 layer copies")
+                                                   f"routing, T=16384 tokens per step, {PREFILL_COPIES} layer copies")
             del players
             pcfg, players, pxs = build_prefill_layers(device, "prefill", copies, 2, static_scales=True)
             extra["prefill_T16384_static_scales"] = measure_prefill(timer, pcfg, players, pxs, K, W, 0, stream,
@@ -628,6 +631,15 @@ def run_gpu(args):
                 "prefill_T16384 with static per-expert input scales: every expert quantises its own rows "
                 "(moe_expert_ffn_static), no per-call activation quantisation")
             del players
+            wcfg, players, pxs = build_prefill_layers(device, "wide", None, 2)
+            extra[f"wide_T{pxs[0].shape[0]}"] = measure_prefill(timer, wcfg, players, pxs, K, W, e2e_steps, stream,
+                                                                world, peaks)
+            extra[f"wide_T{pxs[0].shape[0]}"]["workload"] = (
+                f"wide chunked prefill MoE layer: d={wcfg.d}, {wcfg.E} experts, top-{wcfg.k} + 1 shared, "
+                f"I={wcfg.I}, NVFP4 weights, T={pxs[0].shape[0]} tokens per step (512 + 2048 + 8192 + 16384 + 4), "
+                "uniform routing, 2 layer copies")
+            del players
+            torch.cuda.empty_cache()
             if not args.no_stack:
                 del copies, xs
                 torch.cuda.empty_cache()

@@ -148,8 +148,12 @@ __global__ void __launch_bounds__(1024) tc_schedule_kernel(TcParams p) {
 // the warp then copies the rows kGatherRows at a time, all their loads issued before the
 // stores.
 constexpr int kGatherRows = 8;
+constexpr int kGatherQuantMaxD = 2048;  // static input scales need the m-tile kernel: d <= its limit
 
-__global__ void __launch_bounds__(256) tc_row_gather_kernel(TcParams p) {
+// QUANT: the static-input-scale form (rows quantised from p.x_bf16), a kernel of its own so
+// that its registers do not lower the plain copy's occupancy.
+template <bool QUANT>
+__global__ void __launch_bounds__(256, QUANT ? 2 : 3) tc_row_gather_kernel(TcParams p) {
   MOE_PDL_PROLOGUE();
   const int n_m = *p.n_mtiles;
   const int lane = threadIdx.x & 31;
@@ -180,58 +184,79 @@ __global__ void __launch_bounds__(256) tc_row_gather_kernel(TcParams p) {
       p.row_weight[prow] = wgt;
       p.row_slot[prow] = slot;
     }
-    if (p.x_bf16) {
+    if constexpr (QUANT) {
       // static input scales: each token's bf16 row quantised with its expert's own tensor
       // scale. Lane l takes 16-element blocks l, l + 32, ...: its 8 code bytes go to the
       // gathered row, its scale byte into the m-tile's scale atom.
+      // (d <= kGatherQuantMaxD: at most kQBlk blocks per lane; the loads of two rows go out first)
+      constexpr int kQBlk = kGatherQuantMaxD / kBlock / 32;
       const float ts = p.in_gu[e];
-      for (int j = 0; j < nr; ++j) {
-        const int tj = __shfl_sync(0xffffffffu, t, j);
-        const int rj = r0 + j;
-        const uint4* xsrc = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)tj * d);
-        uint2* cdst = reinterpret_cast<uint2*>(p.a1 + ((size_t)m * kTileM + rj) * (d / 2));
-        for (int blk = lane; blk < d / kBlock; blk += 32) {
-          const uint4 lo = __ldg(xsrc + 2 * blk), hi = __ldg(xsrc + 2 * blk + 1);
-          const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-          float v[16];
+      const int nblk = d / kBlock;
+      for (int j0 = 0; j0 < nr; j0 += 2) {
+        uint4 raw[2][kQBlk][2];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[2 * i] = __uint_as_float(wv[i] << 16);
-            v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        for (int u = 0; u < 2; ++u) {
+          const int tj = __shfl_sync(0xffffffffu, t, (j0 + u) & 31);
+          const uint4* xsrc = reinterpret_cast<const uint4*>(p.x_bf16 + (size_t)tj * d);
+#pragma unroll
+          for (int b = 0; b < kQBlk; ++b) {
+            const int blk = lane + 32 * b;
+            const bool ld = j0 + u < nr && blk < nblk;
+            raw[u][b][0] = ld ? __ldg(xsrc + 2 * blk) : make_uint4(0u, 0u, 0u, 0u);
+            raw[u][b][1] = ld ? __ldg(xsrc + 2 * blk + 1) : make_uint4(0u, 0u, 0u, 0u);
           }
-          uint2 cw;
-          const uint32_t sb = quantize_block16(v, ts, &cw);
-          cdst[blk] = cw;
-          p.sfa1[((size_t)m * (d / 64) + blk / 4) * kAtom + (rj % 32) * 16 + (rj / 32) * 4 + blk % 4] = (uint8_t)sb;
         }
-      }
-      continue;
-    }
-    for (int j0 = 0; j0 < nr; j0 += kGatherRows) {
-      int tj[kGatherRows];
 #pragma unroll
-      for (int u = 0; u < kGatherRows; ++u) tj[u] = __shfl_sync(0xffffffffu, t, (j0 + u) & 31);
-      if (p.a1) {
-        for (int c = lane; c < d / 32; c += 32) {
-          uint4 v[kGatherRows];
-#pragma unroll
-          for (int u = 0; u < kGatherRows; ++u)
-            if (j0 + u < nr) v[u] = __ldg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)tj[u] * (d / 2)) + c);
-#pragma unroll
-          for (int u = 0; u < kGatherRows; ++u)
-            if (j0 + u < nr) reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r0 + j0 + u) * (d / 2))[c] = v[u];
-        }
-      }
-      for (int kc = lane; kc < d / 64; kc += 32) {
-        uint32_t v[kGatherRows];
-#pragma unroll
-        for (int u = 0; u < kGatherRows; ++u)
-          if (j0 + u < nr) v[u] = __ldg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)tj[u] * (d / kBlock)) + kc);
-#pragma unroll
-        for (int u = 0; u < kGatherRows; ++u) {
+        for (int u = 0; u < 2; ++u) {
           const int rj = r0 + j0 + u;
-          if (j0 + u < nr)
-            *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (rj % 32) * 16 + (rj / 32) * 4) = v[u];
+          if (j0 + u >= nr) break;
+          uint2* cdst = reinterpret_cast<uint2*>(p.a1 + ((size_t)m * kTileM + rj) * (d / 2));
+#pragma unroll
+          for (int b = 0; b < kQBlk; ++b) {
+            const int blk = lane + 32 * b;
+            if (blk >= nblk) break;
+            const uint4 lo = raw[u][b][0], hi = raw[u][b][1];
+            const uint32_t wv[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            float v[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              v[2 * i] = __uint_as_float(wv[i] << 16);
+              v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+            }
+            uint2 cw;
+            const uint32_t sb = quantize_block16(v, ts, &cw);
+            cdst[blk] = cw;
+            p.sfa1[((size_t)m * (d / 64) + blk / 4) * kAtom + (rj % 32) * 16 + (rj / 32) * 4 + blk % 4] = (uint8_t)sb;
+          }
+        }
+      }
+    } else {
+      for (int j0 = 0; j0 < nr; j0 += kGatherRows) {
+        int tj[kGatherRows];
+#pragma unroll
+        for (int u = 0; u < kGatherRows; ++u) tj[u] = __shfl_sync(0xffffffffu, t, (j0 + u) & 31);
+        if (p.a1) {
+          for (int c = lane; c < d / 32; c += 32) {
+            uint4 v[kGatherRows];
+#pragma unroll
+            for (int u = 0; u < kGatherRows; ++u)
+              if (j0 + u < nr) v[u] = __ldg(reinterpret_cast<const uint4*>(p.xq_codes + (size_t)tj[u] * (d / 2)) + c);
+#pragma unroll
+            for (int u = 0; u < kGatherRows; ++u)
+              if (j0 + u < nr) reinterpret_cast<uint4*>(p.a1 + ((size_t)m * kTileM + r0 + j0 + u) * (d / 2))[c] = v[u];
+          }
+        }
+        for (int kc = lane; kc < d / 64; kc += 32) {
+          uint32_t v[kGatherRows];
+#pragma unroll
+          for (int u = 0; u < kGatherRows; ++u)
+            if (j0 + u < nr) v[u] = __ldg(reinterpret_cast<const uint32_t*>(p.xq_scales + (size_t)tj[u] * (d / kBlock)) + kc);
+#pragma unroll
+          for (int u = 0; u < kGatherRows; ++u) {
+            const int rj = r0 + j0 + u;
+            if (j0 + u < nr)
+              *reinterpret_cast<uint32_t*>(p.sfa1 + ((size_t)m * (d / 64) + kc) * kAtom + (rj % 32) * 16 + (rj / 32) * 4) = v[u];
+          }
         }
       }
     }
@@ -707,6 +732,7 @@ constexpr int kMtSfbBytes = 8 * kAtom;               // 4 KB: two atoms per K = 
 constexpr int kMtStageBytes = kMtABytes + kMtBBytes + kMtSfbBytes;
 constexpr int kMtColSfa = 256, kMtColSfb = 384;      // TMEM columns (accumulator at 0)
 constexpr int kMtMaxD = 2048, kMtMaxI = 768;
+static_assert(kMtMaxD <= kGatherQuantMaxD, "the row gather quantises rows of up to kGatherQuantMaxD");
 constexpr size_t kMtSmemMax = 225 * 1024;  // + 2 KB of static shared memory = the 227 KB limit
 constexpr uint32_t kMtIdesc = idesc_mxf4nvf4(kTileM, kMtN);
 // Down tiles computed transposed, D[output column][token] (weights the A operand, two M = 128
@@ -1326,10 +1352,12 @@ cudaError_t launch_ffn_tc(const FfnArgs& a, void* ws, int num_sms, int32_t* stat
   if ((e = launch_pdl(tc_schedule_kernel, dim3(1 + zc), dim3(1024), 0, st, p)) != cudaSuccess) return e;
   if (mt) {
     // m-tile kernel: rows gathered once per m-tile, then one job per m-tile
-    if ((e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess) return e;
+    e = per_expert ? launch_pdl(tc_row_gather_kernel<true>, dim3(num_sms * 8), dim3(256), 0, st, p)
+                   : launch_pdl(tc_row_gather_kernel<false>, dim3(num_sms * 8), dim3(256), 0, st, p);
+    if (e != cudaSuccess) return e;
     return launch_pdl(tc_ffn_mt_kernel, dim3(num_sms), dim3(kMtThreads), mt_smem_bytes(a.d, a.I), st, maps, p);
   }
-  if (p.a1 && (e = launch_pdl(tc_row_gather_kernel, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess)
+  if (p.a1 && (e = launch_pdl(tc_row_gather_kernel<false>, dim3(num_sms * 8), dim3(256), 0, st, p)) != cudaSuccess)
     return e;
   return launch_pdl(tc_ffn_kernel, dim3(num_sms), dim3(kTcThreads), ffn_tc_smem_bytes(), st, maps, p);
 }
