@@ -739,7 +739,6 @@ constexpr uint32_t kMtIdesc = idesc_mxf4nvf4(kTileM, kMtN);
 // halves of a 256-column tile; h the N = 128 B operand): each thread of the epilogue then
 // holds one output column for 32 tokens, and a warp's reduction covers 32 consecutive floats
 // (128 bytes) of one token's row of y.
-constexpr bool kMtDownTransposed = true;
 constexpr uint32_t kMtIdescDownT = idesc_mxf4nvf4(128, kTileM);
 constexpr bool kMtPregather = true;  // above 64 tokens: one TMA box of pre-gathered rows per stage
 
@@ -937,7 +936,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
             tmem_cp_sf(sfb + 8 * kc, sdesc_sf(aS + kAtom * kc));                        // rows 0-127
             tmem_cp_sf(sfb + 8 * kc + 4, sdesc_sf(aS + kMtSfbBytes / 2 + kAtom * kc));  // rows 128-255
           }
-          if (phase1 || !kMtDownTransposed) {
+          if (phase1) {
 #pragma unroll
             for (int kc = 0; kc < 4; ++kc)
               mma_mxf4nvf4(tmem, sdesc_sw128(aA + 32 * kc), sdesc_sw128(aB + 32 * kc), kMtIdesc,
@@ -1075,12 +1074,7 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
       fence_proxy_async_smem();
       named_bar_sync(2, 32 * kMtEpiWarps);
       if (ew == 0 && lane == 0) mbar_arrive(&h_ready);
-      // ---- down tiles: w * o added into y (or o stored). The warp reads its 32 rows x 64
-      // columns as two 16-row halves in the .16x256b shape (thread t: rows t/4 and t/4 + 8 of
-      // the half, columns 8i + 2(t%4) and +1); neighbouring lanes then swap one pair, so that
-      // each holds 4 consecutive columns of one row: row t/4 + 8(t%2) of the half, columns
-      // 8i + 4((t/2)%2) .. +3. A warp's vector reduction covers 16 rows x 32 contiguous bytes
-      // (two lanes per row) instead of 32 rows x 16 bytes, which L2 absorbs about twice as fast.
+      // ---- down tiles: w * o added into y (or o stored)
       const float ts_o = G.dn_ts[eloc] * ts_h;
       int orow = -1;  // output row of this thread's m-tile row (lane = row), -1 if padding
       float f = 0.0f;
@@ -1090,87 +1084,39 @@ __global__ void __launch_bounds__(kMtThreads, 1) tc_ffn_mt_kernel(const __grid_c
         f = p.mode == 0 ? p.row_weight[prow] * ts_o : ts_o;
       }
       float* const obase = (p.mode != 0 && sh) ? p.shared_out : p.out;
-      if (kMtDownTransposed) {
-        // D[output column][token]: thread = output column 32q + lane of each 128-column half,
-        // its 32 registers = tokens 32cq .. 32cq + 31 (their output rows and factors from
-        // shared memory, published by the first tile's barrier)
-        if (cq == 0) {
-          s_orow[row] = orow;
-          s_f[row] = f;
-        }
-        for (int nq = 0; nq < nt2 && go; ++nq) {
-          const int n = (nq + rn) % nt2;
-          if (!(go = wait_acc())) break;
-          uint32_t v[2][32];
-          tmem_ld32(lane_base + 32 * cq, v[0]);
-          tmem_ld32(lane_base + 128 + 32 * cq, v[1]);
-          tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty);
-          if (ew == 0 && lane == 0) MT_TRACE(kEvDrainEnd, jc, tix);
-          ++tc;
-          const int ocol = kMtN * n + 32 * q + lane;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int orr = s_orow[32 * cq + j];
-            const float fr = s_f[32 * cq + j];
-            if (orr >= 0) {
-              float* o = obase + (size_t)orr * d + ocol;
-              const float a0 = __uint_as_float(v[0][j]) * fr, a1 = __uint_as_float(v[1][j]) * fr;
-              if (p.mode == 0) {
-                red_add_f32(o, a0);
-                red_add_f32(o + 128, a1);
-              } else {
-                o[0] = a0;
-                o[128] = a1;
-              }
-            }
-          }
-          if (ew == 0 && lane == 0) MT_TRACE(kEvEpiEnd, jc, tix);
-          ++tix;
-        }
-        continue;
+      // D[output column][token]: thread = output column 32q + lane of each 128-column half,
+      // its 32 registers = tokens 32cq .. 32cq + 31 (their output rows and factors from
+      // shared memory, published by the first tile's barrier)
+      if (cq == 0) {
+        s_orow[row] = orow;
+        s_f[row] = f;
       }
-      const bool odd = (lane & 1) != 0;
-      const int src0 = (lane >> 2) + 8 * (lane & 1);  // quarter row of half 0 after the swap
-      int orh[2];
-      float fh[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        orh[h] = __shfl_sync(0xffffffffu, orow, src0 + 16 * h);
-        fh[h] = __shfl_sync(0xffffffffu, f, src0 + 16 * h);
-      }
-      const int coff = 4 * ((lane >> 1) & 1);
       for (int nq = 0; nq < nt2 && go; ++nq) {
         const int n = (nq + rn) % nt2;
         if (!(go = wait_acc())) break;
         uint32_t v[2][32];
-        tmem_ld16x256b_x8(lane_base + 64 * cq, v[0]);
-        tmem_ld16x256b_x8(lane_base + (16u << 16) + 64 * cq, v[1]);
+        tmem_ld32(lane_base + 32 * cq, v[0]);
+        tmem_ld32(lane_base + 128 + 32 * cq, v[1]);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty);
         if (ew == 0 && lane == 0) MT_TRACE(kEvDrainEnd, jc, tix);
         ++tc;
+        const int ocol = kMtN * n + 32 * q + lane;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float* o = orh[h] >= 0 ? obase + (size_t)orh[h] * d + kMtN * n + 64 * cq + coff : nullptr;
-          const float fr = fh[h];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t r0 = __shfl_xor_sync(0xffffffffu, odd ? v[h][4 * i] : v[h][4 * i + 2], 1);
-            const uint32_t r1 = __shfl_xor_sync(0xffffffffu, odd ? v[h][4 * i + 1] : v[h][4 * i + 3], 1);
-            const float a0 = __uint_as_float(odd ? r0 : v[h][4 * i]) * fr;
-            const float a1 = __uint_as_float(odd ? r1 : v[h][4 * i + 1]) * fr;
-            const float a2 = __uint_as_float(odd ? v[h][4 * i + 2] : r0) * fr;
-            const float a3 = __uint_as_float(odd ? v[h][4 * i + 3] : r1) * fr;
-            if (o != nullptr) {
-              if (p.mode == 0)
-                red_add_v4(o + 8 * i, a0, a1, a2, a3);
-              else
-                *reinterpret_cast<float4*>(o + 8 * i) = make_float4(a0, a1, a2, a3);
+        for (int j = 0; j < 32; ++j) {
+          const int orr = s_orow[32 * cq + j];
+          const float fr = s_f[32 * cq + j];
+          if (orr >= 0) {
+            float* o = obase + (size_t)orr * d + ocol;
+            const float a0 = __uint_as_float(v[0][j]) * fr, a1 = __uint_as_float(v[1][j]) * fr;
+            if (p.mode == 0) {
+              red_add_f32(o, a0);
+              red_add_f32(o + 128, a1);
+            } else {
+              o[0] = a0;
+              o[128] = a1;
             }
           }
         }
