@@ -792,7 +792,7 @@ def main():
     ap.add_argument("--workload", choices=["decode", "prefill", "wide", "stack48"], default="decode")
     ap.add_argument("--no-hot", action="store_true", help="skip the hot-tier (L2 persisting) measurements")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-steps", type=int, default=4)
+    ap.add_argument("--cpu-steps", type=int, default=16, help="oracle decode forwards timed (about 10 s)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="only the headline workload")
     ap.add_argument("--no-stack", action="store_true", help="leave out the 48-layer decode stack")
